@@ -1,0 +1,413 @@
+"""Benchmark of the FlexPrefill prefill-attention hot path on B200.
+
+One step = one pass of the whole path over one attention layer (all heads):
+fp_estimate -> fp_pattern -> fp_select -> fp_sparse_attn, on seeded synthetic
+Q/K/V shaped like a Llama-3.1-8B layer at 128k tokens (32 q / 8 kv heads,
+d = 128, block 128).  Prints ONE JSON line (rank 0).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+--impl reference times the CPU oracle (the plain fp64 restatement of the
+method) on a bounded sample of the same workload.  Multi-GPU runs (torchrun)
+give every rank its own layer (independent problems, weak scaling); there is
+no exchange on the data path.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from dynamic_block_sparse_fp_b200 import synth  # noqa: E402
+
+METRIC = "prefill-attn tokens/s and effective TFLOPS (% bf16 peak) at 128k; speedup vs dense"
+LAUNCHES_PER_STEP = 12  # estimate 8, pattern 1, select 2, attention 1
+
+
+def load_peaks() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle samples over the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self) -> dict:
+        rows = []
+        if self.path and os.path.exists(self.path):
+            for line in open(self.path):
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+            os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v == "Active"})
+        busy = [s for s in sm if s > 0.5 * (max(mx) if mx else 1)] or sm
+        return {"sm_mhz": statistics.median(busy) if busy else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+def dist_setup():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        import datetime
+        torch.distributed.init_process_group(
+            "nccl" if torch.cuda.is_available() else "gloo",
+            timeout=datetime.timedelta(seconds=600))
+    return ws, rank, local
+
+
+def max_over_ranks(x: float, ws: int, device) -> float:
+    if ws == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(ws: int):
+    if ws > 1:
+        torch.distributed.barrier()
+
+
+# ------------------------------------------------------------ CPU baseline --
+
+def cpu_oracle_sample(w: synth.Workload, heads=(0,), q_blocks=None) -> dict:
+    """Time the oracle on a bounded sample and extrapolate to the full layer.
+
+    Sample: the estimate, pattern and select of ``heads`` (every q head costs
+    the same there) and attention of ``q_blocks`` rows of those heads, scaled
+    by the kept blocks of the whole layer.
+    """
+    import numpy as np
+
+    import oracle
+    kvs = sorted({h // (w.n_q_heads // w.n_kv_heads) for h in heads})
+    inp = synth.make_inputs(w, kv_heads=kvs)
+    g = w.n_q_heads // w.n_kv_heads
+    loc = [kvs.index(h // g) * g + h % g for h in heads]
+    q = inp["q"][:, loc]
+    kk = inp["k"][:, [kvs.index(h // g) for h in heads]]
+    vv = inp["v"][:, [kvs.index(h // g) for h in heads]]
+    # each sampled head gets its own kv head copy (GQA index h // 1)
+    t0 = time.perf_counter()
+    est = oracle.estimate(q, kk, w.block_size)
+    t1 = time.perf_counter()
+    e32 = {x: est[x].astype(np.float32) for x in ("map", "est_last", "true_last", "vert",
+                                                    "slash")}
+    _, pat = oracle.pattern(e32["est_last"], e32["true_last"], w.tau)
+    counts, indices = oracle.select(pat, e32["map"], e32["vert"], e32["slash"], w.n_blocks,
+                                    w.block_size, w.gamma, w.min_budget, w.max_budget)
+    t2 = time.perf_counter()
+    nb = w.n_blocks
+    qbs = q_blocks if q_blocks is not None else [nb - 1, (3 * nb) // 4, nb // 2, nb // 4]
+    oracle.sparse_attention(q, kk, vv, counts, indices, w.block_size, heads=list(range(len(heads))),
+                            q_blocks=qbs)
+    t3 = time.perf_counter()
+    kept_sample = int(sum(counts[0, i, qb] for i in range(len(heads)) for qb in qbs))
+    kept_heads = int(counts.sum())
+    nh = len(heads)
+    t_est = (t1 - t0) / nh * w.n_q_heads
+    t_sel = (t2 - t1) / nh * w.n_q_heads
+    # attention time per kept block, times the kept blocks of every head
+    # (sampled heads' mean stands in for the others)
+    t_att = (t3 - t2) / max(kept_sample, 1) * (kept_heads / nh) * w.n_q_heads
+    total = t_est + t_sel + t_att
+    return {"seconds_measured": t3 - t0, "seconds_extrapolated": total,
+            "tokens_per_s": w.seq_len * w.batch / total,
+            "sample": (f"oracle (numpy fp64) on q heads {list(heads)} of {w.name}: estimate, "
+                       f"pattern and select in full, attention on query blocks {qbs} "
+                       f"({kept_sample} kept blocks); extrapolated to {w.n_q_heads} heads and "
+                       f"all kept blocks")}
+
+
+def cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def workload_config(w: synth.Workload, ws: int) -> dict:
+    return {"workload": w.name, "batch_per_gpu": w.batch, "global_batch": w.batch * ws,
+            "seq_len": w.seq_len, "n_q_heads": w.n_q_heads, "n_kv_heads": w.n_kv_heads,
+            "head_dim": w.head_dim, "block_size": w.block_size, "gamma": w.gamma, "tau": w.tau,
+            "min_budget": w.min_budget, "max_budget": w.max_budget,
+            "parallelism": f"independent layers x{ws}" if ws > 1 else "single GPU",
+            "l2": "no flush: every step streams Q (1.07 GB at 128k) and K/V, inputs larger "
+                  "than the 126 MB L2"}
+
+
+def run_reference(args, w, ws, rank):
+    if rank != 0:
+        return
+    steps = []
+    for i in range(args.warmup + args.steps):
+        r = cpu_oracle_sample(w)
+        if i >= args.warmup:
+            steps.append(r)
+    tps = statistics.mean(r["tokens_per_s"] for r in steps)
+    line = {"impl": "reference", "metric": METRIC, "value": tps, "unit": "tokens/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1000.0 * w.seq_len * w.batch / tps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": workload_config(w, 1),
+            "cpu_baseline": {"value": tps, "unit": "tokens/s", "cores": cores(),
+                             "kind": "oracle", "sample": steps[0]["sample"]},
+            "e2e": {"value": tps, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# --------------------------------------------------------------------- ours --
+
+def run_ours(args, w, ws, rank, local):
+    from dynamic_block_sparse_fp_b200 import build, ops
+
+    build.build()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    peaks = load_peaks()
+    # every rank: its own independent layer (batch index = rank)
+    wr = w.replace(seed=w.seed + 1000 * rank) if rank else w
+    inp = synth.make_inputs(wr)
+    q, k, v = (inp[x].to(dev) for x in ("q", "k", "v"))
+    bt, hq, n, d = q.shape
+    hkv, bs = k.shape[1], w.block_size
+    nb = n // bs
+    s = ops.make_shape(q, k, bs)
+    p = ops.make_params(w.gamma, w.tau, w.min_budget, w.max_budget)
+    f32 = dict(dtype=torch.float32, device=dev)
+    qbar = torch.empty(bt, hq, nb, d, **f32)
+    kbar = torch.empty(bt, hkv, nb, d, **f32)
+    amap = torch.empty(bt, hq, nb * (nb + 1) // 2, **f32)
+    est_last = torch.empty(bt, hq, nb, **f32)
+    true_last = torch.empty(bt, hq, nb, **f32)
+    vert = torch.empty(bt, hq, n, **f32)
+    slash = torch.empty(bt, hq, n, **f32)
+    djs = torch.empty(bt, hq, **f32)
+    pat = torch.empty(bt, hq, dtype=torch.int32, device=dev)
+    counts = torch.empty(bt, hq, nb, dtype=torch.int32, device=dev)
+    indices = torch.empty(bt, hq, nb, nb, dtype=torch.int32, device=dev)
+    out = torch.empty_like(q)
+    ws_est = ops.workspace(s, ops.FP_CALL_ESTIMATE, dev)
+    ws_sel = ops.workspace(s, ops.FP_CALL_SELECT, dev)
+    stream = torch.cuda.current_stream(dev)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)]
+          for _ in range(args.warmup + args.steps)]
+
+    def step(e):
+        e[0].record(stream)
+        ops._check(ops.fp_estimate(s, q, k, qbar, kbar, amap, est_last, true_last, vert, slash,
+                                   ws_est, stream), "fp_estimate")
+        e[1].record(stream)
+        ops._check(ops.fp_pattern(s, p, est_last, true_last, djs, pat, stream), "fp_pattern")
+        e[2].record(stream)
+        ops._check(ops.fp_select(s, p, pat, amap, vert, slash, counts, indices, ws_sel, stream),
+                   "fp_select")
+        e[3].record(stream)
+        ops._check(ops.fp_sparse_attn(s, q, k, v, counts, indices, out, None, None, stream),
+                   "fp_sparse_attn")
+        e[4].record(stream)
+
+    for i in range(args.warmup):
+        step(ev[i])
+    torch.cuda.synchronize()
+    assert ops.fp_last_device_status(stream) == 0
+    barrier(ws)
+    torch.cuda.synchronize()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        t_start.record(stream)
+        for i in range(args.warmup, args.warmup + args.steps):
+            step(ev[i])
+        t_end.record(stream)
+        torch.cuda.synchronize()
+    barrier(ws)
+    status = ops.fp_last_device_status(stream)
+    if status != 0:
+        raise RuntimeError(f"device status {ops.STATUS.get(status, status)}")
+    total_ms = max_over_ranks(t_start.elapsed_time(t_end), ws, dev)
+    ms_step = total_ms / args.steps
+    timed = ev[args.warmup:]
+    stage_ms = [statistics.mean(e[j].elapsed_time(e[j + 1]) for e in timed) for j in range(4)]
+    kept = int(counts.sum())
+    qa_heads = int((pat == ops.FP_PATTERN_QA).sum())
+    t_pairs = nb * (nb + 1) // 2
+    flop_block = 4.0 * bs * bs * d
+    attn_flops = flop_block * kept
+    attn_tflops = attn_flops / (stage_ms[3] * 1e-3) / 1e12
+    tokens = n * bt
+    value = ws * tokens / (ms_step * 1e-3)
+    # dense comparison at the same length (same kernel over every causal block)
+    dense_ms = None
+    if not args.no_dense:
+        dout = torch.empty_like(q)
+        de = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        ops._check(ops.fp_dense_attn(s, q, k, v, dout, None, stream), "fp_dense_attn")
+        de[0].record(stream)
+        reps = 2
+        for _ in range(reps):
+            ops._check(ops.fp_dense_attn(s, q, k, v, dout, None, stream), "fp_dense_attn")
+        de[1].record(stream)
+        torch.cuda.synchronize()
+        dense_ms = de[0].elapsed_time(de[1]) / reps
+        del dout
+    # estimate: algorithmic bytes = read Q and K once + write its outputs
+    eb = q.element_size()
+    est_bytes = (q.numel() + k.numel()) * eb + 4 * (qbar.numel() + kbar.numel() + amap.numel()
+                                                   + est_last.numel() + true_last.numel()
+                                                   + vert.numel() + slash.numel())
+    peak_t = peaks["bf16_tflops_sustained"]
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded Q/K/V with planted query-aware / vertical-slash structure "
+                "and RoPE; no dataset or weights)",
+        "config": workload_config(w, ws),
+        "roofline": {"bound": "tensor", "kernel": "fp_sparse_attn", "achieved": attn_tflops,
+                     "peak": peak_t, "unit": "TFLOP/s", "frac": attn_tflops / peak_t,
+                     "traffic": None,
+                     "peak_kind": f"bf16 dense, sustained ({peaks['source']})",
+                     "algorithmic_flops_per_launch": attn_flops},
+        "gpu_launches": LAUNCHES_PER_STEP * args.steps,
+        "stages_ms": {"estimate": stage_ms[0], "pattern": stage_ms[1], "select": stage_ms[2],
+                      "sparse_attn": stage_ms[3]},
+        "estimate_hbm": {"bytes": est_bytes, "gbs": est_bytes / (stage_ms[0] * 1e-3) / 1e9,
+                         "frac": est_bytes / (stage_ms[0] * 1e-3) / 1e9 / peaks["hbm_gbs"]},
+        "effective_tflops": {"sparse_attn": attn_tflops,
+                             "whole_step": attn_flops / (ms_step * 1e-3) / 1e12},
+        "kept_blocks": kept, "causal_blocks": t_pairs * hq * bt,
+        "kept_fraction": kept / (t_pairs * hq * bt), "qa_heads": qa_heads,
+        "sparsity_implied_ratio": t_pairs * hq * bt / kept,
+    }
+    if dense_ms is not None:
+        line["dense_attn_ms"] = dense_ms
+        line["dense_tflops"] = flop_block * t_pairs * hq * bt / (dense_ms * 1e-3) / 1e12
+        line["speedup_vs_dense"] = {"whole_step": dense_ms / ms_step,
+                                    "sparse_attn_only": dense_ms / stage_ms[3]}
+    line["clocks"] = clk.summary()
+    # ---- end to end through the C ABI with host buffers ----
+    if not args.no_e2e:
+        qh, kh, vh = (inp[x].contiguous().pin_memory() for x in ("q", "k", "v"))
+        oh = torch.empty_like(qh).pin_memory()
+        del out, indices
+        torch.cuda.empty_cache()
+        wsh = ops.workspace(s, ops.FP_CALL_PREFILL_HOST, dev)
+        ops._check(ops.fp_prefill_attn_host(s, p, qh, kh, vh, oh, wsh, stream), "host")
+        torch.cuda.synchronize()
+        a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier(ws)
+        a.record(stream)
+        for _ in range(args.e2e_steps):
+            ops._check(ops.fp_prefill_attn_host(s, p, qh, kh, vh, oh, wsh, stream), "host")
+        b_.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = max_over_ranks(a.elapsed_time(b_) / args.e2e_steps, ws, dev)
+        h2d = (qh.numel() + kh.numel() + vh.numel()) * qh.element_size()
+        line["e2e"] = {"value": ws * tokens / (e2e_ms * 1e-3), "unit": "tokens/s",
+                       "h2d_bytes_per_step": h2d,
+                       "d2h_bytes_per_step": oh.numel() * oh.element_size(),
+                       "ms_per_step": e2e_ms, "steps": args.e2e_steps,
+                       "api": "fp_prefill_attn_host (pinned host q/k/v in, out back)"}
+    if rank == 0 and not args.no_cpu_baseline:
+        cb = cpu_oracle_sample(w)
+        line["cpu_baseline"] = {"value": cb["tokens_per_s"], "unit": "tokens/s",
+                                "cores": cores(), "kind": "oracle", "sample": cb["sample"],
+                                "seconds_measured": cb["seconds_measured"]}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="llama8b_n131072", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--gamma", type=float)
+    ap.add_argument("--tau", type=float)
+    ap.add_argument("--min-budget", type=int)
+    ap.add_argument("--max-budget", type=int)
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-dense", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    w = synth.WORKLOADS[args.workload]
+    over = {k: v for k, v in (("gamma", args.gamma), ("tau", args.tau),
+                              ("min_budget", args.min_budget),
+                              ("max_budget", args.max_budget)) if v is not None}
+    if over:
+        w = w.replace(**over)
+    ws, rank, local = dist_setup()
+    try:
+        if args.impl == "reference":
+            run_reference(args, w, ws, rank)
+        else:
+            run_ours(args, w, ws, rank, local)
+    finally:
+        if ws > 1 and torch.distributed.is_initialized():
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

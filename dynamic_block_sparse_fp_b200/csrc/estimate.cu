@@ -1,0 +1,402 @@
+// estimate.cu -- fp_estimate: block pooling, the estimated block map, and the
+// true attention of the last query block with its vertical / slash sums.
+//
+// FlexPrefill (atlas.scime.ai summary, "Approach"): per head, a block-pooled
+// attention estimate from the last query block is compared with the true
+// distribution; the vertical-slash fallback is driven by column and diagonal
+// attention sums of the same last block.
+//
+// Kernels (all reductions in a fixed order, so results are reproducible):
+//   pool_kernel          mean of each B-token block of q and k (HBM stream)
+//   map_logits_kernel    scaled qbar.kbar^T for the causal block pairs
+//   map_softmax_kernel   in-place row softmax of the packed map, + est_last
+//   last_pass1_kernel    per (head, key block): row max / sum of exp of the
+//                        last query block's logits (online-softmax partials)
+//   last_lse_kernel      combine partials -> log-sum-exp of each last-block row
+//   last_pass2_kernel    per (head, key block): P = exp(logit - lse); column
+//                        sums (vert), block mass (true_last), diagonal partials
+//   slash_combine_kernel diagonal partials of neighbouring key blocks -> slash
+#include <math.h>
+
+#include "fp_internal.cuh"
+
+namespace fpi {
+namespace {
+
+template <class T>
+__device__ __forceinline__ float ld_f(const T *p);
+template <>
+__device__ __forceinline__ float ld_f<float>(const float *p) { return *p; }
+template <>
+__device__ __forceinline__ float ld_f<__nv_bfloat16>(const __nv_bfloat16 *p) {
+  return __bfloat162float(*p);
+}
+
+// 8 consecutive elements as fp32 (16 B for bf16, 32 B for fp32).
+__device__ __forceinline__ void ld8(const float *p, float (&x)[8]) {
+  float4 a = *reinterpret_cast<const float4 *>(p);
+  float4 b = *reinterpret_cast<const float4 *>(p + 4);
+  x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
+  x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+}
+__device__ __forceinline__ void ld8(const __nv_bfloat16 *p, float (&x)[8]) {
+  uint4 u = *reinterpret_cast<const uint4 *>(p);
+  const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&u);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    float2 f = __bfloat1622float2(h[i]);
+    x[2 * i] = f.x;
+    x[2 * i + 1] = f.y;
+  }
+}
+
+// ------------------------------------------------------------------ pooling --
+// grid (nb, heads, Bt), 256 threads.  x [Bt, heads, N, d] -> out [Bt, heads, nb, d].
+template <class T>
+__global__ void __launch_bounds__(256) pool_kernel(const T *__restrict__ x, float *__restrict__ out,
+                                                   int n, int d, int bs) {
+  __shared__ float part[32][128];
+  const int blk = blockIdx.x, head = blockIdx.y, b = blockIdx.z;
+  const int heads = gridDim.y, nb = gridDim.x;
+  const int vec_per_row = d / 8;
+  const int rows_per_it = 256 / vec_per_row;
+  const int tv = threadIdx.x % vec_per_row, tr = threadIdx.x / vec_per_row;
+  const T *base = x + ((size_t(b) * heads + head) * n + size_t(blk) * bs) * d;
+  float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  for (int r = tr; r < bs; r += rows_per_it) {
+    float v[8];
+    ld8(base + size_t(r) * d + tv * 8, v);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i] += v[i];
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) part[tr][tv * 8 + i] = acc[i];
+  __syncthreads();
+  if (threadIdx.x < d) {
+    float s = 0.f;
+    for (int r = 0; r < rows_per_it; ++r) s += part[r][threadIdx.x];
+    out[((size_t(b) * heads + head) * nb + blk) * d + threadIdx.x] = s / float(bs);
+  }
+}
+
+// ------------------------------------------------------------ block map --
+// grid (tiles, tiles, Bt*Hq), 256 threads; 64x64 tile of the nb x nb logit
+// matrix of one q head; tiles above the diagonal exit at once.
+__global__ void __launch_bounds__(256) map_logits_kernel(const float *__restrict__ qbar,
+                                                         const float *__restrict__ kbar,
+                                                         float *__restrict__ map, int hq, int g,
+                                                         int nb, int d, float scale) {
+  const int ti = blockIdx.x, tj = blockIdx.y;
+  if (tj > ti) return;
+  const int bh = blockIdx.z, b = bh / hq, h = bh % hq, kv = h / g;
+  const int hkv = hq / g;
+  __shared__ float As[32][65];
+  __shared__ float Bs[32][65];
+  const float *qa = qbar + (size_t(b) * hq + h) * nb * d;
+  const float *kb = kbar + (size_t(b) * hkv + kv) * nb * d;
+  const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
+  float acc[4][4] = {};
+  for (int k0 = 0; k0 < d; k0 += 32) {
+    for (int e = threadIdx.x; e < 64 * 32; e += 256) {
+      int r = e / 32, c = e % 32;
+      int gi = ti * 64 + r, gj = tj * 64 + r;
+      As[c][r] = gi < nb ? qa[size_t(gi) * d + k0 + c] : 0.f;
+      Bs[c][r] = gj < nb ? kb[size_t(gj) * d + k0 + c] : 0.f;
+    }
+    __syncthreads();
+#pragma unroll 8
+    for (int c = 0; c < 32; ++c) {
+      float a[4], bb[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) a[u] = As[c][ty + 16 * u];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) bb[u] = Bs[c][tx + 16 * u];
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int w = 0; w < 4; ++w) acc[u][w] = fmaf(a[u], bb[w], acc[u][w]);
+    }
+    __syncthreads();
+  }
+  float *m = map + (size_t(b) * hq + h) * (size_t(nb) * (nb + 1) / 2);
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    int i = ti * 64 + ty + 16 * u;
+    if (i >= nb) continue;
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      int j = tj * 64 + tx + 16 * w;
+      if (j <= i) m[size_t(i) * (i + 1) / 2 + j] = acc[u][w] * scale;
+    }
+  }
+}
+
+// One warp per map row; 8 rows per CTA.
+__global__ void __launch_bounds__(256) map_softmax_kernel(float *__restrict__ map,
+                                                          float *__restrict__ est_last,
+                                                          long long rows_total, int nb) {
+  const long long row = (long long)blockIdx.x * 8 + threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+  if (row >= rows_total) return;
+  const long long bh = row / nb;
+  const int i = int(row % nb);
+  float *r = map + bh * ((long long)nb * (nb + 1) / 2) + (long long)i * (i + 1) / 2;
+  const int len = i + 1;
+  float mx = -INFINITY;
+  for (int j = lane; j < len; j += 32) mx = fmaxf(mx, r[j]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  float s = 0.f;
+  for (int j = lane; j < len; j += 32) s += expf(r[j] - mx);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  const float inv = 1.f / s;
+  for (int j = lane; j < len; j += 32) {
+    float p = expf(r[j] - mx) * inv;
+    r[j] = p;
+    if (i == nb - 1) est_last[bh * nb + j] = p;
+  }
+}
+
+// ---------------------------------------------------- last query block --
+// S tile: scale * q_last[BS x D] . k_tile[BS x D]^T into smem S[BS][BS+1],
+// causally masked (-inf) when the key tile is the diagonal one.
+template <int BS, int D, class T>
+struct LastTile {
+  static constexpr int KC = 32;
+  static constexpr int TPR = BS / 16;  // outputs per thread along each axis
+  float A[KC][BS + 1];
+  float Bm[KC][BS + 1];
+  float S[BS][BS + 1];
+};
+
+template <int BS, int D, class T>
+__device__ void last_tile_scores(LastTile<BS, D, T> &sm, const T *__restrict__ qlast,
+                                 const T *__restrict__ ktile, float scale, bool diagonal) {
+  constexpr int KC = LastTile<BS, D, T>::KC;
+  constexpr int TPR = LastTile<BS, D, T>::TPR;
+  const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
+  float acc[TPR][TPR];
+#pragma unroll
+  for (int u = 0; u < TPR; ++u)
+#pragma unroll
+    for (int w = 0; w < TPR; ++w) acc[u][w] = 0.f;
+  for (int k0 = 0; k0 < D; k0 += KC) {
+    for (int e = threadIdx.x; e < BS * KC; e += 256) {
+      int r = e / KC, c = e % KC;
+      sm.A[c][r] = ld_f(qlast + size_t(r) * D + k0 + c);
+      sm.Bm[c][r] = ld_f(ktile + size_t(r) * D + k0 + c);
+    }
+    __syncthreads();
+#pragma unroll 4
+    for (int c = 0; c < KC; ++c) {
+      float a[TPR], bb[TPR];
+#pragma unroll
+      for (int u = 0; u < TPR; ++u) a[u] = sm.A[c][ty + 16 * u];
+#pragma unroll
+      for (int u = 0; u < TPR; ++u) bb[u] = sm.Bm[c][tx + 16 * u];
+#pragma unroll
+      for (int u = 0; u < TPR; ++u)
+#pragma unroll
+        for (int w = 0; w < TPR; ++w) acc[u][w] = fmaf(a[u], bb[w], acc[u][w]);
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int u = 0; u < TPR; ++u)
+#pragma unroll
+    for (int w = 0; w < TPR; ++w) {
+      int r = ty + 16 * u, c = tx + 16 * w;
+      sm.S[r][c] = (diagonal && c > r) ? -INFINITY : acc[u][w] * scale;
+    }
+  __syncthreads();
+}
+
+// grid (nb, Hq, Bt), 256 threads.
+template <int BS, int D, class T>
+__global__ void __launch_bounds__(256) last_pass1_kernel(const T *__restrict__ q,
+                                                         const T *__restrict__ k, int hq, int g,
+                                                         int n, float scale,
+                                                         float *__restrict__ pm,
+                                                         float *__restrict__ pl) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  auto &sm = *reinterpret_cast<LastTile<BS, D, T> *>(smem_raw);
+  const int j = blockIdx.x, h = blockIdx.y, b = blockIdx.z, nb = gridDim.x;
+  const int kv = h / g, hkv = hq / g;
+  const T *qlast = q + ((size_t(b) * hq + h) * n + (n - BS)) * D;
+  const T *kt = k + ((size_t(b) * hkv + kv) * n + size_t(j) * BS) * D;
+  last_tile_scores<BS, D, T>(sm, qlast, kt, scale, j == nb - 1);
+  // 256 threads, BS rows: 256/BS threads per row
+  constexpr int TPRW = 256 / BS;
+  const int r = threadIdx.x / TPRW, part = threadIdx.x % TPRW;
+  float mx = -INFINITY;
+  for (int c = part; c < BS; c += TPRW) mx = fmaxf(mx, sm.S[r][c]);
+#pragma unroll
+  for (int o = TPRW / 2; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  float s = 0.f;
+  if (mx > -INFINITY)
+    for (int c = part; c < BS; c += TPRW) s += expf(sm.S[r][c] - mx);
+#pragma unroll
+  for (int o = TPRW / 2; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  if (part == 0) {
+    size_t o = ((size_t(b) * hq + h) * nb + j) * BS + r;
+    pm[o] = mx;
+    pl[o] = s;
+  }
+}
+
+// one thread per (b, h, r): lse over the nb partials, in key-block order.
+__global__ void last_lse_kernel(const float *__restrict__ pm, const float *__restrict__ pl,
+                                float *__restrict__ lse, int rows, int nb, int bs) {
+  const int t = blockIdx.x * blockDim.x + threadIdx.x;
+  if (t >= rows) return;
+  const int bh = t / bs, r = t % bs;
+  float mx = -INFINITY;
+  for (int j = 0; j < nb; ++j) mx = fmaxf(mx, pm[(size_t(bh) * nb + j) * bs + r]);
+  float s = 0.f;
+  for (int j = 0; j < nb; ++j) {
+    size_t o = (size_t(bh) * nb + j) * bs + r;
+    if (pm[o] > -INFINITY) s += pl[o] * expf(pm[o] - mx);
+  }
+  lse[t] = mx + logf(s);
+}
+
+template <int BS, int D, class T>
+__global__ void __launch_bounds__(256) last_pass2_kernel(
+    const T *__restrict__ q, const T *__restrict__ k, int hq, int g, int n, float scale,
+    const float *__restrict__ lse, float *__restrict__ vert, float *__restrict__ true_last,
+    float *__restrict__ sp) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  auto &sm = *reinterpret_cast<LastTile<BS, D, T> *>(smem_raw);
+  __shared__ float colsum[BS];
+  const int j = blockIdx.x, h = blockIdx.y, b = blockIdx.z, nb = gridDim.x;
+  const int kv = h / g, hkv = hq / g;
+  const size_t bh = size_t(b) * hq + h;
+  const T *qlast = q + (bh * n + (n - BS)) * D;
+  const T *kt = k + ((size_t(b) * hkv + kv) * n + size_t(j) * BS) * D;
+  last_tile_scores<BS, D, T>(sm, qlast, kt, scale, j == nb - 1);
+  for (int e = threadIdx.x; e < BS * BS; e += 256) {
+    int r = e / BS, c = e % BS;
+    float s = sm.S[r][c];
+    sm.S[r][c] = (s == -INFINITY) ? 0.f : expf(s - lse[bh * BS + r]);
+  }
+  __syncthreads();
+  if (threadIdx.x < BS) {
+    const int c = threadIdx.x;
+    float s = 0.f;
+    for (int r = 0; r < BS; ++r) s += sm.S[r][c];
+    colsum[c] = s;
+    vert[bh * n + size_t(j) * BS + c] = s;
+  }
+  // diagonal partials: delta = r - c + BS - 1 in [0, 2BS-2]
+  if (threadIdx.x < 2 * BS - 1) {
+    const int delta = threadIdx.x;
+    float s = 0.f;
+    int r0 = delta - (BS - 1) > 0 ? delta - (BS - 1) : 0;
+    int r1 = delta < BS - 1 ? delta : BS - 1;
+    for (int r = r0; r <= r1; ++r) s += sm.S[r][r - delta + BS - 1];
+    sp[(bh * nb + j) * (2 * BS - 1) + delta] = s;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float s = 0.f;
+    for (int c = 0; c < BS; ++c) s += colsum[c];
+    true_last[bh * nb + j] = s / float(BS);
+  }
+}
+
+// one thread per (b, h, o): slash[o] from the (at most two) key blocks whose
+// diagonal partials hold offset o.
+__global__ void slash_combine_kernel(const float *__restrict__ sp, float *__restrict__ slash,
+                                     long long total, int n, int nb, int bs) {
+  const long long t = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (t >= total) return;
+  const long long bh = t / n;
+  const int o = int(t % n);
+  // tile j holds o at delta = o - n + (j + 2) * bs - 1, valid in [0, 2bs-2]
+  int jlo = (n - o + 1 + bs - 1) / bs - 2;
+  if (jlo < 0) jlo = 0;
+  int jhi = (n - o - 1) / bs;
+  if (jhi > nb - 1) jhi = nb - 1;
+  float s = 0.f;
+  for (int j = jlo; j <= jhi; ++j) {
+    int delta = o - n + (j + 2) * bs - 1;
+    if (delta >= 0 && delta <= 2 * bs - 2) s += sp[(bh * nb + j) * (2 * bs - 1) + delta];
+  }
+  slash[t] = s;
+}
+
+template <int BS, int D, class T>
+cudaError_t run_last(const Dims &Dm, const T *q, const T *k, float *true_last, float *vert,
+                     float *slash, void *ws, cudaStream_t st) {
+  Carver c{static_cast<char *>(ws), 0};
+  const size_t rows = size_t(Dm.bt) * Dm.hq;
+  float *pm = c.take<float>(rows * Dm.nb * BS);
+  float *pl = c.take<float>(rows * Dm.nb * BS);
+  float *lse = c.take<float>(rows * BS);
+  float *sp = c.take<float>(rows * Dm.nb * (2 * BS - 1));
+  const float scale = 1.f / sqrtf(float(D));
+  const size_t smem = sizeof(LastTile<BS, D, T>);
+  cudaFuncSetAttribute(last_pass1_kernel<BS, D, T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                       int(smem));
+  cudaFuncSetAttribute(last_pass2_kernel<BS, D, T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                       int(smem));
+  dim3 grid(Dm.nb, Dm.hq, Dm.bt);
+  last_pass1_kernel<BS, D, T><<<grid, 256, smem, st>>>(q, k, Dm.hq, Dm.g, Dm.n, scale, pm, pl);
+  const int lrows = int(rows * BS);
+  last_lse_kernel<<<(lrows + 127) / 128, 128, 0, st>>>(pm, pl, lse, lrows, Dm.nb, BS);
+  last_pass2_kernel<BS, D, T><<<grid, 256, smem, st>>>(q, k, Dm.hq, Dm.g, Dm.n, scale, lse, vert,
+                                                       true_last, sp);
+  const long long tot = (long long)rows * Dm.n;
+  slash_combine_kernel<<<unsigned((tot + 255) / 256), 256, 0, st>>>(sp, slash, tot, Dm.n, Dm.nb,
+                                                                    BS);
+  return cudaGetLastError();
+}
+
+template <class T>
+cudaError_t run_estimate(const Dims &Dm, const T *q, const T *k, float *qbar, float *kbar,
+                         float *map, float *est_last, float *true_last, float *vert,
+                         float *slash, void *ws, cudaStream_t st) {
+  pool_kernel<T><<<dim3(Dm.nb, Dm.hq, Dm.bt), 256, 0, st>>>(q, qbar, Dm.n, Dm.d, Dm.bs);
+  pool_kernel<T><<<dim3(Dm.nb, Dm.hkv, Dm.bt), 256, 0, st>>>(k, kbar, Dm.n, Dm.d, Dm.bs);
+  const int tiles = (Dm.nb + 63) / 64;
+  const float scale = 1.f / sqrtf(float(Dm.d));
+  map_logits_kernel<<<dim3(tiles, tiles, Dm.bt * Dm.hq), 256, 0, st>>>(qbar, kbar, map, Dm.hq,
+                                                                      Dm.g, Dm.nb, Dm.d, scale);
+  const long long rows = (long long)Dm.bt * Dm.hq * Dm.nb;
+  map_softmax_kernel<<<unsigned((rows + 7) / 8), 256, 0, st>>>(map, est_last, rows, Dm.nb);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  if (Dm.bs == 128 && Dm.d == 128)
+    return run_last<128, 128, T>(Dm, q, k, true_last, vert, slash, ws, st);
+  if (Dm.bs == 128 && Dm.d == 64)
+    return run_last<128, 64, T>(Dm, q, k, true_last, vert, slash, ws, st);
+  if (Dm.bs == 64 && Dm.d == 128)
+    return run_last<64, 128, T>(Dm, q, k, true_last, vert, slash, ws, st);
+  return run_last<64, 64, T>(Dm, q, k, true_last, vert, slash, ws, st);
+}
+
+}  // namespace
+
+size_t estimate_ws_bytes(const Dims &D) {
+  Carver c{nullptr, 0};
+  const size_t rows = size_t(D.bt) * D.hq;
+  c.take<float>(rows * D.nb * D.bs);
+  c.take<float>(rows * D.nb * D.bs);
+  c.take<float>(rows * D.bs);
+  c.take<float>(rows * D.nb * (2 * D.bs - 1));
+  return c.off + 256;
+}
+
+cudaError_t launch_estimate(const Dims &D, const void *q, const void *k, float *qbar,
+                            float *kbar, float *map, float *est_last, float *true_last,
+                            float *vert, float *slash, void *ws, cudaStream_t st) {
+  if (D.dtype == FP_F32)
+    return run_estimate<float>(D, static_cast<const float *>(q), static_cast<const float *>(k),
+                               qbar, kbar, map, est_last, true_last, vert, slash, ws, st);
+  return run_estimate<__nv_bfloat16>(D, static_cast<const __nv_bfloat16 *>(q),
+                                     static_cast<const __nv_bfloat16 *>(k), qbar, kbar, map,
+                                     est_last, true_last, vert, slash, ws, st);
+}
+
+}  // namespace fpi

@@ -1,0 +1,351 @@
+// fp_api.cu -- the extern "C" entry points of include/fp.h: argument
+// validation (on the host, before any launch), workspace layout, dispatch to
+// the stage launchers, and the per-device status word.
+#include <math.h>
+
+#include <algorithm>
+
+#include "fp_internal.cuh"
+
+#define FP_API extern "C" __attribute__((visibility("default")))
+
+namespace fpi {
+
+__device__ int g_fp_status;  // first device-side error since the last read
+
+int *device_status_ptr() {
+  static int *ptrs[64] = {nullptr};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  if (!ptrs[dev]) {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_fp_status) == cudaSuccess) ptrs[dev] = static_cast<int *>(p);
+  }
+  return ptrs[dev];
+}
+
+namespace {
+
+fp_status check_shape(const fp_shape *s, Dims *D) {
+  if (!s) return FP_ERR_NULL;
+  if (s->dtype != FP_BF16 && s->dtype != FP_F32) return FP_ERR_DTYPE;
+  if (s->batch < 1 || s->n_q_heads < 1 || s->n_kv_heads < 1 || s->seq_len < 1)
+    return FP_ERR_SHAPE;
+  if (s->n_q_heads % s->n_kv_heads != 0) return FP_ERR_SHAPE;
+  if (s->block_size != 64 && s->block_size != 128) return FP_ERR_SHAPE;
+  if (s->head_dim != 64 && s->head_dim != 128) return FP_ERR_SHAPE;
+  if (s->seq_len % s->block_size != 0) return FP_ERR_SHAPE;
+  const long long nb = s->seq_len / s->block_size;
+  if (nb > 4096) return FP_ERR_SHAPE;
+  // row coordinates of every (batch, head, token) must fit in int32
+  if ((long long)s->batch * s->n_q_heads * s->seq_len >= (1ll << 31)) return FP_ERR_SHAPE;
+  D->bt = s->batch;
+  D->hq = s->n_q_heads;
+  D->hkv = s->n_kv_heads;
+  D->n = s->seq_len;
+  D->d = s->head_dim;
+  D->bs = s->block_size;
+  D->nb = int(nb);
+  D->g = s->n_q_heads / s->n_kv_heads;
+  D->t_pairs = nb * (nb + 1) / 2;
+  D->dtype = s->dtype;
+  return FP_OK;
+}
+
+fp_status check_attn_shape(const Dims &D) {
+  if (D.dtype == FP_BF16 && (D.d != 128 || D.bs != 128)) return FP_ERR_SHAPE;
+  return FP_OK;
+}
+
+fp_status check_params(const fp_params *p) {
+  if (!p) return FP_ERR_NULL;
+  if (!(p->gamma > 0.f) || !(p->gamma <= 1.f)) return FP_ERR_PARAM;
+  if (!(p->tau >= 0.f) || isinf(p->tau)) return FP_ERR_PARAM;
+  if (p->min_budget < 0) return FP_ERR_PARAM;
+  return FP_OK;
+}
+
+SelectBudgets budgets(const Dims &D, const fp_params &p) {
+  SelectBudgets b;
+  const long long T = D.t_pairs, nb = D.nb, bs = D.bs;
+  long long lo = nb * ((p.min_budget + bs - 1) / bs);
+  if (lo > T) lo = T;
+  long long hi = p.max_budget <= 0 ? T : nb * (p.max_budget / bs);
+  if (hi > T) hi = T;
+  b.qa_lo = lo < hi ? lo : hi;
+  b.qa_hi = hi;
+  int vlo = p.min_budget < D.n ? p.min_budget : D.n;
+  int vhi = p.max_budget <= 0 ? D.n : (p.max_budget < D.n ? p.max_budget : D.n);
+  b.vs_lo = vlo < vhi ? vlo : vhi;
+  b.vs_hi = vhi;
+  return b;
+}
+
+fp_status check_ws(void *ws, size_t have, size_t need) {
+  if (need == 0) return FP_OK;
+  if (!ws) return FP_ERR_WORKSPACE;
+  if (reinterpret_cast<uintptr_t>(ws) % 256 != 0) return FP_ERR_WORKSPACE;
+  if (have < need) return FP_ERR_WORKSPACE;
+  return FP_OK;
+}
+
+fp_status check_device() {
+  static int cc[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return FP_ERR_CUDA;
+  if (cc[dev] == 0) {
+    int major = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
+      return FP_ERR_CUDA;
+    cc[dev] = major;
+  }
+  return cc[dev] == 10 ? FP_OK : FP_ERR_UNSUPPORTED;
+}
+
+fp_status cuda_status(cudaError_t e) { return e == cudaSuccess ? FP_OK : FP_ERR_CUDA; }
+
+// Intermediates of the whole path, carved from a workspace.
+struct Prefill {
+  float *qbar, *kbar, *map, *est_last, *true_last, *vert, *slash, *djs;
+  int32_t *pattern, *counts, *indices;
+  void *stage_ws;
+};
+
+size_t carve_prefill(const Dims &D, void *ws, Prefill *P) {
+  Carver c{static_cast<char *>(ws), 0};
+  const size_t heads = size_t(D.bt) * D.hq;
+  P->qbar = c.take<float>(heads * D.nb * D.d);
+  P->kbar = c.take<float>(size_t(D.bt) * D.hkv * D.nb * D.d);
+  P->map = c.take<float>(heads * D.t_pairs);
+  P->est_last = c.take<float>(heads * D.nb);
+  P->true_last = c.take<float>(heads * D.nb);
+  P->vert = c.take<float>(heads * D.n);
+  P->slash = c.take<float>(heads * D.n);
+  P->djs = c.take<float>(heads);
+  P->pattern = c.take<int32_t>(heads);
+  P->counts = c.take<int32_t>(heads * D.nb);
+  P->indices = c.take<int32_t>(heads * D.nb * size_t(D.nb));
+  const size_t stage = std::max(estimate_ws_bytes(D), std::max(select_ws_bytes(D),
+                                                               attn_ws_bytes(D)));
+  P->stage_ws = c.take<char>(stage);
+  return c.off + 256;
+}
+
+size_t elem_bytes(const Dims &D) { return D.dtype == FP_BF16 ? 2 : 4; }
+
+fp_status run_attn(const Dims &D, const void *q, const void *k, const void *v,
+                   const int32_t *counts, const int32_t *indices, void *out, float *lse,
+                   bool dense, void *ws, cudaStream_t st) {
+  if (D.dtype == FP_F32)
+    return cuda_status(launch_attn_f32(D, static_cast<const float *>(q),
+                                       static_cast<const float *>(k),
+                                       static_cast<const float *>(v), counts, indices,
+                                       static_cast<float *>(out), lse, dense, st));
+  return cuda_status(launch_attn_bf16(D, q, k, v, counts, indices, out, lse, dense, ws, st));
+}
+
+fp_status run_prefill(const Dims &D, const fp_params &p, const void *q, const void *k,
+                      const void *v, void *out, float *lse, int64_t *stats, const Prefill &P,
+                      cudaStream_t st) {
+  cudaError_t e = launch_estimate(D, q, k, P.qbar, P.kbar, P.map, P.est_last, P.true_last,
+                                  P.vert, P.slash, P.stage_ws, st);
+  if (e != cudaSuccess) return FP_ERR_CUDA;
+  e = launch_pattern(D, p.tau, P.est_last, P.true_last, P.djs, P.pattern, st);
+  if (e != cudaSuccess) return FP_ERR_CUDA;
+  e = launch_select(D, p.gamma, budgets(D, p), P.pattern, P.map, P.vert, P.slash, P.counts,
+                    P.indices, P.stage_ws, st);
+  if (e != cudaSuccess) return FP_ERR_CUDA;
+  if (stats && launch_stats(D, P.counts, P.pattern, stats, st) != cudaSuccess)
+    return FP_ERR_CUDA;
+  return run_attn(D, q, k, v, P.counts, P.indices, out, lse, false, P.stage_ws, st);
+}
+
+}  // namespace
+}  // namespace fpi
+
+using namespace fpi;
+
+FP_API size_t fp_workspace_size(const fp_shape *shape, int which_call) {
+  Dims D;
+  if (check_shape(shape, &D) != FP_OK) return 0;
+  switch (which_call) {
+    case FP_CALL_ESTIMATE:
+      return estimate_ws_bytes(D);
+    case FP_CALL_SELECT:
+      return select_ws_bytes(D);
+    case FP_CALL_SPARSE_ATTN:
+      return attn_ws_bytes(D);
+    case FP_CALL_PREFILL: {
+      Prefill P;
+      return carve_prefill(D, nullptr, &P);
+    }
+    case FP_CALL_PREFILL_HOST: {
+      Prefill P;
+      Carver c{nullptr, 0};
+      const size_t eb = elem_bytes(D);
+      c.take<char>(size_t(D.bt) * D.hq * D.n * D.d * eb);
+      c.take<char>(size_t(D.bt) * D.hkv * D.n * D.d * eb);
+      c.take<char>(size_t(D.bt) * D.hkv * D.n * D.d * eb);
+      c.take<char>(size_t(D.bt) * D.hq * D.n * D.d * eb);
+      c.take<char>(carve_prefill(D, nullptr, &P));
+      return c.off + 256;
+    }
+    default:
+      return 0;
+  }
+}
+
+FP_API fp_status fp_estimate(const fp_shape *shape, const void *q, const void *k, float *qbar,
+                             float *kbar, float *map, float *est_last, float *true_last,
+                             float *vert, float *slash, void *ws, size_t ws_bytes,
+                             fp_stream_t stream) {
+  Dims D;
+  fp_status s = check_shape(shape, &D);
+  if (s != FP_OK) return s;
+  if (!q || !k || !qbar || !kbar || !map || !est_last || !true_last || !vert || !slash)
+    return FP_ERR_NULL;
+  if ((s = check_ws(ws, ws_bytes, estimate_ws_bytes(D))) != FP_OK) return s;
+  if ((s = check_device()) != FP_OK) return s;
+  return cuda_status(launch_estimate(D, q, k, qbar, kbar, map, est_last, true_last, vert, slash,
+                                     ws, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+FP_API fp_status fp_pattern(const fp_shape *shape, const fp_params *params,
+                            const float *est_last, const float *true_last, float *djs,
+                            int32_t *pattern, fp_stream_t stream) {
+  Dims D;
+  fp_status s = check_shape(shape, &D);
+  if (s != FP_OK) return s;
+  if ((s = check_params(params)) != FP_OK) return s;
+  if (!est_last || !true_last || !djs || !pattern) return FP_ERR_NULL;
+  if ((s = check_device()) != FP_OK) return s;
+  return cuda_status(launch_pattern(D, params->tau, est_last, true_last, djs, pattern,
+                                    reinterpret_cast<cudaStream_t>(stream)));
+}
+
+FP_API fp_status fp_select(const fp_shape *shape, const fp_params *params,
+                           const int32_t *pattern, const float *map, const float *vert,
+                           const float *slash, int32_t *counts, int32_t *indices, void *ws,
+                           size_t ws_bytes, fp_stream_t stream) {
+  Dims D;
+  fp_status s = check_shape(shape, &D);
+  if (s != FP_OK) return s;
+  if ((s = check_params(params)) != FP_OK) return s;
+  if (!pattern || !map || !vert || !slash || !counts || !indices) return FP_ERR_NULL;
+  if ((s = check_ws(ws, ws_bytes, select_ws_bytes(D))) != FP_OK) return s;
+  if ((s = check_device()) != FP_OK) return s;
+  return cuda_status(launch_select(D, params->gamma, budgets(D, *params), pattern, map, vert,
+                                   slash, counts, indices, ws,
+                                   reinterpret_cast<cudaStream_t>(stream)));
+}
+
+FP_API fp_status fp_sparse_attn(const fp_shape *shape, const void *q, const void *k,
+                                const void *v, const int32_t *counts, const int32_t *indices,
+                                void *out, float *lse, void *ws, size_t ws_bytes,
+                                fp_stream_t stream) {
+  Dims D;
+  fp_status s = check_shape(shape, &D);
+  if (s != FP_OK) return s;
+  if ((s = check_attn_shape(D)) != FP_OK) return s;
+  if (!q || !k || !v || !counts || !indices || !out) return FP_ERR_NULL;
+  if ((s = check_ws(ws, ws_bytes, attn_ws_bytes(D))) != FP_OK) return s;
+  if ((s = check_device()) != FP_OK) return s;
+  return run_attn(D, q, k, v, counts, indices, out, lse, false, ws,
+                  reinterpret_cast<cudaStream_t>(stream));
+}
+
+FP_API fp_status fp_dense_attn(const fp_shape *shape, const void *q, const void *k,
+                               const void *v, void *out, float *lse, fp_stream_t stream) {
+  Dims D;
+  fp_status s = check_shape(shape, &D);
+  if (s != FP_OK) return s;
+  if ((s = check_attn_shape(D)) != FP_OK) return s;
+  if (!q || !k || !v || !out) return FP_ERR_NULL;
+  if ((s = check_device()) != FP_OK) return s;
+  // dense lists are implicit: counts / indices are never read
+  static const int32_t dummy = 0;
+  return run_attn(D, q, k, v, &dummy, &dummy, out, lse, true, nullptr,
+                  reinterpret_cast<cudaStream_t>(stream));
+}
+
+FP_API fp_status fp_prefill_attn(const fp_shape *shape, const fp_params *params, const void *q,
+                                 const void *k, const void *v, void *out, float *lse,
+                                 int64_t *stats, void *ws, size_t ws_bytes,
+                                 fp_stream_t stream) {
+  Dims D;
+  fp_status s = check_shape(shape, &D);
+  if (s != FP_OK) return s;
+  if ((s = check_attn_shape(D)) != FP_OK) return s;
+  if ((s = check_params(params)) != FP_OK) return s;
+  if (!q || !k || !v || !out) return FP_ERR_NULL;
+  Prefill P;
+  if ((s = check_ws(ws, ws_bytes, carve_prefill(D, nullptr, &P))) != FP_OK) return s;
+  if ((s = check_device()) != FP_OK) return s;
+  carve_prefill(D, ws, &P);
+  return run_prefill(D, *params, q, k, v, out, lse, stats, P,
+                     reinterpret_cast<cudaStream_t>(stream));
+}
+
+FP_API fp_status fp_prefill_attn_host(const fp_shape *shape, const fp_params *params,
+                                      const void *q_host, const void *k_host,
+                                      const void *v_host, void *out_host, void *ws,
+                                      size_t ws_bytes, fp_stream_t stream) {
+  Dims D;
+  fp_status s = check_shape(shape, &D);
+  if (s != FP_OK) return s;
+  if ((s = check_attn_shape(D)) != FP_OK) return s;
+  if ((s = check_params(params)) != FP_OK) return s;
+  if (!q_host || !k_host || !v_host || !out_host) return FP_ERR_NULL;
+  if ((s = check_ws(ws, ws_bytes, fp_workspace_size(shape, FP_CALL_PREFILL_HOST))) != FP_OK)
+    return s;
+  if ((s = check_device()) != FP_OK) return s;
+  const size_t eb = elem_bytes(D);
+  const size_t qbytes = size_t(D.bt) * D.hq * D.n * D.d * eb;
+  const size_t kvbytes = size_t(D.bt) * D.hkv * D.n * D.d * eb;
+  Carver c{static_cast<char *>(ws), 0};
+  char *qd = c.take<char>(qbytes);
+  char *kd = c.take<char>(kvbytes);
+  char *vd = c.take<char>(kvbytes);
+  char *od = c.take<char>(qbytes);
+  Prefill P;
+  carve_prefill(D, c.take<char>(carve_prefill(D, nullptr, &P)), &P);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaMemcpyAsync(qd, q_host, qbytes, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+      cudaMemcpyAsync(kd, k_host, kvbytes, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+      cudaMemcpyAsync(vd, v_host, kvbytes, cudaMemcpyHostToDevice, st) != cudaSuccess)
+    return FP_ERR_CUDA;
+  s = run_prefill(D, *params, qd, kd, vd, od, nullptr, nullptr, P, st);
+  if (s != FP_OK) return s;
+  if (cudaMemcpyAsync(out_host, od, qbytes, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    return FP_ERR_CUDA;
+  return FP_OK;
+}
+
+FP_API fp_status fp_last_device_status(fp_stream_t stream) {
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return FP_ERR_CUDA;
+  int *p = device_status_ptr();
+  if (!p) return FP_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpy(&v, p, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return FP_ERR_CUDA;
+  const int zero = 0;
+  if (cudaMemcpy(p, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess)
+    return FP_ERR_CUDA;
+  return static_cast<fp_status>(v);
+}
+
+FP_API const char *fp_status_string(fp_status status) {
+  switch (status) {
+    case FP_OK: return "FP_OK";
+    case FP_ERR_NULL: return "FP_ERR_NULL: a required pointer is NULL";
+    case FP_ERR_SHAPE: return "FP_ERR_SHAPE: unsupported or inconsistent shape";
+    case FP_ERR_DTYPE: return "FP_ERR_DTYPE: unsupported dtype";
+    case FP_ERR_PARAM: return "FP_ERR_PARAM: gamma, tau or budget out of range";
+    case FP_ERR_WORKSPACE: return "FP_ERR_WORKSPACE: workspace NULL, misaligned or too small";
+    case FP_ERR_CUDA: return "FP_ERR_CUDA: a CUDA call or launch failed";
+    case FP_ERR_TIMEOUT: return "FP_ERR_TIMEOUT: a device pipeline wait ran out of time";
+    case FP_ERR_DEVICE_CHECK: return "FP_ERR_DEVICE_CHECK: an argument failed a device check";
+    case FP_ERR_UNSUPPORTED: return "FP_ERR_UNSUPPORTED: the device is not sm_100";
+  }
+  return "unknown fp_status";
+}

@@ -1,0 +1,421 @@
+// select.cu -- fp_select: cumulative-attention index selection.
+//
+// FlexPrefill (atlas.scime.ai summary, "Approach"): keep the smallest set of
+// blocks (query-aware heads, over the flattened estimated map) or lines
+// (vertical-slash heads, over column and diagonal sums) whose cumulative
+// normalised attention reaches gamma; the summary's "Measured effects" table
+// adds min / max computational budgets.
+//
+// Exact rule on a list of fp32 scores s_i (finite, >= 0):
+//   order       score descending, then index ascending;
+//   mass        w_i = ceil(s_i * 2^32), an integer, summed exactly (W);
+//   k_gamma     smallest k with (double)(sum of the first k masses) >=
+//               (double)gamma * (double)W; gamma >= 1 keeps everything;
+//   k           clamp(k_gamma, lo, hi);
+//   kept        the first k entries of the order.
+// Because non-negative fp32 scores order like their bit patterns, the kept
+// set is {bits_i > b} u {bits_i == b and i <= idx} for one threshold pair
+// (b, idx).  select_head_kernel finds it with a three-level radix descent on
+// the bit patterns (12 + 12 + 8 bits), weighted by mass to find k_gamma and by
+// count when the clamp moves k, and one ordered count for the tie rank.  All
+// of it is integer arithmetic, so the result does not depend on thread order.
+// emit_rows_kernel then writes every row's ascending block list.
+#include "fp_internal.cuh"
+
+namespace fpi {
+namespace {
+
+constexpr int kThreads = 1024;
+constexpr int kMaxBlocks = 4096;  // nb limit (flags live in shared memory)
+
+enum : int { SEL_THRESHOLD = 0, SEL_NONE = 1, SEL_ALL = 2 };
+
+struct HeadSel {
+  int mode;
+  uint32_t bits;
+  uint32_t idx;
+  int pad;
+};
+
+__device__ __forceinline__ uint32_t score_bits(float s) {
+  return s > 0.f ? __float_as_uint(s) : 0u;  // negative zero / NaN / negatives -> 0
+}
+__device__ __forceinline__ uint64_t score_mass(uint32_t bits) {
+  return (uint64_t)ceil((double)__uint_as_float(bits) * 4294967296.0);
+}
+__device__ __forceinline__ bool kept(uint32_t bits, uint32_t i, const HeadSel &s) {
+  if (s.mode == SEL_ALL) return true;
+  if (s.mode == SEL_NONE) return false;
+  return bits > s.bits || (bits == s.bits && i <= s.idx);
+}
+
+struct SelSmem {
+  unsigned long long hmass[4096];
+  unsigned int hcnt[4096];
+  unsigned long long warp_tot[32];
+  unsigned long long res[4];
+  uint8_t colflag[kMaxBlocks];
+  uint8_t distflag[kMaxBlocks];
+};
+
+// Block-wide exclusive prefix sum (thread order) of one value per thread.
+__device__ unsigned long long block_excl_scan(unsigned long long v, SelSmem &sm,
+                                              unsigned long long *total) {
+  const int lane = threadIdx.x % 32, w = threadIdx.x / 32;
+  unsigned long long x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    unsigned long long y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  __syncthreads();
+  if (lane == 31) sm.warp_tot[w] = x;
+  __syncthreads();
+  if (w == 0) {
+    unsigned long long t = sm.warp_tot[lane];
+    unsigned long long s = t;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      unsigned long long y = __shfl_up_sync(0xffffffffu, s, o);
+      if (lane >= o) s += y;
+    }
+    sm.warp_tot[lane] = s - t;  // exclusive over warps
+    if (lane == 31) sm.res[3] = s;
+  }
+  __syncthreads();
+  unsigned long long r = sm.warp_tot[w] + x - v;
+  *total = sm.res[3];
+  __syncthreads();
+  return r;
+}
+
+// Histogram of (bits >> shift) & (nbins-1) over entries whose masked bits
+// equal `prefix`, mass and count, warp-aggregated shared-memory atomics.
+__device__ void histogram(const float *__restrict__ s, uint32_t n, uint32_t prefix,
+                          uint32_t pmask, int shift, uint32_t nbins, SelSmem &sm) {
+  for (uint32_t i = threadIdx.x; i < nbins; i += kThreads) {
+    sm.hmass[i] = 0;
+    sm.hcnt[i] = 0;
+  }
+  __syncthreads();
+  const int lane = threadIdx.x % 32;
+  for (uint32_t base = (threadIdx.x / 32) * 32; base < n; base += kThreads) {
+    const uint32_t i = base + lane;
+    uint32_t bin = 0xFFFFFFFFu;
+    uint64_t w = 0;
+    if (i < n) {
+      const uint32_t b = score_bits(s[i]);
+      if ((b & pmask) == prefix) {
+        bin = (b >> shift) & (nbins - 1);
+        w = score_mass(b);
+      }
+    }
+    const unsigned peers = __match_any_sync(0xffffffffu, bin);
+    const unsigned lo = __reduce_add_sync(peers, unsigned(w & 0xFFFFFFull));
+    const unsigned hi = __reduce_add_sync(peers, unsigned(w >> 24));
+    if (bin != 0xFFFFFFFFu && lane == __ffs(peers) - 1) {
+      atomicAdd(&sm.hmass[bin], ((unsigned long long)hi << 24) + lo);
+      atomicAdd(&sm.hcnt[bin], unsigned(__popc(peers)));
+    }
+  }
+  __syncthreads();
+}
+
+// Scan the histogram from the highest bin down; find the first bin at which
+// above + (inclusive cumulative) reaches the target.  Updates *above_m /
+// *above_c to include every bin strictly higher, returns the bin.
+__device__ uint32_t find_crossing(uint32_t nbins, bool by_mass, double target_m,
+                                  unsigned long long target_c, unsigned long long *above_m,
+                                  unsigned long long *above_c, SelSmem &sm) {
+  const uint32_t per = nbins >= kThreads ? nbins / kThreads : 1;
+  const uint32_t p0 = threadIdx.x * per;  // positions in descending-bin order
+  unsigned long long lm = 0, lc = 0;
+  if (p0 < nbins)
+    for (uint32_t p = p0; p < p0 + per; ++p) {
+      const uint32_t b = nbins - 1 - p;
+      lm += sm.hmass[b];
+      lc += sm.hcnt[b];
+    }
+  unsigned long long tm, tc;
+  const unsigned long long em = block_excl_scan(lm, sm, &tm);
+  const unsigned long long ec = block_excl_scan(lc, sm, &tc);
+  if (threadIdx.x == 0) {
+    sm.res[0] = 0;  // fallback: lowest bin (unreachable for valid targets)
+    sm.res[1] = tm - sm.hmass[0];
+    sm.res[2] = tc - sm.hcnt[0];
+  }
+  __syncthreads();
+  const unsigned long long am = *above_m, ac = *above_c;
+  auto reach = [&](unsigned long long m, unsigned long long c) {
+    return by_mass ? (double)(am + m) >= target_m : (ac + c) >= target_c;
+  };
+  if (p0 < nbins && !reach(em, ec) && reach(em + lm, ec + lc)) {
+    unsigned long long cm = em, cc = ec;
+    for (uint32_t p = p0; p < p0 + per; ++p) {
+      const uint32_t b = nbins - 1 - p;
+      if (reach(cm + sm.hmass[b], cc + sm.hcnt[b])) {
+        sm.res[0] = b;
+        sm.res[1] = cm;
+        sm.res[2] = cc;
+        break;
+      }
+      cm += sm.hmass[b];
+      cc += sm.hcnt[b];
+    }
+  }
+  __syncthreads();
+  const uint32_t bin = uint32_t(sm.res[0]);
+  *above_m = am + sm.res[1];
+  *above_c = ac + sm.res[2];
+  __syncthreads();
+  return bin;
+}
+
+// Radix descent; returns the threshold bit pattern and the mass / count of
+// every entry with larger bits.  Sets *total_m to W when first_pass_total.
+__device__ uint32_t descend(const float *s, uint32_t n, bool by_mass, float gamma,
+                            unsigned long long target_c, unsigned long long *above_m,
+                            unsigned long long *above_c, unsigned long long *total_m,
+                            double *target_m_out, SelSmem &sm) {
+  const int shifts[3] = {20, 8, 0};
+  const int widths[3] = {12, 12, 8};
+  uint32_t prefix = 0, pmask = 0;
+  *above_m = 0;
+  *above_c = 0;
+  double target_m = 0.0;
+  for (int lv = 0; lv < 3; ++lv) {
+    const uint32_t nbins = 1u << widths[lv];
+    histogram(s, n, prefix, pmask, shifts[lv], nbins, sm);
+    if (lv == 0 && by_mass) {
+      // W = every mass (the first level sees every entry)
+      unsigned long long part = 0;
+      for (uint32_t b = threadIdx.x; b < nbins; b += kThreads) part += sm.hmass[b];
+      unsigned long long tot;
+      block_excl_scan(part, sm, &tot);
+      *total_m = tot;
+      target_m = (double)gamma * (double)tot;
+      *target_m_out = target_m;
+    }
+    const uint32_t bin = find_crossing(nbins, by_mass, target_m, target_c, above_m, above_c, sm);
+    prefix |= bin << shifts[lv];
+    pmask |= (nbins - 1) << shifts[lv];
+  }
+  return prefix;
+}
+
+// Index of the m-th (1-based) entry with bit pattern == b, in index order.
+__device__ uint32_t tie_index(const float *s, uint32_t n, uint32_t b, unsigned long long m,
+                              SelSmem &sm) {
+  const uint32_t per = (n + kThreads - 1) / kThreads;
+  const uint32_t i0 = threadIdx.x * per;
+  const uint32_t i1 = min(n, i0 + per);
+  unsigned long long c = 0;
+  for (uint32_t i = i0; i < i1; ++i) c += score_bits(s[i]) == b;
+  unsigned long long tot;
+  const unsigned long long e = block_excl_scan(c, sm, &tot);
+  if (threadIdx.x == 0) sm.res[0] = n - 1;
+  __syncthreads();
+  if (e < m && m <= e + c) {
+    unsigned long long r = e;
+    for (uint32_t i = i0; i < i1; ++i)
+      if (score_bits(s[i]) == b && ++r == m) {
+        sm.res[0] = i;
+        break;
+      }
+  }
+  __syncthreads();
+  const uint32_t idx = uint32_t(sm.res[0]);
+  __syncthreads();
+  return idx;
+}
+
+__device__ HeadSel select_list(const float *s, uint32_t n, float gamma, unsigned long long lo,
+                               unsigned long long hi, SelSmem &sm) {
+  HeadSel r{SEL_NONE, 0u, 0u, 0};
+  if (n == 0) return r;
+  unsigned long long am = 0, ac = 0, wtot = 0, k;
+  double target = 0.0;
+  uint32_t b = 0;
+  unsigned long long m = 0;
+  bool have_threshold = false;
+  if (gamma >= 1.f) {
+    k = n;
+  } else {
+    b = descend(s, n, true, gamma, 0, &am, &ac, &wtot, &target, sm);
+    if (target <= 0.0) {
+      k = 0;
+    } else {
+      const unsigned long long w = score_mass(b);
+      // smallest m >= 1 with am + m * w >= target (w >= 1 here: a zero-mass
+      // bin cannot be the crossing one for a positive target)
+      unsigned long long mm = 1;
+      if (w > 0) {
+        double need = (target - (double)am) / (double)w;
+        mm = need <= 1.0 ? 1ull : (unsigned long long)ceil(need);
+        while (mm > 1 && (double)(am + (mm - 1) * w) >= target) --mm;
+        while ((double)(am + mm * w) < target) ++mm;
+      }
+      k = ac + mm;
+      m = mm;
+      have_threshold = true;
+    }
+  }
+  const unsigned long long kc = k < lo ? lo : (k > hi ? hi : k);
+  if (kc == 0) return r;
+  if (kc >= n) {
+    r.mode = SEL_ALL;
+    return r;
+  }
+  if (!(have_threshold && kc == k)) {
+    b = descend(s, n, false, gamma, kc, &am, &ac, &wtot, &target, sm);
+    m = kc - ac;
+  }
+  r.mode = SEL_THRESHOLD;
+  r.bits = b;
+  r.idx = tie_index(s, n, b, m, sm);
+  return r;
+}
+
+// grid (Hq, Bt), 1024 threads, dynamic shared memory SelSmem.
+__global__ void __launch_bounds__(kThreads) select_head_kernel(
+    const int32_t *__restrict__ pattern, const float *__restrict__ map,
+    const float *__restrict__ vert, const float *__restrict__ slash, int n, int nb, int bs,
+    float gamma, long long qa_lo, long long qa_hi, int vs_lo, int vs_hi,
+    HeadSel *__restrict__ sel, uint8_t *__restrict__ colflag, uint8_t *__restrict__ distflag) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  SelSmem &sm = *reinterpret_cast<SelSmem *>(smem_raw);
+  const size_t bh = size_t(blockIdx.y) * gridDim.x + blockIdx.x;
+  const size_t t_pairs = size_t(nb) * (nb + 1) / 2;
+  if (pattern[bh] == FP_PATTERN_QA) {
+    HeadSel r = select_list(map + bh * t_pairs, uint32_t(t_pairs), gamma, qa_lo, qa_hi, sm);
+    if (threadIdx.x == 0) sel[2 * bh] = r;
+    return;
+  }
+  for (int i = threadIdx.x; i < nb; i += kThreads) {
+    sm.colflag[i] = 0;
+    sm.distflag[i] = 0;
+  }
+  __syncthreads();
+  const float *vv = vert + bh * n;
+  const float *ss = slash + bh * n;
+  HeadSel rv = select_list(vv, uint32_t(n), gamma, vs_lo, vs_hi, sm);
+  for (int t = threadIdx.x; t < n; t += kThreads)
+    if (kept(score_bits(vv[t]), uint32_t(t), rv)) sm.colflag[t / bs] = 1;
+  HeadSel rs = select_list(ss, uint32_t(n), gamma, vs_lo, vs_hi, sm);
+  for (int o = threadIdx.x; o < n; o += kThreads)
+    if (kept(score_bits(ss[o]), uint32_t(o), rs)) {
+      const int d0 = o / bs;
+      sm.distflag[d0] = 1;
+      if (o % bs != 0 && d0 + 1 < nb) sm.distflag[d0 + 1] = 1;
+    }
+  __syncthreads();
+  for (int i = threadIdx.x; i < nb; i += kThreads) {
+    colflag[bh * nb + i] = sm.colflag[i];
+    distflag[bh * nb + i] = sm.distflag[i];
+  }
+  if (threadIdx.x == 0) {
+    sel[2 * bh] = rv;
+    sel[2 * bh + 1] = rs;
+  }
+}
+
+// grid (ceil(nb/8), Hq, Bt), 256 threads: one warp per row.
+__global__ void __launch_bounds__(256) emit_rows_kernel(
+    const int32_t *__restrict__ pattern, const float *__restrict__ map, int nb,
+    const HeadSel *__restrict__ sel, const uint8_t *__restrict__ colflag,
+    const uint8_t *__restrict__ distflag, int32_t *__restrict__ counts,
+    int32_t *__restrict__ indices) {
+  const int qi = blockIdx.x * 8 + threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+  if (qi >= nb) return;
+  const size_t bh = size_t(blockIdx.z) * gridDim.y + blockIdx.y;
+  const bool qa = pattern[bh] == FP_PATTERN_QA;
+  const HeadSel s = sel[2 * bh];
+  const size_t rowbase = size_t(qi) * (qi + 1) / 2;
+  const float *mrow = map + bh * (size_t(nb) * (nb + 1) / 2) + rowbase;
+  const uint8_t *cf = colflag + bh * nb;
+  const uint8_t *df = distflag + bh * nb;
+  int32_t *out = indices + (bh * nb + qi) * size_t(nb);
+  int cnt = 0;
+  for (int j0 = 0; j0 <= qi; j0 += 32) {
+    const int j = j0 + lane;
+    bool keep = false;
+    if (j <= qi) {
+      if (j == qi)
+        keep = true;
+      else if (qa)
+        keep = kept(score_bits(mrow[j]), uint32_t(rowbase + j), s);
+      else
+        keep = cf[j] || df[qi - j];
+    }
+    const unsigned bal = __ballot_sync(0xffffffffu, keep);
+    if (keep) out[cnt + __popc(bal & ((1u << lane) - 1u))] = j;
+    cnt += __popc(bal);
+  }
+  if (lane == 0) counts[bh * nb + qi] = cnt;
+}
+
+__global__ void stats_kernel(const int32_t *__restrict__ counts,
+                             const int32_t *__restrict__ pattern, long long rows, int heads,
+                             int64_t *__restrict__ stats) {
+  __shared__ unsigned long long red[32];
+  unsigned long long s = 0, qa = 0;
+  for (long long i = threadIdx.x; i < rows; i += blockDim.x) s += (unsigned)counts[i];
+  for (int i = threadIdx.x; i < heads; i += blockDim.x) qa += pattern[i] == FP_PATTERN_QA;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    s += __shfl_xor_sync(0xffffffffu, s, o);
+    qa += __shfl_xor_sync(0xffffffffu, qa, o);
+  }
+  if (threadIdx.x % 32 == 0) red[threadIdx.x / 32] = (qa << 40) | s;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    unsigned long long ts = 0, tq = 0;
+    for (int w = 0; w < int(blockDim.x / 32); ++w) {
+      ts += red[w] & ((1ull << 40) - 1);
+      tq += red[w] >> 40;
+    }
+    stats[0] = (int64_t)ts;
+    stats[1] = (int64_t)tq;
+  }
+}
+
+}  // namespace
+
+size_t select_ws_bytes(const Dims &D) {
+  Carver c{nullptr, 0};
+  const size_t heads = size_t(D.bt) * D.hq;
+  c.take<HeadSel>(2 * heads);
+  c.take<uint8_t>(heads * D.nb);
+  c.take<uint8_t>(heads * D.nb);
+  return c.off + 256;
+}
+
+cudaError_t launch_select(const Dims &D, float gamma, const SelectBudgets &bud,
+                          const int32_t *pattern, const float *map, const float *vert,
+                          const float *slash, int32_t *counts, int32_t *indices, void *ws,
+                          cudaStream_t st) {
+  if (D.nb > kMaxBlocks) return cudaErrorInvalidValue;
+  Carver c{static_cast<char *>(ws), 0};
+  const size_t heads = size_t(D.bt) * D.hq;
+  HeadSel *sel = c.take<HeadSel>(2 * heads);
+  uint8_t *cf = c.take<uint8_t>(heads * D.nb);
+  uint8_t *df = c.take<uint8_t>(heads * D.nb);
+  const int smem = int(sizeof(SelSmem));
+  cudaFuncSetAttribute(select_head_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  select_head_kernel<<<dim3(D.hq, D.bt), kThreads, smem, st>>>(
+      pattern, map, vert, slash, D.n, D.nb, D.bs, gamma, bud.qa_lo, bud.qa_hi, bud.vs_lo,
+      bud.vs_hi, sel, cf, df);
+  emit_rows_kernel<<<dim3((D.nb + 7) / 8, D.hq, D.bt), 256, 0, st>>>(pattern, map, D.nb, sel, cf,
+                                                                    df, counts, indices);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_stats(const Dims &D, const int32_t *counts, const int32_t *pattern,
+                         int64_t *stats, cudaStream_t st) {
+  stats_kernel<<<1, 1024, 0, st>>>(counts, pattern, (long long)D.bt * D.hq * D.nb, D.bt * D.hq,
+                                   stats);
+  return cudaGetLastError();
+}
+
+}  // namespace fpi

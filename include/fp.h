@@ -1,0 +1,230 @@
+/*
+ * fp.h -- C ABI of the FlexPrefill prefill-attention hot path on B200 (sm_100a).
+ *
+ * The method (FlexPrefill: A Context-Aware Sparse Attention Mechanism for
+ * Efficient Long-Sequence Inference; atlas.scime.ai summary, "Approach"):
+ * for every attention head, estimate block-pooled attention from the last
+ * query block, compare it with the true distribution by the square root of
+ * the Jensen-Shannon divergence, choose query-aware block selection when the
+ * estimate is accurate and a vertical-slash pattern otherwise, keep the
+ * smallest set of blocks/lines whose cumulative normalised attention reaches
+ * gamma (within min/max token budgets), and run causal block-sparse
+ * attention over the kept blocks.  The abstract (same title; OpenReview and
+ * codewithpapers pages) names the two parts "Query-Aware Sparse Pattern
+ * Determination" and "Cumulative-Attention Based Index Selection".
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  * Layouts are dense and row-major (C order):
+ *      q            [Bt, Hq,  N, d]   (fp_shape.dtype: bf16 or fp32)
+ *      k, v         [Bt, Hkv, N, d]
+ *      out          [Bt, Hq,  N, d]   (same dtype as q)
+ *    with N = seq_len, d = head_dim, B = block_size, nb = N / B,
+ *    T = nb (nb + 1) / 2 and g = Hq / Hkv; query head h reads kv head h / g.
+ *  * Every data pointer is DEVICE memory owned by the caller, except the
+ *    *_host pointers of fp_prefill_attn_host.  The library allocates no
+ *    device memory; scratch space is the caller's workspace (`ws`, at least
+ *    fp_workspace_size() bytes, 256-byte aligned).  A workspace must not be
+ *    shared by calls that may run concurrently.
+ *  * Arguments are validated on the host before anything is launched; a
+ *    failed check returns an error code and launches nothing.
+ *  * Kernels run asynchronously on `stream` (NULL = the legacy default
+ *    stream).  A launch failure returns FP_ERR_CUDA.  Errors found on the
+ *    device (an index outside the causal range, a pipeline wait that ran out
+ *    of time) are recorded in a per-device status word and read with
+ *    fp_last_device_status().
+ *  * No C++ exception crosses this ABI.  Calls on distinct streams with
+ *    distinct workspaces may run from several host threads.
+ *  * Supported shapes: N % B == 0, Hq % Hkv == 0, B in {64, 128},
+ *    d in {64, 128}.  The bf16 path (tensor cores) needs d == 128 and
+ *    B == 128; fp32 (the debug path, CUDA cores) takes every listed shape.
+ */
+#ifndef FP_H_
+#define FP_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t (struct CUstream_st *). */
+typedef struct CUstream_st *fp_stream_t;
+
+typedef enum {
+  FP_OK = 0,
+  FP_ERR_NULL = 1,          /* a required pointer is NULL                        */
+  FP_ERR_SHAPE = 2,         /* unsupported or inconsistent shape                 */
+  FP_ERR_DTYPE = 3,         /* unsupported dtype for this call                   */
+  FP_ERR_PARAM = 4,         /* gamma / tau / budget out of range                 */
+  FP_ERR_WORKSPACE = 5,     /* workspace NULL, misaligned or too small          */
+  FP_ERR_CUDA = 6,          /* a CUDA runtime call or launch failed              */
+  FP_ERR_TIMEOUT = 7,       /* device: a pipeline wait ran out of time           */
+  FP_ERR_DEVICE_CHECK = 8,  /* device: an argument failed an on-device check     */
+  FP_ERR_UNSUPPORTED = 9    /* the current device is not sm_100                  */
+} fp_status;
+
+typedef enum { FP_BF16 = 0, FP_F32 = 1 } fp_dtype;
+
+typedef struct {
+  int batch;       /* Bt                                    */
+  int n_q_heads;   /* Hq                                    */
+  int n_kv_heads;  /* Hkv, divides Hq (grouped-query heads) */
+  int seq_len;     /* N, a multiple of block_size           */
+  int head_dim;    /* d                                     */
+  int block_size;  /* B                                     */
+  fp_dtype dtype;  /* element type of q, k, v and out       */
+} fp_shape;
+
+typedef struct {
+  float gamma;     /* cumulative-attention threshold, 0 < gamma <= 1 (>= 1 keeps all) */
+  float tau;       /* JS-distance threshold, >= 0; tau == 0 disables query-aware mode   */
+  int min_budget;  /* tokens per query row, >= 0 (0: no minimum)                        */
+  int max_budget;  /* tokens per query row; <= 0: uncapped                              */
+} fp_params;
+
+enum { FP_PATTERN_QA = 0, FP_PATTERN_VS = 1 };
+
+/* Calls that take a workspace, for fp_workspace_size(). */
+enum {
+  FP_CALL_ESTIMATE = 0,
+  FP_CALL_SELECT = 1,
+  FP_CALL_SPARSE_ATTN = 2,
+  FP_CALL_PREFILL = 3,      /* fp_prefill_attn: every intermediate lives in ws     */
+  FP_CALL_PREFILL_HOST = 4  /* fp_prefill_attn_host: also device copies of q,k,v,out */
+};
+
+/* Bytes of workspace `which_call` needs for `shape` (0 if the shape is invalid). */
+size_t fp_workspace_size(const fp_shape *shape, int which_call);
+
+/*
+ * fp_estimate -- the pattern-determination inputs of every head.
+ * Source: atlas.scime.ai summary, "Approach" (block-pooled estimate from the
+ * last query block; the true distribution; vertical-slash lines).
+ *   qbar      [Bt,Hq,nb,d]  fp32  mean of q over each block of B tokens
+ *   kbar      [Bt,Hkv,nb,d] fp32  mean of k over each block
+ *   map       [Bt,Hq,T]     fp32  estimated block map: row i (stored at
+ *             i(i+1)/2 .. i(i+1)/2+i) is the softmax over key blocks j <= i of
+ *             qbar[i].kbar[j] / sqrt(d)
+ *   est_last  [Bt,Hq,nb]    fp32  the last row of map (the estimate a-hat)
+ *   true_last [Bt,Hq,nb]    fp32  true attention of the last query block,
+ *             summed over the keys of each block and averaged over its B rows
+ *   vert      [Bt,Hq,N]     fp32  vert[t]  = sum over the last B queries of P[r,t]
+ *   slash     [Bt,Hq,N]     fp32  slash[o] = sum over r of P[r, N-B+r-o]
+ * where P is the causal softmax of q.k/sqrt(d) for the last B queries.
+ * Workspace: fp_workspace_size(shape, FP_CALL_ESTIMATE).
+ */
+fp_status fp_estimate(const fp_shape *shape, const void *q, const void *k,
+                      float *qbar, float *kbar, float *map, float *est_last,
+                      float *true_last, float *vert, float *slash,
+                      void *ws, size_t ws_bytes, fp_stream_t stream);
+
+/*
+ * fp_pattern -- per-head pattern choice.
+ * Source: atlas.scime.ai summary, "Approach" (square-root JS divergence of
+ * the estimate against the true distribution) and its "Measured effects"
+ * table (tau = 0 disables query-aware mode, so the test is strict).
+ *   djs     [Bt,Hq] fp32   sqrt(JSD(est_last, true_last)), natural log, both
+ *                          inputs renormalised; computed in fp64
+ *   pattern [Bt,Hq] int32  FP_PATTERN_QA if djs < tau (fp64 compare), else VS
+ */
+fp_status fp_pattern(const fp_shape *shape, const fp_params *params,
+                     const float *est_last, const float *true_last,
+                     float *djs, int32_t *pattern, fp_stream_t stream);
+
+/*
+ * fp_select -- cumulative-attention index selection.
+ * Source: atlas.scime.ai summary, "Approach" (smallest set of blocks/lines
+ * whose cumulative normalised attention reaches gamma) and "Measured effects"
+ * (min/max budgets; the flattened estimated map).
+ * Rule for one list of fp32 scores: order by score descending, then index
+ * ascending; masses w = ceil(score * 2^32) as integers; keep the shortest
+ * prefix whose mass reaches (double)gamma * (double)sum(w); clamp its length
+ * to [lo, hi].
+ *   QA heads: the list is map[h] flattened (packed index), lo = min(T,
+ *     nb*ceil(min_budget/B)), hi = nb*floor(max_budget/B) (or T), each kept
+ *     pair (i, j) adds block j to row i.
+ *   VS heads: vert[h] and slash[h] are two lists of N lines, lo =
+ *     min(N, min_budget), hi = max_budget (or N); a kept column t adds key
+ *     block t/B to every row; a kept offset o adds every block pair at
+ *     distance o/B (and o/B + 1 when B does not divide o).
+ *   Every row also keeps its diagonal block.
+ *   counts  [Bt,Hq,nb]     int32  blocks kept in row i (1..i+1)
+ *   indices [Bt,Hq,nb,nb]  int32  row i's blocks, ascending, in the first
+ *                                 counts[i] slots (the rest is not written)
+ * The result is exact (integer arithmetic on the given fp32 scores).
+ * Workspace: fp_workspace_size(shape, FP_CALL_SELECT).
+ */
+fp_status fp_select(const fp_shape *shape, const fp_params *params,
+                    const int32_t *pattern, const float *map, const float *vert,
+                    const float *slash, int32_t *counts, int32_t *indices,
+                    void *ws, size_t ws_bytes, fp_stream_t stream);
+
+/*
+ * fp_sparse_attn -- causal block-sparse attention over the given lists.
+ * Source: atlas.scime.ai summary, "Approach" and "Experimental setup" (the
+ * sparse kernel builds on FlashAttention).
+ * Row block i of head h attends to the keys of blocks indices[b,h,i,0..
+ * counts-1] (each 0 <= j <= i; inside block i only keys <= the query), with
+ * softmax(q.k / sqrt(d)) V in fp32 accumulation.
+ *   out [Bt,Hq,N,d] (dtype of q); lse [Bt,Hq,N] fp32, natural-log
+ *   log-sum-exp of the scaled logits, or NULL.
+ * A row with counts == 0 gets zeros and lse = -inf.
+ * Workspace: fp_workspace_size(shape, FP_CALL_SPARSE_ATTN).
+ */
+fp_status fp_sparse_attn(const fp_shape *shape, const void *q, const void *k,
+                         const void *v, const int32_t *counts,
+                         const int32_t *indices, void *out, float *lse,
+                         void *ws, size_t ws_bytes, fp_stream_t stream);
+
+/*
+ * fp_dense_attn -- dense causal attention (every block j <= i), the same
+ * kernels as fp_sparse_attn; the comparison point for the speedup ("full
+ * attention" in the summary's "Key results").  No workspace.
+ */
+fp_status fp_dense_attn(const fp_shape *shape, const void *q, const void *k,
+                        const void *v, void *out, float *lse,
+                        fp_stream_t stream);
+
+/*
+ * fp_prefill_attn -- the whole path for one layer: estimate, pattern,
+ * select, sparse attention, with every intermediate in `ws`
+ * (fp_workspace_size(shape, FP_CALL_PREFILL) bytes).  out/lse as in
+ * fp_sparse_attn.  `stats` (device int64[2], or NULL) is overwritten on
+ * `stream` with {kept blocks summed over every head and row, number of
+ * query-aware heads}.
+ */
+fp_status fp_prefill_attn(const fp_shape *shape, const fp_params *params,
+                          const void *q, const void *k, const void *v,
+                          void *out, float *lse, int64_t *stats,
+                          void *ws, size_t ws_bytes, fp_stream_t stream);
+
+/*
+ * fp_prefill_attn_host -- fp_prefill_attn on HOST buffers: copies q, k, v
+ * to device memory inside `ws` (fp_workspace_size(shape,
+ * FP_CALL_PREFILL_HOST) bytes), runs the path and copies the output back to
+ * out_host, all enqueued on `stream` (one cudaMemcpyAsync per buffer; page-
+ * locked host memory makes the copies asynchronous).  The host buffers must
+ * stay valid until the stream reaches the end of the call.
+ */
+fp_status fp_prefill_attn_host(const fp_shape *shape, const fp_params *params,
+                               const void *q_host, const void *k_host,
+                               const void *v_host, void *out_host,
+                               void *ws, size_t ws_bytes, fp_stream_t stream);
+
+/*
+ * fp_last_device_status -- synchronises `stream`, returns the first error
+ * the kernels recorded on the current device since the last call (FP_OK if
+ * none) and clears it.
+ */
+fp_status fp_last_device_status(fp_stream_t stream);
+
+/* Static, human-readable name of a status code. */
+const char *fp_status_string(fp_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FP_H_ */

@@ -1,0 +1,127 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports
+every function include/fp.h declares, and rejects bad arguments with the
+documented status before touching the device."""
+import ctypes
+import os
+
+import pytest
+
+from dynamic_block_sparse_fp_b200 import build, ops
+
+FAKE = 1 << 20  # a non-null "device pointer" (never dereferenced: validation fails first)
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return ops.lib()
+
+
+def shape(**kw):
+    base = dict(batch=1, n_q_heads=4, n_kv_heads=2, seq_len=1024, head_dim=128, block_size=128,
+                dtype=ops.FP_BF16)
+    base.update(kw)
+    return ops.fp_shape(**base)
+
+
+def test_exports_every_declared_function(L):
+    names = ops.header_functions()
+    assert len(names) == 10, names
+    for n in names:
+        assert hasattr(L, n), n
+    # nothing but the fp_* API is exported (static CUDA runtime stays hidden)
+    out = os.popen(f"nm -D --defined-only {ops.lib_path()}").read().split()
+    exported = [s for s in out if not all(c in "0123456789abcdef" for c in s) and len(s) > 1]
+    exported = [s for s in exported if s not in ("T", "B", "D", "R", "W", "A")]
+    assert sorted(exported) == names
+
+
+def test_status_strings(L):
+    for code, name in ops.STATUS.items():
+        assert ops.fp_status_string(code).startswith(name)
+    assert ops.fp_status_string(99) == "unknown fp_status"
+
+
+def test_workspace_sizes(L):
+    s = shape()
+    assert ops.fp_workspace_size(s, ops.FP_CALL_ESTIMATE) > 0
+    assert ops.fp_workspace_size(s, ops.FP_CALL_SELECT) > 0
+    assert ops.fp_workspace_size(s, ops.FP_CALL_SPARSE_ATTN) == 0
+    pre = ops.fp_workspace_size(s, ops.FP_CALL_PREFILL)
+    host = ops.fp_workspace_size(s, ops.FP_CALL_PREFILL_HOST)
+    io = (2 * 4 + 2 * 2) * 1024 * 128 * 2  # q, out (4 heads) + k, v (2 heads), bf16
+    assert host >= pre + io
+    assert ops.fp_workspace_size(shape(seq_len=1000), ops.FP_CALL_PREFILL) == 0
+    assert ops.fp_workspace_size(s, 17) == 0
+    # larger problems need more
+    assert ops.fp_workspace_size(shape(seq_len=4096), ops.FP_CALL_ESTIMATE) > \
+        ops.fp_workspace_size(s, ops.FP_CALL_ESTIMATE)
+
+
+@pytest.mark.parametrize("bad,code", [
+    (dict(seq_len=1000), 2), (dict(block_size=32), 2), (dict(head_dim=96), 2),
+    (dict(n_q_heads=3), 2), (dict(n_kv_heads=0), 2), (dict(dtype=7), 3),
+    (dict(seq_len=128 * 4097), 2),
+])
+def test_bad_shapes_rejected(L, bad, code):
+    s = shape(**bad)
+    ws = FAKE
+    assert L.fp_estimate(ctypes.byref(s), *([FAKE] * 9), ws, 1 << 40, None) == code
+    assert L.fp_dense_attn(ctypes.byref(s), FAKE, FAKE, FAKE, FAKE, None, None) == code
+
+
+def test_null_pointers_rejected(L):
+    s = shape()
+    p = ops.make_params(0.95, 0.1, 1024, 0)
+    assert L.fp_estimate(None, *([FAKE] * 9), FAKE, 1 << 40, None) == 1
+    assert L.fp_estimate(ctypes.byref(s), FAKE, None, *([FAKE] * 7), FAKE, 1 << 40, None) == 1
+    assert L.fp_pattern(ctypes.byref(s), None, FAKE, FAKE, FAKE, FAKE, None) == 1
+    assert L.fp_pattern(ctypes.byref(s), ctypes.byref(p), FAKE, None, FAKE, FAKE, None) == 1
+    assert L.fp_select(ctypes.byref(s), ctypes.byref(p), FAKE, FAKE, FAKE, FAKE, FAKE, None,
+                       FAKE, 1 << 40, None) == 1
+    assert L.fp_sparse_attn(ctypes.byref(s), FAKE, FAKE, FAKE, None, FAKE, FAKE, None, None, 0,
+                            None) == 1
+    assert L.fp_dense_attn(ctypes.byref(s), FAKE, FAKE, None, FAKE, None, None) == 1
+    assert L.fp_prefill_attn(ctypes.byref(s), ctypes.byref(p), FAKE, FAKE, FAKE, None, None,
+                             None, FAKE, 1 << 40, None) == 1
+    assert L.fp_prefill_attn_host(ctypes.byref(s), ctypes.byref(p), FAKE, FAKE, None, FAKE,
+                                  FAKE, 1 << 40, None) == 1
+
+
+@pytest.mark.parametrize("gamma,tau,lo,code", [
+    (0.0, 0.1, 0, 4), (1.5, 0.1, 0, 4), (float("nan"), 0.1, 0, 4), (0.9, -0.1, 0, 4),
+    (0.9, float("inf"), 0, 4), (0.9, 0.1, -5, 4),
+])
+def test_bad_params_rejected(L, gamma, tau, lo, code):
+    s = shape()
+    p = ops.make_params(gamma, tau, lo, 0)
+    assert L.fp_pattern(ctypes.byref(s), ctypes.byref(p), FAKE, FAKE, FAKE, FAKE, None) == code
+    assert L.fp_select(ctypes.byref(s), ctypes.byref(p), *([FAKE] * 6), FAKE, 1 << 40,
+                       None) == code
+
+
+def test_workspace_checks(L):
+    s = shape()
+    need = ops.fp_workspace_size(s, ops.FP_CALL_ESTIMATE)
+    args = [FAKE] * 9
+    assert L.fp_estimate(ctypes.byref(s), *args, None, need, None) == 5
+    assert L.fp_estimate(ctypes.byref(s), *args, FAKE, need - 1, None) == 5
+    assert L.fp_estimate(ctypes.byref(s), *args, FAKE + 8, need, None) == 5  # misaligned
+    p = ops.make_params(0.9, 0.1, 0, 0)
+    need = ops.fp_workspace_size(s, ops.FP_CALL_PREFILL)
+    assert L.fp_prefill_attn(ctypes.byref(s), ctypes.byref(p), FAKE, FAKE, FAKE, FAKE, None,
+                             None, FAKE, need - 256, None) == 5
+
+
+def test_bf16_attention_shape_limits(L):
+    # the tensor-core path takes d == 128 and B == 128; fp32 takes all four
+    for bs, d in [(64, 128), (128, 64), (64, 64)]:
+        s = shape(block_size=bs, head_dim=d)
+        assert L.fp_dense_attn(ctypes.byref(s), FAKE, FAKE, FAKE, FAKE, None, None) == 2
+
+
+def test_missing_library_fails_loudly(monkeypatch):
+    monkeypatch.setattr(ops, "_LIB", None)
+    monkeypatch.setenv("FP_LIBRARY", "/nonexistent/libfp.so")
+    with pytest.raises(RuntimeError, match="no fallback"):
+        ops.lib()

@@ -1,0 +1,302 @@
+"""GPU parity: every stage of the CUDA path against the CPU oracle, through the
+C ABI (ops.fp_* -> libfp.so).
+
+Tolerances (written here, derived from the arithmetic):
+  estimate     rtol 1e-4 (+ atol 1e-7 for values near 0): fp32 accumulation of
+               bf16/fp32 inputs against fp64;
+  pattern      identical decision wherever |d_JS - tau| > 1e-6; d_JS within 1e-6;
+  select       bit-exact counts and index lists, given the kernels' own fp32
+               scores and pattern (integer rule, no rounding);
+  attention    max |out - oracle| <= 1e-4 on the fp32 path, <= 2e-2 on the
+               bf16 tensor-core path; lse within 1e-4 / 2e-3.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from dynamic_block_sparse_fp_b200 import build, ops, synth
+
+pytestmark = [pytest.mark.gpu,
+              pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA GPU")]
+
+DEV = "cuda:0"
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    build.build()
+    ops.lib()
+    assert ops.fp_last_device_status() == 0
+
+
+def _np(t):
+    return t.detach().float().cpu().numpy()
+
+
+_CACHE = {}
+
+
+def _inputs(name, **kw):
+    key = (name, tuple(sorted(kw.items())))
+    if key not in _CACHE:
+        w = synth.WORKLOADS[name].replace(**kw) if kw else synth.WORKLOADS[name]
+        inp = synth.make_inputs(w)
+        _CACHE.clear()  # keep one workload's tensors alive at a time
+        _CACHE[key] = (w, inp, {x: inp[x].to(DEV) for x in ("q", "k", "v")})
+    return _CACHE[key]
+
+
+def _estimate_close(got, want, name):
+    for key in ("qbar", "kbar", "map", "est_last", "true_last", "vert", "slash"):
+        g, o = _np(got[key]), want[key]
+        np.testing.assert_allclose(g, o, rtol=1e-4, atol=1e-7, err_msg=f"{name}:{key}")
+
+
+@pytest.mark.parametrize("name", ["tiny_n1024", "llama8b_n8192"])
+def test_estimate_parity(name):
+    w, inp, d = _inputs(name)
+    got = ops.estimate(d["q"], d["k"], w.block_size)
+    torch.cuda.synchronize()
+    want = oracle.estimate(inp["q"], inp["k"], w.block_size)
+    _estimate_close(got, want, name)
+    assert ops.fp_last_device_status() == 0
+
+
+def test_estimate_parity_block64_and_d128_fp32():
+    w, inp, d = _inputs("tiny_n1024", head_dim=128, n_q_heads=4, n_kv_heads=2,
+                        fixed_kinds=("qa", "vs"), seq_len=512)
+    got = ops.estimate(d["q"], d["k"], 64)
+    want = oracle.estimate(inp["q"], inp["k"], 64)
+    _estimate_close(got, want, "b64d128")
+    got = ops.estimate(d["q"], d["k"], 128)
+    want = oracle.estimate(inp["q"], inp["k"], 128)
+    _estimate_close(got, want, "b128d128")
+
+
+@pytest.mark.parametrize("tau", [0.0, 0.03, 0.1, 0.9])
+def test_pattern_parity(tau):
+    w, inp, d = _inputs("llama8b_n8192")
+    est = ops.estimate(d["q"], d["k"], w.block_size)
+    s = ops.make_shape(d["q"], d["k"], w.block_size)
+    djs, pat = ops.pattern(s, ops.make_params(0.95, tau), est["est_last"], est["true_last"])
+    odjs, opat = oracle.pattern(_np(est["est_last"]), _np(est["true_last"]), tau)
+    np.testing.assert_allclose(_np(djs), odjs, rtol=0, atol=1e-6)
+    decided = np.abs(odjs - np.float32(tau)) > 1e-6
+    assert (pat.cpu().numpy()[decided] == opat[decided]).all()
+    if tau == 0.0:
+        assert (pat.cpu().numpy() == oracle.PATTERN_VS).all()
+
+
+def _select_case(w, est, pat, gamma, lo, hi):
+    s = ops.fp_shape(w.batch, w.n_q_heads, w.n_kv_heads, w.seq_len, w.head_dim, w.block_size,
+                     ops.FP_BF16 if w.dtype == "bf16" else ops.FP_F32)
+    p = ops.make_params(gamma, 0.1, lo, hi)
+    counts, indices = ops.select(s, p, pat, est["map"], est["vert"], est["slash"])
+    torch.cuda.synchronize()
+    oc, oi = oracle.select(pat.cpu().numpy(), _np(est["map"]), _np(est["vert"]),
+                           _np(est["slash"]), w.n_blocks, w.block_size, gamma, lo, hi)
+    gc = counts.cpu().numpy()
+    gi = indices.cpu().numpy()
+    np.testing.assert_array_equal(gc, oc)
+    bt, hq, nb = gc.shape
+    for b in range(bt):
+        for h in range(hq):
+            for i in range(nb):
+                c = gc[b, h, i]
+                if not np.array_equal(gi[b, h, i, :c], oi[b, h, i, :c]):
+                    raise AssertionError(f"row ({b},{h},{i}) differs")
+    return gc
+
+
+@pytest.mark.parametrize("name", ["tiny_n1024", "llama8b_n8192"])
+@pytest.mark.parametrize("mode", ["natural", "all_vs", "alternate"])
+@pytest.mark.parametrize("gamma,lo,hi", [(0.95, 1024, 0), (0.9, 0, 0), (0.9, 2048, 8192),
+                                         (0.5, 0, 1024), (1.0, 0, 0), (0.999, 256, 0)])
+def test_select_bit_exact(name, mode, gamma, lo, hi):
+    w, inp, d = _inputs(name)
+    est = ops.estimate(d["q"], d["k"], w.block_size)
+    s = ops.make_shape(d["q"], d["k"], w.block_size)
+    _, pat = ops.pattern(s, ops.make_params(0.95, 0.1), est["est_last"], est["true_last"])
+    if mode == "all_vs":
+        pat = torch.full_like(pat, ops.FP_PATTERN_VS)
+    elif mode == "alternate":
+        pat = (torch.arange(pat.numel(), device=DEV, dtype=torch.int32) % 2).reshape(pat.shape)
+    gc = _select_case(w, est, pat, gamma, lo, hi)
+    if gamma >= 1.0:
+        assert (gc == np.arange(1, w.n_blocks + 1)).all()
+
+
+def test_select_ties_and_zero_scores():
+    """Hand-made scores: many exact ties and zero entries (radix tie rank)."""
+    w = synth.WORKLOADS["tiny_n1024"].replace(n_q_heads=2, n_kv_heads=1)
+    nb, n = w.n_blocks, w.seq_len
+    t_pairs = nb * (nb + 1) // 2
+    g = torch.Generator().manual_seed(5)
+    levels = torch.tensor([0.0, 1e-3, 2e-3, 5e-3, 2.0 ** -20], dtype=torch.float32)
+    mp = levels[torch.randint(0, 5, (1, 2, t_pairs), generator=g)]
+    vt = levels[torch.randint(0, 5, (1, 2, n), generator=g)]
+    sl = levels[torch.randint(0, 5, (1, 2, n), generator=g)]
+    est = {"map": mp.to(DEV), "vert": vt.to(DEV), "slash": sl.to(DEV)}
+    pat = torch.tensor([[0, 1]], dtype=torch.int32, device=DEV)
+    for gamma, lo, hi in [(0.9, 0, 0), (0.7, 100, 300), (0.3, 0, 0)]:
+        _select_case(w, est, pat, gamma, lo, hi)
+
+
+def _pipeline(w, d, gamma=None, tau=None, lo=None, hi=None):
+    s = ops.make_shape(d["q"], d["k"], w.block_size)
+    p = ops.make_params(w.gamma if gamma is None else gamma, w.tau if tau is None else tau,
+                        w.min_budget if lo is None else lo, w.max_budget if hi is None else hi)
+    est = ops.estimate(d["q"], d["k"], w.block_size)
+    djs, pat = ops.pattern(s, p, est["est_last"], est["true_last"])
+    counts, indices = ops.select(s, p, pat, est["map"], est["vert"], est["slash"])
+    out, lse = ops.sparse_attn(d["q"], d["k"], d["v"], counts, indices, w.block_size)
+    torch.cuda.synchronize()
+    return dict(est=est, djs=djs, pattern=pat, counts=counts, indices=indices, out=out, lse=lse,
+                shape=s, params=p)
+
+
+def _attn_check(inp, res, w, tol, lse_tol, heads=None, q_blocks=None):
+    o, l = oracle.sparse_attention(inp["q"], inp["k"], inp["v"], res["counts"].cpu().numpy(),
+                                   res["indices"].cpu().numpy(), w.block_size, heads, q_blocks)
+    g, gl = _np(res["out"]), _np(res["lse"])
+    m = ~np.isnan(o)
+    err = np.abs(g[m] - o[m]).max()
+    assert err <= tol, f"max abs err {err}"
+    ml = ~np.isnan(l)
+    lerr = np.abs(gl[ml] - l[ml]).max()
+    assert lerr <= lse_tol, f"lse err {lerr}"
+    return err
+
+
+def test_pipeline_tiny_fp32_parity():
+    w, inp, d = _inputs("tiny_n1024")
+    res = _pipeline(w, d)
+    err = _attn_check(inp, res, w, 1e-4, 1e-4)
+    assert err < 1e-4
+    assert ops.fp_last_device_status() == 0
+
+
+@pytest.mark.parametrize("tau,lo,hi", [(0.1, 1024, 0), (0.0, 1024, 8192), (0.1, 0, 2048)])
+def test_pipeline_llama8k_bf16_parity(tau, lo, hi):
+    w, inp, d = _inputs("llama8b_n8192")
+    res = _pipeline(w, d, tau=tau, lo=lo, hi=hi)
+    # every head, a spread of query blocks (first, diagonal-heavy, last)
+    _attn_check(inp, res, w, 2e-2, 2e-3, heads=list(range(w.n_q_heads)),
+                q_blocks=[0, 1, 17, 40, 63])
+    assert ops.fp_last_device_status() == 0
+
+
+def test_dense_parity():
+    w, inp, d = _inputs("tiny_n1024")
+    out, lse = ops.dense_attn(d["q"], d["k"], d["v"], w.block_size)
+    o, l = oracle.dense_attention(inp["q"], inp["k"], inp["v"], w.block_size)
+    assert np.abs(_np(out) - o).max() <= 1e-4
+    assert np.abs(_np(lse) - l).max() <= 1e-4
+    w, inp, d = _inputs("llama8b_n8192")
+    out, lse = ops.dense_attn(d["q"], d["k"], d["v"], w.block_size)
+    torch.cuda.synchronize()
+    o, l = oracle.dense_attention(inp["q"], inp["k"], inp["v"], w.block_size, heads=[0, 13, 31],
+                                  q_blocks=[0, 31, 63])
+    m = ~np.isnan(o)
+    assert np.abs(_np(out)[m] - o[m]).max() <= 2e-2
+    ml = ~np.isnan(l)
+    assert np.abs(_np(lse)[ml] - l[ml]).max() <= 2e-3
+
+
+def test_gamma_one_equals_dense_bitwise():
+    w, inp, d = _inputs("llama8b_n8192")
+    res = _pipeline(w, d, gamma=1.0)
+    assert (res["counts"].cpu().numpy() == np.arange(1, w.n_blocks + 1)).all()
+    out, lse = ops.dense_attn(d["q"], d["k"], d["v"], w.block_size)
+    assert torch.equal(out, res["out"])
+    assert torch.equal(lse, res["lse"])
+
+
+def test_prefill_matches_stages_and_host_path():
+    w, inp, d = _inputs("llama8b_n8192")
+    res = _pipeline(w, d)
+    out, _, stats = ops.prefill_attn(d["q"], d["k"], d["v"], w.block_size, res["params"])
+    torch.cuda.synchronize()
+    assert torch.equal(out, res["out"])
+    assert int(stats[0]) == int(res["counts"].sum())
+    assert int(stats[1]) == int((res["pattern"] == ops.FP_PATTERN_QA).sum())
+    # host buffers through the C ABI
+    s = res["shape"]
+    qh, kh, vh = (inp[x].contiguous().pin_memory() for x in ("q", "k", "v"))
+    oh = torch.empty_like(qh).pin_memory()
+    ws = ops.workspace(s, ops.FP_CALL_PREFILL_HOST, DEV)
+    assert ops.fp_prefill_attn_host(s, res["params"], qh, kh, vh, oh, ws) == 0
+    torch.cuda.synchronize()
+    assert torch.equal(oh, res["out"].cpu())
+
+
+def test_edge_empty_rows_and_device_checks():
+    for name in ("tiny_n1024", "llama8b_n8192"):
+        w, inp, d = _inputs(name, seq_len=1024) if name != "tiny_n1024" else _inputs(name)
+        nb = w.n_blocks
+        bt, hq = w.batch, w.n_q_heads
+        counts = torch.zeros(bt, hq, nb, dtype=torch.int32, device=DEV)
+        indices = torch.zeros(bt, hq, nb, nb, dtype=torch.int32, device=DEV)
+        counts[:, :, 1::2] = 1  # odd rows: only key block 0; even rows: empty
+        out, lse = ops.sparse_attn(d["q"], d["k"], d["v"], counts, indices, w.block_size)
+        torch.cuda.synchronize()
+        o, l = oracle.sparse_attention(inp["q"], inp["k"], inp["v"], counts.cpu().numpy(),
+                                       indices.cpu().numpy(), w.block_size, heads=[0],
+                                       q_blocks=[1, 3])
+        bs = w.block_size
+        tol = 1e-4 if w.dtype == "f32" else 2e-2
+        for qi in (1, 3):
+            sl = slice(qi * bs, (qi + 1) * bs)
+            assert np.abs(_np(out)[0, 0, sl] - o[0, 0, sl]).max() <= tol
+        even = _np(out).reshape(bt, hq, nb, bs, -1)[:, :, 0::2]
+        assert (even == 0).all()
+        assert torch.isinf(lse.reshape(bt, hq, nb, bs)[:, :, 0::2]).all()
+        assert ops.fp_last_device_status() == 0
+        # an index outside the causal range is flagged (and masked out)
+        indices[0, 0, 1, 0] = 5
+        ops.sparse_attn(d["q"], d["k"], d["v"], counts, indices, w.block_size)
+        assert ops.fp_last_device_status() == ops.STATUS_CODES["FP_ERR_DEVICE_CHECK"]
+        assert ops.fp_last_device_status() == 0
+
+
+def test_single_block_sequence():
+    w, inp, d = _inputs("llama8b_n8192", seq_len=128, n_q_heads=8, n_kv_heads=2)
+    res = _pipeline(w, d)
+    assert (res["counts"].cpu().numpy() == 1).all()
+    _attn_check(inp, res, w, 2e-2, 2e-3)
+
+
+def test_full_size_128k_sampled():
+    """The bench configuration (Llama-3.1-8B heads, N = 131072), sampled checks."""
+    w, inp, d = _inputs("llama8b_n131072")
+    res = _pipeline(w, d)
+    assert ops.fp_last_device_status() == 0
+    hs = [0, 21]  # one head of two different kv groups
+    g = w.n_q_heads // w.n_kv_heads
+    for h in hs:
+        kv = h // g
+        want = oracle.estimate(inp["q"][:, h:h + 1], inp["k"][:, kv:kv + 1], w.block_size)
+        sub = {k2: v2[:, h:h + 1] for k2, v2 in res["est"].items() if k2 not in ("kbar",)}
+        for key in ("map", "est_last", "true_last", "vert", "slash", "qbar"):
+            np.testing.assert_allclose(_np(sub[key]), want[key], rtol=1e-4, atol=1e-7,
+                                       err_msg=key)
+    # selection: the natural patterns, and every head forced to vertical-slash
+    all_vs = torch.full_like(res["pattern"], ops.FP_PATTERN_VS)
+    vs_counts, vs_indices = ops.select(res["shape"], res["params"], all_vs, res["est"]["map"],
+                                       res["est"]["vert"], res["est"]["slash"])
+    torch.cuda.synchronize()
+    for h in hs:
+        for pat, counts, indices in ((res["pattern"], res["counts"], res["indices"]),
+                                     (all_vs, vs_counts, vs_indices)):
+            oc, oi = oracle.select(pat[:, h:h + 1].cpu().numpy(),
+                                   _np(res["est"]["map"][:, h:h + 1]),
+                                   _np(res["est"]["vert"][:, h:h + 1]),
+                                   _np(res["est"]["slash"][:, h:h + 1]), w.n_blocks,
+                                   w.block_size, w.gamma, w.min_budget, w.max_budget)
+            gc = counts[:, h:h + 1].cpu().numpy()
+            gi = indices[:, h:h + 1].cpu().numpy()
+            np.testing.assert_array_equal(gc, oc)
+            for i in range(0, w.n_blocks, 37):
+                np.testing.assert_array_equal(gi[0, 0, i, :gc[0, 0, i]], oi[0, 0, i, :oc[0, 0, i]])
+    _attn_check(inp, res, w, 2e-2, 2e-3, heads=hs, q_blocks=[0, 511, 1023])
