@@ -239,6 +239,22 @@ FP_API fp_status fp_select(const fp_shape *shape, const fp_params *params,
                                    reinterpret_cast<cudaStream_t>(stream)));
 }
 
+FP_API fp_status fp_select_noalloc(const fp_shape *shape, const fp_params *params,
+                                   const int32_t *pattern, const float *map, const float *vert,
+                                   const float *slash, int32_t *counts, int32_t *indices,
+                                   fp_stream_t stream) {
+  Dims D;
+  fp_status s = check_shape(shape, &D);
+  if (s != FP_OK) return s;
+  if ((s = check_params(params)) != FP_OK) return s;
+  if (!pattern || !map || !vert || !slash || !counts || !indices) return FP_ERR_NULL;
+  if (select_ws_bytes(D) > FP_SELECT_NOALLOC_SCRATCH_BYTES) return FP_ERR_WORKSPACE;
+  if ((s = check_device()) != FP_OK) return s;
+  return cuda_status(launch_select_noalloc(D, params->gamma, budgets(D, *params), pattern, map,
+                                           vert, slash, counts, indices,
+                                           reinterpret_cast<cudaStream_t>(stream)));
+}
+
 FP_API fp_status fp_sparse_attn(const fp_shape *shape, const void *q, const void *k,
                                 const void *v, const int32_t *counts, const int32_t *indices,
                                 void *out, float *lse, void *ws, size_t ws_bytes,

@@ -58,6 +58,10 @@ cudaError_t launch_select(const Dims &D, float gamma, const SelectBudgets &bud,
                           const int32_t *pattern, const float *map, const float *vert,
                           const float *slash, int32_t *counts, int32_t *indices, void *ws,
                           cudaStream_t st);
+cudaError_t launch_select_noalloc(const Dims &D, float gamma, const SelectBudgets &bud,
+                                  const int32_t *pattern, const float *map, const float *vert,
+                                  const float *slash, int32_t *counts, int32_t *indices,
+                                  cudaStream_t st);
 cudaError_t launch_stats(const Dims &D, const int32_t *counts, const int32_t *pattern,
                          int64_t *stats, cudaStream_t st);
 

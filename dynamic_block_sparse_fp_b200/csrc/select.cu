@@ -419,3 +419,61 @@ cudaError_t launch_stats(const Dims &D, const int32_t *counts, const int32_t *pa
 }
 
 }  // namespace fpi
+
+// ---------------------------------------------------------------------------
+// fp_select without a workspace argument.  Its scratch (the same layout
+// select_ws_bytes describes) is one fixed array compiled into the library.
+// The array's name is only a host-side stand-in in host code, so the device
+// address is looked up with cudaGetSymbolAddress once per device (on the
+// first call made with that device current) and cached.  Nothing in the
+// scratch has to start at zero: select_head_kernel writes every record and
+// flag that emit_rows_kernel later reads.
+namespace fpi {
+
+static __device__ __align__(256) unsigned char g_select_scratch[FP_SELECT_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+cudaError_t select_scratch_address(void **out) {
+  static void *addr[64] = {nullptr};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (!addr[dev]) {
+    void *p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_select_scratch);
+    if (e != cudaSuccess) return e;
+    addr[dev] = p;
+  }
+  *out = addr[dev];
+  return cudaSuccess;
+}
+
+}  // namespace
+
+cudaError_t launch_select_noalloc(const Dims &D, float gamma, const SelectBudgets &bud,
+                                  const int32_t *pattern, const float *map, const float *vert,
+                                  const float *slash, int32_t *counts, int32_t *indices,
+                                  cudaStream_t st) {
+  if (D.nb > kMaxBlocks || select_ws_bytes(D) > FP_SELECT_NOALLOC_SCRATCH_BYTES)
+    return cudaErrorInvalidValue;
+  void *scratch = nullptr;
+  cudaError_t e = select_scratch_address(&scratch);
+  if (e != cudaSuccess) return e;
+  Carver c{static_cast<char *>(scratch), 0};
+  const size_t heads = size_t(D.bt) * D.hq;
+  HeadSel *sel = c.take<HeadSel>(2 * heads);
+  uint8_t *cf = c.take<uint8_t>(heads * D.nb);
+  uint8_t *df = c.take<uint8_t>(heads * D.nb);
+  const int smem = int(sizeof(SelSmem));
+  cudaFuncSetAttribute(select_head_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  select_head_kernel<<<dim3(D.hq, D.bt), kThreads, smem, st>>>(
+      pattern, map, vert, slash, D.n, D.nb, D.bs, gamma, bud.qa_lo, bud.qa_hi, bud.vs_lo,
+      bud.vs_hi, sel, cf, df);
+  emit_rows_kernel<<<dim3((D.nb + 7) / 8, D.hq, D.bt), 256, 0, st>>>(pattern, map, D.nb, sel, cf,
+                                                                    df, counts, indices);
+  return cudaGetLastError();
+}
+
+}  // namespace fpi

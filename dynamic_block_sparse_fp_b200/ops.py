@@ -59,6 +59,7 @@ _SIG = {
                                    _P]),
     "fp_pattern": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P]),
     "fp_select": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
+    "fp_select_noalloc": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "fp_sparse_attn": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "fp_dense_attn": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P]),
     "fp_prefill_attn": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t,
@@ -162,6 +163,13 @@ def fp_select(shape, params, pattern, map_, vert, slash, counts, indices, ws,
     return lib().fp_select(ctypes.byref(shape), ctypes.byref(params), _addr(pattern),
                            _addr(map_), _addr(vert), _addr(slash), _addr(counts),
                            _addr(indices), _addr(ws), _nbytes(ws), _stream(stream))
+
+
+def fp_select_noalloc(shape, params, pattern, map_, vert, slash, counts, indices,
+                      stream=None) -> int:
+    return lib().fp_select_noalloc(ctypes.byref(shape), ctypes.byref(params), _addr(pattern),
+                                   _addr(map_), _addr(vert), _addr(slash), _addr(counts),
+                                   _addr(indices), _stream(stream))
 
 
 def fp_sparse_attn(shape, q, k, v, counts, indices, out, lse, ws, stream=None) -> int:

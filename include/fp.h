@@ -162,6 +162,38 @@ fp_status fp_select(const fp_shape *shape, const fp_params *params,
                     void *ws, size_t ws_bytes, fp_stream_t stream);
 
 /*
+ * fp_select_noalloc -- fp_select for callers that cannot allocate device
+ * memory when they call in.  Some hosts own every byte of device memory and
+ * plan it before any work starts: an engine plugin's enqueue hook, a serving
+ * loop with a fixed memory budget, a framework whose caching allocator must
+ * stay the only one.  For them a cudaMalloc at call time is either forbidden
+ * or harmful (it can synchronise the device and fragment the plan), and they
+ * may have no spare buffer to hand over as a workspace.  This entry point
+ * takes no workspace: its scratch is one array of
+ * FP_SELECT_NOALLOC_SCRATCH_BYTES compiled into libfp.so, which every GPU
+ * that loads the library holds until the process exits.
+ * The paper has no counterpart to this call; it computes exactly what
+ * fp_select computes, with the same arguments minus the workspace.
+ *   * The scratch needed is fp_workspace_size(shape, FP_CALL_SELECT); a
+ *     problem needing more than FP_SELECT_NOALLOC_SCRATCH_BYTES is rejected
+ *     with FP_ERR_WORKSPACE before anything is launched.
+ *   * It allocates nothing (no cudaMalloc / cudaFree / allocating library
+ *     routine).  The first call on a device looks up the array's device
+ *     address for that device (cudaGetSymbolAddress); make that first call
+ *     before capturing any stream.
+ *   * Every call on a device uses the same array, which keeps the last
+ *     call's contents (nothing in it needs clearing).  Two calls whose work
+ *     can overlap on the GPU (different streams, several host threads) race
+ *     on it: the caller must order them.
+ */
+#define FP_SELECT_NOALLOC_SCRATCH_BYTES (1u << 20)
+fp_status fp_select_noalloc(const fp_shape *shape, const fp_params *params,
+                            const int32_t *pattern, const float *map,
+                            const float *vert, const float *slash,
+                            int32_t *counts, int32_t *indices,
+                            fp_stream_t stream);
+
+/*
  * fp_sparse_attn -- causal block-sparse attention over the given lists.
  * Source: atlas.scime.ai summary, "Approach" and "Experimental setup" (the
  * sparse kernel builds on FlashAttention).
