@@ -21,8 +21,9 @@
 //
 // Per key tile t the softmax warps read S(t) from TMEM, release the buffer,
 // compute p = 2^(s*scale*log2e - m) with a running row max m, rescale O in
-// TMEM when m grows, write P(t) (bf16) to shared memory and signal the MMA
-// warp, which then issues P(t) V(t) while S(t+1) is already in flight.
+// TMEM only when m grows by more than 2^8, write P(t) (bf16) to shared memory
+// and signal the MMA warp, which then issues P(t) V(t) while S(t+1) is
+// already in flight.
 //
 // Every wait is bounded (2 s); on expiry the kernel records FP_ERR_TIMEOUT,
 // raises a CTA-wide abort flag, drains its outstanding TMA loads and frees
@@ -264,9 +265,13 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(
         x[c] = y;
         tmax = fmaxf(tmax, y);
       }
-      const float mnew = fmaxf(m, tmax);
-      const float muse = mnew == -INFINITY ? 0.f : mnew;
-      const float alpha = ex2(m - muse);
+      // lazy rescale: keep the old max unless the row max grew by more than
+      // 2^8 (p <= 256 is exact enough in fp32 and bf16; the final 1/l uses
+      // the same stale max, so the result is unchanged)
+      float muse = m;
+      if (tmax > m + 8.0f || m == -INFINITY) muse = fmaxf(m, tmax);
+      if (muse == -INFINITY) muse = 0.f;  // every key so far masked
+      const float alpha = ex2(m - muse);  // 1 when unchanged, 0 on the first tile
       float ps = 0.f;
 #pragma unroll
       for (int c = 0; c < BN; ++c) {

@@ -367,6 +367,15 @@ cudaError_t run_estimate(const Dims &Dm, const T *q, const T *k, float *qbar, fl
   map_softmax_kernel<<<unsigned((rows + 7) / 8), 256, 0, st>>>(map, est_last, rows, Dm.nb);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
+  if (last_block_tc_supported(Dm)) {
+    float *sp = nullptr;
+    e = launch_last_block_tc(Dm, q, k, true_last, vert, &sp, ws, st);
+    if (e != cudaSuccess) return e;
+    const long long tot = (long long)Dm.bt * Dm.hq * Dm.n;
+    slash_combine_kernel<<<unsigned((tot + 255) / 256), 256, 0, st>>>(sp, slash, tot, Dm.n,
+                                                                      Dm.nb, Dm.bs);
+    return cudaGetLastError();
+  }
   if (Dm.bs == 128 && Dm.d == 128)
     return run_last<128, 128, T>(Dm, q, k, true_last, vert, slash, ws, st);
   if (Dm.bs == 128 && Dm.d == 64)
@@ -379,6 +388,7 @@ cudaError_t run_estimate(const Dims &Dm, const T *q, const T *k, float *qbar, fl
 }  // namespace
 
 size_t estimate_ws_bytes(const Dims &D) {
+  if (last_block_tc_supported(D)) return last_block_tc_ws_bytes(D);
   Carver c{nullptr, 0};
   const size_t rows = size_t(D.bt) * D.hq;
   c.take<float>(rows * D.nb * D.bs);

@@ -45,6 +45,13 @@ cudaError_t launch_estimate(const Dims &D, const void *q, const void *k, float *
                             float *kbar, float *map, float *est_last, float *true_last,
                             float *vert, float *slash, void *ws, cudaStream_t st);
 
+// Tensor-core passes over the last query block (estimate_tc.cu): bf16,
+// block 128, head dim 128.
+bool last_block_tc_supported(const Dims &D);
+size_t last_block_tc_ws_bytes(const Dims &D);
+cudaError_t launch_last_block_tc(const Dims &D, const void *q, const void *k, float *true_last,
+                                 float *vert, float **sp_out, void *ws, cudaStream_t st);
+
 cudaError_t launch_pattern(const Dims &D, float tau, const float *est_last,
                            const float *true_last, float *djs, int32_t *pattern,
                            cudaStream_t st);
