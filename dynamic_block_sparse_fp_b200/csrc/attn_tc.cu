@@ -77,6 +77,57 @@ __device__ __forceinline__ int list_block(const Item &it, int t, bool dense) {
   return dense ? t : __ldg(it.list + t);
 }
 
+// One S tile of one row (TMEM lane): the row max over the tile (read once,
+// 8 independent chains), the lazy-rescale decision, then the exponentials
+// (S read again 32 columns at a time, so few scores are live), packed to bf16
+// pairs, with the row sum in 8 chains.  MASK: keys c > lim contribute 0.
+template <bool MASK>
+__device__ __forceinline__ void softmax_tile(uint32_t s_addr, int lim, float sl2, float m,
+                                             float &muse, float &alpha, float (&sm8)[8],
+                                             uint32_t (&pk)[BN / 2]) {
+  float mx[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) mx[k] = -INFINITY;
+#pragma unroll
+  for (int c0 = 0; c0 < BN; c0 += 32) {
+    uint32_t u[32];
+    tmem_ld32(s_addr + uint32_t(c0), u);
+    tc_wait_ld();
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const float y = (MASK && c0 + i > lim) ? -INFINITY : __uint_as_float(u[i]);
+      mx[i % 8] = fmaxf(mx[i % 8], y);
+    }
+  }
+  const float tmax = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                           fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * sl2;
+  // lazy rescale: keep the old max unless the row max grew by more than 2^8
+  // (p <= 256 is exact enough in fp32 and bf16; the final 1/l uses the same
+  // stale max, so the result is unchanged)
+  muse = m;
+  if (tmax > m + 8.0f || m == -INFINITY) muse = fmaxf(m, tmax);
+  if (muse == -INFINITY) muse = 0.f;  // every key so far masked
+  alpha = ex2(m - muse);              // 1 when unchanged, 0 on the first tile
+#pragma unroll
+  for (int c0 = 0; c0 < BN; c0 += 32) {
+    uint32_t u[32];
+    tmem_ld32(s_addr + uint32_t(c0), u);
+    tc_wait_ld();
+#pragma unroll
+    for (int i = 0; i < 32; i += 2) {
+      float p0 = ex2(fmaf(__uint_as_float(u[i]), sl2, -muse));
+      float p1 = ex2(fmaf(__uint_as_float(u[i + 1]), sl2, -muse));
+      if (MASK) {
+        p0 = c0 + i > lim ? 0.f : p0;
+        p1 = c0 + i + 1 > lim ? 0.f : p1;
+      }
+      sm8[i % 8] += p0;
+      sm8[(i + 1) % 8] += p1;
+      pk[(c0 + i) / 2] = pack_bf16(p0, p1);
+    }
+  }
+}
+
 __global__ void __launch_bounds__(192, 1) attn_tc_kernel(
     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
     const __grid_constant__ CUtensorMap tm_v, const int32_t *__restrict__ counts,
@@ -242,42 +293,25 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(
         break;
       }
       tc_fence_after();
-      float x[BN];
-#pragma unroll
-      for (int c0 = 0; c0 < BN; c0 += 32) {
-        uint32_t u[32];
-        tmem_ld32(lane_base + uint32_t(sb * BN + c0), u);
-        tc_wait_ld();
-#pragma unroll
-        for (int i = 0; i < 32; ++i) x[c0 + i] = __uint_as_float(u[i]);
-      }
-      tc_fence_before();
-      mbar_arrive(&sm.s_free[sb]);
       const int j = list_block(it, t, dense);
       const bool valid = j >= 0 && j <= it.qi;
       if (!valid && r == 0) report(status, FP_ERR_DEVICE_CHECK);
-      const bool diag = j == it.qi;
-      float tmax = -INFINITY;
-#pragma unroll
-      for (int c = 0; c < BN; ++c) {
-        float y = x[c] * sl2;
-        if (!valid || (diag && c > r)) y = -INFINITY;
-        x[c] = y;
-        tmax = fmaxf(tmax, y);
-      }
-      // lazy rescale: keep the old max unless the row max grew by more than
-      // 2^8 (p <= 256 is exact enough in fp32 and bf16; the final 1/l uses
-      // the same stale max, so the result is unchanged)
-      float muse = m;
-      if (tmax > m + 8.0f || m == -INFINITY) muse = fmaxf(m, tmax);
-      if (muse == -INFINITY) muse = 0.f;  // every key so far masked
-      const float alpha = ex2(m - muse);  // 1 when unchanged, 0 on the first tile
-      float ps = 0.f;
-#pragma unroll
-      for (int c = 0; c < BN; ++c) {
-        x[c] = ex2(x[c] - muse);
-        ps += x[c];
-      }
+      // keys c > lim are masked: the diagonal block hides keys after the query
+      // row, an invalid entry hides all; other tiles take the unmasked path
+      const bool masked = !valid || j == it.qi;
+      const int lim = valid ? r : -1;
+      const uint32_t s_addr = lane_base + uint32_t(sb * BN);
+      float muse, alpha;
+      float sm8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      uint32_t pk[BN / 2];
+      if (masked)
+        softmax_tile<true>(s_addr, lim, sl2, m, muse, alpha, sm8, pk);
+      else
+        softmax_tile<false>(s_addr, lim, sl2, m, muse, alpha, sm8, pk);
+      tc_fence_before();
+      mbar_arrive(&sm.s_free[sb]);
+      const float ps = ((sm8[0] + sm8[1]) + (sm8[2] + sm8[3])) +
+                       ((sm8[4] + sm8[5]) + (sm8[6] + sm8[7]));
       l = l * alpha + ps;
       // wait until P(t-1) V(t-1) finished: P buffer free, O up to date
       if (!__all_sync(0xffffffffu, mbar_wait(&sm.p_empty, (t & 1) ^ 1, abort_flag))) {
@@ -303,11 +337,7 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(
       // (8 keys) c stored at chunk c ^ (row % 8)
 #pragma unroll
       for (int ch = 0; ch < BN / 8; ++ch) {
-        uint4 w;
-        w.x = pack_bf16(x[ch * 8 + 0], x[ch * 8 + 1]);
-        w.y = pack_bf16(x[ch * 8 + 2], x[ch * 8 + 3]);
-        w.z = pack_bf16(x[ch * 8 + 4], x[ch * 8 + 5]);
-        w.w = pack_bf16(x[ch * 8 + 6], x[ch * 8 + 7]);
+        const uint4 w = make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
         const int half = ch / 8, c = ch % 8;
         uint8_t *dst = sm.p + half * HALF_BYTES + r * 128 + ((c ^ (r & 7)) * 16);
         *reinterpret_cast<uint4 *>(dst) = w;

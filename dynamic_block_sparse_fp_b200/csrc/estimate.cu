@@ -80,8 +80,10 @@ __global__ void __launch_bounds__(256) pool_kernel(const T *__restrict__ x, floa
 }
 
 // ------------------------------------------------------------ block map --
-// grid (tiles, tiles, Bt*Hq), 256 threads; 64x64 tile of the nb x nb logit
-// matrix of one q head; tiles above the diagonal exit at once.
+// grid (tiles, tiles, Bt*Hq), 256 threads; a 128x128 tile of the nb x nb
+// logit matrix of one q head (tiles above the diagonal exit at once).  Each
+// thread accumulates an 8x8 register block (rows ty*4+{0..3} and 64+ty*4+..,
+// columns likewise) over d in steps of 8; fp32 fused multiply-adds.
 __global__ void __launch_bounds__(256) map_logits_kernel(const float *__restrict__ qbar,
                                                          const float *__restrict__ kbar,
                                                          float *__restrict__ map, int hq, int g,
@@ -90,42 +92,56 @@ __global__ void __launch_bounds__(256) map_logits_kernel(const float *__restrict
   if (tj > ti) return;
   const int bh = blockIdx.z, b = bh / hq, h = bh % hq, kv = h / g;
   const int hkv = hq / g;
-  __shared__ float As[32][65];
-  __shared__ float Bs[32][65];
+  __shared__ __align__(16) float As[8][128];
+  __shared__ __align__(16) float Bs[8][128];
   const float *qa = qbar + (size_t(b) * hq + h) * nb * d;
   const float *kb = kbar + (size_t(b) * hkv + kv) * nb * d;
   const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
-  float acc[4][4] = {};
-  for (int k0 = 0; k0 < d; k0 += 32) {
-    for (int e = threadIdx.x; e < 64 * 32; e += 256) {
-      int r = e / 32, c = e % 32;
-      int gi = ti * 64 + r, gj = tj * 64 + r;
-      As[c][r] = gi < nb ? qa[size_t(gi) * d + k0 + c] : 0.f;
-      Bs[c][r] = gj < nb ? kb[size_t(gj) * d + k0 + c] : 0.f;
-    }
+  // loader: thread -> (row, 4 consecutive k of the 8-wide chunk)
+  const int lr = threadIdx.x / 2, lk = (threadIdx.x % 2) * 4;
+  const int gi = ti * 128 + lr, gj = tj * 128 + lr;
+  float acc[8][8];
+#pragma unroll
+  for (int u = 0; u < 8; ++u)
+#pragma unroll
+    for (int w = 0; w < 8; ++w) acc[u][w] = 0.f;
+  for (int k0 = 0; k0 < d; k0 += 8) {
+    const float4 av = gi < nb ? *reinterpret_cast<const float4 *>(qa + size_t(gi) * d + k0 + lk)
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
+    const float4 bv = gj < nb ? *reinterpret_cast<const float4 *>(kb + size_t(gj) * d + k0 + lk)
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
     __syncthreads();
-#pragma unroll 8
-    for (int c = 0; c < 32; ++c) {
-      float a[4], bb[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) a[u] = As[c][ty + 16 * u];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) bb[u] = Bs[c][tx + 16 * u];
-#pragma unroll
-      for (int u = 0; u < 4; ++u)
-#pragma unroll
-        for (int w = 0; w < 4; ++w) acc[u][w] = fmaf(a[u], bb[w], acc[u][w]);
-    }
+    As[lk + 0][lr] = av.x;
+    As[lk + 1][lr] = av.y;
+    As[lk + 2][lr] = av.z;
+    As[lk + 3][lr] = av.w;
+    Bs[lk + 0][lr] = bv.x;
+    Bs[lk + 1][lr] = bv.y;
+    Bs[lk + 2][lr] = bv.z;
+    Bs[lk + 3][lr] = bv.w;
     __syncthreads();
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const float4 a0 = *reinterpret_cast<const float4 *>(&As[k][ty * 4]);
+      const float4 a1 = *reinterpret_cast<const float4 *>(&As[k][64 + ty * 4]);
+      const float4 b0 = *reinterpret_cast<const float4 *>(&Bs[k][tx * 4]);
+      const float4 b1 = *reinterpret_cast<const float4 *>(&Bs[k][64 + tx * 4]);
+      const float a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+      const float bb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+#pragma unroll
+        for (int w = 0; w < 8; ++w) acc[u][w] = fmaf(a[u], bb[w], acc[u][w]);
+    }
   }
   float *m = map + (size_t(b) * hq + h) * (size_t(nb) * (nb + 1) / 2);
 #pragma unroll
-  for (int u = 0; u < 4; ++u) {
-    int i = ti * 64 + ty + 16 * u;
+  for (int u = 0; u < 8; ++u) {
+    const int i = ti * 128 + (u < 4 ? ty * 4 + u : 64 + ty * 4 + u - 4);
     if (i >= nb) continue;
 #pragma unroll
-    for (int w = 0; w < 4; ++w) {
-      int j = tj * 64 + tx + 16 * w;
+    for (int w = 0; w < 8; ++w) {
+      const int j = tj * 128 + (w < 4 ? tx * 4 + w : 64 + tx * 4 + w - 4);
       if (j <= i) m[size_t(i) * (i + 1) / 2 + j] = acc[u][w] * scale;
     }
   }
@@ -359,7 +375,7 @@ cudaError_t run_estimate(const Dims &Dm, const T *q, const T *k, float *qbar, fl
                          float *slash, void *ws, cudaStream_t st) {
   pool_kernel<T><<<dim3(Dm.nb, Dm.hq, Dm.bt), 256, 0, st>>>(q, qbar, Dm.n, Dm.d, Dm.bs);
   pool_kernel<T><<<dim3(Dm.nb, Dm.hkv, Dm.bt), 256, 0, st>>>(k, kbar, Dm.n, Dm.d, Dm.bs);
-  const int tiles = (Dm.nb + 63) / 64;
+  const int tiles = (Dm.nb + 127) / 128;
   const float scale = 1.f / sqrtf(float(Dm.d));
   map_logits_kernel<<<dim3(tiles, tiles, Dm.bt * Dm.hq), 256, 0, st>>>(qbar, kbar, map, Dm.hq,
                                                                       Dm.g, Dm.nb, Dm.d, scale);

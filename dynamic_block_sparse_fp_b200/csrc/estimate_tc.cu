@@ -217,41 +217,48 @@ __global__ void __launch_bounds__(kThreads, 1) last_block_tc_kernel(
       const bool diag = j == nb - 1;
       if (PASS == 1) {
         // row r of the last block sees key c of the diagonal tile iff c <= r
-        float tmax = -INFINITY;
+        if (diag) {
 #pragma unroll
-        for (int c = 0; c < BS; ++c) {
-          const float y = (diag && c > r) ? -INFINITY : x[c] * sl2;
-          x[c] = y;
-          tmax = fmaxf(tmax, y);
+          for (int c = 0; c < BS; ++c)
+            if (c > r) x[c] = -INFINITY;
         }
-        const float mnew = fmaxf(m, tmax);
-        float s = 0.f;
+        // 8 independent chains for the max and the sum, then trees
+        float mx[8], sm8[8];
 #pragma unroll
-        for (int c = 0; c < BS; ++c) s += ex2(x[c] - mnew);
+        for (int k = 0; k < 8; ++k) {
+          mx[k] = x[k];
+          sm8[k] = 0.f;
+        }
+#pragma unroll
+        for (int c = 8; c < BS; ++c) mx[c % 8] = fmaxf(mx[c % 8], x[c]);
+        const float tmax = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                                 fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+        const float mnew = fmaxf(m, tmax * sl2);
+#pragma unroll
+        for (int c = 0; c < BS; ++c) sm8[c % 8] += ex2(fmaf(x[c], sl2, -mnew));
+        const float s = ((sm8[0] + sm8[1]) + (sm8[2] + sm8[3])) +
+                        ((sm8[4] + sm8[5]) + (sm8[6] + sm8[7]));
         l = l * ex2(m - mnew) + s;
         m = mnew;
       } else {
-        // key r of the tile, query c of the last block: visible iff r <= c
-        float v = 0.f;
-        float acc = 0.f;  // systolic diagonal accumulator
+        // key r of the tile, query c of the last block: visible iff r <= c.
+        // Diagonal sums (query - key) by a register-systolic chain per warp:
+        // at step c lane l holds the diagonal c - l and passes it one lane up;
+        // lane 31 completes one diagonal per step.  The vertical sum of the
+        // key runs in 4 independent chains.
+        float v4[4] = {0.f, 0.f, 0.f, 0.f};
+        float acc = 0.f;
         float *bins = sm.bins[hh][wq];
 #pragma unroll
-        for (int c4 = 0; c4 < BS; c4 += 4) {
-          const float4 ls = *reinterpret_cast<const float4 *>(&sm.lse2[hh][c4]);
-          const float lv[4] = {ls.x, ls.y, ls.z, ls.w};
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int c = c4 + i;
-            const float p = (diag && r > c) ? 0.f : ex2(fmaf(x[c], sl2, -lv[i]));
-            v += p;
-            // lane l holds the diagonal (c - l); shift it one lane up
-            acc = __shfl_up_sync(0xffffffffu, acc, 1);
-            if (lane == 0) acc = 0.f;
-            acc += p;
-            if (lane == 31) bins[c] = acc;  // diagonal c - 31 is complete
-          }
+        for (int c = 0; c < BS; ++c) {
+          const float p = (diag && r > c) ? 0.f : ex2(fmaf(x[c], sl2, -sm.lse2[hh][c]));
+          v4[c % 4] += p;
+          float a = __shfl_up_sync(0xffffffffu, acc, 1);
+          acc = (lane == 0 ? 0.f : a) + p;
+          if (lane == 31) bins[c] = acc;  // diagonal c - 31 is complete
         }
         if (lane < 31) bins[BS + 30 - lane] = acc;  // diagonals 127 - lane
+        const float v = (v4[0] + v4[1]) + (v4[2] + v4[3]);
         vert[bh * n_tok + size_t(j) * BS + r] = v;
         // tile mass, fixed order: lanes (xor tree), then warps
         float wsum = v;
