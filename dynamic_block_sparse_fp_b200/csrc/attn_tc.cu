@@ -88,15 +88,17 @@ __device__ __forceinline__ void softmax_tile(uint32_t s_addr, int lim, float sl2
   float mx[8];
 #pragma unroll
   for (int k = 0; k < 8; ++k) mx[k] = -INFINITY;
+  {
+    // all four 32-column loads in flight, one wait
+    uint32_t u[BN];
 #pragma unroll
-  for (int c0 = 0; c0 < BN; c0 += 32) {
-    uint32_t u[32];
-    tmem_ld32(s_addr + uint32_t(c0), u);
+    for (int c0 = 0; c0 < BN; c0 += 32)
+      tmem_ld32(s_addr + uint32_t(c0), *reinterpret_cast<uint32_t(*)[32]>(&u[c0]));
     tc_wait_ld();
 #pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      const float y = (MASK && c0 + i > lim) ? -INFINITY : __uint_as_float(u[i]);
-      mx[i % 8] = fmaxf(mx[i % 8], y);
+    for (int c = 0; c < BN; ++c) {
+      const float y = (MASK && c > lim) ? -INFINITY : __uint_as_float(u[c]);
+      mx[c % 8] = fmaxf(mx[c % 8], y);
     }
   }
   const float tmax = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
@@ -109,12 +111,14 @@ __device__ __forceinline__ void softmax_tile(uint32_t s_addr, int lim, float sl2
   if (muse == -INFINITY) muse = 0.f;  // every key so far masked
   alpha = ex2(m - muse);              // 1 when unchanged, 0 on the first tile
 #pragma unroll
-  for (int c0 = 0; c0 < BN; c0 += 32) {
-    uint32_t u[32];
-    tmem_ld32(s_addr + uint32_t(c0), u);
+  for (int c0 = 0; c0 < BN; c0 += 64) {
+    // two 32-column loads in flight, one wait
+    uint32_t u[64];
+    tmem_ld32(s_addr + uint32_t(c0), *reinterpret_cast<uint32_t(*)[32]>(&u[0]));
+    tmem_ld32(s_addr + uint32_t(c0 + 32), *reinterpret_cast<uint32_t(*)[32]>(&u[32]));
     tc_wait_ld();
 #pragma unroll
-    for (int i = 0; i < 32; i += 2) {
+    for (int i = 0; i < 64; i += 2) {
       float p0 = ex2(fmaf(__uint_as_float(u[i]), sl2, -muse));
       float p1 = ex2(fmaf(__uint_as_float(u[i + 1]), sl2, -muse));
       if (MASK) {

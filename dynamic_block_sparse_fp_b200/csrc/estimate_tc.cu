@@ -247,11 +247,19 @@ __global__ void __launch_bounds__(kThreads, 1) last_block_tc_kernel(
         // lane 31 completes one diagonal per step.  The vertical sum of the
         // key runs in 4 independent chains.
         float v4[4] = {0.f, 0.f, 0.f, 0.f};
+        float lq[4];
         float acc = 0.f;
         float *bins = sm.bins[hh][wq];
 #pragma unroll
         for (int c = 0; c < BS; ++c) {
-          const float p = (diag && r > c) ? 0.f : ex2(fmaf(x[c], sl2, -sm.lse2[hh][c]));
+          if (c % 4 == 0) {
+            const float4 ls = *reinterpret_cast<const float4 *>(&sm.lse2[hh][c]);
+            lq[0] = ls.x;
+            lq[1] = ls.y;
+            lq[2] = ls.z;
+            lq[3] = ls.w;
+          }
+          const float p = (diag && r > c) ? 0.f : ex2(fmaf(x[c], sl2, -lq[c % 4]));
           v4[c % 4] += p;
           float a = __shfl_up_sync(0xffffffffu, acc, 1);
           acc = (lane == 0 ? 0.f : a) + p;
