@@ -112,6 +112,16 @@ def dist_setup():
     return ws, rank, local
 
 
+def rank_workload(w: synth.Workload, rank: int) -> synth.Workload:
+    """The independent layer rank `rank` runs (its own seed; rank 0 = w)."""
+    return w.replace(seed=w.seed + 1000 * rank) if rank else w
+
+
+def job_value(tokens_per_rank: int, ws: int, ms_per_step: float) -> float:
+    """Whole-job tokens/s: every rank's tokens over the slowest rank's time."""
+    return ws * tokens_per_rank / (ms_per_step * 1e-3)
+
+
 def max_over_ranks(x: float, ws: int, device) -> float:
     if ws == 1:
         return x
@@ -223,9 +233,8 @@ def run_ours(args, w, ws, rank, local):
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     peaks = load_peaks()
-    # every rank: its own independent layer (batch index = rank)
-    wr = w.replace(seed=w.seed + 1000 * rank) if rank else w
-    inp = synth.make_inputs(wr)
+    # every rank: its own independent layer
+    inp = synth.make_inputs(rank_workload(w, rank))
     q, k, v = (inp[x].to(dev) for x in ("q", "k", "v"))
     bt, hq, n, d = q.shape
     hkv, bs = k.shape[1], w.block_size
@@ -294,7 +303,7 @@ def run_ours(args, w, ws, rank, local):
     attn_flops = flop_block * kept
     attn_tflops = attn_flops / (stage_ms[3] * 1e-3) / 1e12
     tokens = n * bt
-    value = ws * tokens / (ms_step * 1e-3)
+    value = job_value(tokens, ws, ms_step)
     # dense comparison at the same length (same kernel over every causal block)
     dense_ms = None
     if not args.no_dense:

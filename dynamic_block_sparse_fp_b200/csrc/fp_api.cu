@@ -104,6 +104,21 @@ fp_status check_device() {
 
 fp_status cuda_status(cudaError_t e) { return e == cudaSuccess ? FP_OK : FP_ERR_CUDA; }
 
+// One thread waits on an mbarrier that nothing arrives at, with the bounded
+// wait of the pipelined kernels, and records FP_ERR_TIMEOUT when it gives up.
+__global__ void watchdog_selftest_kernel(int *status, unsigned long long limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    mbar_fence_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0 && !mbar_wait(&bar, 0, &abort_flag, limit_ns))
+    report(status, FP_ERR_TIMEOUT);
+}
+
 // Intermediates of the whole path, carved from a workspace.
 struct Prefill {
   float *qbar, *kbar, *map, *est_last, *true_last, *vert, *slash, *djs;
@@ -348,6 +363,15 @@ FP_API fp_status fp_last_device_status(fp_stream_t stream) {
   if (cudaMemcpy(p, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess)
     return FP_ERR_CUDA;
   return static_cast<fp_status>(v);
+}
+
+FP_API fp_status fp_selftest_watchdog(unsigned int limit_us, fp_stream_t stream) {
+  if (limit_us == 0 || limit_us > 1000000u) return FP_ERR_PARAM;
+  fp_status s = check_device();
+  if (s != FP_OK) return s;
+  watchdog_selftest_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      device_status_ptr(), 1000ull * limit_us);
+  return cuda_status(cudaGetLastError());
 }
 
 FP_API const char *fp_status_string(fp_status status) {

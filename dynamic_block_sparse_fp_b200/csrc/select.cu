@@ -20,12 +20,15 @@
 // count when the clamp moves k, and one ordered count for the tie rank.  All
 // of it is integer arithmetic, so the result does not depend on thread order.
 // emit_rows_kernel then writes every row's ascending block list.
+#include <cooperative_groups.h>
+
 #include "fp_internal.cuh"
+
+namespace cg = cooperative_groups;
 
 namespace fpi {
 namespace {
 
-constexpr int kThreads = 1024;
 constexpr int kMaxBlocks = 4096;  // nb limit (flags live in shared memory)
 
 enum : int { SEL_THRESHOLD = 0, SEL_NONE = 1, SEL_ALL = 2 };
@@ -49,13 +52,33 @@ __device__ __forceinline__ bool kept(uint32_t bits, uint32_t i, const HeadSel &s
   return bits > s.bits || (bits == s.bits && i <= s.idx);
 }
 
+
+// ---------------------------------------------------------------------------
+// One selection problem per head, spread over a cluster of kCluster CTAs.
+// Rank r of the cluster owns the contiguous slice [r*ceil(n/C), ...) of the
+// list.  Each histogram level is built per slice, then every rank sums its
+// share of the bins over all ranks (distributed shared memory) into rank 0's
+// copy; rank 0 finds the crossing bin and the other ranks read the result.
+// Integer arithmetic throughout: the result does not depend on the split.
+
+constexpr int kCluster = 8;
+constexpr int kCThreads = 512;
+constexpr int kCWarps = kCThreads / 32;
+
 struct SelSmem {
   unsigned long long hmass[4096];
   unsigned int hcnt[4096];
   unsigned long long warp_tot[32];
-  unsigned long long res[4];
+  unsigned long long res[8];  // [0..2] crossing, [3] scan total, [4] slice count, [5] tie index
   uint8_t colflag[kMaxBlocks];
   uint8_t distflag[kMaxBlocks];
+};
+
+struct Ctx {
+  cg::cluster_group cl;
+  unsigned rank;
+  SelSmem *sm;
+  __device__ SelSmem *peer(unsigned q) const { return cl.map_shared_rank(sm, int(q)); }
 };
 
 // Block-wide exclusive prefix sum (thread order) of one value per thread.
@@ -72,14 +95,14 @@ __device__ unsigned long long block_excl_scan(unsigned long long v, SelSmem &sm,
   if (lane == 31) sm.warp_tot[w] = x;
   __syncthreads();
   if (w == 0) {
-    unsigned long long t = sm.warp_tot[lane];
+    unsigned long long t = lane < kCWarps ? sm.warp_tot[lane] : 0ull;
     unsigned long long s = t;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       unsigned long long y = __shfl_up_sync(0xffffffffu, s, o);
       if (lane >= o) s += y;
     }
-    sm.warp_tot[lane] = s - t;  // exclusive over warps
+    if (lane < kCWarps) sm.warp_tot[lane] = s - t;  // exclusive over warps
     if (lane == 31) sm.res[3] = s;
   }
   __syncthreads();
@@ -89,21 +112,23 @@ __device__ unsigned long long block_excl_scan(unsigned long long v, SelSmem &sm,
   return r;
 }
 
-// Histogram of (bits >> shift) & (nbins-1) over entries whose masked bits
-// equal `prefix`, mass and count, warp-aggregated shared-memory atomics.
-__device__ void histogram(const float *__restrict__ s, uint32_t n, uint32_t prefix,
-                          uint32_t pmask, int shift, uint32_t nbins, SelSmem &sm) {
-  for (uint32_t i = threadIdx.x; i < nbins; i += kThreads) {
+// Histogram of (bits >> shift) & (nbins-1) over the slice [i0, i1), entries
+// whose masked bits equal `prefix`; mass and count, warp-aggregated
+// shared-memory atomics.  Then the cluster-wide merge into rank 0.
+__device__ void histogram(const Ctx &cx, const float *__restrict__ s, uint32_t i0, uint32_t i1,
+                          uint32_t prefix, uint32_t pmask, int shift, uint32_t nbins) {
+  SelSmem &sm = *cx.sm;
+  for (uint32_t i = threadIdx.x; i < nbins; i += kCThreads) {
     sm.hmass[i] = 0;
     sm.hcnt[i] = 0;
   }
   __syncthreads();
   const int lane = threadIdx.x % 32;
-  for (uint32_t base = (threadIdx.x / 32) * 32; base < n; base += kThreads) {
+  for (uint32_t base = i0 + (threadIdx.x / 32) * 32; base < i1; base += kCThreads) {
     const uint32_t i = base + lane;
     uint32_t bin = 0xFFFFFFFFu;
     uint64_t w = 0;
-    if (i < n) {
+    if (i < i1) {
       const uint32_t b = score_bits(s[i]);
       if ((b & pmask) == prefix) {
         bin = (b >> shift) & (nbins - 1);
@@ -118,65 +143,101 @@ __device__ void histogram(const float *__restrict__ s, uint32_t n, uint32_t pref
       atomicAdd(&sm.hcnt[bin], unsigned(__popc(peers)));
     }
   }
-  __syncthreads();
+  // merge: rank r sums bins [r*nbins/C, (r+1)*nbins/C) of every rank into rank 0
+  cx.cl.sync();
+  const uint32_t per = nbins / kCluster;
+  SelSmem *root = cx.peer(0);
+  for (uint32_t b = cx.rank * per + threadIdx.x; b < (cx.rank + 1) * per; b += kCThreads) {
+    unsigned long long m = 0;
+    unsigned int c = 0;
+#pragma unroll
+    for (unsigned q = 0; q < kCluster; ++q) {
+      const SelSmem *pq = cx.peer(q);
+      m += pq->hmass[b];
+      c += pq->hcnt[b];
+    }
+    root->hmass[b] = m;
+    root->hcnt[b] = c;
+  }
+  cx.cl.sync();
 }
 
-// Scan the histogram from the highest bin down; find the first bin at which
-// above + (inclusive cumulative) reaches the target.  Updates *above_m /
-// *above_c to include every bin strictly higher, returns the bin.
-__device__ uint32_t find_crossing(uint32_t nbins, bool by_mass, double target_m,
+// Rank 0: scan the merged histogram from the highest bin down and find the
+// first bin at which above + (inclusive cumulative) reaches the target.  Every
+// rank then reads the bin and the mass / count of the bins strictly higher.
+__device__ uint32_t find_crossing(const Ctx &cx, uint32_t nbins, bool by_mass, double target_m,
                                   unsigned long long target_c, unsigned long long *above_m,
-                                  unsigned long long *above_c, SelSmem &sm) {
-  const uint32_t per = nbins >= kThreads ? nbins / kThreads : 1;
-  const uint32_t p0 = threadIdx.x * per;  // positions in descending-bin order
-  unsigned long long lm = 0, lc = 0;
-  if (p0 < nbins)
-    for (uint32_t p = p0; p < p0 + per; ++p) {
-      const uint32_t b = nbins - 1 - p;
-      lm += sm.hmass[b];
-      lc += sm.hcnt[b];
-    }
-  unsigned long long tm, tc;
-  const unsigned long long em = block_excl_scan(lm, sm, &tm);
-  const unsigned long long ec = block_excl_scan(lc, sm, &tc);
-  if (threadIdx.x == 0) {
-    sm.res[0] = 0;  // fallback: lowest bin (unreachable for valid targets)
-    sm.res[1] = tm - sm.hmass[0];
-    sm.res[2] = tc - sm.hcnt[0];
-  }
-  __syncthreads();
-  const unsigned long long am = *above_m, ac = *above_c;
-  auto reach = [&](unsigned long long m, unsigned long long c) {
-    return by_mass ? (double)(am + m) >= target_m : (ac + c) >= target_c;
-  };
-  if (p0 < nbins && !reach(em, ec) && reach(em + lm, ec + lc)) {
-    unsigned long long cm = em, cc = ec;
-    for (uint32_t p = p0; p < p0 + per; ++p) {
-      const uint32_t b = nbins - 1 - p;
-      if (reach(cm + sm.hmass[b], cc + sm.hcnt[b])) {
-        sm.res[0] = b;
-        sm.res[1] = cm;
-        sm.res[2] = cc;
-        break;
+                                  unsigned long long *above_c) {
+  SelSmem &sm = *cx.sm;
+  if (cx.rank == 0) {
+    const uint32_t per = nbins >= kCThreads ? nbins / kCThreads : 1;
+    const uint32_t p0 = threadIdx.x * per;  // positions in descending-bin order
+    unsigned long long lm = 0, lc = 0;
+    if (p0 < nbins)
+      for (uint32_t p = p0; p < p0 + per; ++p) {
+        const uint32_t b = nbins - 1 - p;
+        lm += sm.hmass[b];
+        lc += sm.hcnt[b];
       }
-      cm += sm.hmass[b];
-      cc += sm.hcnt[b];
+    unsigned long long tm, tc;
+    const unsigned long long em = block_excl_scan(lm, sm, &tm);
+    const unsigned long long ec = block_excl_scan(lc, sm, &tc);
+    if (threadIdx.x == 0) {
+      sm.res[0] = 0;  // fallback: lowest bin (unreachable for valid targets)
+      sm.res[1] = tm - sm.hmass[0];
+      sm.res[2] = tc - sm.hcnt[0];
+    }
+    __syncthreads();
+    const unsigned long long am = *above_m, ac = *above_c;
+    auto reach = [&](unsigned long long m, unsigned long long c) {
+      return by_mass ? (double)(am + m) >= target_m : (ac + c) >= target_c;
+    };
+    if (p0 < nbins && !reach(em, ec) && reach(em + lm, ec + lc)) {
+      unsigned long long cm = em, cc = ec;
+      for (uint32_t p = p0; p < p0 + per; ++p) {
+        const uint32_t b = nbins - 1 - p;
+        if (reach(cm + sm.hmass[b], cc + sm.hcnt[b])) {
+          sm.res[0] = b;
+          sm.res[1] = cm;
+          sm.res[2] = cc;
+          break;
+        }
+        cm += sm.hmass[b];
+        cc += sm.hcnt[b];
+      }
     }
   }
-  __syncthreads();
-  const uint32_t bin = uint32_t(sm.res[0]);
-  *above_m = am + sm.res[1];
-  *above_c = ac + sm.res[2];
-  __syncthreads();
+  cx.cl.sync();
+  const SelSmem *root = cx.peer(0);
+  const uint32_t bin = uint32_t(root->res[0]);
+  *above_m += root->res[1];
+  *above_c += root->res[2];
+  cx.cl.sync();  // rank 0 may reuse res afterwards
   return bin;
 }
 
+// Rank 0 sums the merged level-1 histogram (every entry is in it): W.
+__device__ unsigned long long total_mass(const Ctx &cx, uint32_t nbins) {
+  SelSmem &sm = *cx.sm;
+  if (cx.rank == 0) {
+    unsigned long long part = 0;
+    for (uint32_t b = threadIdx.x; b < nbins; b += kCThreads) part += sm.hmass[b];
+    unsigned long long tot;
+    block_excl_scan(part, sm, &tot);
+    if (threadIdx.x == 0) sm.res[6] = tot;
+  }
+  cx.cl.sync();
+  const unsigned long long w = cx.peer(0)->res[6];
+  cx.cl.sync();
+  return w;
+}
+
 // Radix descent; returns the threshold bit pattern and the mass / count of
-// every entry with larger bits.  Sets *total_m to W when first_pass_total.
-__device__ uint32_t descend(const float *s, uint32_t n, bool by_mass, float gamma,
-                            unsigned long long target_c, unsigned long long *above_m,
-                            unsigned long long *above_c, unsigned long long *total_m,
-                            double *target_m_out, SelSmem &sm) {
+// every entry with larger bits.  By mass the target is gamma * W.
+__device__ uint32_t descend(const Ctx &cx, const float *s, uint32_t i0, uint32_t i1,
+                            bool by_mass, float gamma, unsigned long long target_c,
+                            unsigned long long *above_m, unsigned long long *above_c,
+                            double *target_m_out) {
   const int shifts[3] = {20, 8, 0};
   const int widths[3] = {12, 12, 8};
   uint32_t prefix = 0, pmask = 0;
@@ -185,55 +246,60 @@ __device__ uint32_t descend(const float *s, uint32_t n, bool by_mass, float gamm
   double target_m = 0.0;
   for (int lv = 0; lv < 3; ++lv) {
     const uint32_t nbins = 1u << widths[lv];
-    histogram(s, n, prefix, pmask, shifts[lv], nbins, sm);
+    histogram(cx, s, i0, i1, prefix, pmask, shifts[lv], nbins);
     if (lv == 0 && by_mass) {
-      // W = every mass (the first level sees every entry)
-      unsigned long long part = 0;
-      for (uint32_t b = threadIdx.x; b < nbins; b += kThreads) part += sm.hmass[b];
-      unsigned long long tot;
-      block_excl_scan(part, sm, &tot);
-      *total_m = tot;
+      const unsigned long long tot = total_mass(cx, nbins);
       target_m = (double)gamma * (double)tot;
       *target_m_out = target_m;
     }
-    const uint32_t bin = find_crossing(nbins, by_mass, target_m, target_c, above_m, above_c, sm);
+    const uint32_t bin = find_crossing(cx, nbins, by_mass, target_m, target_c, above_m, above_c);
     prefix |= bin << shifts[lv];
     pmask |= (nbins - 1) << shifts[lv];
   }
   return prefix;
 }
 
-// Index of the m-th (1-based) entry with bit pattern == b, in index order.
-__device__ uint32_t tie_index(const float *s, uint32_t n, uint32_t b, unsigned long long m,
-                              SelSmem &sm) {
-  const uint32_t per = (n + kThreads - 1) / kThreads;
-  const uint32_t i0 = threadIdx.x * per;
-  const uint32_t i1 = min(n, i0 + per);
+// Index of the m-th (1-based) entry with bit pattern == b, in index order,
+// over the whole list (the slices are in index order across ranks).
+__device__ uint32_t tie_index(const Ctx &cx, const float *s, uint32_t n, uint32_t i0,
+                              uint32_t i1, uint32_t b, unsigned long long m) {
+  SelSmem &sm = *cx.sm;
+  const uint32_t len = i1 > i0 ? i1 - i0 : 0;
+  const uint32_t per = (len + kCThreads - 1) / kCThreads;
+  const uint32_t t0 = i0 + threadIdx.x * per;
+  const uint32_t t1 = min(i1, t0 + per);
   unsigned long long c = 0;
-  for (uint32_t i = i0; i < i1; ++i) c += score_bits(s[i]) == b;
+  for (uint32_t i = t0; i < t1; ++i) c += score_bits(s[i]) == b;
   unsigned long long tot;
   const unsigned long long e = block_excl_scan(c, sm, &tot);
-  if (threadIdx.x == 0) sm.res[0] = n - 1;
-  __syncthreads();
-  if (e < m && m <= e + c) {
-    unsigned long long r = e;
-    for (uint32_t i = i0; i < i1; ++i)
+  if (threadIdx.x == 0) {
+    sm.res[4] = tot;
+    if (cx.rank == 0) sm.res[5] = n - 1;
+  }
+  cx.cl.sync();
+  unsigned long long off = 0;  // matches in the slices of lower ranks
+  for (unsigned q = 0; q < cx.rank; ++q) off += cx.peer(q)->res[4];
+  if (off + e < m && m <= off + e + c) {
+    unsigned long long r = off + e;
+    for (uint32_t i = t0; i < t1; ++i)
       if (score_bits(s[i]) == b && ++r == m) {
-        sm.res[0] = i;
+        cx.peer(0)->res[5] = i;
         break;
       }
   }
-  __syncthreads();
-  const uint32_t idx = uint32_t(sm.res[0]);
-  __syncthreads();
+  cx.cl.sync();
+  const uint32_t idx = uint32_t(cx.peer(0)->res[5]);
+  cx.cl.sync();
   return idx;
 }
 
-__device__ HeadSel select_list(const float *s, uint32_t n, float gamma, unsigned long long lo,
-                               unsigned long long hi, SelSmem &sm) {
+__device__ HeadSel select_list(const Ctx &cx, const float *s, uint32_t n, float gamma,
+                               unsigned long long lo, unsigned long long hi) {
   HeadSel r{SEL_NONE, 0u, 0u, 0};
   if (n == 0) return r;
-  unsigned long long am = 0, ac = 0, wtot = 0, k;
+  const uint32_t chunk = (n + kCluster - 1) / kCluster;
+  const uint32_t i0 = min(n, cx.rank * chunk), i1 = min(n, i0 + chunk);
+  unsigned long long am = 0, ac = 0, k;
   double target = 0.0;
   uint32_t b = 0;
   unsigned long long m = 0;
@@ -241,7 +307,7 @@ __device__ HeadSel select_list(const float *s, uint32_t n, float gamma, unsigned
   if (gamma >= 1.f) {
     k = n;
   } else {
-    b = descend(s, n, true, gamma, 0, &am, &ac, &wtot, &target, sm);
+    b = descend(cx, s, i0, i1, true, gamma, 0, &am, &ac, &target);
     if (target <= 0.0) {
       k = 0;
     } else {
@@ -267,56 +333,73 @@ __device__ HeadSel select_list(const float *s, uint32_t n, float gamma, unsigned
     return r;
   }
   if (!(have_threshold && kc == k)) {
-    b = descend(s, n, false, gamma, kc, &am, &ac, &wtot, &target, sm);
+    b = descend(cx, s, i0, i1, false, gamma, kc, &am, &ac, &target);
     m = kc - ac;
   }
   r.mode = SEL_THRESHOLD;
   r.bits = b;
-  r.idx = tie_index(s, n, b, m, sm);
+  r.idx = tie_index(cx, s, n, i0, i1, b, m);
   return r;
 }
 
-// grid (Hq, Bt), 1024 threads, dynamic shared memory SelSmem.
-__global__ void __launch_bounds__(kThreads) select_head_kernel(
-    const int32_t *__restrict__ pattern, const float *__restrict__ map,
-    const float *__restrict__ vert, const float *__restrict__ slash, int n, int nb, int bs,
-    float gamma, long long qa_lo, long long qa_hi, int vs_lo, int vs_hi,
-    HeadSel *__restrict__ sel, uint8_t *__restrict__ colflag, uint8_t *__restrict__ distflag) {
+// grid (kCluster * Hq, Bt), clusters of kCluster CTAs along x, kCThreads
+// threads, dynamic shared memory SelSmem.  Cluster h selects head h.
+__global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kCThreads)
+    select_head_kernel(const int32_t *__restrict__ pattern, const float *__restrict__ map,
+                       const float *__restrict__ vert, const float *__restrict__ slash, int n,
+                       int nb, int bs, float gamma, long long qa_lo, long long qa_hi, int vs_lo,
+                       int vs_hi, HeadSel *__restrict__ sel, uint8_t *__restrict__ colflag,
+                       uint8_t *__restrict__ distflag) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
-  SelSmem &sm = *reinterpret_cast<SelSmem *>(smem_raw);
-  const size_t bh = size_t(blockIdx.y) * gridDim.x + blockIdx.x;
+  Ctx cx{cg::this_cluster(), 0u, reinterpret_cast<SelSmem *>(smem_raw)};
+  cx.rank = cx.cl.block_rank();
+  SelSmem &sm = *cx.sm;
+  const size_t heads_x = gridDim.x / kCluster;
+  const size_t bh = size_t(blockIdx.y) * heads_x + blockIdx.x / kCluster;
   const size_t t_pairs = size_t(nb) * (nb + 1) / 2;
-  if (pattern[bh] == FP_PATTERN_QA) {
-    HeadSel r = select_list(map + bh * t_pairs, uint32_t(t_pairs), gamma, qa_lo, qa_hi, sm);
-    if (threadIdx.x == 0) sel[2 * bh] = r;
+  if (pattern[bh] == FP_PATTERN_QA) {  // uniform over the cluster
+    HeadSel r = select_list(cx, map + bh * t_pairs, uint32_t(t_pairs), gamma, qa_lo, qa_hi);
+    if (cx.rank == 0 && threadIdx.x == 0) sel[2 * bh] = r;
     return;
   }
-  for (int i = threadIdx.x; i < nb; i += kThreads) {
+  for (int i = threadIdx.x; i < nb; i += kCThreads) {
     sm.colflag[i] = 0;
     sm.distflag[i] = 0;
   }
   __syncthreads();
   const float *vv = vert + bh * n;
   const float *ss = slash + bh * n;
-  HeadSel rv = select_list(vv, uint32_t(n), gamma, vs_lo, vs_hi, sm);
-  for (int t = threadIdx.x; t < n; t += kThreads)
+  const uint32_t chunk = (uint32_t(n) + kCluster - 1) / kCluster;
+  const int s0 = int(min(uint32_t(n), cx.rank * chunk)), s1 = int(min(uint32_t(n), s0 + chunk));
+  HeadSel rv = select_list(cx, vv, uint32_t(n), gamma, vs_lo, vs_hi);
+  for (int t = s0 + threadIdx.x; t < s1; t += kCThreads)
     if (kept(score_bits(vv[t]), uint32_t(t), rv)) sm.colflag[t / bs] = 1;
-  HeadSel rs = select_list(ss, uint32_t(n), gamma, vs_lo, vs_hi, sm);
-  for (int o = threadIdx.x; o < n; o += kThreads)
+  HeadSel rs = select_list(cx, ss, uint32_t(n), gamma, vs_lo, vs_hi);
+  for (int o = s0 + threadIdx.x; o < s1; o += kCThreads)
     if (kept(score_bits(ss[o]), uint32_t(o), rs)) {
       const int d0 = o / bs;
       sm.distflag[d0] = 1;
       if (o % bs != 0 && d0 + 1 < nb) sm.distflag[d0 + 1] = 1;
     }
-  __syncthreads();
-  for (int i = threadIdx.x; i < nb; i += kThreads) {
-    colflag[bh * nb + i] = sm.colflag[i];
-    distflag[bh * nb + i] = sm.distflag[i];
+  // OR the slices' flags: rank r writes blocks [r*per, (r+1)*per)
+  cx.cl.sync();
+  const int per = (nb + kCluster - 1) / kCluster;
+  for (int i = int(cx.rank) * per + threadIdx.x; i < min(nb, int(cx.rank + 1) * per);
+       i += kCThreads) {
+    uint8_t c = 0, d = 0;
+#pragma unroll
+    for (unsigned q = 0; q < kCluster; ++q) {
+      c |= cx.peer(q)->colflag[i];
+      d |= cx.peer(q)->distflag[i];
+    }
+    colflag[bh * nb + i] = c;
+    distflag[bh * nb + i] = d;
   }
-  if (threadIdx.x == 0) {
+  if (cx.rank == 0 && threadIdx.x == 0) {
     sel[2 * bh] = rv;
     sel[2 * bh + 1] = rs;
   }
+  cx.cl.sync();  // peers' flags stay readable until every rank is done
 }
 
 // grid (ceil(nb/8), Hq, Bt), 256 threads: one warp per row.
@@ -403,7 +486,7 @@ cudaError_t launch_select(const Dims &D, float gamma, const SelectBudgets &bud,
   uint8_t *df = c.take<uint8_t>(heads * D.nb);
   const int smem = int(sizeof(SelSmem));
   cudaFuncSetAttribute(select_head_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  select_head_kernel<<<dim3(D.hq, D.bt), kThreads, smem, st>>>(
+  select_head_kernel<<<dim3(kCluster * D.hq, D.bt), kCThreads, smem, st>>>(
       pattern, map, vert, slash, D.n, D.nb, D.bs, gamma, bud.qa_lo, bud.qa_hi, bud.vs_lo,
       bud.vs_hi, sel, cf, df);
   emit_rows_kernel<<<dim3((D.nb + 7) / 8, D.hq, D.bt), 256, 0, st>>>(pattern, map, D.nb, sel, cf,
@@ -468,7 +551,7 @@ cudaError_t launch_select_noalloc(const Dims &D, float gamma, const SelectBudget
   uint8_t *df = c.take<uint8_t>(heads * D.nb);
   const int smem = int(sizeof(SelSmem));
   cudaFuncSetAttribute(select_head_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  select_head_kernel<<<dim3(D.hq, D.bt), kThreads, smem, st>>>(
+  select_head_kernel<<<dim3(kCluster * D.hq, D.bt), kCThreads, smem, st>>>(
       pattern, map, vert, slash, D.n, D.nb, D.bs, gamma, bud.qa_lo, bud.qa_hi, bud.vs_lo,
       bud.vs_hi, sel, cf, df);
   emit_rows_kernel<<<dim3((D.nb + 7) / 8, D.hq, D.bt), 256, 0, st>>>(pattern, map, D.nb, sel, cf,

@@ -66,6 +66,7 @@ _SIG = {
                                        _P]),
     "fp_prefill_attn_host": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "fp_last_device_status": (ctypes.c_int, [_P]),
+    "fp_selftest_watchdog": (ctypes.c_int, [ctypes.c_uint, _P]),
     "fp_status_string": (ctypes.c_char_p, [ctypes.c_int]),
 }
 
@@ -194,6 +195,10 @@ def fp_prefill_attn_host(shape, params, q_host, k_host, v_host, out_host, ws,
     return lib().fp_prefill_attn_host(ctypes.byref(shape), ctypes.byref(params), _addr(q_host),
                                       _addr(k_host), _addr(v_host), _addr(out_host), _addr(ws),
                                       _nbytes(ws), _stream(stream))
+
+
+def fp_selftest_watchdog(limit_us: int, stream=None) -> int:
+    return lib().fp_selftest_watchdog(limit_us, _stream(stream))
 
 
 def fp_last_device_status(stream=None) -> int:

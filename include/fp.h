@@ -252,6 +252,16 @@ fp_status fp_prefill_attn_host(const fp_shape *shape, const fp_params *params,
  */
 fp_status fp_last_device_status(fp_stream_t stream);
 
+/*
+ * fp_selftest_watchdog -- exercises the failure detection every pipelined
+ * kernel here relies on: one thread waits, with the same bounded wait the
+ * kernels use, on an mbarrier that nothing ever arrives at, gives up after
+ * limit_us microseconds (1 .. 1000000) and records FP_ERR_TIMEOUT in the
+ * device status word, which fp_last_device_status() then returns.  The
+ * device stays usable.  No counterpart in the pages (an engineering check).
+ */
+fp_status fp_selftest_watchdog(unsigned int limit_us, fp_stream_t stream);
+
 /* Static, human-readable name of a status code. */
 const char *fp_status_string(fp_status status);
 

@@ -26,7 +26,7 @@ def shape(**kw):
 
 def test_exports_every_declared_function(L):
     names = ops.header_functions()
-    assert len(names) == 11, names
+    assert len(names) == 12, names
     for n in names:
         assert hasattr(L, n), n
     # nothing but the fp_* API is exported (static CUDA runtime stays hidden)
@@ -118,6 +118,11 @@ def test_bf16_attention_shape_limits(L):
     for bs, d in [(64, 128), (128, 64), (64, 64)]:
         s = shape(block_size=bs, head_dim=d)
         assert L.fp_dense_attn(ctypes.byref(s), FAKE, FAKE, FAKE, FAKE, None, None) == 2
+
+
+def test_watchdog_selftest_rejects_bad_limits(L):
+    assert L.fp_selftest_watchdog(0, None) == 4
+    assert L.fp_selftest_watchdog(2000000, None) == 4
 
 
 def test_missing_library_fails_loudly(monkeypatch):
