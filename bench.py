@@ -36,6 +36,26 @@ METRIC = "prefill-attn tokens/s and effective TFLOPS (% bf16 peak) at 128k; spee
 LAUNCHES_PER_STEP = 12  # estimate 8, pattern 1, select 2, attention 1
 
 
+def kernel_traffic(source: str, workload: str):
+    """DRAM bytes per launch of a kernel from a committed ncu capture.
+
+    profiles/<name>_traffic.json holds {"source_sha256", "workload",
+    "bytes_per_launch", ...}; the figure is used only while the kernel source
+    still hashes to the captured one (else None: the counters are stale).
+    """
+    import hashlib
+    name = os.path.splitext(os.path.basename(source))[0]
+    rec_path = os.path.join(ROOT, "profiles", f"{name}_traffic.json")
+    src_path = os.path.join(ROOT, "dynamic_block_sparse_fp_b200", "csrc", source)
+    if not (os.path.exists(rec_path) and os.path.exists(src_path)):
+        return None
+    rec = json.load(open(rec_path))
+    sha = hashlib.sha256(open(src_path, "rb").read()).hexdigest()
+    if rec.get("source_sha256") != sha or rec.get("workload") != workload:
+        return None
+    return rec.get("bytes_per_launch")
+
+
 def load_peaks() -> dict:
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -333,7 +353,7 @@ def run_ours(args, w, ws, rank, local):
         "config": workload_config(w, ws),
         "roofline": {"bound": "tensor", "kernel": "fp_sparse_attn", "achieved": attn_tflops,
                      "peak": peak_t, "unit": "TFLOP/s", "frac": attn_tflops / peak_t,
-                     "traffic": None,
+                     "traffic": kernel_traffic("attn_tc.cu", w.name),
                      "peak_kind": f"bf16 dense, sustained ({peaks['source']})",
                      "algorithmic_flops_per_launch": attn_flops},
         "gpu_launches": LAUNCHES_PER_STEP * args.steps,

@@ -41,7 +41,6 @@ namespace fpi {
 namespace {
 
 constexpr int BM = 128;   // query rows per tile (= block size)
-constexpr int BLK = 128;  // keys per listed block
 constexpr int BN = 64;    // keys per tile (half a block)
 constexpr int HD = 128;   // head dim
 constexpr int NS = 2;     // K/V pipeline stages
@@ -60,6 +59,7 @@ struct TcSmem {
   uint64_t s_full[2], s_free[2];
   uint64_t p_full, p_empty, o_full;
   uint32_t tmem_base;
+  int ntile;  // key tiles of this CTA
   int abort_flag;
 };
 constexpr size_t kSmemBytes = sizeof(TcSmem) + 1024;  // + alignment slack
@@ -77,15 +77,48 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   return *reinterpret_cast<uint32_t *>(&h);
 }
 
-struct Item {
-  int qi, h, b, kv, n;  // n = listed blocks; 2n tiles
-  size_t bh;
-  const int32_t *list;
+// The key tiles of one CTA, in order.
+//  Block size 128 (PAIR = false): the CTA's 128 query rows are one block qa;
+//    tile t is half (t & 1) of listed block list_a[t / 2]: 2 n tiles.
+//  Block size 64 (PAIR = true): the 128 rows are blocks qa = 2p and qb = 2p+1
+//    (qb may be past the end); the tiles are the blocks of the ascending union
+//    of both lists, one 64-key block each; in_a / in_b say whose list holds it.
+struct Tile {
+  int j;     // key block
+  int sub;   // 64-key half of a 128-key block (PAIR = false), else 0
+  bool in_a, in_b;
 };
 
-__device__ __forceinline__ int list_block(const Item &it, int t, bool dense) {
-  return dense ? t : __ldg(it.list + t);
-}
+template <bool PAIR>
+struct Walker {
+  const int32_t *la, *lb;
+  int na, nb2, ia, ib;
+  bool dense;
+  int t;
+  __device__ Walker(const int32_t *la_, int na_, const int32_t *lb_, int nb_, bool dense_)
+      : la(la_), lb(lb_), na(na_), nb2(nb_), ia(0), ib(0), dense(dense_), t(0) {}
+  __device__ int entry(const int32_t *l, int i) const { return dense ? i : __ldg(l + i); }
+  __device__ Tile next() {
+    Tile x;
+    if (!PAIR) {
+      x.j = entry(la, t / 2);
+      x.sub = t & 1;
+      x.in_a = true;
+      x.in_b = false;
+    } else {
+      const int ja = ia < na ? entry(la, ia) : 0x7fffffff;
+      const int jb = ib < nb2 ? entry(lb, ib) : 0x7fffffff;
+      x.j = ja < jb ? ja : jb;
+      x.sub = 0;
+      x.in_a = ja == x.j;
+      x.in_b = jb == x.j;
+      ia += x.in_a;
+      ib += x.in_b;
+    }
+    ++t;
+    return x;
+  }
+};
 
 // One S tile (64 keys) of one row (TMEM lane): the row max over the tile,
 // the lazy-rescale decision, then the exponentials packed to bf16 pairs,
@@ -129,31 +162,37 @@ __device__ __forceinline__ void softmax_tile(uint32_t s_addr, int lim, float sl2
   }
 }
 
+template <bool PAIR>
 __global__ void __launch_bounds__(192, 2) attn_tc_kernel(
     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
     const __grid_constant__ CUtensorMap tm_v, const int32_t *__restrict__ counts,
     const int32_t *__restrict__ indices, __nv_bfloat16 *__restrict__ out,
-    float *__restrict__ lse, int hq, int g, int n_tok, bool dense, int *status) {
+    float *__restrict__ lse, int hq, int g, int n_tok, int nb, bool dense, int *status) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   TcSmem &sm = *reinterpret_cast<TcSmem *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int nb = gridDim.x;
+  constexpr int KB = PAIR ? 64 : 128;  // tokens per block
 
-  Item it;
-  it.qi = nb - 1 - blockIdx.x;  // longest rows first
-  it.h = blockIdx.y;
-  it.b = blockIdx.z;
-  it.kv = it.h / g;
-  it.bh = size_t(it.b) * hq + it.h;
-  it.n = dense ? it.qi + 1 : counts[it.bh * nb + it.qi];
-  if (it.n < 0 || it.n > it.qi + 1) {  // a row holds at most qi + 1 causal blocks
-    if (threadIdx.x == 0) report(status, FP_ERR_DEVICE_CHECK);
-    it.n = it.n < 0 ? 0 : it.qi + 1;
-  }
-  it.list = indices + (it.bh * nb + it.qi) * size_t(nb);
-  const int hkv = hq / g;
-  const int ntile = 2 * it.n;  // tile t: half (t & 1) of listed block t / 2
+  // the CTA's query blocks (longest rows first)
+  const int h = blockIdx.y, b = blockIdx.z, kv = h / g, hkv = hq / g;
+  const size_t bh = size_t(b) * hq + h;
+  const int qa = PAIR ? 2 * (int(gridDim.x) - 1 - int(blockIdx.x)) : nb - 1 - int(blockIdx.x);
+  const int qb = qa + 1;
+  const bool has_b = PAIR && qb < nb;
+  auto row_count = [&](int qblk) {
+    int n = dense ? qblk + 1 : counts[bh * nb + qblk];
+    if (n < 0 || n > qblk + 1) {  // a row holds at most qblk + 1 causal blocks
+      if (threadIdx.x == 0) report(status, FP_ERR_DEVICE_CHECK);
+      n = n < 0 ? 0 : qblk + 1;
+    }
+    return n;
+  };
+  const int na = row_count(qa);
+  const int nbb = has_b ? row_count(qb) : 0;
+  const int32_t *la = indices + (bh * nb + qa) * size_t(nb);
+  const int32_t *lb = has_b ? indices + (bh * nb + qb) * size_t(nb) : la;
+  const int qlast = has_b ? qb : qa;  // largest valid key block of the CTA
 
   if (threadIdx.x == 0) {
     mbar_init(&sm.bar_q, 1);
@@ -170,6 +209,16 @@ __global__ void __launch_bounds__(192, 2) attn_tc_kernel(
     mbar_init(&sm.p_empty, 1);
     mbar_init(&sm.o_full, 1);
     sm.abort_flag = 0;
+    int nt = 2 * na;
+    if (PAIR) {  // size of the union of the two lists
+      Walker<true> w(la, na, lb, nbb, dense);
+      nt = 0;
+      while (w.ia < w.na || w.ib < w.nb2) {
+        w.next();
+        ++nt;
+      }
+    }
+    sm.ntile = nt;
     mbar_fence_init();
   }
   if (warp == 5) {
@@ -180,6 +229,7 @@ __global__ void __launch_bounds__(192, 2) attn_tc_kernel(
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
+  const int ntile = sm.ntile;
   volatile int *abort_flag = &sm.abort_flag;
 
   auto fail = [&](int code) {
@@ -193,21 +243,23 @@ __global__ void __launch_bounds__(192, 2) attn_tc_kernel(
       prefetch_tmap(&tm_q);
       prefetch_tmap(&tm_k);
       prefetch_tmap(&tm_v);
-      const int qrow = int((it.bh * n_tok) + size_t(it.qi) * BM);
+      const int qrow = int((bh * n_tok) + size_t(qa) * KB);
       mbar_arrive_expect_tx(&sm.bar_q, Q_BYTES);
       tma_load_2d(sm.q, &tm_q, &sm.bar_q, 0, qrow);
       tma_load_2d(sm.q + Q_HALF, &tm_q, &sm.bar_q, 64, qrow);
-      const size_t kvrow0 = (size_t(it.b) * hkv + it.kv) * n_tok;
+      const size_t kvrow0 = (size_t(b) * hkv + kv) * n_tok;
+      Walker<PAIR> walk(la, na, lb, nbb, dense);
       int issued = 0;
       for (int t = 0; t < ntile; ++t) {
         const int s = t % NS;
+        const Tile x = walk.next();
         if (!mbar_wait(&sm.kv_empty[s], ((t / NS) & 1) ^ 1, abort_flag)) {
           fail(FP_ERR_TIMEOUT);
           break;
         }
-        int j = list_block(it, t / 2, dense);
-        j = j < 0 ? 0 : (j > it.qi ? it.qi : j);  // invalid entries are masked by softmax
-        const int krow = int(kvrow0 + size_t(j) * BLK + size_t(t & 1) * BN);
+        // invalid entries load any in-range block; the softmax masks them
+        const int j = x.j < 0 ? 0 : (x.j > qlast ? qlast : x.j);
+        const int krow = int(kvrow0 + size_t(j) * KB + size_t(x.sub) * BN);
         mbar_arrive_expect_tx(&sm.k_full[s], KV_BYTES);
         tma_load_2d(sm.k[s], &tm_k, &sm.k_full[s], 0, krow);
         tma_load_2d(sm.k[s] + KV_HALF, &tm_k, &sm.k_full[s], 64, krow);
@@ -289,22 +341,31 @@ __global__ void __launch_bounds__(192, 2) attn_tc_kernel(
     const float sl2 = 1.4426950408889634f / sqrtf(float(HD));  // scale * log2(e)
     float m = -INFINITY, l = 0.f;
     bool ok = true;
+    // rows of this warp: block qa (PAIR: rows 0-63) or qb (PAIR: rows 64-127)
+    const int half = PAIR ? r / 64 : 0;
+    const int qh = PAIR ? qa + half : qa;
+    const int rl = r - 64 * half;  // row inside its block
+    Walker<PAIR> walk(la, na, lb, nbb, dense);
+    Tile x = walk.next();  // prefetched one tile ahead
     for (int t = 0; t < ntile; ++t) {
       const int sb = t & 1, s = t % NS;
+      const Tile cur = x;
+      if (t + 1 < ntile) x = walk.next();
       // waits are made warp-uniform: tcgen05.ld/st below are .sync.aligned
       if (!__all_sync(0xffffffffu, mbar_wait(&sm.s_full[sb], (t >> 1) & 1, abort_flag))) {
         ok = false;
         break;
       }
       tc_fence_after();
-      const int j = list_block(it, t / 2, dense);
-      const bool valid = j >= 0 && j <= it.qi;
-      if (!valid && r == 0 && (t & 1) == 0) report(status, FP_ERR_DEVICE_CHECK);
-      // keys c > lim of this tile are masked: in the diagonal block the tile
-      // holds keys 64 (t & 1) + c, hidden after the query row; an invalid
-      // entry hides all; other tiles take the unmasked path
-      const bool masked = !valid || j == it.qi;
-      const int lim = valid ? r - BN * (t & 1) : -1;
+      const bool mine = PAIR ? (half ? cur.in_b : cur.in_a) : true;
+      const bool inrange = cur.j >= 0 && cur.j <= qh;
+      if (mine && !inrange && rl == 0 && cur.sub == 0) report(status, FP_ERR_DEVICE_CHECK);
+      const bool valid = mine && inrange;
+      // keys c > lim of this 64-key tile are masked: the diagonal block hides
+      // keys after the query row (tile keys start at 64 sub); a tile off this
+      // row's list, or an invalid entry, hides all; other tiles are unmasked
+      const bool masked = !valid || cur.j == qh;
+      const int lim = valid ? rl - BN * cur.sub : -1;
       float muse, alpha;
       float sm8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
       uint32_t pk[BN / 2];
@@ -318,16 +379,18 @@ __global__ void __launch_bounds__(192, 2) attn_tc_kernel(
       const float ps = ((sm8[0] + sm8[1]) + (sm8[2] + sm8[3])) +
                        ((sm8[4] + sm8[5]) + (sm8[6] + sm8[7]));
       l = l * alpha + ps;
-      // wait until P(t-1) V(t-1) finished: O is up to date.  The slot P(t)
-      // goes to held K(t), which S(t) (waited for above) has read.
-      if (!__all_sync(0xffffffffu, mbar_wait(&sm.p_empty, (t & 1) ^ 1, abort_flag))) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      // the whole warp rescales if any of its rows' max grew (alpha == 1 for
-      // the others)
+      // O is rescaled (rarely: lazy) by the whole warp if any of its rows'
+      // max grew; that needs P(t-1) V(t-1) finished.  p_empty completes once
+      // per P V; S(t), waited for above, was issued after P(t-2) V(t-2), so
+      // the barrier is at most one phase behind and the parity wait for
+      // phase t-1 is exact.  Without a rescale nothing waits here: P(t) goes
+      // to the K(t) slot, which P(t-1) V(t-1) does not read.
       if (__any_sync(0xffffffffu, t > 0 && alpha != 1.f)) {
+        if (!__all_sync(0xffffffffu, mbar_wait(&sm.p_empty, (t & 1) ^ 1, abort_flag))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
 #pragma unroll
         for (int c0 = 0; c0 < HD; c0 += 32) {
           uint32_t u[32];
@@ -352,7 +415,8 @@ __global__ void __launch_bounds__(192, 2) attn_tc_kernel(
       m = muse;
     }
     // ------------------------------------------------------------ epilogue --
-    const size_t orow = it.bh * n_tok + size_t(it.qi) * BM + r;
+    const size_t orow = bh * n_tok + size_t(qa) * KB + r;
+    const bool row_exists = !PAIR || half == 0 || has_b;
     if (ok && ntile > 0 && !__all_sync(0xffffffffu, mbar_wait(&sm.o_full, 0, abort_flag)))
       ok = false;
     if (!ok) fail(FP_ERR_TIMEOUT);
@@ -377,10 +441,10 @@ __global__ void __launch_bounds__(192, 2) attn_tc_kernel(
         w.y = pack_bf16(__uint_as_float(u[i + 2]) * inv, __uint_as_float(u[i + 3]) * inv);
         w.z = pack_bf16(__uint_as_float(u[i + 4]) * inv, __uint_as_float(u[i + 5]) * inv);
         w.w = pack_bf16(__uint_as_float(u[i + 6]) * inv, __uint_as_float(u[i + 7]) * inv);
-        dst[(c0 + i) / 8] = w;
+        if (row_exists) dst[(c0 + i) / 8] = w;
       }
     }
-    if (lse) lse[orow] = good ? (m + log2f(l)) * 0.6931471805599453f : -INFINITY;
+    if (lse && row_exists) lse[orow] = good ? (m + log2f(l)) * 0.6931471805599453f : -INFINITY;
   }
   tc_fence_before();
   __syncthreads();
@@ -419,17 +483,25 @@ size_t attn_ws_bytes(const Dims &) { return 0; }
 cudaError_t launch_attn_bf16(const Dims &D, const void *q, const void *k, const void *v,
                              const int32_t *counts, const int32_t *indices, void *out,
                              float *lse, bool dense, void *, cudaStream_t st) {
-  if (D.bs != BLK || D.d != HD) return cudaErrorInvalidValue;
+  if ((D.bs != 128 && D.bs != 64) || D.d != HD) return cudaErrorInvalidValue;
   CUtensorMap mq, mk, mv;
   if (!encode_map(&mq, q, uint64_t(D.bt) * D.hq * D.n, BM) ||
       !encode_map(&mk, k, uint64_t(D.bt) * D.hkv * D.n, BN) ||
       !encode_map(&mv, v, uint64_t(D.bt) * D.hkv * D.n, BN))
     return cudaErrorInvalidValue;
-  cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                       int(kSmemBytes));
-  attn_tc_kernel<<<dim3(D.nb, D.hq, D.bt), 192, kSmemBytes, st>>>(
-      mq, mk, mv, counts, indices, static_cast<__nv_bfloat16 *>(out), lse, D.hq, D.g, D.n,
-      dense, device_status_ptr());
+  int *status = device_status_ptr();
+  __nv_bfloat16 *o = static_cast<__nv_bfloat16 *>(out);
+  if (D.bs == 128) {
+    cudaFuncSetAttribute(attn_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         int(kSmemBytes));
+    attn_tc_kernel<false><<<dim3(D.nb, D.hq, D.bt), 192, kSmemBytes, st>>>(
+        mq, mk, mv, counts, indices, o, lse, D.hq, D.g, D.n, D.nb, dense, status);
+  } else {
+    cudaFuncSetAttribute(attn_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         int(kSmemBytes));
+    attn_tc_kernel<true><<<dim3((D.nb + 1) / 2, D.hq, D.bt), 192, kSmemBytes, st>>>(
+        mq, mk, mv, counts, indices, o, lse, D.hq, D.g, D.n, D.nb, dense, status);
+  }
   return cudaGetLastError();
 }
 

@@ -53,7 +53,7 @@ fp_status check_shape(const fp_shape *s, Dims *D) {
 }
 
 fp_status check_attn_shape(const Dims &D) {
-  if (D.dtype == FP_BF16 && (D.d != 128 || D.bs != 128)) return FP_ERR_SHAPE;
+  if (D.dtype == FP_BF16 && D.d != 128) return FP_ERR_SHAPE;
   return FP_OK;
 }
 

@@ -36,8 +36,8 @@
  *  * No C++ exception crosses this ABI.  Calls on distinct streams with
  *    distinct workspaces may run from several host threads.
  *  * Supported shapes: N % B == 0, Hq % Hkv == 0, B in {64, 128},
- *    d in {64, 128}.  The bf16 path (tensor cores) needs d == 128 and
- *    B == 128; fp32 (the debug path, CUDA cores) takes every listed shape.
+ *    d in {64, 128}.  The bf16 attention (tensor cores) needs d == 128;
+ *    fp32 (the debug path, CUDA cores) takes every listed shape.
  */
 #ifndef FP_H_
 #define FP_H_

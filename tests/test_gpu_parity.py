@@ -187,6 +187,27 @@ def test_pipeline_llama8k_bf16_parity(tau, lo, hi):
     assert ops.fp_last_device_status() == 0
 
 
+@pytest.mark.parametrize("n,tau,hi", [(4096, 0.1, 0), (4096, 0.0, 1024), (4032, 0.1, 0)])
+def test_pipeline_glm_block64_bf16_parity(n, tau, hi):
+    """Block size 64 on the tensor cores (GLM-4-9B heads: 32 q / 2 kv), N with
+    an even and an odd number of blocks."""
+    w, inp, d = _inputs("glm9b_n65536_b64", seq_len=n, n_q_heads=8, n_kv_heads=2)
+    res = _pipeline(w, d, tau=tau, hi=hi)
+    nb = w.n_blocks
+    _attn_check(inp, res, w, 2e-2, 2e-3, heads=list(range(w.n_q_heads)),
+                q_blocks=[0, 1, 2, nb // 2, nb - 2, nb - 1])
+    # dense at block 64 against the oracle
+    out, lse = ops.dense_attn(d["q"], d["k"], d["v"], 64)
+    torch.cuda.synchronize()
+    o, l = oracle.dense_attention(inp["q"], inp["k"], inp["v"], 64, heads=[0, 5],
+                                  q_blocks=[0, 3, nb - 1])
+    m = ~np.isnan(o)
+    assert np.abs(_np(out)[m] - o[m]).max() <= 2e-2
+    ml = ~np.isnan(l)
+    assert np.abs(_np(lse)[ml] - l[ml]).max() <= 2e-3
+    assert ops.fp_last_device_status() == 0
+
+
 def test_dense_parity():
     w, inp, d = _inputs("tiny_n1024")
     out, lse = ops.dense_attn(d["q"], d["k"], d["v"], w.block_size)
