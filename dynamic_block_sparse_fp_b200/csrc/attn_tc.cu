@@ -7,23 +7,29 @@
 // FlashAttention's online softmax.  Block size 128, head dim 128.
 //
 // One CTA handles one (query block, head, batch) item and is small enough
-// (96 KB of shared memory, 256 TMEM columns, <= 168 registers per thread)
+// (112 KB of shared memory, 256 TMEM columns, <= 168 registers per thread)
 // that two CTAs share an SM, so one CTA's softmax overlaps the other's MMAs.
 // Every listed key block (128 keys) is processed as two 64-key tiles.
 // 6 warps, specialised:
 //   warps 0-3  softmax + epilogue: thread r owns query row r, which is TMEM
 //              lane r (warp w may only touch lanes 32w..32w+31);
-//   warp 4     TMA producer: Q once, then K and V tiles through a 2-stage ring;
+//   warp 4     TMA producer: Q once, then K tiles through a 3-slot ring and
+//              V tiles through a 2-slot ring;
 //   warp 5     MMA issuer (one thread): S = Q K^T (N = 64) into one of two
 //              TMEM buffers, O += P V (K = 64) into a TMEM accumulator.
 // TMEM (256 columns): S0 [0,64), S1 [64,128), O [128,256).
 // Shared memory (1024-B aligned, 128-B swizzle everywhere):
-//   Q 32 KB (two halves [128 rows x 64 d]) | K x2 16 KB | V x2 16 KB
+//   Q 32 KB (two halves [128 rows x 64 d]) | K x3 16 KB | V x2 16 KB
+// (112 KB in all, with no room for alignment slack: the kernel requires the
+// dynamic shared-memory window to start 1024-B aligned, which it is when the
+// kernel declares no static shared memory, and checks it).
 // K and V tiles are two 8-KB halves [64 keys x 64 d]; Q and K are K-major
 // operands of S, V is the MN-major B operand of P V.  P(t) ([128 rows x 64
 // keys], 16 KB, K-major) is written into the shared-memory slot of K(t),
 // which S(t) no longer needs: the producer refills that slot only after
-// P(t) V(t) has completed.
+// P(t) V(t) has completed.  With three K slots the load of K(t+2) waits only
+// for P(t-1) V(t-1), so it is in flight while the softmax works on S(t) and
+// S(t+1) instead of sitting on the path between P(t) V(t) and S(t+2).
 //
 // Per key tile t the softmax warps read S(t) from TMEM, release the buffer,
 // compute p = 2^(s*scale*log2e - m) with a running row max m, rescale O in
@@ -43,7 +49,8 @@ namespace {
 constexpr int BM = 128;   // query rows per tile (= block size)
 constexpr int BN = 64;    // keys per tile (half a block)
 constexpr int HD = 128;   // head dim
-constexpr int NS = 2;     // K/V pipeline stages
+constexpr int NK = 3;     // K slots (K(t), then P(t))
+constexpr int NV = 2;     // V slots
 constexpr uint32_t Q_BYTES = BM * HD * 2;   // 32 KB
 constexpr uint32_t Q_HALF = Q_BYTES / 2;    // [128 rows x 64 d]
 constexpr uint32_t KV_BYTES = BN * HD * 2;  // 16 KB
@@ -52,17 +59,18 @@ constexpr uint32_t TMEM_COLS = 256;
 
 struct TcSmem {
   uint8_t q[Q_BYTES];
-  uint8_t k[NS][KV_BYTES];  // K(t), then P(t)
-  uint8_t v[NS][KV_BYTES];
+  uint8_t k[NK][KV_BYTES];  // K(t), then P(t)
+  uint8_t v[NV][KV_BYTES];
   uint64_t bar_q;
-  uint64_t k_full[NS], v_full[NS], kv_empty[NS];
+  uint64_t k_full[NK], k_empty[NK], v_full[NV], v_empty[NV];
   uint64_t s_full[2], s_free[2];
   uint64_t p_full, p_empty, o_full;
   uint32_t tmem_base;
   int ntile;  // key tiles of this CTA
   int abort_flag;
 };
-constexpr size_t kSmemBytes = sizeof(TcSmem) + 1024;  // + alignment slack
+constexpr size_t kSmemBytes = sizeof(TcSmem);  // no slack: the base is 1024-B aligned
+// two CTAs per SM: 228 KB of shared memory, 1 KB of it reserved per CTA
 static_assert(2 * (kSmemBytes + 1024) <= 233472, "two CTAs must fit in one SM");
 static_assert(BM * BN * 2 == KV_BYTES, "P(t) must fit the K(t) slot");
 
@@ -169,8 +177,13 @@ __global__ void __launch_bounds__(192, 2) attn_tc_kernel(
     const int32_t *__restrict__ indices, __nv_bfloat16 *__restrict__ out,
     float *__restrict__ lse, int hq, int g, int n_tok, int nb, bool dense, int *status) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
-  TcSmem &sm = *reinterpret_cast<TcSmem *>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // the 128-B swizzled operand tiles need 1024-B alignment and there is no
+  // slack to realign: refuse (before touching shared memory) if it is missing
+  if (smem_u32(smem_raw) & 1023u) {
+    if (threadIdx.x == 0) report(status, FP_ERR_UNSUPPORTED);
+    return;
+  }
+  TcSmem &sm = *reinterpret_cast<TcSmem *>(smem_raw);
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   constexpr int KB = PAIR ? 64 : 128;  // tokens per block
 
@@ -196,10 +209,13 @@ __global__ void __launch_bounds__(192, 2) attn_tc_kernel(
 
   if (threadIdx.x == 0) {
     mbar_init(&sm.bar_q, 1);
-    for (int s = 0; s < NS; ++s) {
+    for (int s = 0; s < NK; ++s) {
       mbar_init(&sm.k_full[s], 1);
+      mbar_init(&sm.k_empty[s], 1);
+    }
+    for (int s = 0; s < NV; ++s) {
       mbar_init(&sm.v_full[s], 1);
-      mbar_init(&sm.kv_empty[s], 1);
+      mbar_init(&sm.v_empty[s], 1);
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&sm.s_full[s], 1);
@@ -250,33 +266,42 @@ __global__ void __launch_bounds__(192, 2) attn_tc_kernel(
       const size_t kvrow0 = (size_t(b) * hkv + kv) * n_tok;
       Walker<PAIR> walk(la, na, lb, nbb, dense);
       int issued = 0;
+      // K(t) waits for P(t-3) V(t-3) (its slot held P(t-3)), V(t) for
+      // P(t-2) V(t-2); in program order K(t+1) follows V(t), which waited
+      // for the same P V, so neither load waits longer than its slot needs
+      int issued_k = 0, issued_v = 0;
       for (int t = 0; t < ntile; ++t) {
-        const int s = t % NS;
+        const int sk = t % NK, sv = t % NV;
         const Tile x = walk.next();
-        if (!mbar_wait(&sm.kv_empty[s], ((t / NS) & 1) ^ 1, abort_flag)) {
-          fail(FP_ERR_TIMEOUT);
-          break;
-        }
         // invalid entries load any in-range block; the softmax masks them
         const int j = x.j < 0 ? 0 : (x.j > qlast ? qlast : x.j);
         const int krow = int(kvrow0 + size_t(j) * KB + size_t(x.sub) * BN);
-        mbar_arrive_expect_tx(&sm.k_full[s], KV_BYTES);
-        tma_load_2d(sm.k[s], &tm_k, &sm.k_full[s], 0, krow);
-        tma_load_2d(sm.k[s] + KV_HALF, &tm_k, &sm.k_full[s], 64, krow);
-        mbar_arrive_expect_tx(&sm.v_full[s], KV_BYTES);
-        tma_load_2d(sm.v[s], &tm_v, &sm.v_full[s], 0, krow);
-        tma_load_2d(sm.v[s] + KV_HALF, &tm_v, &sm.v_full[s], 64, krow);
-        issued = t + 1;
+        if (!mbar_wait(&sm.k_empty[sk], ((t / NK) & 1) ^ 1, abort_flag)) {
+          fail(FP_ERR_TIMEOUT);
+          break;
+        }
+        mbar_arrive_expect_tx(&sm.k_full[sk], KV_BYTES);
+        tma_load_2d(sm.k[sk], &tm_k, &sm.k_full[sk], 0, krow);
+        tma_load_2d(sm.k[sk] + KV_HALF, &tm_k, &sm.k_full[sk], 64, krow);
+        issued_k = t + 1;
+        if (!mbar_wait(&sm.v_empty[sv], ((t / NV) & 1) ^ 1, abort_flag)) {
+          fail(FP_ERR_TIMEOUT);
+          break;
+        }
+        mbar_arrive_expect_tx(&sm.v_full[sv], KV_BYTES);
+        tma_load_2d(sm.v[sv], &tm_v, &sm.v_full[sv], 0, krow);
+        tma_load_2d(sm.v[sv] + KV_HALF, &tm_v, &sm.v_full[sv], 64, krow);
+        issued_v = t + 1;
       }
       if (*abort_flag) {
-        // drain: wait (bounded) for the loads still in flight
+        // drain: wait (bounded) for the loads still in flight, the last load
+        // of each slot
         volatile int never = 0;
         mbar_wait(&sm.bar_q, 0, &never, 100000000ull);
-        for (int t = issued - NS > 0 ? issued - NS : 0; t < issued; ++t) {
-          const int s = t % NS;
-          mbar_wait(&sm.k_full[s], (t / NS) & 1, &never, 100000000ull);
-          mbar_wait(&sm.v_full[s], (t / NS) & 1, &never, 100000000ull);
-        }
+        for (int t = issued_k - NK > 0 ? issued_k - NK : 0; t < issued_k; ++t)
+          mbar_wait(&sm.k_full[t % NK], (t / NK) & 1, &never, 100000000ull);
+        for (int t = issued_v - NV > 0 ? issued_v - NV : 0; t < issued_v; ++t)
+          mbar_wait(&sm.v_full[t % NV], (t / NV) & 1, &never, 100000000ull);
       }
     }
   } else if (warp == 5) {
@@ -287,12 +312,12 @@ __global__ void __launch_bounds__(192, 2) attn_tc_kernel(
       const uint32_t q_addr = smem_u32(sm.q);
       bool ok = mbar_wait(&sm.bar_q, 0, abort_flag);
       auto issue_pv = [&](int u) -> bool {
-        const int s = u % NS;
+        const int sk = u % NK, sv = u % NV;
         if (!mbar_wait(&sm.p_full, u & 1, abort_flag)) return false;
-        if (!mbar_wait(&sm.v_full[s], (u / NS) & 1, abort_flag)) return false;
+        if (!mbar_wait(&sm.v_full[sv], (u / NV) & 1, abort_flag)) return false;
         tc_fence_after();
-        const uint32_t p_addr = smem_u32(sm.k[s]);  // P(u) sits in K(u)'s slot
-        const uint32_t v_addr = smem_u32(sm.v[s]);
+        const uint32_t p_addr = smem_u32(sm.k[sk]);  // P(u) sits in K(u)'s slot
+        const uint32_t v_addr = smem_u32(sm.v[sv]);
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk) {
           // A = P [128 rows x 64 keys]: K-major, 16 keys = 32 B along a row
@@ -302,13 +327,14 @@ __global__ void __launch_bounds__(192, 2) attn_tc_kernel(
           const uint64_t bd = umma_desc_sw128(v_addr + kk * 16 * 128, KV_HALF, 1024);
           tc_mma_ss(tmem + 2 * BN, ad, bd, idesc_o, (u > 0 || kk > 0) ? 1u : 0u);
         }
-        tc_commit(&sm.kv_empty[s]);
+        tc_commit(&sm.k_empty[sk]);
+        tc_commit(&sm.v_empty[sv]);
         tc_commit(&sm.p_empty);
         return true;
       };
       for (int t = 0; ok && t < ntile; ++t) {
-        const int s = t % NS, sb = t & 1;
-        if (!mbar_wait(&sm.k_full[s], (t / NS) & 1, abort_flag) ||
+        const int s = t % NK, sb = t & 1;
+        if (!mbar_wait(&sm.k_full[s], (t / NK) & 1, abort_flag) ||
             !mbar_wait(&sm.s_free[sb], ((t >> 1) & 1) ^ 1, abort_flag)) {
           ok = false;
           break;
@@ -348,7 +374,7 @@ __global__ void __launch_bounds__(192, 2) attn_tc_kernel(
     Walker<PAIR> walk(la, na, lb, nbb, dense);
     Tile x = walk.next();  // prefetched one tile ahead
     for (int t = 0; t < ntile; ++t) {
-      const int sb = t & 1, s = t % NS;
+      const int sb = t & 1, s = t % NK;
       const Tile cur = x;
       if (t + 1 < ntile) x = walk.next();
       // waits are made warp-uniform: tcgen05.ld/st below are .sync.aligned
