@@ -7,34 +7,37 @@
 // FlashAttention's online softmax.  Block size 128, head dim 128.
 //
 // One CTA handles one (query block, head, batch) item and is small enough
-// (112 KB of shared memory, 256 TMEM columns, <= 168 registers per thread)
+// (112 KB of shared memory, 256 TMEM columns, <= 144 registers per thread)
 // that two CTAs share an SM, so one CTA's softmax overlaps the other's MMAs.
 // Every listed key block (128 keys) is processed as two 64-key tiles.
-// 6 warps, specialised:
+// 7 warps, specialised:
 //   warps 0-3  softmax + epilogue: thread r owns query row r, which is TMEM
 //              lane r (warp w may only touch lanes 32w..32w+31);
-//   warp 4     TMA producer: Q once, then K tiles through a 3-slot ring and
-//              V tiles through a 2-slot ring;
-//   warp 5     MMA issuer (one thread): S = Q K^T (N = 64) into one of two
-//              TMEM buffers, O += P V (K = 64) into a TMEM accumulator.
-// TMEM (256 columns): S0 [0,64), S1 [64,128), O [128,256).
+//   warp 4     TMA producer: Q once, then K tiles through a 3-slot ring;
+//   warp 6     TMA producer: V tiles through a 2-slot ring;
+//   warp 5     MMA issuer (one thread): S = Q K^T (N = 64, both operands in
+//              shared memory) into TMEM, O += P V (K = 64, P from TMEM, V
+//              from shared memory) into a TMEM accumulator.
+// TMEM (256 columns): S [0,64) fp32, P0 [64,96) and P1 [96,128) (bf16 pairs),
+// O [128,256) fp32.
 // Shared memory (1024-B aligned, 128-B swizzle everywhere):
 //   Q 32 KB (two halves [128 rows x 64 d]) | K x3 16 KB | V x2 16 KB
 // (112 KB in all, with no room for alignment slack: the kernel requires the
 // dynamic shared-memory window to start 1024-B aligned, which it is when the
 // kernel declares no static shared memory, and checks it).
 // K and V tiles are two 8-KB halves [64 keys x 64 d]; Q and K are K-major
-// operands of S, V is the MN-major B operand of P V.  P(t) ([128 rows x 64
-// keys], 16 KB, K-major) is written into the shared-memory slot of K(t),
-// which S(t) no longer needs: the producer refills that slot only after
-// P(t) V(t) has completed.  With three K slots the load of K(t+2) waits only
-// for P(t-1) V(t-1), so it is in flight while the softmax works on S(t) and
-// S(t+1) instead of sitting on the path between P(t) V(t) and S(t+2).
+// operands of S, V is the MN-major B operand of P V.  A K slot is refilled as
+// soon as S of its tile has completed, a V slot once P V of its tile has.
+// Keeping P in TMEM (rather than staging it in shared memory for an SS MMA)
+// takes 16 KB of stores and 16 KB of tensor-core operand reads per tile off
+// the shared memory, whose bandwidth the operand reads of Q, K and V and the
+// TMA writes of K and V already nearly fill.
 //
-// Per key tile t the softmax warps read S(t) from TMEM, release the buffer,
-// compute p = 2^(s*scale*log2e - m) with a running row max m, rescale O in
-// TMEM only when m grows by more than 2^8, write P(t) (bf16) and signal the
-// MMA warp, which then issues P(t) V(t) while S(t+1) is already in flight.
+// Per key tile t the softmax warps read S(t) from TMEM into registers and
+// release it (so S(t+1) = Q K(t+1)^T runs during the exponentials), compute
+// p = 2^(s*scale*log2e - m) with a running row max m, rescale O in TMEM only
+// when m grows by more than 2^8, store P(t) (bf16) into P(t mod 2) and signal
+// the MMA warp, which issues P(t) V(t).
 //
 // Every wait is bounded (2 s); on expiry the kernel records FP_ERR_TIMEOUT,
 // raises a CTA-wide abort flag, drains its outstanding TMA loads and frees
@@ -59,12 +62,14 @@ constexpr uint32_t TMEM_COLS = 256;
 
 struct TcSmem {
   uint8_t q[Q_BYTES];
-  uint8_t k[NK][KV_BYTES];  // K(t), then P(t)
+  uint8_t k[NK][KV_BYTES];
   uint8_t v[NV][KV_BYTES];
   uint64_t bar_q;
   uint64_t k_full[NK], k_empty[NK], v_full[NV], v_empty[NV];
-  uint64_t s_full[2], s_free[2];
-  uint64_t p_full, p_empty, o_full;
+  uint64_t s_full, s_free;   // S(t) written / read out
+  // P(t) stored / P(t) V(t) done, both per P buffer (t mod 2): a barrier is
+  // then never more than one phase ahead of its waiter
+  uint64_t p_full[2], p_empty[2], o_full;
   uint32_t tmem_base;
   int ntile;  // key tiles of this CTA
   int abort_flag;
@@ -72,7 +77,8 @@ struct TcSmem {
 constexpr size_t kSmemBytes = sizeof(TcSmem);  // no slack: the base is 1024-B aligned
 // two CTAs per SM: 228 KB of shared memory, 1 KB of it reserved per CTA
 static_assert(2 * (kSmemBytes + 1024) <= 233472, "two CTAs must fit in one SM");
-static_assert(BM * BN * 2 == KV_BYTES, "P(t) must fit the K(t) slot");
+constexpr uint32_t S_COL = 0, P_COL = BN, O_COL = 2 * BN;  // TMEM columns
+static_assert(P_COL + 2 * (BN / 2) <= O_COL && O_COL + HD <= TMEM_COLS, "TMEM layout");
 
 __device__ __forceinline__ float ex2(float x) {
   float y;
@@ -128,27 +134,99 @@ struct Walker {
   }
 };
 
-// One S tile (64 keys) of one row (TMEM lane): the row max over the tile,
-// the lazy-rescale decision, then the exponentials packed to bf16 pairs,
-// with the row sum in 8 chains.  MASK: keys c > lim contribute 0.
+// Two-lane fp32 arithmetic (one f32x2 instruction for both lanes).
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return d;
+}
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+__device__ __forceinline__ float2 fsub2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "sub.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// 2^x on the FMA pipe (no MUFU), for the share of the exponentials that the
+// MUFU unit would otherwise queue: x = j + f with j the nearest integer (adding
+// 1.5 * 2^23 rounds x and leaves j in the low mantissa bits of the sum) and
+// |f| <= 1/2 (Cody-Waite range reduction); 2^f by a cubic whose coefficients
+// were fitted here by Remez exchange for least maximum relative error on
+// [-1/2, 1/2] (7.5e-5 evaluated in fp32: far below the bf16 rounding of P);
+// then j is added to the exponent field.  Inputs here are <= 8; x is clamped
+// below at -126 (the result there is < 2^-125, i.e. nothing next to the row
+// maximum's 1).
+constexpr float kPolyC0 = 0x1.fff692p-1f, kPolyC1 = 0x1.62f31ap-1f, kPolyC2 = 0x1.f0de1ap-3f,
+                kPolyC3 = 0x1.c3f76p-5f;
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+  constexpr float kShift = 12582912.f;  // 1.5 * 2^23
+  x.x = fmaxf(x.x, -126.f);
+  x.y = fmaxf(x.y, -126.f);
+  const float2 t = fadd2(x, make_float2(kShift, kShift));
+  const float2 f = fsub2(x, fsub2(t, make_float2(kShift, kShift)));
+  float2 p = ffma2(make_float2(kPolyC3, kPolyC3), f, make_float2(kPolyC2, kPolyC2));
+  p = ffma2(p, f, make_float2(kPolyC1, kPolyC1));
+  p = ffma2(p, f, make_float2(kPolyC0, kPolyC0));
+  // t's bits are 0x4B400000 + j; shifted by 23 only j * 2^23 survives
+  return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
+                     __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
+}
+
+// Of every 4 column pairs of an S row, how many take exp2_poly2 rather than
+// the MUFU ex2 (the MUFU unit, 16 lanes per clock per SM, would otherwise be
+// as busy as the tensor cores).
+#ifndef FP_ATTN_POLY_PAIRS
+#define FP_ATTN_POLY_PAIRS 0
+#endif
+constexpr int kPolyPairs = FP_ATTN_POLY_PAIRS;
+static_assert(kPolyPairs >= 0 && kPolyPairs <= 4, "poly pairs per 4");
+
+// One S tile (64 keys) of one row (TMEM lane): read out (then released), the
+// row max over the tile, the lazy-rescale decision, then the exponentials
+// packed to bf16 pairs, with the row sum in 4 two-lane chains.  MASK: keys
+// c > lim contribute 0.
 template <bool MASK>
-__device__ __forceinline__ void softmax_tile(uint32_t s_addr, int lim, float sl2, float m,
-                                             float &muse, float &alpha, float (&sm8)[8],
-                                             uint32_t (&pk)[BN / 2]) {
+__device__ __forceinline__ void softmax_tile(uint32_t s_addr, uint64_t *s_free, int lim,
+                                             float sl2, float m, float &muse, float &alpha,
+                                             float2 (&acc)[4], uint32_t (&pk)[BN / 2]) {
   uint32_t u[BN];
   tmem_ld32(s_addr, *reinterpret_cast<uint32_t(*)[32]>(&u[0]));
   tmem_ld32(s_addr + 32u, *reinterpret_cast<uint32_t(*)[32]>(&u[32]));
   tc_wait_ld();
+  // S is in registers: the next S may overwrite the TMEM buffer
+  tc_fence_before();
+  mbar_arrive(s_free);
+  float y[BN];
+#pragma unroll
+  for (int c = 0; c < BN; ++c) y[c] = (MASK && c > lim) ? -INFINITY : __uint_as_float(u[c]);
   float mx[8];
 #pragma unroll
   for (int k = 0; k < 8; ++k) mx[k] = -INFINITY;
 #pragma unroll
-  for (int c = 0; c < BN; ++c) {
-    const float y = (MASK && c > lim) ? -INFINITY : __uint_as_float(u[c]);
-    mx[c % 8] = fmaxf(mx[c % 8], y);
-  }
-  const float tmax = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                           fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * sl2;
+  for (int c = 0; c < BN; c += 2) mx[(c / 2) % 8] = max3f(mx[(c / 2) % 8], y[c], y[c + 1]);
+  const float tmax =
+      max3f(max3f(mx[0], mx[1], mx[2]), max3f(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7])) * sl2;
   // lazy rescale: keep the old max unless the row max grew by more than 2^8
   // (p <= 256 is exact enough in fp32 and bf16; the final 1/l uses the same
   // stale max, so the result is unchanged)
@@ -156,22 +234,28 @@ __device__ __forceinline__ void softmax_tile(uint32_t s_addr, int lim, float sl2
   if (tmax > m + 8.0f || m == -INFINITY) muse = fmaxf(m, tmax);
   if (muse == -INFINITY) muse = 0.f;  // every key so far masked
   alpha = ex2(m - muse);              // 1 when unchanged, 0 on the first tile
+  const float2 sc = make_float2(sl2, sl2), nm = make_float2(-muse, -muse);
 #pragma unroll
   for (int i = 0; i < BN; i += 2) {
-    float p0 = ex2(fmaf(__uint_as_float(u[i]), sl2, -muse));
-    float p1 = ex2(fmaf(__uint_as_float(u[i + 1]), sl2, -muse));
-    if (MASK) {
-      p0 = i > lim ? 0.f : p0;
-      p1 = i + 1 > lim ? 0.f : p1;
+    const float2 x = ffma2(make_float2(__uint_as_float(u[i]), __uint_as_float(u[i + 1])), sc, nm);
+    float2 p;
+    if ((i / 2) % 4 < kPolyPairs) {
+      p = exp2_poly2(x);
+    } else {
+      p.x = ex2(x.x);
+      p.y = ex2(x.y);
     }
-    sm8[i % 8] += p0;
-    sm8[(i + 1) % 8] += p1;
-    pk[i / 2] = pack_bf16(p0, p1);
+    if (MASK) {
+      p.x = i > lim ? 0.f : p.x;
+      p.y = i + 1 > lim ? 0.f : p.y;
+    }
+    acc[(i / 2) % 4] = fadd2(acc[(i / 2) % 4], p);
+    pk[i / 2] = pack_bf16(p.x, p.y);
   }
 }
 
 template <bool PAIR>
-__global__ void __launch_bounds__(192, 2) attn_tc_kernel(
+__global__ void __launch_bounds__(224, 2) attn_tc_kernel(
     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
     const __grid_constant__ CUtensorMap tm_v, const int32_t *__restrict__ counts,
     const int32_t *__restrict__ indices, __nv_bfloat16 *__restrict__ out,
@@ -217,12 +301,12 @@ __global__ void __launch_bounds__(192, 2) attn_tc_kernel(
       mbar_init(&sm.v_full[s], 1);
       mbar_init(&sm.v_empty[s], 1);
     }
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&sm.s_full[s], 1);
-      mbar_init(&sm.s_free[s], 128);
-    }
-    mbar_init(&sm.p_full, 128);
-    mbar_init(&sm.p_empty, 1);
+    mbar_init(&sm.s_full, 1);
+    mbar_init(&sm.s_free, 128);
+    mbar_init(&sm.p_full[0], 128);
+    mbar_init(&sm.p_full[1], 128);
+    mbar_init(&sm.p_empty[0], 1);
+    mbar_init(&sm.p_empty[1], 1);
     mbar_init(&sm.o_full, 1);
     sm.abort_flag = 0;
     int nt = 2 * na;
@@ -253,55 +337,51 @@ __global__ void __launch_bounds__(192, 2) attn_tc_kernel(
     *abort_flag = 1;
   };
 
-  if (warp == 4) {
-    // ------------------------------------------------------- TMA producer --
+  if (warp == 4 || warp == 6) {
+    // ------------------------------------------ TMA producers (K, then V) --
+    // two threads, so that neither ring waits on the other: K(t) waits for
+    // S(t-3) to finish with its slot, V(t) for P(t-2) V(t-2)
     if (lane == 0 && ntile > 0) {
-      prefetch_tmap(&tm_q);
-      prefetch_tmap(&tm_k);
-      prefetch_tmap(&tm_v);
-      const int qrow = int((bh * n_tok) + size_t(qa) * KB);
-      mbar_arrive_expect_tx(&sm.bar_q, Q_BYTES);
-      tma_load_2d(sm.q, &tm_q, &sm.bar_q, 0, qrow);
-      tma_load_2d(sm.q + Q_HALF, &tm_q, &sm.bar_q, 64, qrow);
+      const bool is_k = warp == 4;
+      const CUtensorMap *tm = is_k ? &tm_k : &tm_v;
+      const int nslot = is_k ? NK : NV;
+      uint8_t *const base = is_k ? sm.k[0] : sm.v[0];
+      uint64_t *const full = is_k ? sm.k_full : sm.v_full;
+      uint64_t *const empty = is_k ? sm.k_empty : sm.v_empty;
+      prefetch_tmap(tm);
+      if (is_k) {
+        prefetch_tmap(&tm_q);
+        const int qrow = int((bh * n_tok) + size_t(qa) * KB);
+        mbar_arrive_expect_tx(&sm.bar_q, Q_BYTES);
+        tma_load_2d(sm.q, &tm_q, &sm.bar_q, 0, qrow);
+        tma_load_2d(sm.q + Q_HALF, &tm_q, &sm.bar_q, 64, qrow);
+      }
       const size_t kvrow0 = (size_t(b) * hkv + kv) * n_tok;
       Walker<PAIR> walk(la, na, lb, nbb, dense);
       int issued = 0;
-      // K(t) waits for P(t-3) V(t-3) (its slot held P(t-3)), V(t) for
-      // P(t-2) V(t-2); in program order K(t+1) follows V(t), which waited
-      // for the same P V, so neither load waits longer than its slot needs
-      int issued_k = 0, issued_v = 0;
       for (int t = 0; t < ntile; ++t) {
-        const int sk = t % NK, sv = t % NV;
+        const int sl = t % nslot;
         const Tile x = walk.next();
         // invalid entries load any in-range block; the softmax masks them
         const int j = x.j < 0 ? 0 : (x.j > qlast ? qlast : x.j);
         const int krow = int(kvrow0 + size_t(j) * KB + size_t(x.sub) * BN);
-        if (!mbar_wait(&sm.k_empty[sk], ((t / NK) & 1) ^ 1, abort_flag)) {
+        if (!mbar_wait(&empty[sl], ((t / nslot) & 1) ^ 1, abort_flag)) {
           fail(FP_ERR_TIMEOUT);
           break;
         }
-        mbar_arrive_expect_tx(&sm.k_full[sk], KV_BYTES);
-        tma_load_2d(sm.k[sk], &tm_k, &sm.k_full[sk], 0, krow);
-        tma_load_2d(sm.k[sk] + KV_HALF, &tm_k, &sm.k_full[sk], 64, krow);
-        issued_k = t + 1;
-        if (!mbar_wait(&sm.v_empty[sv], ((t / NV) & 1) ^ 1, abort_flag)) {
-          fail(FP_ERR_TIMEOUT);
-          break;
-        }
-        mbar_arrive_expect_tx(&sm.v_full[sv], KV_BYTES);
-        tma_load_2d(sm.v[sv], &tm_v, &sm.v_full[sv], 0, krow);
-        tma_load_2d(sm.v[sv] + KV_HALF, &tm_v, &sm.v_full[sv], 64, krow);
-        issued_v = t + 1;
+        uint8_t *dst = base + size_t(sl) * KV_BYTES;
+        mbar_arrive_expect_tx(&full[sl], KV_BYTES);
+        tma_load_2d(dst, tm, &full[sl], 0, krow);
+        tma_load_2d(dst + KV_HALF, tm, &full[sl], 64, krow);
+        issued = t + 1;
       }
       if (*abort_flag) {
         // drain: wait (bounded) for the loads still in flight, the last load
         // of each slot
         volatile int never = 0;
-        mbar_wait(&sm.bar_q, 0, &never, 100000000ull);
-        for (int t = issued_k - NK > 0 ? issued_k - NK : 0; t < issued_k; ++t)
-          mbar_wait(&sm.k_full[t % NK], (t / NK) & 1, &never, 100000000ull);
-        for (int t = issued_v - NV > 0 ? issued_v - NV : 0; t < issued_v; ++t)
-          mbar_wait(&sm.v_full[t % NV], (t / NV) & 1, &never, 100000000ull);
+        if (is_k) mbar_wait(&sm.bar_q, 0, &never, 100000000ull);
+        for (int t = issued - nslot > 0 ? issued - nslot : 0; t < issued; ++t)
+          mbar_wait(&full[t % nslot], (t / nslot) & 1, &never, 100000000ull);
       }
     }
   } else if (warp == 5) {
@@ -312,30 +392,29 @@ __global__ void __launch_bounds__(192, 2) attn_tc_kernel(
       const uint32_t q_addr = smem_u32(sm.q);
       bool ok = mbar_wait(&sm.bar_q, 0, abort_flag);
       auto issue_pv = [&](int u) -> bool {
-        const int sk = u % NK, sv = u % NV;
-        if (!mbar_wait(&sm.p_full, u & 1, abort_flag)) return false;
+        const int sv = u % NV, pb = u & 1;
+        if (!mbar_wait(&sm.p_full[pb], (u >> 1) & 1, abort_flag)) return false;
         if (!mbar_wait(&sm.v_full[sv], (u / NV) & 1, abort_flag)) return false;
         tc_fence_after();
-        const uint32_t p_addr = smem_u32(sm.k[sk]);  // P(u) sits in K(u)'s slot
         const uint32_t v_addr = smem_u32(sm.v[sv]);
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk) {
-          // A = P [128 rows x 64 keys]: K-major, 16 keys = 32 B along a row
-          const uint64_t ad = umma_desc_sw128(p_addr + kk * 32, 16, 1024);
+          // A = P(u) [128 lanes x 64 keys] in TMEM: 16 keys = 8 columns;
           // B = V [64 keys x 128 d]: MN-major, 64-d halves KV_HALF apart,
           // 16 keys = 16 rows of 128 B
           const uint64_t bd = umma_desc_sw128(v_addr + kk * 16 * 128, KV_HALF, 1024);
-          tc_mma_ss(tmem + 2 * BN, ad, bd, idesc_o, (u > 0 || kk > 0) ? 1u : 0u);
+          tc_mma_ts(tmem + O_COL, tmem + P_COL + uint32_t(pb * (BN / 2) + kk * 8), bd, idesc_o,
+                    (u > 0 || kk > 0) ? 1u : 0u);
         }
-        tc_commit(&sm.k_empty[sk]);
         tc_commit(&sm.v_empty[sv]);
-        tc_commit(&sm.p_empty);
+        tc_commit(&sm.p_empty[pb]);
         return true;
       };
       for (int t = 0; ok && t < ntile; ++t) {
-        const int s = t % NK, sb = t & 1;
+        const int s = t % NK;
+        // S(t) overwrites S(t-1): the softmax must have read it out
         if (!mbar_wait(&sm.k_full[s], (t / NK) & 1, abort_flag) ||
-            !mbar_wait(&sm.s_free[sb], ((t >> 1) & 1) ^ 1, abort_flag)) {
+            !mbar_wait(&sm.s_free, (t & 1) ^ 1, abort_flag)) {
           ok = false;
           break;
         }
@@ -348,9 +427,10 @@ __global__ void __launch_bounds__(192, 2) attn_tc_kernel(
               umma_desc_sw128(q_addr + (kk / 4) * Q_HALF + (kk % 4) * 32, 16, 1024);
           const uint64_t bd =
               umma_desc_sw128(k_addr + (kk / 4) * KV_HALF + (kk % 4) * 32, 16, 1024);
-          tc_mma_ss(tmem + uint32_t(sb * BN), ad, bd, idesc_s, kk > 0 ? 1u : 0u);
+          tc_mma_ss(tmem + S_COL, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
         }
-        tc_commit(&sm.s_full[sb]);
+        tc_commit(&sm.s_full);
+        tc_commit(&sm.k_empty[s]);
         if (t >= 1 && !issue_pv(t - 1)) {
           ok = false;
           break;
@@ -374,11 +454,11 @@ __global__ void __launch_bounds__(192, 2) attn_tc_kernel(
     Walker<PAIR> walk(la, na, lb, nbb, dense);
     Tile x = walk.next();  // prefetched one tile ahead
     for (int t = 0; t < ntile; ++t) {
-      const int sb = t & 1, s = t % NK;
+      const int pb = t & 1;
       const Tile cur = x;
       if (t + 1 < ntile) x = walk.next();
       // waits are made warp-uniform: tcgen05.ld/st below are .sync.aligned
-      if (!__all_sync(0xffffffffu, mbar_wait(&sm.s_full[sb], (t >> 1) & 1, abort_flag))) {
+      if (!__all_sync(0xffffffffu, mbar_wait(&sm.s_full, t & 1, abort_flag))) {
         ok = false;
         break;
       }
@@ -393,26 +473,23 @@ __global__ void __launch_bounds__(192, 2) attn_tc_kernel(
       const bool masked = !valid || cur.j == qh;
       const int lim = valid ? rl - BN * cur.sub : -1;
       float muse, alpha;
-      float sm8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                       make_float2(0.f, 0.f)};
       uint32_t pk[BN / 2];
-      const uint32_t s_addr = lane_base + uint32_t(sb * BN);
+      const uint32_t s_addr = lane_base + S_COL;
       if (masked)
-        softmax_tile<true>(s_addr, lim, sl2, m, muse, alpha, sm8, pk);
+        softmax_tile<true>(s_addr, &sm.s_free, lim, sl2, m, muse, alpha, acc, pk);
       else
-        softmax_tile<false>(s_addr, lim, sl2, m, muse, alpha, sm8, pk);
-      tc_fence_before();
-      mbar_arrive(&sm.s_free[sb]);
-      const float ps = ((sm8[0] + sm8[1]) + (sm8[2] + sm8[3])) +
-                       ((sm8[4] + sm8[5]) + (sm8[6] + sm8[7]));
+        softmax_tile<false>(s_addr, &sm.s_free, lim, sl2, m, muse, alpha, acc, pk);
+      const float ps = ((acc[0].x + acc[0].y) + (acc[1].x + acc[1].y)) +
+                       ((acc[2].x + acc[2].y) + (acc[3].x + acc[3].y));
       l = l * alpha + ps;
       // O is rescaled (rarely: lazy) by the whole warp if any of its rows'
-      // max grew; that needs P(t-1) V(t-1) finished.  p_empty completes once
-      // per P V; S(t), waited for above, was issued after P(t-2) V(t-2), so
-      // the barrier is at most one phase behind and the parity wait for
-      // phase t-1 is exact.  Without a rescale nothing waits here: P(t) goes
-      // to the K(t) slot, which P(t-1) V(t-1) does not read.
+      // max grew; that needs P(t-1) V(t-1) finished (p_empty of buffer
+      // (t-1) mod 2, its ((t-1)/2)-th completion)
       if (__any_sync(0xffffffffu, t > 0 && alpha != 1.f)) {
-        if (!__all_sync(0xffffffffu, mbar_wait(&sm.p_empty, (t & 1) ^ 1, abort_flag))) {
+        if (!__all_sync(0xffffffffu,
+                        mbar_wait(&sm.p_empty[pb ^ 1], ((t - 1) >> 1) & 1, abort_flag))) {
           ok = false;
           break;
         }
@@ -420,24 +497,24 @@ __global__ void __launch_bounds__(192, 2) attn_tc_kernel(
 #pragma unroll
         for (int c0 = 0; c0 < HD; c0 += 32) {
           uint32_t u[32];
-          tmem_ld32(lane_base + uint32_t(2 * BN + c0), u);
+          tmem_ld32(lane_base + O_COL + uint32_t(c0), u);
           tc_wait_ld();
 #pragma unroll
           for (int i = 0; i < 32; ++i) u[i] = __float_as_uint(__uint_as_float(u[i]) * alpha);
-          tmem_st32(lane_base + uint32_t(2 * BN + c0), u);
+          tmem_st32(lane_base + O_COL + uint32_t(c0), u);
         }
-        tc_wait_st();
       }
-      // P row -> the K(t) slot, K-major SW128 [128 rows x 64 keys]: 16-B chunk
-      // (8 keys) c of row r stored at chunk c ^ (r % 8)
-#pragma unroll
-      for (int c = 0; c < BN / 8; ++c) {
-        const uint4 w = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-        *reinterpret_cast<uint4 *>(sm.k[s] + r * 128 + ((c ^ (r & 7)) * 16)) = w;
+      // P(t) goes to buffer t mod 2 once P(t-2) V(t-2) has read it out (for
+      // t < 2 the wait is on the phase before the first and returns at once)
+      if (!__all_sync(0xffffffffu, mbar_wait(&sm.p_empty[pb], ((t >> 1) & 1) ^ 1, abort_flag))) {
+        ok = false;
+        break;
       }
-      fence_async_smem();
+      tc_fence_after();
+      tmem_st32(lane_base + P_COL + uint32_t(pb * (BN / 2)), pk);
+      tc_wait_st();
       tc_fence_before();
-      mbar_arrive(&sm.p_full);
+      mbar_arrive(&sm.p_full[pb]);
       m = muse;
     }
     // ------------------------------------------------------------ epilogue --
@@ -454,7 +531,7 @@ __global__ void __launch_bounds__(192, 2) attn_tc_kernel(
     for (int c0 = 0; c0 < HD; c0 += 32) {
       uint32_t u[32];
       if (ok && ntile > 0) {
-        tmem_ld32(lane_base + uint32_t(2 * BN + c0), u);
+        tmem_ld32(lane_base + O_COL + uint32_t(c0), u);
         tc_wait_ld();
       } else {
 #pragma unroll
@@ -520,12 +597,12 @@ cudaError_t launch_attn_bf16(const Dims &D, const void *q, const void *k, const 
   if (D.bs == 128) {
     cudaFuncSetAttribute(attn_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          int(kSmemBytes));
-    attn_tc_kernel<false><<<dim3(D.nb, D.hq, D.bt), 192, kSmemBytes, st>>>(
+    attn_tc_kernel<false><<<dim3(D.nb, D.hq, D.bt), 224, kSmemBytes, st>>>(
         mq, mk, mv, counts, indices, o, lse, D.hq, D.g, D.n, D.nb, dense, status);
   } else {
     cudaFuncSetAttribute(attn_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          int(kSmemBytes));
-    attn_tc_kernel<true><<<dim3((D.nb + 1) / 2, D.hq, D.bt), 192, kSmemBytes, st>>>(
+    attn_tc_kernel<true><<<dim3((D.nb + 1) / 2, D.hq, D.bt), 224, kSmemBytes, st>>>(
         mq, mk, mv, counts, indices, o, lse, D.hq, D.g, D.n, D.nb, dense, status);
   }
   return cudaGetLastError();
