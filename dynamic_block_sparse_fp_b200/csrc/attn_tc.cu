@@ -7,37 +7,41 @@
 // FlashAttention's online softmax.  Block size 128, head dim 128.
 //
 // One CTA handles one (query block, head, batch) item and is small enough
-// (112 KB of shared memory, 256 TMEM columns, <= 144 registers per thread)
+// (112 KB of shared memory, 256 TMEM columns, <= 168 registers per thread)
 // that two CTAs share an SM, so one CTA's softmax overlaps the other's MMAs.
 // Every listed key block (128 keys) is processed as two 64-key tiles.
-// 7 warps, specialised:
+// 6 warps, specialised:
 //   warps 0-3  softmax + epilogue: thread r owns query row r, which is TMEM
 //              lane r (warp w may only touch lanes 32w..32w+31);
-//   warp 4     TMA producer: Q once, then K tiles through a 3-slot ring;
-//   warp 6     TMA producer: V tiles through a 2-slot ring;
-//   warp 5     MMA issuer (one thread): S = Q K^T (N = 64, both operands in
-//              shared memory) into TMEM, O += P V (K = 64, P from TMEM, V
-//              from shared memory) into a TMEM accumulator.
-// TMEM (256 columns): S [0,64) fp32, P0 [64,96) and P1 [96,128) (bf16 pairs),
-// O [128,256) fp32.
+//   warp 4     TMA producer (one thread): Q's second half once, then K tiles
+//              through a 3-slot ring and V tiles through a 3-slot ring;
+//   warp 5     MMA issuer (one thread): S = Q K^T (N = 64) into TMEM and
+//              O += P V (K = 64, P from TMEM) into a TMEM accumulator.
+// TMEM (256 columns): S [0,64) fp32 | P [64,96) bf16 pairs | Q d 0..63
+// [96,128) bf16 pairs | O [128,256) fp32.
 // Shared memory (1024-B aligned, 128-B swizzle everywhere):
-//   Q 32 KB (two halves [128 rows x 64 d]) | K x3 16 KB | V x2 16 KB
+//   Q d 64..127 16 KB [128 rows x 64 d] | K x3 16 KB | V x3 16 KB
 // (112 KB in all, with no room for alignment slack: the kernel requires the
 // dynamic shared-memory window to start 1024-B aligned, which it is when the
 // kernel declares no static shared memory, and checks it).
-// K and V tiles are two 8-KB halves [64 keys x 64 d]; Q and K are K-major
-// operands of S, V is the MN-major B operand of P V.  A K slot is refilled as
-// soon as S of its tile has completed, a V slot once P V of its tile has.
-// Keeping P in TMEM (rather than staging it in shared memory for an SS MMA)
-// takes 16 KB of stores and 16 KB of tensor-core operand reads per tile off
-// the shared memory, whose bandwidth the operand reads of Q, K and V and the
-// TMA writes of K and V already nearly fill.
+// K and V tiles are two 8-KB halves [64 keys x 64 d]; K is the K-major B
+// operand of S, V the MN-major B operand of P V.  S takes its first 64 d
+// with A = Q from TMEM and the other 64 with A = Q from shared memory.  A K
+// slot is refilled as soon as S of its tile has completed, a V slot once P V
+// of its tile has.
+// Why this split: an MMA of N = 64 whose operands both come from shared memory
+// reads A (all of Q) for every 64 keys, 192 B per clock at full rate, more
+// than the 128 B per clock shared memory delivers, and the K and V tile writes
+// share that bandwidth.  Keeping P and half of Q in TMEM cuts the shared
+// memory traffic per tile from 128 KB (Q, K, P, V operand reads, P stores,
+// K/V writes) to 80 KB; all of Q plus a second P buffer would not fit in 256
+// columns.
 //
 // Per key tile t the softmax warps read S(t) from TMEM into registers and
 // release it (so S(t+1) = Q K(t+1)^T runs during the exponentials), compute
 // p = 2^(s*scale*log2e - m) with a running row max m, rescale O in TMEM only
-// when m grows by more than 2^8, store P(t) (bf16) into P(t mod 2) and signal
-// the MMA warp, which issues P(t) V(t).
+// when m grows by more than 2^8, store P(t) (bf16) once P(t-1) V(t-1) has
+// read P(t-1), and signal the MMA warp, which issues P(t) V(t).
 //
 // Every wait is bounded (2 s); on expiry the kernel records FP_ERR_TIMEOUT,
 // raises a CTA-wide abort flag, drains its outstanding TMA loads and frees
@@ -52,8 +56,8 @@ namespace {
 constexpr int BM = 128;   // query rows per tile (= block size)
 constexpr int BN = 64;    // keys per tile (half a block)
 constexpr int HD = 128;   // head dim
-constexpr int NK = 3;     // K slots (K(t), then P(t))
-constexpr int NV = 2;     // V slots
+constexpr int NK = 3;     // K slots
+constexpr int NV = 3;     // V slots
 constexpr uint32_t Q_BYTES = BM * HD * 2;   // 32 KB
 constexpr uint32_t Q_HALF = Q_BYTES / 2;    // [128 rows x 64 d]
 constexpr uint32_t KV_BYTES = BN * HD * 2;  // 16 KB
@@ -61,15 +65,13 @@ constexpr uint32_t KV_HALF = KV_BYTES / 2;  // [64 keys x 64 d]
 constexpr uint32_t TMEM_COLS = 256;
 
 struct TcSmem {
-  uint8_t q[Q_BYTES];
+  uint8_t q[Q_HALF];  // Q, d 64..127 (d 0..63 lives in TMEM)
   uint8_t k[NK][KV_BYTES];
   uint8_t v[NV][KV_BYTES];
-  uint64_t bar_q;
+  uint64_t bar_q, q_tmem;    // Q's shared-memory half loaded / TMEM half stored
   uint64_t k_full[NK], k_empty[NK], v_full[NV], v_empty[NV];
   uint64_t s_full, s_free;   // S(t) written / read out
-  // P(t) stored / P(t) V(t) done, both per P buffer (t mod 2): a barrier is
-  // then never more than one phase ahead of its waiter
-  uint64_t p_full[2], p_empty[2], o_full;
+  uint64_t p_full, p_empty, o_full;  // P(t) stored / P(t) V(t) done / all done
   uint32_t tmem_base;
   int ntile;  // key tiles of this CTA
   int abort_flag;
@@ -77,8 +79,9 @@ struct TcSmem {
 constexpr size_t kSmemBytes = sizeof(TcSmem);  // no slack: the base is 1024-B aligned
 // two CTAs per SM: 228 KB of shared memory, 1 KB of it reserved per CTA
 static_assert(2 * (kSmemBytes + 1024) <= 233472, "two CTAs must fit in one SM");
-constexpr uint32_t S_COL = 0, P_COL = BN, O_COL = 2 * BN;  // TMEM columns
-static_assert(P_COL + 2 * (BN / 2) <= O_COL && O_COL + HD <= TMEM_COLS, "TMEM layout");
+// TMEM columns: S fp32, P bf16 pairs, the first 64 d of Q bf16 pairs, O fp32
+constexpr uint32_t S_COL = 0, P_COL = BN, Q0_COL = BN + BN / 2, O_COL = 2 * BN;
+static_assert(Q0_COL + HD / 4 <= O_COL && O_COL + HD <= TMEM_COLS, "TMEM layout");
 
 __device__ __forceinline__ float ex2(float x) {
   float y;
@@ -202,38 +205,27 @@ __device__ __forceinline__ float2 exp2_poly2(float2 x) {
 constexpr int kPolyPairs = FP_ATTN_POLY_PAIRS;
 static_assert(kPolyPairs >= 0 && kPolyPairs <= 4, "poly pairs per 4");
 
-// One S tile (64 keys) of one row (TMEM lane): read out (then released), the
-// row max over the tile, the lazy-rescale decision, then the exponentials
-// packed to bf16 pairs, with the row sum in 4 two-lane chains.  MASK: keys
-// c > lim contribute 0.
+// The maximum of one S row over a 64-key tile (raw scores); MASK: keys
+// c > lim are left out.
 template <bool MASK>
-__device__ __forceinline__ void softmax_tile(uint32_t s_addr, uint64_t *s_free, int lim,
-                                             float sl2, float m, float &muse, float &alpha,
-                                             float2 (&acc)[4], uint32_t (&pk)[BN / 2]) {
-  uint32_t u[BN];
-  tmem_ld32(s_addr, *reinterpret_cast<uint32_t(*)[32]>(&u[0]));
-  tmem_ld32(s_addr + 32u, *reinterpret_cast<uint32_t(*)[32]>(&u[32]));
-  tc_wait_ld();
-  // S is in registers: the next S may overwrite the TMEM buffer
-  tc_fence_before();
-  mbar_arrive(s_free);
-  float y[BN];
-#pragma unroll
-  for (int c = 0; c < BN; ++c) y[c] = (MASK && c > lim) ? -INFINITY : __uint_as_float(u[c]);
+__device__ __forceinline__ float tile_max(const uint32_t (&u)[BN], int lim) {
   float mx[8];
 #pragma unroll
   for (int k = 0; k < 8; ++k) mx[k] = -INFINITY;
 #pragma unroll
-  for (int c = 0; c < BN; c += 2) mx[(c / 2) % 8] = max3f(mx[(c / 2) % 8], y[c], y[c + 1]);
-  const float tmax =
-      max3f(max3f(mx[0], mx[1], mx[2]), max3f(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7])) * sl2;
-  // lazy rescale: keep the old max unless the row max grew by more than 2^8
-  // (p <= 256 is exact enough in fp32 and bf16; the final 1/l uses the same
-  // stale max, so the result is unchanged)
-  muse = m;
-  if (tmax > m + 8.0f || m == -INFINITY) muse = fmaxf(m, tmax);
-  if (muse == -INFINITY) muse = 0.f;  // every key so far masked
-  alpha = ex2(m - muse);              // 1 when unchanged, 0 on the first tile
+  for (int c = 0; c < BN; c += 2) {
+    const float y0 = (MASK && c > lim) ? -INFINITY : __uint_as_float(u[c]);
+    const float y1 = (MASK && c + 1 > lim) ? -INFINITY : __uint_as_float(u[c + 1]);
+    mx[(c / 2) % 8] = max3f(mx[(c / 2) % 8], y0, y1);
+  }
+  return max3f(max3f(mx[0], mx[1], mx[2]), max3f(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
+}
+
+// p = 2^(s * sl2 - muse) for one S row over a 64-key tile, packed to bf16
+// pairs, and its sum in 4 two-lane chains; MASK: keys c > lim give 0.
+template <bool MASK>
+__device__ __forceinline__ void tile_exp(const uint32_t (&u)[BN], int lim, float sl2, float muse,
+                                         float2 (&acc)[4], uint32_t (&pk)[BN / 2]) {
   const float2 sc = make_float2(sl2, sl2), nm = make_float2(-muse, -muse);
 #pragma unroll
   for (int i = 0; i < BN; i += 2) {
@@ -254,11 +246,44 @@ __device__ __forceinline__ void softmax_tile(uint32_t s_addr, uint64_t *s_free, 
   }
 }
 
+// One S tile of one row (TMEM lane): read out (then released); the row max
+// and the exponentials against the running max m are computed side by side
+// (independent instruction streams), and the exponentials are redone only
+// if some row of the warp needs a new max: the max grew by more than 2^8
+// (lazy rescale: p <= 256 is exact enough in fp32 and bf16, and the final
+// 1/l uses the same stale max, so the result is unchanged), or this is the
+// first tile.
+template <bool MASK>
+__device__ __forceinline__ void softmax_tile(uint32_t s_addr, uint64_t *s_free, bool first,
+                                             int lim, float sl2, float m, float &muse,
+                                             float &alpha, float2 (&acc)[4],
+                                             uint32_t (&pk)[BN / 2]) {
+  uint32_t u[BN];
+  tmem_ld32(s_addr, *reinterpret_cast<uint32_t(*)[32]>(&u[0]));
+  tmem_ld32(s_addr + 32u, *reinterpret_cast<uint32_t(*)[32]>(&u[32]));
+  tc_wait_ld();
+  // S is in registers: the next S may overwrite the TMEM buffer
+  tc_fence_before();
+  mbar_arrive(s_free);
+  if (!first) tile_exp<MASK>(u, lim, sl2, m, acc, pk);
+  const float tmax = tile_max<MASK>(u, lim) * sl2;
+  muse = m;
+  if (tmax > m + 8.0f || m == -INFINITY) muse = fmaxf(m, tmax);
+  if (muse == -INFINITY) muse = 0.f;  // every key so far masked
+  if (__any_sync(0xffffffffu, first || muse != m)) {
+#pragma unroll
+    for (int k = 0; k < 4; ++k) acc[k] = make_float2(0.f, 0.f);
+    tile_exp<MASK>(u, lim, sl2, muse, acc, pk);
+  }
+  alpha = muse != m ? ex2(m - muse) : 1.f;  // 0 on the first tile
+}
+
 template <bool PAIR>
-__global__ void __launch_bounds__(224, 2) attn_tc_kernel(
+__global__ void __launch_bounds__(192, 2) attn_tc_kernel(
     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-    const __grid_constant__ CUtensorMap tm_v, const int32_t *__restrict__ counts,
-    const int32_t *__restrict__ indices, __nv_bfloat16 *__restrict__ out,
+    const __grid_constant__ CUtensorMap tm_v, const __nv_bfloat16 *__restrict__ qg,
+    const int32_t *__restrict__ counts, const int32_t *__restrict__ indices,
+    __nv_bfloat16 *__restrict__ out,
     float *__restrict__ lse, int hq, int g, int n_tok, int nb, bool dense, int *status) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   // the 128-B swizzled operand tiles need 1024-B alignment and there is no
@@ -293,6 +318,7 @@ __global__ void __launch_bounds__(224, 2) attn_tc_kernel(
 
   if (threadIdx.x == 0) {
     mbar_init(&sm.bar_q, 1);
+    mbar_init(&sm.q_tmem, 128);
     for (int s = 0; s < NK; ++s) {
       mbar_init(&sm.k_full[s], 1);
       mbar_init(&sm.k_empty[s], 1);
@@ -303,10 +329,8 @@ __global__ void __launch_bounds__(224, 2) attn_tc_kernel(
     }
     mbar_init(&sm.s_full, 1);
     mbar_init(&sm.s_free, 128);
-    mbar_init(&sm.p_full[0], 128);
-    mbar_init(&sm.p_full[1], 128);
-    mbar_init(&sm.p_empty[0], 1);
-    mbar_init(&sm.p_empty[1], 1);
+    mbar_init(&sm.p_full, 128);
+    mbar_init(&sm.p_empty, 1);
     mbar_init(&sm.o_full, 1);
     sm.abort_flag = 0;
     int nt = 2 * na;
@@ -337,51 +361,63 @@ __global__ void __launch_bounds__(224, 2) attn_tc_kernel(
     *abort_flag = 1;
   };
 
-  if (warp == 4 || warp == 6) {
-    // ------------------------------------------ TMA producers (K, then V) --
-    // two threads, so that neither ring waits on the other: K(t) waits for
-    // S(t-3) to finish with its slot, V(t) for P(t-2) V(t-2)
+  if (warp == 4) {
+    // ------------------------------------------------------- TMA producer --
+    // Q's second half once, then K(i) and V(i - 2) in turn.  K(i) waits for
+    // S(i-3) to finish with its slot, V(i-2) for P(i-5) V(i-5), which was
+    // issued before S(i-3) and is covered by its commit: by the time K(i) may
+    // load, V(i-2) may too, so the interleaving delays neither.
     if (lane == 0 && ntile > 0) {
-      const bool is_k = warp == 4;
-      const CUtensorMap *tm = is_k ? &tm_k : &tm_v;
-      const int nslot = is_k ? NK : NV;
-      uint8_t *const base = is_k ? sm.k[0] : sm.v[0];
-      uint64_t *const full = is_k ? sm.k_full : sm.v_full;
-      uint64_t *const empty = is_k ? sm.k_empty : sm.v_empty;
-      prefetch_tmap(tm);
-      if (is_k) {
-        prefetch_tmap(&tm_q);
-        const int qrow = int((bh * n_tok) + size_t(qa) * KB);
-        mbar_arrive_expect_tx(&sm.bar_q, Q_BYTES);
-        tma_load_2d(sm.q, &tm_q, &sm.bar_q, 0, qrow);
-        tma_load_2d(sm.q + Q_HALF, &tm_q, &sm.bar_q, 64, qrow);
-      }
+      prefetch_tmap(&tm_q);
+      prefetch_tmap(&tm_k);
+      prefetch_tmap(&tm_v);
+      const int qrow = int((bh * n_tok) + size_t(qa) * KB);
+      mbar_arrive_expect_tx(&sm.bar_q, Q_HALF);
+      tma_load_2d(sm.q, &tm_q, &sm.bar_q, 64, qrow);
       const size_t kvrow0 = (size_t(b) * hkv + kv) * n_tok;
-      Walker<PAIR> walk(la, na, lb, nbb, dense);
-      int issued = 0;
-      for (int t = 0; t < ntile; ++t) {
-        const int sl = t % nslot;
-        const Tile x = walk.next();
-        // invalid entries load any in-range block; the softmax masks them
+      Walker<PAIR> walk_k(la, na, lb, nbb, dense), walk_v(la, na, lb, nbb, dense);
+      // first row of key tile x: invalid entries load any in-range block (the
+      // softmax masks them)
+      auto tile_row = [&](const Tile &x) {
         const int j = x.j < 0 ? 0 : (x.j > qlast ? qlast : x.j);
-        const int krow = int(kvrow0 + size_t(j) * KB + size_t(x.sub) * BN);
-        if (!mbar_wait(&empty[sl], ((t / nslot) & 1) ^ 1, abort_flag)) {
-          fail(FP_ERR_TIMEOUT);
-          break;
+        return int(kvrow0 + size_t(j) * KB + size_t(x.sub) * BN);
+      };
+      int issued_k = 0, issued_v = 0;
+      for (int i = 0; i < ntile + 2 && !*abort_flag; ++i) {
+        if (i < ntile) {
+          const int sl = i % NK;
+          const int row = tile_row(walk_k.next());
+          if (!mbar_wait(&sm.k_empty[sl], ((i / NK) & 1) ^ 1, abort_flag)) {
+            fail(FP_ERR_TIMEOUT);
+            break;
+          }
+          mbar_arrive_expect_tx(&sm.k_full[sl], KV_BYTES);
+          tma_load_2d(sm.k[sl], &tm_k, &sm.k_full[sl], 0, row);
+          tma_load_2d(sm.k[sl] + KV_HALF, &tm_k, &sm.k_full[sl], 64, row);
+          issued_k = i + 1;
         }
-        uint8_t *dst = base + size_t(sl) * KV_BYTES;
-        mbar_arrive_expect_tx(&full[sl], KV_BYTES);
-        tma_load_2d(dst, tm, &full[sl], 0, krow);
-        tma_load_2d(dst + KV_HALF, tm, &full[sl], 64, krow);
-        issued = t + 1;
+        if (i >= 2) {
+          const int t = i - 2, sl = t % NV;
+          const int row = tile_row(walk_v.next());
+          if (!mbar_wait(&sm.v_empty[sl], ((t / NV) & 1) ^ 1, abort_flag)) {
+            fail(FP_ERR_TIMEOUT);
+            break;
+          }
+          mbar_arrive_expect_tx(&sm.v_full[sl], KV_BYTES);
+          tma_load_2d(sm.v[sl], &tm_v, &sm.v_full[sl], 0, row);
+          tma_load_2d(sm.v[sl] + KV_HALF, &tm_v, &sm.v_full[sl], 64, row);
+          issued_v = t + 1;
+        }
       }
       if (*abort_flag) {
         // drain: wait (bounded) for the loads still in flight, the last load
         // of each slot
         volatile int never = 0;
-        if (is_k) mbar_wait(&sm.bar_q, 0, &never, 100000000ull);
-        for (int t = issued - nslot > 0 ? issued - nslot : 0; t < issued; ++t)
-          mbar_wait(&full[t % nslot], (t / nslot) & 1, &never, 100000000ull);
+        mbar_wait(&sm.bar_q, 0, &never, 100000000ull);
+        for (int t = issued_k - NK > 0 ? issued_k - NK : 0; t < issued_k; ++t)
+          mbar_wait(&sm.k_full[t % NK], (t / NK) & 1, &never, 100000000ull);
+        for (int t = issued_v - NV > 0 ? issued_v - NV : 0; t < issued_v; ++t)
+          mbar_wait(&sm.v_full[t % NV], (t / NV) & 1, &never, 100000000ull);
       }
     }
   } else if (warp == 5) {
@@ -390,10 +426,10 @@ __global__ void __launch_bounds__(224, 2) attn_tc_kernel(
       constexpr uint32_t idesc_s = umma_idesc_bf16(BM, BN, 0);
       constexpr uint32_t idesc_o = umma_idesc_bf16(BM, HD, 1);
       const uint32_t q_addr = smem_u32(sm.q);
-      bool ok = mbar_wait(&sm.bar_q, 0, abort_flag);
+      bool ok = mbar_wait(&sm.bar_q, 0, abort_flag) && mbar_wait(&sm.q_tmem, 0, abort_flag);
       auto issue_pv = [&](int u) -> bool {
-        const int sv = u % NV, pb = u & 1;
-        if (!mbar_wait(&sm.p_full[pb], (u >> 1) & 1, abort_flag)) return false;
+        const int sv = u % NV;
+        if (!mbar_wait(&sm.p_full, u & 1, abort_flag)) return false;
         if (!mbar_wait(&sm.v_full[sv], (u / NV) & 1, abort_flag)) return false;
         tc_fence_after();
         const uint32_t v_addr = smem_u32(sm.v[sv]);
@@ -403,11 +439,11 @@ __global__ void __launch_bounds__(224, 2) attn_tc_kernel(
           // B = V [64 keys x 128 d]: MN-major, 64-d halves KV_HALF apart,
           // 16 keys = 16 rows of 128 B
           const uint64_t bd = umma_desc_sw128(v_addr + kk * 16 * 128, KV_HALF, 1024);
-          tc_mma_ts(tmem + O_COL, tmem + P_COL + uint32_t(pb * (BN / 2) + kk * 8), bd, idesc_o,
+          tc_mma_ts(tmem + O_COL, tmem + P_COL + uint32_t(kk * 8), bd, idesc_o,
                     (u > 0 || kk > 0) ? 1u : 0u);
         }
         tc_commit(&sm.v_empty[sv]);
-        tc_commit(&sm.p_empty[pb]);
+        tc_commit(&sm.p_empty);
         return true;
       };
       for (int t = 0; ok && t < ntile; ++t) {
@@ -420,15 +456,17 @@ __global__ void __launch_bounds__(224, 2) attn_tc_kernel(
         }
         tc_fence_after();
         const uint32_t k_addr = smem_u32(sm.k[s]);
+        // d 0..63: A = Q from TMEM (16 d = 8 columns), B = K's first half;
+        // d 64..127: A = Q's second half in shared memory, B = K's second half
+        // (16 d = 32 B inside a 64-d half)
 #pragma unroll
-        for (int kk = 0; kk < HD / 16; ++kk) {
-          // 16 d = 32 B inside a 64-d half; Q halves Q_HALF apart, K halves KV_HALF
-          const uint64_t ad =
-              umma_desc_sw128(q_addr + (kk / 4) * Q_HALF + (kk % 4) * 32, 16, 1024);
-          const uint64_t bd =
-              umma_desc_sw128(k_addr + (kk / 4) * KV_HALF + (kk % 4) * 32, 16, 1024);
-          tc_mma_ss(tmem + S_COL, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
-        }
+        for (int kk = 0; kk < 4; ++kk)
+          tc_mma_ts(tmem + S_COL, tmem + Q0_COL + uint32_t(kk * 8),
+                    umma_desc_sw128(k_addr + kk * 32, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          tc_mma_ss(tmem + S_COL, umma_desc_sw128(q_addr + kk * 32, 16, 1024),
+                    umma_desc_sw128(k_addr + KV_HALF + kk * 32, 16, 1024), idesc_s, 1u);
         tc_commit(&sm.s_full);
         tc_commit(&sm.k_empty[s]);
         if (t >= 1 && !issue_pv(t - 1)) {
@@ -451,10 +489,28 @@ __global__ void __launch_bounds__(224, 2) attn_tc_kernel(
     const int half = PAIR ? r / 64 : 0;
     const int qh = PAIR ? qa + half : qa;
     const int rl = r - 64 * half;  // row inside its block
+    const bool row_exists = !PAIR || half == 0 || has_b;
+    {
+      // the first 64 d of this row's query -> TMEM (A operand of Q K^T);
+      // 32-bit column c holds d 2c (low half) and 2c + 1
+      uint32_t qw[32];
+      const uint4 *src = reinterpret_cast<const uint4 *>(qg + (bh * n_tok + size_t(qa) * KB + r) * HD);
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        const uint4 w = row_exists ? __ldg(src + c) : make_uint4(0u, 0u, 0u, 0u);
+        qw[4 * c] = w.x;
+        qw[4 * c + 1] = w.y;
+        qw[4 * c + 2] = w.z;
+        qw[4 * c + 3] = w.w;
+      }
+      tmem_st32(lane_base + Q0_COL, qw);
+      tc_wait_st();
+      tc_fence_before();
+      mbar_arrive(&sm.q_tmem);
+    }
     Walker<PAIR> walk(la, na, lb, nbb, dense);
     Tile x = walk.next();  // prefetched one tile ahead
     for (int t = 0; t < ntile; ++t) {
-      const int pb = t & 1;
       const Tile cur = x;
       if (t + 1 < ntile) x = walk.next();
       // waits are made warp-uniform: tcgen05.ld/st below are .sync.aligned
@@ -478,22 +534,23 @@ __global__ void __launch_bounds__(224, 2) attn_tc_kernel(
       uint32_t pk[BN / 2];
       const uint32_t s_addr = lane_base + S_COL;
       if (masked)
-        softmax_tile<true>(s_addr, &sm.s_free, lim, sl2, m, muse, alpha, acc, pk);
+        softmax_tile<true>(s_addr, &sm.s_free, t == 0, lim, sl2, m, muse, alpha, acc, pk);
       else
-        softmax_tile<false>(s_addr, &sm.s_free, lim, sl2, m, muse, alpha, acc, pk);
+        softmax_tile<false>(s_addr, &sm.s_free, t == 0, lim, sl2, m, muse, alpha, acc, pk);
       const float ps = ((acc[0].x + acc[0].y) + (acc[1].x + acc[1].y)) +
                        ((acc[2].x + acc[2].y) + (acc[3].x + acc[3].y));
       l = l * alpha + ps;
+      // P(t) overwrites P(t-1), and O may be rescaled: both need P(t-1) V(t-1)
+      // finished (for t = 0 the wait is on the phase before the first and
+      // returns at once)
+      if (!__all_sync(0xffffffffu, mbar_wait(&sm.p_empty, (t & 1) ^ 1, abort_flag))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
       // O is rescaled (rarely: lazy) by the whole warp if any of its rows'
-      // max grew; that needs P(t-1) V(t-1) finished (p_empty of buffer
-      // (t-1) mod 2, its ((t-1)/2)-th completion)
+      // max grew
       if (__any_sync(0xffffffffu, t > 0 && alpha != 1.f)) {
-        if (!__all_sync(0xffffffffu,
-                        mbar_wait(&sm.p_empty[pb ^ 1], ((t - 1) >> 1) & 1, abort_flag))) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
 #pragma unroll
         for (int c0 = 0; c0 < HD; c0 += 32) {
           uint32_t u[32];
@@ -504,22 +561,14 @@ __global__ void __launch_bounds__(224, 2) attn_tc_kernel(
           tmem_st32(lane_base + O_COL + uint32_t(c0), u);
         }
       }
-      // P(t) goes to buffer t mod 2 once P(t-2) V(t-2) has read it out (for
-      // t < 2 the wait is on the phase before the first and returns at once)
-      if (!__all_sync(0xffffffffu, mbar_wait(&sm.p_empty[pb], ((t >> 1) & 1) ^ 1, abort_flag))) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      tmem_st32(lane_base + P_COL + uint32_t(pb * (BN / 2)), pk);
+      tmem_st32(lane_base + P_COL, pk);
       tc_wait_st();
       tc_fence_before();
-      mbar_arrive(&sm.p_full[pb]);
+      mbar_arrive(&sm.p_full);
       m = muse;
     }
     // ------------------------------------------------------------ epilogue --
     const size_t orow = bh * n_tok + size_t(qa) * KB + r;
-    const bool row_exists = !PAIR || half == 0 || has_b;
     if (ok && ntile > 0 && !__all_sync(0xffffffffu, mbar_wait(&sm.o_full, 0, abort_flag)))
       ok = false;
     if (!ok) fail(FP_ERR_TIMEOUT);
@@ -597,13 +646,15 @@ cudaError_t launch_attn_bf16(const Dims &D, const void *q, const void *k, const 
   if (D.bs == 128) {
     cudaFuncSetAttribute(attn_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          int(kSmemBytes));
-    attn_tc_kernel<false><<<dim3(D.nb, D.hq, D.bt), 224, kSmemBytes, st>>>(
-        mq, mk, mv, counts, indices, o, lse, D.hq, D.g, D.n, D.nb, dense, status);
+    attn_tc_kernel<false><<<dim3(D.nb, D.hq, D.bt), 192, kSmemBytes, st>>>(
+        mq, mk, mv, static_cast<const __nv_bfloat16 *>(q), counts, indices, o, lse, D.hq, D.g,
+        D.n, D.nb, dense, status);
   } else {
     cudaFuncSetAttribute(attn_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          int(kSmemBytes));
-    attn_tc_kernel<true><<<dim3((D.nb + 1) / 2, D.hq, D.bt), 224, kSmemBytes, st>>>(
-        mq, mk, mv, counts, indices, o, lse, D.hq, D.g, D.n, D.nb, dense, status);
+    attn_tc_kernel<true><<<dim3((D.nb + 1) / 2, D.hq, D.bt), 192, kSmemBytes, st>>>(
+        mq, mk, mv, static_cast<const __nv_bfloat16 *>(q), counts, indices, o, lse, D.hq, D.g,
+        D.n, D.nb, dense, status);
   }
   return cudaGetLastError();
 }
