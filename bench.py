@@ -157,24 +157,29 @@ def barrier(ws: int):
 
 # ------------------------------------------------------------ CPU baseline --
 
-def cpu_oracle_sample(w: synth.Workload, heads=(0,), q_blocks=None) -> dict:
+def cpu_oracle_sample(w: synth.Workload, heads=(0,), budget_s: float = 10.0,
+                      inputs=None) -> dict:
     """Time the oracle on a bounded sample and extrapolate to the full layer.
 
     Sample: the estimate, pattern and select of ``heads`` (every q head costs
-    the same there) and attention of ``q_blocks`` rows of those heads, scaled
-    by the kept blocks of the whole layer.
+    the same there), then attention of those heads' query blocks, taken in a
+    fixed spread-out order, 4 blocks at a time, until ``budget_s`` seconds of
+    oracle work have passed.  Attention time is scaled by the kept blocks of
+    the whole layer.  ``inputs`` may carry the sampled heads' tensors from an
+    earlier call.
     """
     import numpy as np
 
     import oracle
-    kvs = sorted({h // (w.n_q_heads // w.n_kv_heads) for h in heads})
-    inp = synth.make_inputs(w, kv_heads=kvs)
     g = w.n_q_heads // w.n_kv_heads
-    loc = [kvs.index(h // g) * g + h % g for h in heads]
-    q = inp["q"][:, loc]
-    kk = inp["k"][:, [kvs.index(h // g) for h in heads]]
-    vv = inp["v"][:, [kvs.index(h // g) for h in heads]]
+    kvs = sorted({h // g for h in heads})
+    if inputs is None:
+        inp = synth.make_inputs(w, kv_heads=kvs)
+        loc = [kvs.index(h // g) * g + h % g for h in heads]
+        inputs = (inp["q"][:, loc], inp["k"][:, [kvs.index(h // g) for h in heads]],
+                  inp["v"][:, [kvs.index(h // g) for h in heads]])
     # each sampled head gets its own kv head copy (GQA index h // 1)
+    q, kk, vv = inputs
     t0 = time.perf_counter()
     est = oracle.estimate(q, kk, w.block_size)
     t1 = time.perf_counter()
@@ -185,9 +190,13 @@ def cpu_oracle_sample(w: synth.Workload, heads=(0,), q_blocks=None) -> dict:
                                     w.block_size, w.gamma, w.min_budget, w.max_budget)
     t2 = time.perf_counter()
     nb = w.n_blocks
-    qbs = q_blocks if q_blocks is not None else [nb - 1, (3 * nb) // 4, nb // 2, nb // 4]
-    oracle.sparse_attention(q, kk, vv, counts, indices, w.block_size, heads=list(range(len(heads))),
-                            q_blocks=qbs)
+    order = [int(x) for x in np.random.default_rng(0).permutation(nb)]
+    qbs = []
+    while order and (not qbs or time.perf_counter() - t0 < budget_s):
+        chunk, order = order[:4], order[4:]
+        oracle.sparse_attention(q, kk, vv, counts, indices, w.block_size,
+                                heads=list(range(len(heads))), q_blocks=chunk)
+        qbs += chunk
     t3 = time.perf_counter()
     kept_sample = int(sum(counts[0, i, qb] for i in range(len(heads)) for qb in qbs))
     kept_heads = int(counts.sum())
@@ -199,11 +208,12 @@ def cpu_oracle_sample(w: synth.Workload, heads=(0,), q_blocks=None) -> dict:
     t_att = (t3 - t2) / max(kept_sample, 1) * (kept_heads / nh) * w.n_q_heads
     total = t_est + t_sel + t_att
     return {"seconds_measured": t3 - t0, "seconds_extrapolated": total,
-            "tokens_per_s": w.seq_len * w.batch / total,
+            "tokens_per_s": w.seq_len * w.batch / total, "inputs": inputs,
             "sample": (f"oracle (numpy fp64) on q heads {list(heads)} of {w.name}: estimate, "
-                       f"pattern and select in full, attention on query blocks {qbs} "
-                       f"({kept_sample} kept blocks); extrapolated to {w.n_q_heads} heads and "
-                       f"all kept blocks")}
+                       f"pattern and select in full, then attention on {len(qbs)} query "
+                       f"blocks in a fixed spread order ({kept_sample} kept blocks) until "
+                       f"{budget_s:g} s of oracle work; extrapolated to {w.n_q_heads} heads "
+                       f"and all kept blocks")}
 
 
 def cores() -> int:
@@ -227,8 +237,11 @@ def run_reference(args, w, ws, rank):
     if rank != 0:
         return
     steps = []
+    inputs = None
     for i in range(args.warmup + args.steps):
-        r = cpu_oracle_sample(w)
+        # per step a bounded sample (the whole K + W run stays within minutes)
+        r = cpu_oracle_sample(w, budget_s=args.reference_step_s, inputs=inputs)
+        inputs = r["inputs"]
         if i >= args.warmup:
             steps.append(r)
     tps = statistics.mean(r["tokens_per_s"] for r in steps)
@@ -397,7 +410,7 @@ def run_ours(args, w, ws, rank, local):
                        "ms_per_step": e2e_ms, "steps": args.e2e_steps,
                        "api": "fp_prefill_attn_host (pinned host q/k/v in, out back)"}
     if rank == 0 and not args.no_cpu_baseline:
-        cb = cpu_oracle_sample(w)
+        cb = cpu_oracle_sample(w, budget_s=args.cpu_baseline_s)
         line["cpu_baseline"] = {"value": cb["tokens_per_s"], "unit": "tokens/s",
                                 "cores": cores(), "kind": "oracle", "sample": cb["sample"],
                                 "seconds_measured": cb["seconds_measured"]}
@@ -420,6 +433,10 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-baseline-s", type=float, default=12.0,
+                    help="seconds of oracle work in the cpu_baseline sample")
+    ap.add_argument("--reference-step-s", type=float, default=8.0,
+                    help="seconds of oracle work per step of --impl reference")
     args = ap.parse_args()
     w = synth.WORKLOADS[args.workload]
     over = {k: v for k, v in (("gamma", args.gamma), ("tau", args.tau),
