@@ -62,6 +62,7 @@ fp_status check_params(const fp_params *p) {
   if (!(p->gamma > 0.f) || !(p->gamma <= 1.f)) return FP_ERR_PARAM;
   if (!(p->tau >= 0.f) || isinf(p->tau)) return FP_ERR_PARAM;
   if (p->min_budget < 0) return FP_ERR_PARAM;
+  if (p->qa_mode != FP_QA_FLATTENED && p->qa_mode != FP_QA_QUERYWISE) return FP_ERR_PARAM;
   return FP_OK;
 }
 
@@ -78,6 +79,9 @@ SelectBudgets budgets(const Dims &D, const fp_params &p) {
   int vhi = p.max_budget <= 0 ? D.n : (p.max_budget < D.n ? p.max_budget : D.n);
   b.vs_lo = vlo < vhi ? vlo : vhi;
   b.vs_hi = vhi;
+  b.qa_mode = p.qa_mode;
+  b.row_lo = int((p.min_budget + bs - 1) / bs);
+  b.row_hi = p.max_budget <= 0 ? -1 : int(p.max_budget / bs);
   return b;
 }
 

@@ -57,8 +57,11 @@ cudaError_t launch_pattern(const Dims &D, float tau, const float *est_last,
                            cudaStream_t st);
 
 struct SelectBudgets {
-  long long qa_lo, qa_hi;  // in block pairs
+  long long qa_lo, qa_hi;  // in block pairs (flattened rule)
   int vs_lo, vs_hi;        // in lines
+  int qa_mode;             // FP_QA_FLATTENED or FP_QA_QUERYWISE
+  int row_lo, row_hi;      // query-wise rule: blocks per row before the row-length
+                           // cap; row_hi < 0 means uncapped
 };
 size_t select_ws_bytes(const Dims &D);
 cudaError_t launch_select(const Dims &D, float gamma, const SelectBudgets &bud,

@@ -20,6 +20,13 @@
 // count when the clamp moves k, and one ordered count for the tie rank.  All
 // of it is integer arithmetic, so the result does not depend on thread order.
 // emit_rows_kernel then writes every row's ascending block list.
+//
+// Query-wise rule for query-aware heads ("Measured effects": query-wise index
+// selection instead of the flattened map): the same rule on each row
+// A[i, 0..i] of the map with the row's own total and per-row budgets.
+// select_rows_qa_kernel gives each (row, head) one CTA, which sorts the row's
+// (bit pattern, index) keys in shared memory, finds k by an exact uint64
+// prefix sum of the masses, and writes the row's list itself.
 #include <cooperative_groups.h>
 
 #include "fp_internal.cuh"
@@ -348,8 +355,8 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kCThreads)
     select_head_kernel(const int32_t *__restrict__ pattern, const float *__restrict__ map,
                        const float *__restrict__ vert, const float *__restrict__ slash, int n,
                        int nb, int bs, float gamma, long long qa_lo, long long qa_hi, int vs_lo,
-                       int vs_hi, HeadSel *__restrict__ sel, uint8_t *__restrict__ colflag,
-                       uint8_t *__restrict__ distflag) {
+                       int vs_hi, int qa_mode, HeadSel *__restrict__ sel,
+                       uint8_t *__restrict__ colflag, uint8_t *__restrict__ distflag) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   Ctx cx{cg::this_cluster(), 0u, reinterpret_cast<SelSmem *>(smem_raw)};
   cx.rank = cx.cl.block_rank();
@@ -358,6 +365,7 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kCThreads)
   const size_t bh = size_t(blockIdx.y) * heads_x + blockIdx.x / kCluster;
   const size_t t_pairs = size_t(nb) * (nb + 1) / 2;
   if (pattern[bh] == FP_PATTERN_QA) {  // uniform over the cluster
+    if (qa_mode == FP_QA_QUERYWISE) return;  // rows selected by select_rows_qa_kernel
     HeadSel r = select_list(cx, map + bh * t_pairs, uint32_t(t_pairs), gamma, qa_lo, qa_hi);
     if (cx.rank == 0 && threadIdx.x == 0) sel[2 * bh] = r;
     return;
@@ -406,13 +414,14 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kCThreads)
 __global__ void __launch_bounds__(256) emit_rows_kernel(
     const int32_t *__restrict__ pattern, const float *__restrict__ map, int nb,
     const HeadSel *__restrict__ sel, const uint8_t *__restrict__ colflag,
-    const uint8_t *__restrict__ distflag, int32_t *__restrict__ counts,
+    const uint8_t *__restrict__ distflag, int qa_mode, int32_t *__restrict__ counts,
     int32_t *__restrict__ indices) {
   const int qi = blockIdx.x * 8 + threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
   if (qi >= nb) return;
   const size_t bh = size_t(blockIdx.z) * gridDim.y + blockIdx.y;
   const bool qa = pattern[bh] == FP_PATTERN_QA;
+  if (qa && qa_mode == FP_QA_QUERYWISE) return;  // written by select_rows_qa_kernel
   const HeadSel s = sel[2 * bh];
   const size_t rowbase = size_t(qi) * (qi + 1) / 2;
   const float *mrow = map + bh * (size_t(nb) * (nb + 1) / 2) + rowbase;
@@ -436,6 +445,125 @@ __global__ void __launch_bounds__(256) emit_rows_kernel(
     cnt += __popc(bal);
   }
   if (lane == 0) counts[bh * nb + qi] = cnt;
+}
+
+// Query-wise rule: grid (nb, Hq, Bt), kRowThreads threads, dynamic shared
+// memory for P = (smallest power of two >= nb) 64-bit keys and P flags.
+// Query-aware heads only (others return at once); row qi of head bh:
+//   key_j = (bit pattern of score j) << 32 | (0xFFFFFFFF - j), so a descending
+//   sort is the rule's order (score descending, then j ascending), with the
+//   padding keys (0) last;
+//   k_gamma = smallest k whose exact uint64 mass prefix reaches
+//   (double)gamma * (double)W; k = clamp(k_gamma, lo, hi) with the row's
+//   budgets; the row keeps the first k sorted entries and its diagonal.
+constexpr int kRowThreads = 256;
+
+__global__ void __launch_bounds__(kRowThreads) select_rows_qa_kernel(
+    const int32_t *__restrict__ pattern, const float *__restrict__ map, int nb, int pmax,
+    float gamma, int row_lo, int row_hi, int32_t *__restrict__ counts,
+    int32_t *__restrict__ indices) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  unsigned long long *keys = reinterpret_cast<unsigned long long *>(smem_raw);
+  uint8_t *flag = smem_raw + size_t(pmax) * 8;
+  __shared__ unsigned long long part[kRowThreads];
+  __shared__ int kmin;
+  __shared__ int wcount[kRowThreads / 32];
+  const int qi = blockIdx.x, tid = threadIdx.x;
+  const size_t bh = size_t(blockIdx.z) * gridDim.y + blockIdx.y;
+  if (pattern[bh] != FP_PATTERN_QA) return;
+  const int n = qi + 1;
+  int P = 1;
+  while (P < n) P <<= 1;
+  const float *mrow = map + bh * (size_t(nb) * (nb + 1) / 2) + size_t(qi) * (qi + 1) / 2;
+  for (int i = tid; i < P; i += kRowThreads) {
+    keys[i] = i < n ? ((unsigned long long)score_bits(mrow[i]) << 32) | (0xFFFFFFFFu - uint32_t(i))
+                    : 0ull;
+    flag[i] = 0;
+  }
+  if (tid == 0) kmin = n;
+  __syncthreads();
+  // bitonic sort, descending
+  for (int k = 2; k <= P; k <<= 1)
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      for (int i = tid; i < P; i += kRowThreads) {
+        const int ixj = i ^ j;
+        if (ixj > i) {
+          const unsigned long long x = keys[i], y = keys[ixj];
+          const bool desc = (i & k) == 0;
+          if (desc ? (x < y) : (x > y)) {
+            keys[i] = y;
+            keys[ixj] = x;
+          }
+        }
+      }
+      __syncthreads();
+    }
+  // exact mass prefix: thread t owns sorted entries [t*per, (t+1)*per)
+  const int per = (n + kRowThreads - 1) / kRowThreads;
+  const int e0 = min(n, tid * per), e1 = min(n, e0 + per);
+  unsigned long long loc = 0;
+  for (int e = e0; e < e1; ++e) loc += score_mass(uint32_t(keys[e] >> 32));
+  part[tid] = loc;
+  __syncthreads();
+  // inclusive scan of the thread sums (fixed order)
+  for (int off = 1; off < kRowThreads; off <<= 1) {
+    const unsigned long long v = tid >= off ? part[tid - off] : 0ull;
+    __syncthreads();
+    part[tid] += v;
+    __syncthreads();
+  }
+  const unsigned long long total = part[kRowThreads - 1];
+  int kg;
+  if (gamma >= 1.f) {
+    kg = n;
+  } else {
+    const double target = (double)gamma * (double)total;
+    if (target <= 0.0) {
+      kg = 0;
+    } else {
+      unsigned long long cum = tid > 0 ? part[tid - 1] : 0ull;
+      for (int e = e0; e < e1; ++e) {
+        cum += score_mass(uint32_t(keys[e] >> 32));
+        if ((double)cum >= target) {
+          atomicMin(&kmin, e + 1);
+          break;
+        }
+      }
+      __syncthreads();
+      kg = kmin;
+    }
+  }
+  int lo = row_lo < n ? row_lo : n;
+  const int hi = row_hi < 0 ? n : (row_hi < n ? row_hi : n);
+  lo = lo < hi ? lo : hi;
+  const int kc = kg < lo ? lo : (kg > hi ? hi : kg);
+  for (int e = tid; e < kc; e += kRowThreads) flag[0xFFFFFFFFu - uint32_t(keys[e])] = 1;
+  if (tid == 0) flag[qi] = 1;
+  __syncthreads();
+  // ascending compaction of the flags
+  int32_t *out = indices + (bh * nb + qi) * size_t(nb);
+  const int warp = tid / 32, lane = tid % 32;
+  int base = 0;
+  for (int j0 = 0; j0 < n; j0 += kRowThreads) {
+    const int j = j0 + tid;
+    const bool keep = j < n && flag[j];
+    const unsigned bal = __ballot_sync(0xffffffffu, keep);
+    if (lane == 0) wcount[warp] = __popc(bal);
+    __syncthreads();
+    int before = base;
+    for (int w = 0; w < warp; ++w) before += wcount[w];
+    if (keep) out[before + __popc(bal & ((1u << lane) - 1u))] = j;
+    for (int w = 0; w < kRowThreads / 32; ++w) base += wcount[w];
+    __syncthreads();
+  }
+  if (tid == 0) counts[bh * nb + qi] = base;
+}
+
+size_t rows_qa_smem(int nb, int *pmax) {
+  int p = 1;
+  while (p < nb) p <<= 1;
+  *pmax = p;
+  return size_t(p) * 9;
 }
 
 __global__ void stats_kernel(const int32_t *__restrict__ counts,
@@ -488,9 +616,15 @@ cudaError_t launch_select(const Dims &D, float gamma, const SelectBudgets &bud,
   cudaFuncSetAttribute(select_head_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   select_head_kernel<<<dim3(kCluster * D.hq, D.bt), kCThreads, smem, st>>>(
       pattern, map, vert, slash, D.n, D.nb, D.bs, gamma, bud.qa_lo, bud.qa_hi, bud.vs_lo,
-      bud.vs_hi, sel, cf, df);
-  emit_rows_kernel<<<dim3((D.nb + 7) / 8, D.hq, D.bt), 256, 0, st>>>(pattern, map, D.nb, sel, cf,
-                                                                    df, counts, indices);
+      bud.vs_hi, bud.qa_mode, sel, cf, df);
+  emit_rows_kernel<<<dim3((D.nb + 7) / 8, D.hq, D.bt), 256, 0, st>>>(
+      pattern, map, D.nb, sel, cf, df, bud.qa_mode, counts, indices);
+  if (bud.qa_mode == FP_QA_QUERYWISE) {
+    int pmax;
+    const size_t rsm = rows_qa_smem(D.nb, &pmax);
+    select_rows_qa_kernel<<<dim3(D.nb, D.hq, D.bt), kRowThreads, rsm, st>>>(
+        pattern, map, D.nb, pmax, gamma, bud.row_lo, bud.row_hi, counts, indices);
+  }
   return cudaGetLastError();
 }
 
@@ -553,9 +687,15 @@ cudaError_t launch_select_noalloc(const Dims &D, float gamma, const SelectBudget
   cudaFuncSetAttribute(select_head_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   select_head_kernel<<<dim3(kCluster * D.hq, D.bt), kCThreads, smem, st>>>(
       pattern, map, vert, slash, D.n, D.nb, D.bs, gamma, bud.qa_lo, bud.qa_hi, bud.vs_lo,
-      bud.vs_hi, sel, cf, df);
-  emit_rows_kernel<<<dim3((D.nb + 7) / 8, D.hq, D.bt), 256, 0, st>>>(pattern, map, D.nb, sel, cf,
-                                                                    df, counts, indices);
+      bud.vs_hi, bud.qa_mode, sel, cf, df);
+  emit_rows_kernel<<<dim3((D.nb + 7) / 8, D.hq, D.bt), 256, 0, st>>>(
+      pattern, map, D.nb, sel, cf, df, bud.qa_mode, counts, indices);
+  if (bud.qa_mode == FP_QA_QUERYWISE) {
+    int pmax;
+    const size_t rsm = rows_qa_smem(D.nb, &pmax);
+    select_rows_qa_kernel<<<dim3(D.nb, D.hq, D.bt), kRowThreads, rsm, st>>>(
+        pattern, map, D.nb, pmax, gamma, bud.row_lo, bud.row_hi, counts, indices);
+  }
   return cudaGetLastError();
 }
 

@@ -61,6 +61,7 @@ class Workload:
     n_random_vs_keys: int = 8
     n_planted_blocks: int = 3
     fixed_kinds: tuple | None = None  # per kv head: "qa" / "vs" (overrides p_vs)
+    qa_mode: int = 0  # query-aware heads: 0 flattened map, 1 query-wise rows
 
     def replace(self, **kw) -> "Workload":
         return dataclasses.replace(self, **kw)

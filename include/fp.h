@@ -82,7 +82,22 @@ typedef struct {
   float tau;       /* JS-distance threshold, >= 0; tau == 0 disables query-aware mode   */
   int min_budget;  /* tokens per query row, >= 0 (0: no minimum)                        */
   int max_budget;  /* tokens per query row; <= 0: uncapped                              */
+  int qa_mode;     /* query-aware heads: FP_QA_FLATTENED (0, the default) or
+                      FP_QA_QUERYWISE (1); anything else is FP_ERR_PARAM           */
 } fp_params;
+
+/*
+ * Selection rule for query-aware heads (atlas.scime.ai summary, "Measured
+ * effects": the flattened estimated map, and query-wise index selection as the
+ * alternative the ablation compares):
+ *   FP_QA_FLATTENED  one rule over the whole flattened causal map of the head,
+ *                    budgets nb * ceil(min/B) .. nb * floor(max/B) block pairs;
+ *   FP_QA_QUERYWISE  one rule per query-block row i over A[i, 0..i] with the
+ *                    row's own total, budgets min(i+1, ceil(min/B)) ..
+ *                    min(i+1, floor(max/B)) blocks (i+1 when uncapped).
+ * Both keep every row's diagonal block.  Vertical-slash heads are unaffected.
+ */
+enum { FP_QA_FLATTENED = 0, FP_QA_QUERYWISE = 1 };
 
 enum { FP_PATTERN_QA = 0, FP_PATTERN_VS = 1 };
 

@@ -22,8 +22,8 @@ Sources (cited by page and section):
   [ablations] Same summary, table "Measured effects reported in the paper":
               tau = 0 disables query-aware mode; min budget (1024/2048 tokens);
               max budget (8k/32k tokens); block size 64/128; last (not middle)
-              representative queries; the flattened estimated map (not
-              query-wise selection).
+              representative queries; the flattened estimated map, with
+              query-wise selection as the alternative the ablation compares.
 
 Where the pages are silent the plainest reading is taken; each is named at the
 function that makes it.  Floating point runs in float64 except where a float
@@ -49,6 +49,8 @@ import numpy as np
 
 PATTERN_QA = 0
 PATTERN_VS = 1
+QA_FLATTENED = 0  # query-aware heads: one cumulative rule over the flattened map
+QA_QUERYWISE = 1  # query-aware heads: one cumulative rule per query-block row
 QUANT_SCALE = 2.0 ** 32  # selection masses are integers: ceil(score * 2^32)
 
 
@@ -308,6 +310,39 @@ def select_head_qa(map_row_f32: np.ndarray, n_blocks: int, block: int, gamma: fl
     return [sorted(r) for r in rows]
 
 
+def qa_row_budget(row: int, block: int, min_budget: int, max_budget: int):
+    """(lo, hi) for row ``row`` of a query-wise head, counted in its row+1 key blocks.
+
+    Reading: the same tokens-per-query-row budgets as the flattened rule,
+    applied to the one row: ceil(min_budget / B) blocks at least and
+    floor(max_budget / B) at most, never more than the row holds.
+    """
+    n = row + 1
+    lo = min(n, -(-max(min_budget, 0) // block))
+    hi = n if max_budget <= 0 else min(n, max_budget // block)
+    return min(lo, hi), hi
+
+
+def select_head_qa_querywise(map_row_f32: np.ndarray, n_blocks: int, block: int,
+                             gamma: float, min_budget: int, max_budget: int):
+    """Per-row block lists of one query-aware head, selected row by row.
+
+    [ablations] "query-wise index selection instead of flattening the
+    estimated attention map": the cumulative rule (cumulative_select, same
+    order, masses and target) runs on each query-block row i of the map,
+    A[i, 0..i], with the row's own total, and the row's budgets from
+    qa_row_budget; every row also keeps its diagonal block.
+    """
+    m = np.asarray(map_row_f32, dtype=np.float32)
+    rows = []
+    for i in range(n_blocks):
+        seg = m[tri_offset(i): tri_offset(i) + i + 1]
+        lo, hi = qa_row_budget(i, block, min_budget, max_budget)
+        chosen = cumulative_select(seg, gamma, lo, hi)
+        rows.append(sorted(set(chosen.tolist()) | {i}))
+    return rows
+
+
 def select_head_vs(vert_f32: np.ndarray, slash_f32: np.ndarray, n_blocks: int, block: int,
                    gamma: float, min_budget: int, max_budget: int):
     """Per-row block lists of one vertical-slash head.
@@ -335,11 +370,12 @@ def select_head_vs(vert_f32: np.ndarray, slash_f32: np.ndarray, n_blocks: int, b
 
 
 def select(pattern_arr, amap, vert, slash, n_blocks: int, block: int, gamma: float,
-           min_budget: int, max_budget: int):
+           min_budget: int, max_budget: int, qa_mode: int = QA_FLATTENED):
     """Block lists for every (batch, head): counts [Bt,Hq,nb], indices [Bt,Hq,nb,nb].
 
     Scores are taken as float32 (the precision the kernels decide in).  Unused
-    tail entries of each indices row are set to -1 here.
+    tail entries of each indices row are set to -1 here.  qa_mode picks the
+    flattened or the query-wise rule for query-aware heads.
     """
     pat = np.asarray(pattern_arr)
     m32, v32, s32 = _f32(amap), _f32(vert), _f32(slash)
@@ -348,7 +384,10 @@ def select(pattern_arr, amap, vert, slash, n_blocks: int, block: int, gamma: flo
     indices = np.full((bt, hq, n_blocks, n_blocks), -1, dtype=np.int32)
     for b in range(bt):
         for h in range(hq):
-            if pat[b, h] == PATTERN_QA:
+            if pat[b, h] == PATTERN_QA and qa_mode == QA_QUERYWISE:
+                rows = select_head_qa_querywise(m32[b, h], n_blocks, block, gamma, min_budget,
+                                                max_budget)
+            elif pat[b, h] == PATTERN_QA:
                 rows = select_head_qa(m32[b, h], n_blocks, block, gamma, min_budget, max_budget)
             else:
                 rows = select_head_vs(v32[b, h], s32[b, h], n_blocks, block, gamma,
@@ -419,7 +458,8 @@ def dense_attention(q, k, v, block: int, heads=None, q_blocks=None):
 # ---------------------------------------------------------------- pipeline --
 
 def flexprefill(q, k, v, block: int, gamma: float, tau: float, min_budget: int,
-                max_budget: int, attention: bool = True, heads=None, q_blocks=None):
+                max_budget: int, attention: bool = True, heads=None, q_blocks=None,
+                qa_mode: int = QA_FLATTENED):
     """Whole hot path: estimate -> pattern -> select -> sparse attention.
 
     The selection stage sees float32 copies of the estimate (the precision the
@@ -431,7 +471,7 @@ def flexprefill(q, k, v, block: int, gamma: float, tau: float, min_budget: int,
     djs, pat = pattern(e32["est_last"], e32["true_last"], tau)
     nb = _f64(q).shape[2] // block
     counts, indices = select(pat, e32["map"], e32["vert"], e32["slash"], nb, block, gamma,
-                             min_budget, max_budget)
+                             min_budget, max_budget, qa_mode)
     res = dict(est)
     res.update(djs=djs, pattern=pat, counts=counts, indices=indices)
     if attention:

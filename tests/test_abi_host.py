@@ -100,6 +100,16 @@ def test_bad_params_rejected(L, gamma, tau, lo, code):
                        None) == code
 
 
+@pytest.mark.parametrize("qa_mode", [-1, 2, 7])
+def test_bad_qa_mode_rejected(L, qa_mode):
+    s = shape()
+    p = ops.make_params(0.9, 0.1, 0, 0, qa_mode)
+    assert L.fp_select(ctypes.byref(s), ctypes.byref(p), *([FAKE] * 6), FAKE, 1 << 40,
+                       None) == ops.STATUS_CODES["FP_ERR_PARAM"]
+    assert L.fp_pattern(ctypes.byref(s), ctypes.byref(p), FAKE, FAKE, FAKE, FAKE,
+                        None) == ops.STATUS_CODES["FP_ERR_PARAM"]
+
+
 def test_workspace_checks(L):
     s = shape()
     need = ops.fp_workspace_size(s, ops.FP_CALL_ESTIMATE)

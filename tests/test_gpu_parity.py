@@ -88,14 +88,14 @@ def test_pattern_parity(tau):
         assert (pat.cpu().numpy() == oracle.PATTERN_VS).all()
 
 
-def _select_case(w, est, pat, gamma, lo, hi):
+def _select_case(w, est, pat, gamma, lo, hi, qa_mode=0):
     s = ops.fp_shape(w.batch, w.n_q_heads, w.n_kv_heads, w.seq_len, w.head_dim, w.block_size,
                      ops.FP_BF16 if w.dtype == "bf16" else ops.FP_F32)
-    p = ops.make_params(gamma, 0.1, lo, hi)
+    p = ops.make_params(gamma, 0.1, lo, hi, qa_mode)
     counts, indices = ops.select(s, p, pat, est["map"], est["vert"], est["slash"])
     torch.cuda.synchronize()
     oc, oi = oracle.select(pat.cpu().numpy(), _np(est["map"]), _np(est["vert"]),
-                           _np(est["slash"]), w.n_blocks, w.block_size, gamma, lo, hi)
+                           _np(est["slash"]), w.n_blocks, w.block_size, gamma, lo, hi, qa_mode)
     gc = counts.cpu().numpy()
     gi = indices.cpu().numpy()
     np.testing.assert_array_equal(gc, oc)
@@ -125,6 +125,41 @@ def test_select_bit_exact(name, mode, gamma, lo, hi):
     gc = _select_case(w, est, pat, gamma, lo, hi)
     if gamma >= 1.0:
         assert (gc == np.arange(1, w.n_blocks + 1)).all()
+
+
+@pytest.mark.parametrize("name", ["tiny_n1024", "llama8b_n8192"])
+@pytest.mark.parametrize("mode", ["natural", "alternate"])
+@pytest.mark.parametrize("gamma,lo,hi", [(0.95, 1024, 0), (0.9, 0, 0), (0.9, 2048, 8192),
+                                         (0.5, 0, 1024), (1.0, 0, 0), (0.999, 256, 0),
+                                         (0.9, 0, 100)])
+def test_select_querywise_bit_exact(name, mode, gamma, lo, hi):
+    """Query-wise rule for query-aware heads (one cumulative rule per map row)."""
+    w, inp, d = _inputs(name)
+    est = ops.estimate(d["q"], d["k"], w.block_size)
+    s = ops.make_shape(d["q"], d["k"], w.block_size)
+    _, pat = ops.pattern(s, ops.make_params(0.95, 0.1), est["est_last"], est["true_last"])
+    if mode == "alternate":
+        pat = (torch.arange(pat.numel(), device=DEV, dtype=torch.int32) % 2).reshape(pat.shape)
+    gc = _select_case(w, est, pat, gamma, lo, hi, ops.FP_QA_QUERYWISE)
+    if gamma >= 1.0:
+        assert (gc == np.arange(1, w.n_blocks + 1)).all()
+
+
+def test_select_querywise_ties_and_long_rows():
+    """Hand-made map rows with exact ties and zeros, nb = 256 (rows up to 256
+    entries, several sort stages past one thread's share)."""
+    w = synth.WORKLOADS["llama8b_n8192"].replace(seq_len=256 * 64, block_size=64, n_q_heads=2,
+                                                 n_kv_heads=1)
+    nb, n = w.n_blocks, w.seq_len
+    t_pairs = nb * (nb + 1) // 2
+    g = torch.Generator().manual_seed(9)
+    levels = torch.tensor([0.0, 1e-4, 3e-4, 1e-3, 2.0 ** -20], dtype=torch.float32)
+    mp = levels[torch.randint(0, 5, (1, 2, t_pairs), generator=g)]
+    est = {"map": mp.to(DEV), "vert": torch.rand(1, 2, n).to(DEV),
+           "slash": torch.rand(1, 2, n).to(DEV)}
+    pat = torch.zeros(1, 2, dtype=torch.int32, device=DEV)
+    for gamma, lo, hi in [(0.9, 0, 0), (0.7, 640, 1280), (0.3, 0, 0), (0.99, 0, 64)]:
+        _select_case(w, est, pat, gamma, lo, hi, ops.FP_QA_QUERYWISE)
 
 
 def test_select_ties_and_zero_scores():
@@ -250,6 +285,30 @@ def test_prefill_matches_stages_and_host_path():
     assert ops.fp_prefill_attn_host(s, res["params"], qh, kh, vh, oh, ws) == 0
     torch.cuda.synchronize()
     assert torch.equal(oh, res["out"].cpu())
+
+
+def test_prefill_querywise_pipeline():
+    """The whole path with the query-wise rule: the selection against the
+    oracle's query-wise rule on the same estimate, sampled attention against
+    the oracle, and fp_prefill_attn against the staged calls."""
+    w, inp, d = _inputs("llama8b_n8192")
+    s = ops.make_shape(d["q"], d["k"], w.block_size)
+    p = ops.make_params(w.gamma, w.tau, w.min_budget, w.max_budget, ops.FP_QA_QUERYWISE)
+    est = ops.estimate(d["q"], d["k"], w.block_size)
+    _, pat = ops.pattern(s, p, est["est_last"], est["true_last"])
+    counts, indices = ops.select(s, p, pat, est["map"], est["vert"], est["slash"])
+    out, lse = ops.sparse_attn(d["q"], d["k"], d["v"], counts, indices, w.block_size)
+    torch.cuda.synchronize()
+    oc, _ = oracle.select(pat.cpu().numpy(), _np(est["map"]), _np(est["vert"]), _np(est["slash"]),
+                          w.n_blocks, w.block_size, w.gamma, w.min_budget, w.max_budget,
+                          oracle.QA_QUERYWISE)
+    np.testing.assert_array_equal(counts.cpu().numpy(), oc)
+    res = dict(counts=counts, indices=indices, out=out, lse=lse)
+    _attn_check(inp, res, w, 2e-2, 2e-3, heads=[0, 13, 31], q_blocks=[0, 17, 63])
+    out2, _, stats = ops.prefill_attn(d["q"], d["k"], d["v"], w.block_size, p)
+    torch.cuda.synchronize()
+    assert torch.equal(out2, out)
+    assert int(stats[0]) == int(counts.sum())
 
 
 def test_edge_empty_rows_and_device_checks():
