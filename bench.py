@@ -188,7 +188,7 @@ def cpu_oracle_sample(w: synth.Workload, heads=(0,), budget_s: float = 10.0,
     _, pat = oracle.pattern(e32["est_last"], e32["true_last"], w.tau)
     counts, indices = oracle.select(pat, e32["map"], e32["vert"], e32["slash"], w.n_blocks,
                                     w.block_size, w.gamma, w.min_budget, w.max_budget,
-                                    w.qa_mode)
+                                    w.qa_mode, w.vs_mode)
     t2 = time.perf_counter()
     nb = w.n_blocks
     order = [int(x) for x in np.random.default_rng(0).permutation(nb)]
@@ -230,6 +230,7 @@ def workload_config(w: synth.Workload, ws: int) -> dict:
             "head_dim": w.head_dim, "block_size": w.block_size, "gamma": w.gamma, "tau": w.tau,
             "min_budget": w.min_budget, "max_budget": w.max_budget,
             "qa_selection": "query-wise" if w.qa_mode == 1 else "flattened",
+            "vs_lines": "blocks" if w.vs_mode == 1 else "tokens",
             "parallelism": f"independent layers x{ws}" if ws > 1 else "single GPU",
             "l2": "no flush: every step streams Q (1.07 GB at 128k) and K/V, inputs larger "
                   "than the 126 MB L2"}
@@ -275,7 +276,7 @@ def run_ours(args, w, ws, rank, local):
     hkv, bs = k.shape[1], w.block_size
     nb = n // bs
     s = ops.make_shape(q, k, bs)
-    p = ops.make_params(w.gamma, w.tau, w.min_budget, w.max_budget, w.qa_mode)
+    p = ops.make_params(w.gamma, w.tau, w.min_budget, w.max_budget, w.qa_mode, w.vs_mode)
     f32 = dict(dtype=torch.float32, device=dev)
     qbar = torch.empty(bt, hq, nb, d, **f32)
     kbar = torch.empty(bt, hkv, nb, d, **f32)
@@ -433,6 +434,8 @@ def main():
     ap.add_argument("--max-budget", type=int)
     ap.add_argument("--qa-mode", choices=["flattened", "query-wise"],
                     help="selection rule for query-aware heads (default: flattened)")
+    ap.add_argument("--vs-mode", choices=["tokens", "blocks"],
+                    help="line granularity for vertical-slash heads (default: tokens)")
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
@@ -447,7 +450,9 @@ def main():
                               ("min_budget", args.min_budget),
                               ("max_budget", args.max_budget),
                               ("qa_mode", None if args.qa_mode is None
-                               else int(args.qa_mode == "query-wise"))) if v is not None}
+                               else int(args.qa_mode == "query-wise")),
+                              ("vs_mode", None if args.vs_mode is None
+                               else int(args.vs_mode == "blocks"))) if v is not None}
     if over:
         w = w.replace(**over)
     ws, rank, local = dist_setup()

@@ -63,6 +63,7 @@ fp_status check_params(const fp_params *p) {
   if (!(p->tau >= 0.f) || isinf(p->tau)) return FP_ERR_PARAM;
   if (p->min_budget < 0) return FP_ERR_PARAM;
   if (p->qa_mode != FP_QA_FLATTENED && p->qa_mode != FP_QA_QUERYWISE) return FP_ERR_PARAM;
+  if (p->vs_mode != FP_VS_TOKENS && p->vs_mode != FP_VS_BLOCKS) return FP_ERR_PARAM;
   return FP_OK;
 }
 
@@ -82,6 +83,13 @@ SelectBudgets budgets(const Dims &D, const fp_params &p) {
   b.qa_mode = p.qa_mode;
   b.row_lo = int((p.min_budget + bs - 1) / bs);
   b.row_hi = p.max_budget <= 0 ? -1 : int(p.max_budget / bs);
+  b.vs_mode = p.vs_mode;
+  long long blo = (p.min_budget + bs - 1) / bs;
+  if (blo > nb) blo = nb;
+  long long bhi = p.max_budget <= 0 ? nb : p.max_budget / bs;
+  if (bhi > nb) bhi = nb;
+  b.vsb_lo = int(blo < bhi ? blo : bhi);
+  b.vsb_hi = int(bhi);
   return b;
 }
 

@@ -62,6 +62,8 @@ struct SelectBudgets {
   int qa_mode;             // FP_QA_FLATTENED or FP_QA_QUERYWISE
   int row_lo, row_hi;      // query-wise rule: blocks per row before the row-length
                            // cap; row_hi < 0 means uncapped
+  int vs_mode;             // FP_VS_TOKENS or FP_VS_BLOCKS
+  int vsb_lo, vsb_hi;      // block-pooled lines: budgets in blocks
 };
 size_t select_ws_bytes(const Dims &D);
 cudaError_t launch_select(const Dims &D, float gamma, const SelectBudgets &bud,

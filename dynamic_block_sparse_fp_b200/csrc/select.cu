@@ -27,6 +27,11 @@
 // select_rows_qa_kernel gives each (row, head) one CTA, which sorts the row's
 // (bit pattern, index) keys in shared memory, finds k by an exact uint64
 // prefix sum of the masses, and writes the row's list itself.
+//
+// Block-pooled lines for vertical-slash heads (FP_VS_BLOCKS): pool_lines_kernel
+// sums vert per key block and slash per block distance into nb-entry lists,
+// which select_head_kernel then selects as lines of a sequence of nb tokens
+// with block size 1 (a column is a key block, an offset one block distance).
 #include <cooperative_groups.h>
 
 #include "fp_internal.cuh"
@@ -447,6 +452,29 @@ __global__ void __launch_bounds__(256) emit_rows_kernel(
   if (lane == 0) counts[bh * nb + qi] = cnt;
 }
 
+// Block-pooled lines for vertical-slash heads (FP_VS_BLOCKS): grid
+// (ceil(nb/256), Hq, Bt), 256 threads; thread c of head bh writes
+// pv[bh][c] = sum of vert[bh][c*B .. c*B+B-1] and ps[bh][c] likewise for slash,
+// each summed in double, one add at a time in ascending order, and rounded to
+// float once.  Query-aware heads are skipped.
+__global__ void __launch_bounds__(256) pool_lines_kernel(
+    const int32_t *__restrict__ pattern, const float *__restrict__ vert,
+    const float *__restrict__ slash, int n, int nb, int bs, float *__restrict__ pv,
+    float *__restrict__ ps) {
+  const int c = blockIdx.x * 256 + threadIdx.x;
+  const size_t bh = size_t(blockIdx.z) * gridDim.y + blockIdx.y;
+  if (c >= nb || pattern[bh] == FP_PATTERN_QA) return;
+  const float *v = vert + bh * n + size_t(c) * bs;
+  const float *s = slash + bh * n + size_t(c) * bs;
+  double av = 0.0, as = 0.0;
+  for (int t = 0; t < bs; ++t) {
+    av += (double)v[t];
+    as += (double)s[t];
+  }
+  pv[bh * nb + c] = __double2float_rn(av);
+  ps[bh * nb + c] = __double2float_rn(as);
+}
+
 // Query-wise rule: grid (nb, Hq, Bt), kRowThreads threads, dynamic shared
 // memory for P = (smallest power of two >= nb) 64-bit keys and P flags.
 // Query-aware heads only (others return at once); row qi of head bh:
@@ -614,9 +642,21 @@ cudaError_t launch_select(const Dims &D, float gamma, const SelectBudgets &bud,
   uint8_t *df = c.take<uint8_t>(heads * D.nb);
   const int smem = int(sizeof(SelSmem));
   cudaFuncSetAttribute(select_head_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  select_head_kernel<<<dim3(kCluster * D.hq, D.bt), kCThreads, smem, st>>>(
-      pattern, map, vert, slash, D.n, D.nb, D.bs, gamma, bud.qa_lo, bud.qa_hi, bud.vs_lo,
-      bud.vs_hi, bud.qa_mode, sel, cf, df);
+  if (bud.vs_mode == FP_VS_BLOCKS) {
+    // pooled lines live in the outputs until emit_rows_kernel overwrites them:
+    // vert sums in indices (>= Bt*Hq*nb entries), slash sums in counts
+    float *pv = reinterpret_cast<float *>(indices);
+    float *ps = reinterpret_cast<float *>(counts);
+    pool_lines_kernel<<<dim3((D.nb + 255) / 256, D.hq, D.bt), 256, 0, st>>>(
+        pattern, vert, slash, D.n, D.nb, D.bs, pv, ps);
+    select_head_kernel<<<dim3(kCluster * D.hq, D.bt), kCThreads, smem, st>>>(
+        pattern, map, pv, ps, D.nb, D.nb, 1, gamma, bud.qa_lo, bud.qa_hi, bud.vsb_lo,
+        bud.vsb_hi, bud.qa_mode, sel, cf, df);
+  } else {
+    select_head_kernel<<<dim3(kCluster * D.hq, D.bt), kCThreads, smem, st>>>(
+        pattern, map, vert, slash, D.n, D.nb, D.bs, gamma, bud.qa_lo, bud.qa_hi, bud.vs_lo,
+        bud.vs_hi, bud.qa_mode, sel, cf, df);
+  }
   emit_rows_kernel<<<dim3((D.nb + 7) / 8, D.hq, D.bt), 256, 0, st>>>(
       pattern, map, D.nb, sel, cf, df, bud.qa_mode, counts, indices);
   if (bud.qa_mode == FP_QA_QUERYWISE) {
@@ -685,9 +725,21 @@ cudaError_t launch_select_noalloc(const Dims &D, float gamma, const SelectBudget
   uint8_t *df = c.take<uint8_t>(heads * D.nb);
   const int smem = int(sizeof(SelSmem));
   cudaFuncSetAttribute(select_head_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  select_head_kernel<<<dim3(kCluster * D.hq, D.bt), kCThreads, smem, st>>>(
-      pattern, map, vert, slash, D.n, D.nb, D.bs, gamma, bud.qa_lo, bud.qa_hi, bud.vs_lo,
-      bud.vs_hi, bud.qa_mode, sel, cf, df);
+  if (bud.vs_mode == FP_VS_BLOCKS) {
+    // pooled lines live in the outputs until emit_rows_kernel overwrites them:
+    // vert sums in indices (>= Bt*Hq*nb entries), slash sums in counts
+    float *pv = reinterpret_cast<float *>(indices);
+    float *ps = reinterpret_cast<float *>(counts);
+    pool_lines_kernel<<<dim3((D.nb + 255) / 256, D.hq, D.bt), 256, 0, st>>>(
+        pattern, vert, slash, D.n, D.nb, D.bs, pv, ps);
+    select_head_kernel<<<dim3(kCluster * D.hq, D.bt), kCThreads, smem, st>>>(
+        pattern, map, pv, ps, D.nb, D.nb, 1, gamma, bud.qa_lo, bud.qa_hi, bud.vsb_lo,
+        bud.vsb_hi, bud.qa_mode, sel, cf, df);
+  } else {
+    select_head_kernel<<<dim3(kCluster * D.hq, D.bt), kCThreads, smem, st>>>(
+        pattern, map, vert, slash, D.n, D.nb, D.bs, gamma, bud.qa_lo, bud.qa_hi, bud.vs_lo,
+        bud.vs_hi, bud.qa_mode, sel, cf, df);
+  }
   emit_rows_kernel<<<dim3((D.nb + 7) / 8, D.hq, D.bt), 256, 0, st>>>(
       pattern, map, D.nb, sel, cf, df, bud.qa_mode, counts, indices);
   if (bud.qa_mode == FP_QA_QUERYWISE) {

@@ -25,6 +25,7 @@ from . import build as _build
 FP_BF16, FP_F32 = 0, 1
 FP_PATTERN_QA, FP_PATTERN_VS = 0, 1
 FP_QA_FLATTENED, FP_QA_QUERYWISE = 0, 1
+FP_VS_TOKENS, FP_VS_BLOCKS = 0, 1
 FP_CALL_ESTIMATE, FP_CALL_SELECT, FP_CALL_SPARSE_ATTN, FP_CALL_PREFILL, FP_CALL_PREFILL_HOST = (
     0, 1, 2, 3, 4)
 STATUS = {0: "FP_OK", 1: "FP_ERR_NULL", 2: "FP_ERR_SHAPE", 3: "FP_ERR_DTYPE", 4: "FP_ERR_PARAM",
@@ -45,7 +46,7 @@ class fp_shape(ctypes.Structure):
 class fp_params(ctypes.Structure):
     _fields_ = [("gamma", ctypes.c_float), ("tau", ctypes.c_float),
                 ("min_budget", ctypes.c_int), ("max_budget", ctypes.c_int),
-                ("qa_mode", ctypes.c_int)]
+                ("qa_mode", ctypes.c_int), ("vs_mode", ctypes.c_int)]
 
 
 class FPError(RuntimeError):
@@ -142,8 +143,8 @@ def make_shape(q, k, block_size: int) -> fp_shape:
 
 
 def make_params(gamma: float, tau: float, min_budget: int = 0, max_budget: int = 0,
-                qa_mode: int = 0) -> fp_params:
-    return fp_params(gamma, tau, min_budget, max_budget, qa_mode)
+                qa_mode: int = 0, vs_mode: int = 0) -> fp_params:
+    return fp_params(gamma, tau, min_budget, max_budget, qa_mode, vs_mode)
 
 
 def fp_workspace_size(shape: fp_shape, which_call: int) -> int:

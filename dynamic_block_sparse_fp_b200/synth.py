@@ -62,6 +62,7 @@ class Workload:
     n_planted_blocks: int = 3
     fixed_kinds: tuple | None = None  # per kv head: "qa" / "vs" (overrides p_vs)
     qa_mode: int = 0  # query-aware heads: 0 flattened map, 1 query-wise rows
+    vs_mode: int = 0  # vertical-slash heads: 0 token lines, 1 block-pooled lines
 
     def replace(self, **kw) -> "Workload":
         return dataclasses.replace(self, **kw)

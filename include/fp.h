@@ -84,6 +84,8 @@ typedef struct {
   int max_budget;  /* tokens per query row; <= 0: uncapped                              */
   int qa_mode;     /* query-aware heads: FP_QA_FLATTENED (0, the default) or
                       FP_QA_QUERYWISE (1); anything else is FP_ERR_PARAM           */
+  int vs_mode;     /* vertical-slash heads: FP_VS_TOKENS (0, the default) or
+                      FP_VS_BLOCKS (1); anything else is FP_ERR_PARAM              */
 } fp_params;
 
 /*
@@ -98,6 +100,23 @@ typedef struct {
  * Both keep every row's diagonal block.  Vertical-slash heads are unaffected.
  */
 enum { FP_QA_FLATTENED = 0, FP_QA_QUERYWISE = 1 };
+
+/*
+ * Line granularity for vertical-slash heads (atlas.scime.ai summary,
+ * "Approach": the smallest set of "blocks/lines" reaching gamma):
+ *   FP_VS_TOKENS  lines are tokens: columns t and offsets o are selected from
+ *                 vert[N] and slash[N] with budgets min .. max lines, then
+ *                 column t covers key block t/B and offset o the block
+ *                 distances floor(o/B) and, if B does not divide o, +1;
+ *   FP_VS_BLOCKS  lines are blocks: vert is summed per key block and slash per
+ *                 block distance floor(o/B) (float64, one add at a time in
+ *                 ascending order, rounded to float32 once), and the rule picks
+ *                 key blocks and block distances directly with budgets
+ *                 ceil(min/B) .. floor(max/B) blocks.
+ * With FP_VS_BLOCKS, fp_select uses counts and indices as scratch for the
+ * pooled lines before it writes the lists.
+ */
+enum { FP_VS_TOKENS = 0, FP_VS_BLOCKS = 1 };
 
 enum { FP_PATTERN_QA = 0, FP_PATTERN_VS = 1 };
 

@@ -51,6 +51,8 @@ PATTERN_QA = 0
 PATTERN_VS = 1
 QA_FLATTENED = 0  # query-aware heads: one cumulative rule over the flattened map
 QA_QUERYWISE = 1  # query-aware heads: one cumulative rule per query-block row
+VS_TOKENS = 0     # vertical-slash heads: lines chosen per token, then a block cover
+VS_BLOCKS = 1     # vertical-slash heads: lines pooled per block before the rule
 QUANT_SCALE = 2.0 ** 32  # selection masses are integers: ceil(score * 2^32)
 
 
@@ -369,13 +371,60 @@ def select_head_vs(vert_f32: np.ndarray, slash_f32: np.ndarray, n_blocks: int, b
     return rows
 
 
+def pool_lines(line_f32: np.ndarray, n_blocks: int, block: int) -> np.ndarray:
+    """Block sums of a vertical (per key) or slash (per offset) score line.
+
+    Entry c of the result sums the scores of tokens / offsets c*B .. c*B+B-1:
+    a key block's column mass, or the mass of the offsets whose primary block
+    distance is c (floor(o / B)).  Reading: the sum runs in float64, one add
+    at a time in ascending order, and is rounded to float32 once at the end;
+    the kernels take the same steps, so both select on identical scores.
+    """
+    x = np.asarray(line_f32, dtype=np.float32)
+    out = np.empty(n_blocks, dtype=np.float32)
+    for c in range(n_blocks):
+        acc = 0.0
+        for v in x[c * block: (c + 1) * block].tolist():
+            acc += v
+        out[c] = np.float32(acc)
+    return out
+
+
+def vs_block_budget(n_blocks: int, block: int, min_budget: int, max_budget: int):
+    """(lo, hi) for each pooled line list, counted in blocks (tokens / B)."""
+    lo = min(n_blocks, -(-max(min_budget, 0) // block))
+    hi = n_blocks if max_budget <= 0 else min(n_blocks, max_budget // block)
+    return min(lo, hi), hi
+
+
+def select_head_vs_blocks(vert_f32: np.ndarray, slash_f32: np.ndarray, n_blocks: int,
+                          block: int, gamma: float, min_budget: int, max_budget: int):
+    """Per-row block lists of one vertical-slash head, from block-pooled lines.
+
+    The block-level reading of "blocks/lines" [approach]: the vertical
+    scores are summed per key block and the slash scores per block distance
+    (pool_lines) before the cumulative rule, so the rule and its budgets count
+    whole blocks.  Column block j is kept in every row; block
+    distance d keeps the pairs (qi, qi - d); every row keeps its diagonal.
+    """
+    vb = pool_lines(vert_f32, n_blocks, block)
+    sb = pool_lines(slash_f32, n_blocks, block)
+    lo, hi = vs_block_budget(n_blocks, block, min_budget, max_budget)
+    cols = set(cumulative_select(vb, gamma, lo, hi).tolist())
+    dists = set(cumulative_select(sb, gamma, lo, hi).tolist())
+    return [sorted({j for j in range(qi + 1) if j in cols or (qi - j) in dists} | {qi})
+            for qi in range(n_blocks)]
+
+
 def select(pattern_arr, amap, vert, slash, n_blocks: int, block: int, gamma: float,
-           min_budget: int, max_budget: int, qa_mode: int = QA_FLATTENED):
+           min_budget: int, max_budget: int, qa_mode: int = QA_FLATTENED,
+           vs_mode: int = VS_TOKENS):
     """Block lists for every (batch, head): counts [Bt,Hq,nb], indices [Bt,Hq,nb,nb].
 
     Scores are taken as float32 (the precision the kernels decide in).  Unused
     tail entries of each indices row are set to -1 here.  qa_mode picks the
-    flattened or the query-wise rule for query-aware heads.
+    flattened or the query-wise rule for query-aware heads, vs_mode the token
+    or the block-pooled lines for vertical-slash heads.
     """
     pat = np.asarray(pattern_arr)
     m32, v32, s32 = _f32(amap), _f32(vert), _f32(slash)
@@ -389,6 +438,9 @@ def select(pattern_arr, amap, vert, slash, n_blocks: int, block: int, gamma: flo
                                                 max_budget)
             elif pat[b, h] == PATTERN_QA:
                 rows = select_head_qa(m32[b, h], n_blocks, block, gamma, min_budget, max_budget)
+            elif vs_mode == VS_BLOCKS:
+                rows = select_head_vs_blocks(v32[b, h], s32[b, h], n_blocks, block, gamma,
+                                             min_budget, max_budget)
             else:
                 rows = select_head_vs(v32[b, h], s32[b, h], n_blocks, block, gamma,
                                       min_budget, max_budget)
@@ -459,7 +511,7 @@ def dense_attention(q, k, v, block: int, heads=None, q_blocks=None):
 
 def flexprefill(q, k, v, block: int, gamma: float, tau: float, min_budget: int,
                 max_budget: int, attention: bool = True, heads=None, q_blocks=None,
-                qa_mode: int = QA_FLATTENED):
+                qa_mode: int = QA_FLATTENED, vs_mode: int = VS_TOKENS):
     """Whole hot path: estimate -> pattern -> select -> sparse attention.
 
     The selection stage sees float32 copies of the estimate (the precision the
@@ -471,7 +523,7 @@ def flexprefill(q, k, v, block: int, gamma: float, tau: float, min_budget: int,
     djs, pat = pattern(e32["est_last"], e32["true_last"], tau)
     nb = _f64(q).shape[2] // block
     counts, indices = select(pat, e32["map"], e32["vert"], e32["slash"], nb, block, gamma,
-                             min_budget, max_budget, qa_mode)
+                             min_budget, max_budget, qa_mode, vs_mode)
     res = dict(est)
     res.update(djs=djs, pattern=pat, counts=counts, indices=indices)
     if attention:

@@ -110,6 +110,14 @@ def test_bad_qa_mode_rejected(L, qa_mode):
                         None) == ops.STATUS_CODES["FP_ERR_PARAM"]
 
 
+@pytest.mark.parametrize("vs_mode", [-1, 2])
+def test_bad_vs_mode_rejected(L, vs_mode):
+    s = shape()
+    p = ops.make_params(0.9, 0.1, 0, 0, 0, vs_mode)
+    assert L.fp_select(ctypes.byref(s), ctypes.byref(p), *([FAKE] * 6), FAKE, 1 << 40,
+                       None) == ops.STATUS_CODES["FP_ERR_PARAM"]
+
+
 def test_workspace_checks(L):
     s = shape()
     need = ops.fp_workspace_size(s, ops.FP_CALL_ESTIMATE)

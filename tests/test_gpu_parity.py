@@ -88,14 +88,15 @@ def test_pattern_parity(tau):
         assert (pat.cpu().numpy() == oracle.PATTERN_VS).all()
 
 
-def _select_case(w, est, pat, gamma, lo, hi, qa_mode=0):
+def _select_case(w, est, pat, gamma, lo, hi, qa_mode=0, vs_mode=0):
     s = ops.fp_shape(w.batch, w.n_q_heads, w.n_kv_heads, w.seq_len, w.head_dim, w.block_size,
                      ops.FP_BF16 if w.dtype == "bf16" else ops.FP_F32)
-    p = ops.make_params(gamma, 0.1, lo, hi, qa_mode)
+    p = ops.make_params(gamma, 0.1, lo, hi, qa_mode, vs_mode)
     counts, indices = ops.select(s, p, pat, est["map"], est["vert"], est["slash"])
     torch.cuda.synchronize()
     oc, oi = oracle.select(pat.cpu().numpy(), _np(est["map"]), _np(est["vert"]),
-                           _np(est["slash"]), w.n_blocks, w.block_size, gamma, lo, hi, qa_mode)
+                           _np(est["slash"]), w.n_blocks, w.block_size, gamma, lo, hi, qa_mode,
+                           vs_mode)
     gc = counts.cpu().numpy()
     gi = indices.cpu().numpy()
     np.testing.assert_array_equal(gc, oc)
@@ -160,6 +161,50 @@ def test_select_querywise_ties_and_long_rows():
     pat = torch.zeros(1, 2, dtype=torch.int32, device=DEV)
     for gamma, lo, hi in [(0.9, 0, 0), (0.7, 640, 1280), (0.3, 0, 0), (0.99, 0, 64)]:
         _select_case(w, est, pat, gamma, lo, hi, ops.FP_QA_QUERYWISE)
+
+
+@pytest.mark.parametrize("name", ["tiny_n1024", "llama8b_n8192"])
+@pytest.mark.parametrize("mode", ["all_vs", "alternate"])
+@pytest.mark.parametrize("gamma,lo,hi", [(0.95, 1024, 0), (0.9, 0, 0), (0.9, 2048, 8192),
+                                         (0.5, 0, 1000), (1.0, 0, 0), (0.999, 200, 0)])
+def test_select_vs_blocks_bit_exact(name, mode, gamma, lo, hi):
+    """Block-pooled vertical-slash lines (sums per key block / block distance)."""
+    w, inp, d = _inputs(name)
+    est = ops.estimate(d["q"], d["k"], w.block_size)
+    if mode == "all_vs":
+        pat = torch.full((w.batch, w.n_q_heads), ops.FP_PATTERN_VS, dtype=torch.int32, device=DEV)
+    else:
+        pat = (torch.arange(w.batch * w.n_q_heads, device=DEV, dtype=torch.int32) % 2).reshape(
+            w.batch, w.n_q_heads)
+    for qa_mode in (ops.FP_QA_FLATTENED, ops.FP_QA_QUERYWISE):
+        gc = _select_case(w, est, pat, gamma, lo, hi, qa_mode, ops.FP_VS_BLOCKS)
+    if gamma >= 1.0:
+        assert (gc == np.arange(1, w.n_blocks + 1)).all()
+
+
+def test_prefill_vs_blocks_pipeline():
+    """tau = 0 (every head vertical-slash) with block-pooled lines: the
+    selection against the oracle on the same estimate, sampled attention, and
+    fp_prefill_attn against the staged calls."""
+    w, inp, d = _inputs("llama8b_n8192")
+    s = ops.make_shape(d["q"], d["k"], w.block_size)
+    p = ops.make_params(w.gamma, 0.0, w.min_budget, 4096, 0, ops.FP_VS_BLOCKS)
+    est = ops.estimate(d["q"], d["k"], w.block_size)
+    _, pat = ops.pattern(s, p, est["est_last"], est["true_last"])
+    assert (pat == ops.FP_PATTERN_VS).all()
+    counts, indices = ops.select(s, p, pat, est["map"], est["vert"], est["slash"])
+    out, lse = ops.sparse_attn(d["q"], d["k"], d["v"], counts, indices, w.block_size)
+    torch.cuda.synchronize()
+    oc, _ = oracle.select(pat.cpu().numpy(), _np(est["map"]), _np(est["vert"]), _np(est["slash"]),
+                          w.n_blocks, w.block_size, w.gamma, w.min_budget, 4096,
+                          oracle.QA_FLATTENED, oracle.VS_BLOCKS)
+    np.testing.assert_array_equal(counts.cpu().numpy(), oc)
+    res = dict(counts=counts, indices=indices, out=out, lse=lse)
+    _attn_check(inp, res, w, 2e-2, 2e-3, heads=[1, 30], q_blocks=[5, 40, 63])
+    out2, _, stats = ops.prefill_attn(d["q"], d["k"], d["v"], w.block_size, p)
+    torch.cuda.synchronize()
+    assert torch.equal(out2, out)
+    assert int(stats[0]) == int(counts.sum())
 
 
 def test_select_ties_and_zero_scores():
