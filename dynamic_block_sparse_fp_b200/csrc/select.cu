@@ -136,23 +136,34 @@ __device__ void histogram(const Ctx &cx, const float *__restrict__ s, uint32_t i
   }
   __syncthreads();
   const int lane = threadIdx.x % 32;
-  for (uint32_t base = i0 + (threadIdx.x / 32) * 32; base < i1; base += kCThreads) {
-    const uint32_t i = base + lane;
-    uint32_t bin = 0xFFFFFFFFu;
-    uint64_t w = 0;
-    if (i < i1) {
-      const uint32_t b = score_bits(s[i]);
-      if ((b & pmask) == prefix) {
-        bin = (b >> shift) & (nbins - 1);
-        w = score_mass(b);
-      }
+  // each warp takes kHistU consecutive groups of 32 entries per round and
+  // issues all their loads before using any, so the scan is not one load
+  // latency per 32 entries
+  constexpr uint32_t kHistU = 8;
+  for (uint32_t base = i0 + (threadIdx.x / 32) * 32 * kHistU; base < i1;
+       base += kCThreads * kHistU) {
+    uint32_t bits[kHistU];
+#pragma unroll
+    for (uint32_t u = 0; u < kHistU; ++u) {
+      const uint32_t i = base + u * 32 + lane;
+      bits[u] = i < i1 ? score_bits(s[i]) : 0u;
     }
-    const unsigned peers = __match_any_sync(0xffffffffu, bin);
-    const unsigned lo = __reduce_add_sync(peers, unsigned(w & 0xFFFFFFull));
-    const unsigned hi = __reduce_add_sync(peers, unsigned(w >> 24));
-    if (bin != 0xFFFFFFFFu && lane == __ffs(peers) - 1) {
-      atomicAdd(&sm.hmass[bin], ((unsigned long long)hi << 24) + lo);
-      atomicAdd(&sm.hcnt[bin], unsigned(__popc(peers)));
+#pragma unroll
+    for (uint32_t u = 0; u < kHistU; ++u) {
+      const uint32_t i = base + u * 32 + lane;
+      uint32_t bin = 0xFFFFFFFFu;
+      uint64_t w = 0;
+      if (i < i1 && (bits[u] & pmask) == prefix) {
+        bin = (bits[u] >> shift) & (nbins - 1);
+        w = score_mass(bits[u]);
+      }
+      const unsigned peers = __match_any_sync(0xffffffffu, bin);
+      const unsigned lo = __reduce_add_sync(peers, unsigned(w & 0xFFFFFFull));
+      const unsigned hi = __reduce_add_sync(peers, unsigned(w >> 24));
+      if (bin != 0xFFFFFFFFu && lane == __ffs(peers) - 1) {
+        atomicAdd(&sm.hmass[bin], ((unsigned long long)hi << 24) + lo);
+        atomicAdd(&sm.hcnt[bin], unsigned(__popc(peers)));
+      }
     }
   }
   // merge: rank r sums bins [r*nbins/C, (r+1)*nbins/C) of every rank into rank 0
@@ -272,18 +283,35 @@ __device__ uint32_t descend(const Ctx &cx, const float *s, uint32_t i0, uint32_t
 }
 
 // Index of the m-th (1-based) entry with bit pattern == b, in index order,
-// over the whole list (the slices are in index order across ranks).
+// over the whole list (the slices are in index order across ranks).  Warp w
+// of a rank scans its contiguous chunk of the rank's slice 32 entries at a
+// time (coalesced, kTieU groups in flight) and counts matches by ballot; an
+// exclusive scan over the warps and the ranks' totals place the m-th match,
+// and the warp holding it rescans its chunk to find it.
 __device__ uint32_t tie_index(const Ctx &cx, const float *s, uint32_t n, uint32_t i0,
                               uint32_t i1, uint32_t b, unsigned long long m) {
   SelSmem &sm = *cx.sm;
+  constexpr uint32_t kTieU = 8;
+  const int lane = threadIdx.x % 32, warp = threadIdx.x / 32;
   const uint32_t len = i1 > i0 ? i1 - i0 : 0;
-  const uint32_t per = (len + kCThreads - 1) / kCThreads;
-  const uint32_t t0 = i0 + threadIdx.x * per;
-  const uint32_t t1 = min(i1, t0 + per);
+  const uint32_t per = ((len + kCWarps - 1) / kCWarps + 31u) & ~31u;
+  const uint32_t w0 = min(i1, i0 + uint32_t(warp) * per), w1 = min(i1, w0 + per);
+  auto matches = [&](uint32_t g) -> unsigned {  // ballot of group g (32 entries from w0)
+    const uint32_t i = w0 + g * 32 + lane;
+    return __ballot_sync(0xffffffffu, i < w1 && score_bits(s[i]) == b);
+  };
+  const uint32_t ngroups = (w1 - w0 + 31) / 32;
   unsigned long long c = 0;
-  for (uint32_t i = t0; i < t1; ++i) c += score_bits(s[i]) == b;
+  for (uint32_t g0 = 0; g0 < ngroups; g0 += kTieU) {
+    unsigned bal[kTieU];
+#pragma unroll
+    for (uint32_t u = 0; u < kTieU; ++u) bal[u] = g0 + u < ngroups ? matches(g0 + u) : 0u;
+#pragma unroll
+    for (uint32_t u = 0; u < kTieU; ++u) c += __popc(bal[u]);
+  }
   unsigned long long tot;
-  const unsigned long long e = block_excl_scan(c, sm, &tot);
+  const unsigned long long e = __shfl_sync(0xffffffffu,
+                                           block_excl_scan(lane == 0 ? c : 0ull, sm, &tot), 0);
   if (threadIdx.x == 0) {
     sm.res[4] = tot;
     if (cx.rank == 0) sm.res[5] = n - 1;
@@ -291,13 +319,20 @@ __device__ uint32_t tie_index(const Ctx &cx, const float *s, uint32_t n, uint32_
   cx.cl.sync();
   unsigned long long off = 0;  // matches in the slices of lower ranks
   for (unsigned q = 0; q < cx.rank; ++q) off += cx.peer(q)->res[4];
-  if (off + e < m && m <= off + e + c) {
+  if (off + e < m && m <= off + e + c) {  // warp-uniform
     unsigned long long r = off + e;
-    for (uint32_t i = t0; i < t1; ++i)
-      if (score_bits(s[i]) == b && ++r == m) {
-        cx.peer(0)->res[5] = i;
+    for (uint32_t g = 0; g < ngroups; ++g) {
+      const unsigned bal = matches(g);
+      const unsigned cnt = __popc(bal);
+      if (r + cnt >= m) {
+        // the (m - r)-th set bit of bal
+        unsigned x = bal;
+        for (unsigned long long k = r + 1; k < m; ++k) x &= x - 1;
+        if (lane == 0) cx.peer(0)->res[5] = w0 + g * 32 + uint32_t(__ffs(x) - 1);
         break;
       }
+      r += cnt;
+    }
   }
   cx.cl.sync();
   const uint32_t idx = uint32_t(cx.peer(0)->res[5]);
