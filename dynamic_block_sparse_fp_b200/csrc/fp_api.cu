@@ -4,6 +4,8 @@
 #include <math.h>
 
 #include <algorithm>
+#include <mutex>
+#include <vector>
 
 #include "fp_internal.cuh"
 
@@ -22,6 +24,24 @@ int *device_status_ptr() {
     if (cudaGetSymbolAddress(&p, g_fp_status) == cudaSuccess) ptrs[dev] = static_cast<int *>(p);
   }
   return ptrs[dev];
+}
+
+// The two copy streams fp_prefill_attn_host overlaps its transfers on (host to
+// device, device to host), created once per device on first use and kept
+// for the life of the process, like the status word.
+bool copy_streams(cudaStream_t *in, cudaStream_t *out) {
+  static std::mutex mu;
+  static cudaStream_t s_in[64] = {nullptr}, s_out[64] = {nullptr};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!s_in[dev] && cudaStreamCreateWithFlags(&s_in[dev], cudaStreamNonBlocking) != cudaSuccess)
+    return false;
+  if (!s_out[dev] && cudaStreamCreateWithFlags(&s_out[dev], cudaStreamNonBlocking) != cudaSuccess)
+    return false;
+  *in = s_in[dev];
+  *out = s_out[dev];
+  return true;
 }
 
 namespace {
@@ -137,6 +157,8 @@ struct Prefill {
   int32_t *pattern, *counts, *indices;
   void *stage_ws;
 };
+
+constexpr int kHostUnits = 4;  // fp_prefill_attn_host: pipelined units per batch entry
 
 size_t carve_prefill(const Dims &D, void *ws, Prefill *P) {
   Carver c{static_cast<char *>(ws), 0};
@@ -350,18 +372,75 @@ FP_API fp_status fp_prefill_attn_host(const fp_shape *shape, const fp_params *pa
   char *kd = c.take<char>(kvbytes);
   char *vd = c.take<char>(kvbytes);
   char *od = c.take<char>(qbytes);
-  Prefill P;
-  carve_prefill(D, c.take<char>(carve_prefill(D, nullptr, &P)), &P);
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  if (cudaMemcpyAsync(qd, q_host, qbytes, cudaMemcpyHostToDevice, st) != cudaSuccess ||
-      cudaMemcpyAsync(kd, k_host, kvbytes, cudaMemcpyHostToDevice, st) != cudaSuccess ||
-      cudaMemcpyAsync(vd, v_host, kvbytes, cudaMemcpyHostToDevice, st) != cudaSuccess)
-    return FP_ERR_CUDA;
-  s = run_prefill(D, *params, qd, kd, vd, od, nullptr, nullptr, P, st);
-  if (s != FP_OK) return s;
-  if (cudaMemcpyAsync(out_host, od, qbytes, cudaMemcpyDeviceToHost, st) != cudaSuccess)
-    return FP_ERR_CUDA;
-  return FP_OK;
+  Prefill Pfull;
+  char *pre = c.take<char>(carve_prefill(D, nullptr, &Pfull));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream), sin = nullptr, sout = nullptr;
+  if (!copy_streams(&sin, &sout)) return FP_ERR_CUDA;
+  // Every stage is independent per (batch, kv head) with its query heads, so
+  // the call runs as units of consecutive kv heads (about a quarter of them
+  // per batch entry): the inputs of unit u+1 are copied in while unit u
+  // computes on `stream`, and its output is copied out while unit u+1
+  // computes.  The caller's stream forks to the copy streams and joins them
+  // at the end through events, so `stream` still orders the whole call.
+  const int per_unit = (D.hkv + kHostUnits - 1) / kHostUnits;
+  const int units_per_batch = (D.hkv + per_unit - 1) / per_unit;
+  const int nunits = D.bt * units_per_batch;
+  std::vector<cudaEvent_t> ev;
+  auto event = [&](cudaEvent_t *e) {
+    if (cudaEventCreateWithFlags(e, cudaEventDisableTiming) != cudaSuccess) return false;
+    ev.push_back(*e);
+    return true;
+  };
+  auto finish = [&](fp_status r) {
+    for (cudaEvent_t e : ev) cudaEventDestroy(e);  // released once they complete
+    return r;
+  };
+  cudaEvent_t e_start, e_end;
+  if (!event(&e_start) || cudaEventRecord(e_start, st) != cudaSuccess ||
+      cudaStreamWaitEvent(sin, e_start, 0) != cudaSuccess ||
+      cudaStreamWaitEvent(sout, e_start, 0) != cudaSuccess)
+    return finish(FP_ERR_CUDA);
+  const size_t head_bytes = size_t(D.n) * D.d * eb;
+  const char *qh = static_cast<const char *>(q_host);
+  const char *kh = static_cast<const char *>(k_host);
+  const char *vh = static_cast<const char *>(v_host);
+  char *oh = static_cast<char *>(out_host);
+  for (int u = 0; u < nunits; ++u) {
+    const int b = u / units_per_batch;
+    const int kv0 = (u % units_per_batch) * per_unit;
+    const int nk = std::min(per_unit, D.hkv - kv0);
+    fp_shape us = *shape;
+    us.batch = 1;
+    us.n_kv_heads = nk;
+    us.n_q_heads = nk * D.g;
+    Dims Du;
+    if (check_shape(&us, &Du) != FP_OK) return finish(FP_ERR_SHAPE);
+    const size_t qoff = (size_t(b) * D.hq + size_t(kv0) * D.g) * head_bytes;
+    const size_t kvoff = (size_t(b) * D.hkv + kv0) * head_bytes;
+    const size_t qlen = size_t(nk) * D.g * head_bytes, kvlen = size_t(nk) * head_bytes;
+    cudaEvent_t e_in, e_comp;
+    if (!event(&e_in) || !event(&e_comp) ||
+        cudaMemcpyAsync(qd + qoff, qh + qoff, qlen, cudaMemcpyHostToDevice, sin) != cudaSuccess ||
+        cudaMemcpyAsync(kd + kvoff, kh + kvoff, kvlen, cudaMemcpyHostToDevice, sin) !=
+            cudaSuccess ||
+        cudaMemcpyAsync(vd + kvoff, vh + kvoff, kvlen, cudaMemcpyHostToDevice, sin) !=
+            cudaSuccess ||
+        cudaEventRecord(e_in, sin) != cudaSuccess || cudaStreamWaitEvent(st, e_in, 0) != cudaSuccess)
+      return finish(FP_ERR_CUDA);
+    Prefill Pu;
+    carve_prefill(Du, pre, &Pu);  // units run one after another on `stream`
+    const fp_status r = run_prefill(Du, *params, qd + qoff, kd + kvoff, vd + kvoff, od + qoff,
+                                    nullptr, nullptr, Pu, st);
+    if (r != FP_OK) return finish(r);
+    if (cudaEventRecord(e_comp, st) != cudaSuccess ||
+        cudaStreamWaitEvent(sout, e_comp, 0) != cudaSuccess ||
+        cudaMemcpyAsync(oh + qoff, od + qoff, qlen, cudaMemcpyDeviceToHost, sout) != cudaSuccess)
+      return finish(FP_ERR_CUDA);
+  }
+  if (!event(&e_end) || cudaEventRecord(e_end, sout) != cudaSuccess ||
+      cudaStreamWaitEvent(st, e_end, 0) != cudaSuccess)
+    return finish(FP_ERR_CUDA);
+  return finish(FP_OK);
 }
 
 FP_API fp_status fp_last_device_status(fp_stream_t stream) {

@@ -270,9 +270,17 @@ fp_status fp_prefill_attn(const fp_shape *shape, const fp_params *params,
  * fp_prefill_attn_host -- fp_prefill_attn on HOST buffers: copies q, k, v
  * to device memory inside `ws` (fp_workspace_size(shape,
  * FP_CALL_PREFILL_HOST) bytes), runs the path and copies the output back to
- * out_host, all enqueued on `stream` (one cudaMemcpyAsync per buffer; page-
- * locked host memory makes the copies asynchronous).  The host buffers must
- * stay valid until the stream reaches the end of the call.
+ * out_host.  Every stage is independent per (batch entry, kv head), so the
+ * call runs as units of about a quarter of the kv heads of one batch entry:
+ * the inputs of a unit are copied in (one cudaMemcpyAsync per buffer slice)
+ * while the previous unit computes on `stream`, and each unit's output is
+ * copied out while the next one computes.  The copies run on two streams of
+ * the library's own, created once per device on first use and kept until the
+ * process exits; `stream` forks to them and joins them through events, so
+ * work enqueued on `stream` after this call sees the finished output.
+ * Page-locked host memory makes the copies asynchronous and lets them
+ * overlap.  The host buffers must stay valid until `stream` reaches the end
+ * of the call.  The result is bitwise that of fp_prefill_attn.
  */
 fp_status fp_prefill_attn_host(const fp_shape *shape, const fp_params *params,
                                const void *q_host, const void *k_host,

@@ -356,6 +356,25 @@ def test_prefill_querywise_pipeline():
     assert int(stats[0]) == int(counts.sum())
 
 
+def test_host_path_batch2_fp32_matches_device_path():
+    """fp_prefill_attn_host runs as pipelined units of (batch entry, kv heads):
+    with two batch entries and two kv heads (four units) its output must be
+    bitwise the device path's."""
+    w = synth.WORKLOADS["tiny_n1024"].replace(batch=2)
+    inp = synth.make_inputs(w)
+    d = {x: inp[x].to(DEV) for x in ("q", "k", "v")}
+    s = ops.make_shape(d["q"], d["k"], w.block_size)
+    p = ops.make_params(w.gamma, w.tau, w.min_budget, w.max_budget)
+    out, _, _ = ops.prefill_attn(d["q"], d["k"], d["v"], w.block_size, p)
+    qh, kh, vh = (inp[x].contiguous().pin_memory() for x in ("q", "k", "v"))
+    oh = torch.empty_like(qh).pin_memory()
+    ws = ops.workspace(s, ops.FP_CALL_PREFILL_HOST, DEV)
+    assert ops.fp_prefill_attn_host(s, p, qh, kh, vh, oh, ws) == 0
+    torch.cuda.synchronize()
+    assert torch.equal(oh, out.cpu())
+    assert ops.fp_last_device_status() == 0
+
+
 def test_edge_empty_rows_and_device_checks():
     for name in ("tiny_n1024", "llama8b_n8192"):
         w, inp, d = _inputs(name, seq_len=1024) if name != "tiny_n1024" else _inputs(name)
