@@ -224,14 +224,19 @@ def cores() -> int:
         return os.cpu_count() or 1
 
 
-def workload_config(w: synth.Workload, ws: int) -> dict:
-    return {"workload": w.name, "batch_per_gpu": w.batch, "global_batch": w.batch * ws,
+def workload_config(w: synth.Workload, ws: int, heads: bool = False) -> dict:
+    if heads:
+        par = f"kv heads split over {ws} ranks, outputs all-gathered (NCCL)"
+    else:
+        par = f"independent layers x{ws}" if ws > 1 else "single GPU"
+    return {"workload": w.name, "batch_per_gpu": w.batch,
+            "global_batch": w.batch if heads else w.batch * ws,
             "seq_len": w.seq_len, "n_q_heads": w.n_q_heads, "n_kv_heads": w.n_kv_heads,
             "head_dim": w.head_dim, "block_size": w.block_size, "gamma": w.gamma, "tau": w.tau,
             "min_budget": w.min_budget, "max_budget": w.max_budget,
             "qa_selection": "query-wise" if w.qa_mode == 1 else "flattened",
             "vs_lines": "blocks" if w.vs_mode == 1 else "tokens",
-            "parallelism": f"independent layers x{ws}" if ws > 1 else "single GPU",
+            "parallelism": par,
             "l2": "no flush: every step streams Q (1.07 GB at 128k) and K/V, inputs larger "
                   "than the 126 MB L2"}
 
@@ -263,14 +268,21 @@ def run_reference(args, w, ws, rank):
 # --------------------------------------------------------------------- ours --
 
 def run_ours(args, w, ws, rank, local):
-    from dynamic_block_sparse_fp_b200 import build, ops
+    from dynamic_block_sparse_fp_b200 import build, ops, sharded
 
     build.build()
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     peaks = load_peaks()
-    # every rank: its own independent layer
-    inp = synth.make_inputs(rank_workload(w, rank))
+    heads = args.shard == "heads"
+    if heads:
+        # one layer, its kv heads split over the ranks; outputs all-gathered
+        inp = synth.make_inputs(w)
+        inp.update(zip(("q", "k", "v"), sharded.shard_inputs(inp["q"], inp["k"], inp["v"],
+                                                             ws, rank)))
+    else:
+        # every rank: its own independent layer
+        inp = synth.make_inputs(rank_workload(w, rank))
     q, k, v = (inp[x].to(dev) for x in ("q", "k", "v"))
     bt, hq, n, d = q.shape
     hkv, bs = k.shape[1], w.block_size
@@ -309,6 +321,8 @@ def run_ours(args, w, ws, rank, local):
         ops._check(ops.fp_sparse_attn(s, q, k, v, counts, indices, out, None, None, stream),
                    "fp_sparse_attn")
         e[4].record(stream)
+        if heads and ws > 1:
+            sharded.gather_heads(out, ws)  # the whole layer's output on every rank
 
     for i in range(args.warmup):
         step(ev[i])
@@ -339,7 +353,8 @@ def run_ours(args, w, ws, rank, local):
     attn_flops = flop_block * kept
     attn_tflops = attn_flops / (stage_ms[3] * 1e-3) / 1e12
     tokens = n * bt
-    value = job_value(tokens, ws, ms_step)
+    # weak scaling: every rank's own layer; head sharding: one layer in all
+    value = tokens / (ms_step * 1e-3) if heads else job_value(tokens, ws, ms_step)
     # dense comparison at the same length (same kernel over every causal block)
     dense_ms = None
     if not args.no_dense:
@@ -363,10 +378,11 @@ def run_ours(args, w, ws, rank, local):
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "higher_is_better": True, "scaling": "strong" if heads else "weak",
+        "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded Q/K/V with planted query-aware / vertical-slash structure "
                 "and RoPE; no dataset or weights)",
-        "config": workload_config(w, ws),
+        "config": workload_config(w, ws, heads),
         "roofline": {"bound": "tensor", "kernel": "fp_sparse_attn", "achieved": attn_tflops,
                      "peak": peak_t, "unit": "TFLOP/s", "frac": attn_tflops / peak_t,
                      "traffic": kernel_traffic("attn_tc.cu", w.name),
@@ -407,7 +423,9 @@ def run_ours(args, w, ws, rank, local):
         torch.cuda.synchronize()
         e2e_ms = max_over_ranks(a.elapsed_time(b_) / args.e2e_steps, ws, dev)
         h2d = (qh.numel() + kh.numel() + vh.numel()) * qh.element_size()
-        line["e2e"] = {"value": ws * tokens / (e2e_ms * 1e-3), "unit": "tokens/s",
+        # head sharding: each rank copies its own heads in and out
+        e2e_tok = tokens if heads else ws * tokens
+        line["e2e"] = {"value": e2e_tok / (e2e_ms * 1e-3), "unit": "tokens/s",
                        "h2d_bytes_per_step": h2d,
                        "d2h_bytes_per_step": oh.numel() * oh.element_size(),
                        "ms_per_step": e2e_ms, "steps": args.e2e_steps,
@@ -440,6 +458,9 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--shard", choices=["layers", "heads"], default="layers",
+                    help="N > 1: independent layers per rank (weak scaling, default) or one "
+                         "layer's kv heads split over the ranks (strong scaling)")
     ap.add_argument("--cpu-baseline-s", type=float, default=12.0,
                     help="seconds of oracle work in the cpu_baseline sample")
     ap.add_argument("--reference-step-s", type=float, default=8.0,

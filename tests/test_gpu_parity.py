@@ -375,6 +375,20 @@ def test_host_path_batch2_fp32_matches_device_path():
     assert ops.fp_last_device_status() == 0
 
 
+def test_sharded_single_rank_is_the_whole_path():
+    """With one rank the head-sharded entry is fp_prefill_attn, bitwise."""
+    from dynamic_block_sparse_fp_b200 import sharded
+    w, inp, d = _inputs("llama8b_n8192")
+    p = ops.make_params(w.gamma, w.tau, w.min_budget, w.max_budget)
+    want, _, _ = ops.prefill_attn(d["q"], d["k"], d["v"], w.block_size, p)
+    got = sharded.sharded_prefill_attn(d["q"], d["k"], d["v"], w.block_size, p)
+    qs, ks, vs = sharded.shard_inputs(d["q"], d["k"], d["v"], 2, 1)  # rank 1 of 2: heads 16-31
+    half, _, _ = ops.prefill_attn(qs, ks, vs, w.block_size, p)
+    torch.cuda.synchronize()
+    assert torch.equal(got, want)
+    assert torch.equal(half, want[:, 16:])
+
+
 def test_edge_empty_rows_and_device_checks():
     for name in ("tiny_n1024", "llama8b_n8192"):
         w, inp, d = _inputs(name, seq_len=1024) if name != "tiny_n1024" else _inputs(name)

@@ -60,3 +60,54 @@ def test_job_value_is_whole_job_tokens_per_second():
     assert bench.job_value(131072, 8, 100.0) == pytest.approx(8 * 1310720.0)
     w = __import__("dynamic_block_sparse_fp_b200.synth", fromlist=["x"]).WORKLOADS["tiny_n1024"]
     assert bench.rank_workload(w, 0) is w
+
+
+def _fake_prefill(q, k, v, block_size, params):
+    """Stand-in for the library call (no GPU here): a per-head function of the
+    head's own q and its kv head's k and v, so that a wrong slice shows."""
+    g = q.shape[1] // k.shape[1]
+    kk = k.repeat_interleave(g, dim=1)
+    vv = v.repeat_interleave(g, dim=1)
+    return 2.0 * q + 3.0 * kk - vv, None, None
+
+
+def _shard_worker(rank, ws, port, out):
+    import datetime
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    from dynamic_block_sparse_fp_b200 import ops, sharded
+    dist.init_process_group("gloo", rank=rank, world_size=ws,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        ops.prefill_attn = _fake_prefill  # this process only
+        g = torch.Generator().manual_seed(3)
+        q = torch.randn(2, 8, 16, 4, generator=g)   # Bt 2, Hq 8
+        k = torch.randn(2, 4, 16, 4, generator=g)   # Hkv 4: 2 kv heads per rank
+        v = torch.randn(2, 4, 16, 4, generator=g)
+        full = sharded.sharded_prefill_attn(q, k, v, 8, None)
+        local = sharded.sharded_prefill_attn(q, k, v, 8, None, gather=False)
+        want = _fake_prefill(q, k, v, 8, None)[0]
+        kv0, nk = sharded.head_shard(4, ws, rank)
+        out[rank] = (bool(torch.equal(full, want)),
+                     bool(torch.equal(local, want[:, kv0 * 2:(kv0 + nk) * 2])))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_ranks_head_sharded_layer_gathers_every_head():
+    ws = 2
+    with mp.Manager() as mgr:
+        out = mgr.dict()
+        mp.start_processes(_shard_worker, args=(ws, _free_port(), out), nprocs=ws, join=True,
+                           start_method="spawn")
+        res = dict(out)
+    assert res[0] == res[1] == (True, True)
+
+
+def test_head_shard_rule():
+    from dynamic_block_sparse_fp_b200 import sharded
+    assert [sharded.head_shard(8, 4, r) for r in range(4)] == [(0, 2), (2, 2), (4, 2), (6, 2)]
+    assert sharded.head_shard(8, 1, 0) == (0, 8)
+    with pytest.raises(ValueError):
+        sharded.head_shard(8, 3, 0)
+    with pytest.raises(ValueError):
+        sharded.head_shard(8, 2, 2)
