@@ -51,13 +51,17 @@ __device__ __forceinline__ void ld8(const __nv_bfloat16 *p, float (&x)[8]) {
 }
 
 // ------------------------------------------------------------------ pooling --
-// grid (nb, heads, Bt), 256 threads.  x [Bt, heads, N, d] -> out [Bt, heads, nb, d].
+// grid (blocks, heads, Bt), 256 threads.  x [Bt, heads, N, d] -> out [Bt, heads,
+// nb, d], blocks blk0 .. blk0 + gridDim.x - 1.  With `qa_only` (a pattern
+// array, or null), heads whose pattern is not query-aware are skipped.
 template <class T>
 __global__ void __launch_bounds__(256) pool_kernel(const T *__restrict__ x, float *__restrict__ out,
-                                                   int n, int d, int bs) {
+                                                   int n, int d, int bs, int nb, int blk0,
+                                                   const int32_t *__restrict__ qa_only) {
   __shared__ float part[32][128];
-  const int blk = blockIdx.x, head = blockIdx.y, b = blockIdx.z;
-  const int heads = gridDim.y, nb = gridDim.x;
+  const int blk = blk0 + int(blockIdx.x), head = blockIdx.y, b = blockIdx.z;
+  const int heads = gridDim.y;
+  if (qa_only && qa_only[size_t(b) * heads + head] != FP_PATTERN_QA) return;
   const int vec_per_row = d / 8;
   const int rows_per_it = 256 / vec_per_row;
   const int tv = threadIdx.x % vec_per_row, tr = threadIdx.x / vec_per_row;
@@ -87,10 +91,12 @@ __global__ void __launch_bounds__(256) pool_kernel(const T *__restrict__ x, floa
 __global__ void __launch_bounds__(256) map_logits_kernel(const float *__restrict__ qbar,
                                                          const float *__restrict__ kbar,
                                                          float *__restrict__ map, int hq, int g,
-                                                         int nb, int d, float scale) {
+                                                         int nb, int d, float scale,
+                                                         const int32_t *__restrict__ qa_only) {
   const int ti = blockIdx.x, tj = blockIdx.y;
   if (tj > ti) return;
   const int bh = blockIdx.z, b = bh / hq, h = bh % hq, kv = h / g;
+  if (qa_only && qa_only[bh] != FP_PATTERN_QA) return;
   const int hkv = hq / g;
   __shared__ __align__(16) float As[8][128];
   __shared__ __align__(16) float Bs[8][128];
@@ -147,17 +153,10 @@ __global__ void __launch_bounds__(256) map_logits_kernel(const float *__restrict
   }
 }
 
-// One warp per map row; 8 rows per CTA.
-__global__ void __launch_bounds__(256) map_softmax_kernel(float *__restrict__ map,
-                                                          float *__restrict__ est_last,
-                                                          long long rows_total, int nb) {
-  const long long row = (long long)blockIdx.x * 8 + threadIdx.x / 32;
-  const int lane = threadIdx.x % 32;
-  if (row >= rows_total) return;
-  const long long bh = row / nb;
-  const int i = int(row % nb);
-  float *r = map + bh * ((long long)nb * (nb + 1) / 2) + (long long)i * (i + 1) / 2;
-  const int len = i + 1;
+// Softmax of one map row in place (one warp; the same steps for every row,
+// whichever kernel runs them); the last row also goes to est_last.
+__device__ __forceinline__ void map_row_softmax(float *r, int len, float *est_last_row,
+                                                int lane) {
   float mx = -INFINITY;
   for (int j = lane; j < len; j += 32) mx = fmaxf(mx, r[j]);
 #pragma unroll
@@ -170,8 +169,64 @@ __global__ void __launch_bounds__(256) map_softmax_kernel(float *__restrict__ ma
   for (int j = lane; j < len; j += 32) {
     float p = expf(r[j] - mx) * inv;
     r[j] = p;
-    if (i == nb - 1) est_last[bh * nb + j] = p;
+    if (est_last_row) est_last_row[j] = p;
   }
+}
+
+// One warp per map row; 8 rows per CTA.  `qa_only`: as for pool_kernel.
+__global__ void __launch_bounds__(256) map_softmax_kernel(float *__restrict__ map,
+                                                          float *__restrict__ est_last,
+                                                          long long rows_total, int nb,
+                                                          const int32_t *__restrict__ qa_only) {
+  const long long row = (long long)blockIdx.x * 8 + threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+  if (row >= rows_total) return;
+  const long long bh = row / nb;
+  if (qa_only && qa_only[bh] != FP_PATTERN_QA) return;
+  const int i = int(row % nb);
+  float *r = map + bh * ((long long)nb * (nb + 1) / 2) + (long long)i * (i + 1) / 2;
+  map_row_softmax(r, i + 1, i == nb - 1 ? est_last + bh * nb : nullptr, lane);
+}
+
+// The last row of the map alone (the estimate a-hat that the pattern test
+// needs), for every head: grid (Hq, Bt), 256 threads.  Logit j is the same
+// fmaf chain over d, in order, times scale, that map_logits_kernel forms, and
+// the softmax is map_row_softmax, so the row is bitwise the full map's.
+__global__ void __launch_bounds__(256) map_last_row_kernel(const float *__restrict__ qbar,
+                                                           const float *__restrict__ kbar,
+                                                           float *__restrict__ map,
+                                                           float *__restrict__ est_last, int hq,
+                                                           int g, int nb, int d, float scale) {
+  const int h = blockIdx.x, b = blockIdx.y, kv = h / g, hkv = hq / g;
+  const size_t bh = size_t(b) * hq + h;
+  __shared__ __align__(16) float qs[128];
+  const float *qa = qbar + (bh * nb + (nb - 1)) * d;
+  const float *kb = kbar + (size_t(b) * hkv + kv) * nb * d;
+  float *r = map + bh * (size_t(nb) * (nb + 1) / 2) + size_t(nb - 1) * nb / 2;
+  if (threadIdx.x < d) qs[threadIdx.x] = qa[threadIdx.x];
+  __syncthreads();
+  for (int j = threadIdx.x; j < nb; j += 256) {
+    // k-bar row j in chunks of 8 float4 loads issued together; the fmaf
+    // chain itself runs over d in order
+    const float4 *kr = reinterpret_cast<const float4 *>(kb + size_t(j) * d);
+    float acc = 0.f;
+    for (int c = 0; c < d / 4; c += 8) {
+      float4 t[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) t[u] = kr[c + u];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const float *x = &qs[4 * (c + u)];
+        acc = fmaf(x[0], t[u].x, acc);
+        acc = fmaf(x[1], t[u].y, acc);
+        acc = fmaf(x[2], t[u].z, acc);
+        acc = fmaf(x[3], t[u].w, acc);
+      }
+    }
+    r[j] = acc * scale;
+  }
+  __syncthreads();
+  if (threadIdx.x < 32) map_row_softmax(r, nb, est_last + bh * nb, threadIdx.x);
 }
 
 // ---------------------------------------------------- last query block --
@@ -369,23 +424,29 @@ cudaError_t run_last(const Dims &Dm, const T *q, const T *k, float *true_last, f
   return cudaGetLastError();
 }
 
+// Q pooling and the block map; with `qa_only`, for query-aware heads only.
 template <class T>
-cudaError_t run_estimate(const Dims &Dm, const T *q, const T *k, float *qbar, float *kbar,
-                         float *map, float *est_last, float *true_last, float *vert,
-                         float *slash, void *ws, cudaStream_t st) {
-  pool_kernel<T><<<dim3(Dm.nb, Dm.hq, Dm.bt), 256, 0, st>>>(q, qbar, Dm.n, Dm.d, Dm.bs);
-  pool_kernel<T><<<dim3(Dm.nb, Dm.hkv, Dm.bt), 256, 0, st>>>(k, kbar, Dm.n, Dm.d, Dm.bs);
+cudaError_t run_map(const Dims &Dm, const T *q, float *qbar, const float *kbar, float *map,
+                    float *est_last, const int32_t *qa_only, cudaStream_t st) {
+  pool_kernel<T><<<dim3(Dm.nb, Dm.hq, Dm.bt), 256, 0, st>>>(q, qbar, Dm.n, Dm.d, Dm.bs, Dm.nb,
+                                                             0, qa_only);
   const int tiles = (Dm.nb + 127) / 128;
   const float scale = 1.f / sqrtf(float(Dm.d));
-  map_logits_kernel<<<dim3(tiles, tiles, Dm.bt * Dm.hq), 256, 0, st>>>(qbar, kbar, map, Dm.hq,
-                                                                      Dm.g, Dm.nb, Dm.d, scale);
+  map_logits_kernel<<<dim3(tiles, tiles, Dm.bt * Dm.hq), 256, 0, st>>>(
+      qbar, kbar, map, Dm.hq, Dm.g, Dm.nb, Dm.d, scale, qa_only);
   const long long rows = (long long)Dm.bt * Dm.hq * Dm.nb;
-  map_softmax_kernel<<<unsigned((rows + 7) / 8), 256, 0, st>>>(map, est_last, rows, Dm.nb);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
+  map_softmax_kernel<<<unsigned((rows + 7) / 8), 256, 0, st>>>(map, est_last, rows, Dm.nb,
+                                                               qa_only);
+  return cudaGetLastError();
+}
+
+// The true last-block distribution, vertical and slash sums.
+template <class T>
+cudaError_t run_true_last(const Dims &Dm, const T *q, const T *k, float *true_last,
+                          float *vert, float *slash, void *ws, cudaStream_t st) {
   if (last_block_tc_supported(Dm)) {
     float *sp = nullptr;
-    e = launch_last_block_tc(Dm, q, k, true_last, vert, &sp, ws, st);
+    cudaError_t e = launch_last_block_tc(Dm, q, k, true_last, vert, &sp, ws, st);
     if (e != cudaSuccess) return e;
     const long long tot = (long long)Dm.bt * Dm.hq * Dm.n;
     slash_combine_kernel<<<unsigned((tot + 255) / 256), 256, 0, st>>>(sp, slash, tot, Dm.n,
@@ -401,6 +462,36 @@ cudaError_t run_estimate(const Dims &Dm, const T *q, const T *k, float *qbar, fl
   return run_last<64, 64, T>(Dm, q, k, true_last, vert, slash, ws, st);
 }
 
+template <class T>
+cudaError_t run_estimate(const Dims &Dm, const T *q, const T *k, float *qbar, float *kbar,
+                         float *map, float *est_last, float *true_last, float *vert,
+                         float *slash, void *ws, cudaStream_t st) {
+  pool_kernel<T><<<dim3(Dm.nb, Dm.hkv, Dm.bt), 256, 0, st>>>(k, kbar, Dm.n, Dm.d, Dm.bs, Dm.nb,
+                                                              0, nullptr);
+  cudaError_t e = run_map<T>(Dm, q, qbar, kbar, map, est_last, nullptr, st);
+  if (e != cudaSuccess) return e;
+  return run_true_last<T>(Dm, q, k, true_last, vert, slash, ws, st);
+}
+
+// Pattern-aware first half: everything the pattern test reads, for every head
+// (K pooled, Q pooled over the last block only, the map's last row, the true
+// last-block distribution and the line sums), but not the rest of the map.
+template <class T>
+cudaError_t run_decision(const Dims &Dm, const T *q, const T *k, float *qbar, float *kbar,
+                         float *map, float *est_last, float *true_last, float *vert,
+                         float *slash, void *ws, cudaStream_t st) {
+  pool_kernel<T><<<dim3(Dm.nb, Dm.hkv, Dm.bt), 256, 0, st>>>(k, kbar, Dm.n, Dm.d, Dm.bs, Dm.nb,
+                                                              0, nullptr);
+  pool_kernel<T><<<dim3(1, Dm.hq, Dm.bt), 256, 0, st>>>(q, qbar, Dm.n, Dm.d, Dm.bs, Dm.nb,
+                                                         Dm.nb - 1, nullptr);
+  map_last_row_kernel<<<dim3(Dm.hq, Dm.bt), 256, 0, st>>>(qbar, kbar, map, est_last, Dm.hq,
+                                                           Dm.g, Dm.nb, Dm.d,
+                                                           1.f / sqrtf(float(Dm.d)));
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  return run_true_last<T>(Dm, q, k, true_last, vert, slash, ws, st);
+}
+
 }  // namespace
 
 size_t estimate_ws_bytes(const Dims &D) {
@@ -412,6 +503,28 @@ size_t estimate_ws_bytes(const Dims &D) {
   c.take<float>(rows * D.bs);
   c.take<float>(rows * D.nb * (2 * D.bs - 1));
   return c.off + 256;
+}
+
+cudaError_t launch_estimate_decision(const Dims &D, const void *q, const void *k, float *qbar,
+                                     float *kbar, float *map, float *est_last,
+                                     float *true_last, float *vert, float *slash, void *ws,
+                                     cudaStream_t st) {
+  if (D.dtype == FP_F32)
+    return run_decision<float>(D, static_cast<const float *>(q), static_cast<const float *>(k),
+                               qbar, kbar, map, est_last, true_last, vert, slash, ws, st);
+  return run_decision<__nv_bfloat16>(D, static_cast<const __nv_bfloat16 *>(q),
+                                     static_cast<const __nv_bfloat16 *>(k), qbar, kbar, map,
+                                     est_last, true_last, vert, slash, ws, st);
+}
+
+cudaError_t launch_estimate_map_qa(const Dims &D, const void *q, float *qbar, const float *kbar,
+                                   float *map, float *est_last, const int32_t *pattern,
+                                   cudaStream_t st) {
+  if (D.dtype == FP_F32)
+    return run_map<float>(D, static_cast<const float *>(q), qbar, kbar, map, est_last, pattern,
+                          st);
+  return run_map<__nv_bfloat16>(D, static_cast<const __nv_bfloat16 *>(q), qbar, kbar, map,
+                                est_last, pattern, st);
 }
 
 cudaError_t launch_estimate(const Dims &D, const void *q, const void *k, float *qbar,

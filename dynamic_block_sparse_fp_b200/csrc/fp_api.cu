@@ -193,13 +193,19 @@ fp_status run_attn(const Dims &D, const void *q, const void *k, const void *v,
   return cuda_status(launch_attn_bf16(D, q, k, v, counts, indices, out, lse, dense, ws, st));
 }
 
+// The whole path, pattern-aware: the inputs of the pattern test first, for every
+// head; then Q pooling and the block map only for the query-aware heads (the
+// vertical-slash heads' selection never reads them).  Every value is bitwise
+// the one the separate fp_estimate / fp_pattern / fp_select calls produce.
 fp_status run_prefill(const Dims &D, const fp_params &p, const void *q, const void *k,
                       const void *v, void *out, float *lse, int64_t *stats, const Prefill &P,
                       cudaStream_t st) {
-  cudaError_t e = launch_estimate(D, q, k, P.qbar, P.kbar, P.map, P.est_last, P.true_last,
-                                  P.vert, P.slash, P.stage_ws, st);
+  cudaError_t e = launch_estimate_decision(D, q, k, P.qbar, P.kbar, P.map, P.est_last,
+                                           P.true_last, P.vert, P.slash, P.stage_ws, st);
   if (e != cudaSuccess) return FP_ERR_CUDA;
   e = launch_pattern(D, p.tau, P.est_last, P.true_last, P.djs, P.pattern, st);
+  if (e != cudaSuccess) return FP_ERR_CUDA;
+  e = launch_estimate_map_qa(D, q, P.qbar, P.kbar, P.map, P.est_last, P.pattern, st);
   if (e != cudaSuccess) return FP_ERR_CUDA;
   e = launch_select(D, p.gamma, budgets(D, p), P.pattern, P.map, P.vert, P.slash, P.counts,
                     P.indices, P.stage_ws, st);

@@ -44,6 +44,17 @@ size_t estimate_ws_bytes(const Dims &D);
 cudaError_t launch_estimate(const Dims &D, const void *q, const void *k, float *qbar,
                             float *kbar, float *map, float *est_last, float *true_last,
                             float *vert, float *slash, void *ws, cudaStream_t st);
+// Pattern-aware halves of launch_estimate (fp_prefill_attn): everything the
+// pattern test reads for every head (K pooled, Q pooled over the last block,
+// the map's last row, true_last, vert, slash) ...
+cudaError_t launch_estimate_decision(const Dims &D, const void *q, const void *k, float *qbar,
+                                     float *kbar, float *map, float *est_last,
+                                     float *true_last, float *vert, float *slash, void *ws,
+                                     cudaStream_t st);
+// ... and then Q pooling and the map for the query-aware heads of `pattern`.
+cudaError_t launch_estimate_map_qa(const Dims &D, const void *q, float *qbar, const float *kbar,
+                                   float *map, float *est_last, const int32_t *pattern,
+                                   cudaStream_t st);
 
 // Tensor-core passes over the last query block (estimate_tc.cu): bf16,
 // block 128, head dim 128.

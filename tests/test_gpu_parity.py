@@ -389,6 +389,31 @@ def test_sharded_single_rank_is_the_whole_path():
     assert torch.equal(half, want[:, 16:])
 
 
+@pytest.mark.parametrize("name,n", [("llama8b_n8192", None), ("tiny_n1024", None),
+                                    ("glm9b_n65536_b64", 4096)])
+def test_prefill_pattern_aware_mixed_heads_bitwise(name, n):
+    """fp_prefill_attn computes Q pooling and the map only for query-aware
+    heads; with tau between the heads' d_JS values (both patterns present) its
+    output and counts must be bitwise those of the separate calls."""
+    w, inp, d = _inputs(name, **({"seq_len": n, "n_q_heads": 8, "n_kv_heads": 2} if n else {}))
+    s = ops.make_shape(d["q"], d["k"], w.block_size)
+    est = ops.estimate(d["q"], d["k"], w.block_size)
+    djs, _ = ops.pattern(s, ops.make_params(w.gamma, w.tau), est["est_last"], est["true_last"])
+    v = np.sort(np.unique(djs.cpu().numpy().ravel()))
+    assert v.size >= 2
+    tau = float((v[v.size // 2 - 1] + v[v.size // 2]) / 2)
+    p = ops.make_params(w.gamma, tau, w.min_budget, w.max_budget)
+    _, pat = ops.pattern(s, p, est["est_last"], est["true_last"])
+    n_qa = int((pat == ops.FP_PATTERN_QA).sum())
+    assert 0 < n_qa < pat.numel()
+    counts, indices = ops.select(s, p, pat, est["map"], est["vert"], est["slash"])
+    out, _ = ops.sparse_attn(d["q"], d["k"], d["v"], counts, indices, w.block_size)
+    out2, _, stats = ops.prefill_attn(d["q"], d["k"], d["v"], w.block_size, p)
+    torch.cuda.synchronize()
+    assert torch.equal(out2, out)
+    assert int(stats[0]) == int(counts.sum()) and int(stats[1]) == n_qa
+
+
 def test_edge_empty_rows_and_device_checks():
     for name in ("tiny_n1024", "llama8b_n8192"):
         w, inp, d = _inputs(name, seq_len=1024) if name != "tiny_n1024" else _inputs(name)
