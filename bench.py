@@ -388,7 +388,10 @@ def run_ours(args, w, ws, rank, local):
                      "traffic": kernel_traffic("attn_tc.cu", w.name),
                      "peak_kind": f"bf16 dense, sustained ({peaks['source']})",
                      "algorithmic_flops_per_launch": attn_flops},
-        "gpu_launches": LAUNCHES_PER_STEP * args.steps,
+        # the library's kernels per step: 12, plus the query-wise row
+        # selection and the line pooling when those modes are on
+        "gpu_launches": (LAUNCHES_PER_STEP + int(w.qa_mode == 1) + int(w.vs_mode == 1))
+                        * args.steps,
         "stages_ms": {"estimate": stage_ms[0], "pattern": stage_ms[1], "select": stage_ms[2],
                       "sparse_attn": stage_ms[3]},
         "estimate_hbm": {"bytes": est_bytes, "gbs": est_bytes / (stage_ms[0] * 1e-3) / 1e9,
