@@ -483,3 +483,61 @@ def test_full_size_128k_sampled():
             for i in range(0, w.n_blocks, 37):
                 np.testing.assert_array_equal(gi[0, 0, i, :gc[0, 0, i]], oi[0, 0, i, :oc[0, 0, i]])
     _attn_check(inp, res, w, 2e-2, 2e-3, heads=hs, q_blocks=[0, 511, 1023])
+
+
+def _full_size_sampled(name, heads, q_blocks, rows_every=37, **over):
+    """One configuration at its full size: the whole path on the GPU, then per
+    sampled head the estimate (oracle, rtol 1e-4), the selection (bit-exact,
+    on the GPU's own fp32 scores) and sampled attention rows (2e-2)."""
+    w0, inp, d = _inputs(name)
+    w = w0.replace(**over) if over else w0
+    res = _pipeline(w, d)
+    assert ops.fp_last_device_status() == 0
+    g = w.n_q_heads // w.n_kv_heads
+    for h in heads:
+        kv = h // g
+        want = oracle.estimate(inp["q"][:, h:h + 1], inp["k"][:, kv:kv + 1], w.block_size)
+        for key in ("map", "est_last", "true_last", "vert", "slash"):
+            np.testing.assert_allclose(_np(res["est"][key][:, h:h + 1]), want[key], rtol=1e-4,
+                                       atol=1e-7, err_msg=f"{key} head {h}")
+    all_vs = torch.full_like(res["pattern"], ops.FP_PATTERN_VS)
+    vs_counts, vs_indices = ops.select(res["shape"], res["params"], all_vs, res["est"]["map"],
+                                       res["est"]["vert"], res["est"]["slash"])
+    torch.cuda.synchronize()
+    for h in heads:
+        for pat, counts, indices in ((res["pattern"], res["counts"], res["indices"]),
+                                     (all_vs, vs_counts, vs_indices)):
+            oc, oi = oracle.select(pat[:, h:h + 1].cpu().numpy(),
+                                   _np(res["est"]["map"][:, h:h + 1]),
+                                   _np(res["est"]["vert"][:, h:h + 1]),
+                                   _np(res["est"]["slash"][:, h:h + 1]), w.n_blocks,
+                                   w.block_size, w.gamma, w.min_budget, w.max_budget)
+            gc = counts[:, h:h + 1].cpu().numpy()
+            gi = indices[:, h:h + 1].cpu().numpy()
+            np.testing.assert_array_equal(gc, oc)
+            for i in range(0, w.n_blocks, rows_every):
+                np.testing.assert_array_equal(gi[0, 0, i, :gc[0, 0, i]],
+                                              oi[0, 0, i, :oc[0, 0, i]])
+    _attn_check(inp, res, w, 2e-2, 2e-3, heads=heads, q_blocks=q_blocks)
+    return res
+
+
+@pytest.mark.parametrize("name", ["glm9b_n65536_b128", "glm9b_n65536_b64"])
+def test_full_size_glm_64k_sampled(name):
+    """GLM-4-9B heads (32 q / 2 kv), N = 65536, block 128 and 64, max budget
+    32768 tokens, 75 % vertical-slash plantings."""
+    w = synth.WORKLOADS[name]
+    nb = w.n_blocks
+    _full_size_sampled(name, heads=[3, 30], q_blocks=[0, nb // 2, nb - 1])
+
+
+def test_full_size_32k_gamma09_sampled():
+    """N = 32768 at gamma = 0.9 (the 32k sweep's other point)."""
+    _full_size_sampled("llama8b_n32768", heads=[5, 26], q_blocks=[0, 100, 255], gamma=0.9)
+
+
+def test_full_size_128k_vs_capped_sampled():
+    """128k sweep points with every head vertical-slash (tau = 0), gamma = 0.9,
+    min budget 2048 and max budget 8192 tokens."""
+    _full_size_sampled("llama8b_n131072", heads=[2, 17], q_blocks=[1, 640, 1023], rows_every=61,
+                       tau=0.0, gamma=0.9, min_budget=2048, max_budget=8192)
