@@ -357,6 +357,45 @@ FP_API fp_status fp_prefill_attn(const fp_shape *shape, const fp_params *params,
                      reinterpret_cast<cudaStream_t>(stream));
 }
 
+FP_API fp_status fp_prefill_attn_varlen(const fp_shape *shape, const fp_params *params,
+                                        int n_seqs, const int32_t *seq_lens, const void *q,
+                                        const void *k, const void *v, void *out, float *lse,
+                                        int64_t *stats, void *ws, size_t ws_bytes,
+                                        fp_stream_t stream) {
+  Dims D;
+  fp_status s = check_shape(shape, &D);
+  if (s != FP_OK) return s;
+  if (D.bt != 1) return FP_ERR_SHAPE;
+  if ((s = check_attn_shape(D)) != FP_OK) return s;
+  if ((s = check_params(params)) != FP_OK) return s;
+  if (!q || !k || !v || !out || !seq_lens) return FP_ERR_NULL;
+  if (n_seqs < 1) return FP_ERR_SHAPE;
+  for (int i = 0; i < n_seqs; ++i)
+    if (seq_lens[i] <= 0 || seq_lens[i] > D.n || seq_lens[i] % D.bs != 0) return FP_ERR_SHAPE;
+  Prefill Pmax;
+  if ((s = check_ws(ws, ws_bytes, carve_prefill(D, nullptr, &Pmax))) != FP_OK) return s;
+  if ((s = check_device()) != FP_OK) return s;
+  const size_t eb = elem_bytes(D);
+  const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  size_t tok = 0;  // tokens of the sequences before this one
+  for (int i = 0; i < n_seqs; ++i) {
+    fp_shape one = *shape;
+    one.seq_len = seq_lens[i];
+    Dims Ds;
+    if ((s = check_shape(&one, &Ds)) != FP_OK) return s;
+    Prefill P;
+    carve_prefill(Ds, ws, &P);  // fits: a shorter sequence needs less than N_max
+    const size_t qo = tok * D.hq * D.d * eb, kvo = tok * D.hkv * D.d * eb;
+    s = run_prefill(Ds, *params, static_cast<const char *>(q) + qo,
+                    static_cast<const char *>(k) + kvo, static_cast<const char *>(v) + kvo,
+                    static_cast<char *>(out) + qo, lse ? lse + tok * D.hq : nullptr,
+                    stats ? stats + 2 * i : nullptr, P, st);
+    if (s != FP_OK) return s;
+    tok += size_t(seq_lens[i]);
+  }
+  return FP_OK;
+}
+
 FP_API fp_status fp_prefill_attn_host(const fp_shape *shape, const fp_params *params,
                                       const void *q_host, const void *k_host,
                                       const void *v_host, void *out_host, void *ws,

@@ -68,6 +68,8 @@ _SIG = {
     "fp_prefill_attn": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t,
                                        _P]),
     "fp_prefill_attn_host": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
+    "fp_prefill_attn_varlen": (ctypes.c_int, [_P, _P, ctypes.c_int, _P, _P, _P, _P, _P, _P, _P,
+                                              _P, ctypes.c_size_t, _P]),
     "fp_last_device_status": (ctypes.c_int, [_P]),
     "fp_selftest_watchdog": (ctypes.c_int, [ctypes.c_uint, _P]),
     "fp_status_string": (ctypes.c_char_p, [ctypes.c_int]),
@@ -201,6 +203,17 @@ def fp_prefill_attn_host(shape, params, q_host, k_host, v_host, out_host, ws,
                                       _nbytes(ws), _stream(stream))
 
 
+def fp_prefill_attn_varlen(shape, params, seq_lens, q, k, v, out, lse, stats, ws,
+                           stream=None) -> int:
+    """seq_lens: a sequence of Python ints (copied to a host int32 array here)."""
+    n = len(seq_lens)
+    lens = (ctypes.c_int32 * max(n, 1))(*seq_lens)
+    return lib().fp_prefill_attn_varlen(ctypes.byref(shape), ctypes.byref(params), n,
+                                        ctypes.cast(lens, ctypes.c_void_p), _addr(q), _addr(k),
+                                        _addr(v), _addr(out), _addr(lse), _addr(stats),
+                                        _addr(ws), _nbytes(ws), _stream(stream))
+
+
 def fp_selftest_watchdog(limit_us: int, stream=None) -> int:
     return lib().fp_selftest_watchdog(limit_us, _stream(stream))
 
@@ -281,6 +294,35 @@ def dense_attn(q, k, v, block_size: int, with_lse: bool = True, stream=None):
     lse = torch.empty(q.shape[:3], dtype=torch.float32, device=q.device) if with_lse else None
     _check(fp_dense_attn(s, q, k, v, out, lse, stream), "fp_dense_attn")
     return out, lse
+
+
+def prefill_attn_varlen(seqs_q, seqs_k, seqs_v, block_size: int, params: fp_params,
+                        stream=None):
+    """The whole path over sequences of different lengths in one call.
+
+    seqs_*: lists of [1, H, N_s, d] tensors (one per sequence).  They are packed
+    back to back for the call and the outputs are returned as a list of
+    [1, Hq, N_s, d] views of one packed buffer, with per-sequence stats
+    [n_seqs, 2].
+    """
+    lens = [int(x.shape[2]) for x in seqs_q]
+    q = torch.cat([x.reshape(-1) for x in seqs_q])
+    k = torch.cat([x.reshape(-1) for x in seqs_k])
+    v = torch.cat([x.reshape(-1) for x in seqs_v])
+    hq, d = seqs_q[0].shape[1], seqs_q[0].shape[3]
+    hkv = seqs_k[0].shape[1]
+    s = fp_shape(1, hq, hkv, max(lens), d, block_size,
+                 FP_BF16 if seqs_q[0].dtype == torch.bfloat16 else FP_F32)
+    out = torch.empty_like(q)
+    stats = torch.empty(len(lens), 2, dtype=torch.int64, device=q.device)
+    ws = workspace(s, FP_CALL_PREFILL, q.device)
+    _check(fp_prefill_attn_varlen(s, params, lens, q, k, v, out, None, stats, ws, stream),
+           "fp_prefill_attn_varlen")
+    outs, off = [], 0
+    for n in lens:
+        outs.append(out[off: off + hq * n * d].view(1, hq, n, d))
+        off += hq * n * d
+    return outs, stats
 
 
 def prefill_attn(q, k, v, block_size: int, params: fp_params, with_lse: bool = False,

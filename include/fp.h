@@ -267,6 +267,32 @@ fp_status fp_prefill_attn(const fp_shape *shape, const fp_params *params,
                           void *ws, size_t ws_bytes, fp_stream_t stream);
 
 /*
+ * fp_prefill_attn_varlen -- fp_prefill_attn over a batch of sequences of
+ * different lengths (no counterpart in the pages: the method is defined per
+ * sequence; this is the batching a serving caller needs).
+ *   shape     batch must be 1 and seq_len the longest allowed length N_max;
+ *             the other fields as for fp_prefill_attn
+ *   n_seqs    number of sequences, >= 1
+ *   seq_lens  HOST int32[n_seqs]: N_s, each a positive multiple of
+ *             block_size and <= N_max
+ *   q, out    the sequences' [Hq, N_s, d] tensors back to back (sequence s
+ *             starts Hq * d * (N_0 + ... + N_{s-1}) elements in);
+ *   k, v      likewise [Hkv, N_s, d]
+ *   lse       NULL, or [Hq, N_s] fp32 back to back
+ *   stats     NULL, or device int64[n_seqs][2], per sequence as for
+ *             fp_prefill_attn
+ *   ws        fp_workspace_size(shape, FP_CALL_PREFILL) bytes, reused by the
+ *             sequences one after another on `stream`
+ * Every sequence's result is bitwise that of its own fp_prefill_attn call.
+ * A bad length returns FP_ERR_SHAPE before anything is launched.
+ */
+fp_status fp_prefill_attn_varlen(const fp_shape *shape, const fp_params *params,
+                                 int n_seqs, const int32_t *seq_lens,
+                                 const void *q, const void *k, const void *v,
+                                 void *out, float *lse, int64_t *stats,
+                                 void *ws, size_t ws_bytes, fp_stream_t stream);
+
+/*
  * fp_prefill_attn_host -- fp_prefill_attn on HOST buffers: copies q, k, v
  * to device memory inside `ws` (fp_workspace_size(shape,
  * FP_CALL_PREFILL_HOST) bytes), runs the path and copies the output back to

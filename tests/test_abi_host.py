@@ -26,7 +26,7 @@ def shape(**kw):
 
 def test_exports_every_declared_function(L):
     names = ops.header_functions()
-    assert len(names) == 12, names
+    assert len(names) == 13, names
     for n in names:
         assert hasattr(L, n), n
     # nothing but the fp_* API is exported (static CUDA runtime stays hidden)
@@ -116,6 +116,33 @@ def test_bad_vs_mode_rejected(L, vs_mode):
     p = ops.make_params(0.9, 0.1, 0, 0, 0, vs_mode)
     assert L.fp_select(ctypes.byref(s), ctypes.byref(p), *([FAKE] * 6), FAKE, 1 << 40,
                        None) == ops.STATUS_CODES["FP_ERR_PARAM"]
+
+
+@pytest.mark.parametrize("lens,batch,code", [
+    ([1024, 1000], 1, "FP_ERR_SHAPE"),   # not a multiple of the block size
+    ([1024, 0], 1, "FP_ERR_SHAPE"),      # empty sequence
+    ([2048], 1, "FP_ERR_SHAPE"),         # longer than shape.seq_len (1024)
+    ([], 1, "FP_ERR_SHAPE"),             # no sequence
+    ([1024], 2, "FP_ERR_SHAPE"),         # the shape's batch must be 1
+])
+def test_varlen_bad_lengths_rejected(L, lens, batch, code):
+    s = shape(batch=batch)
+    p = ops.make_params(0.9, 0.1, 0, 0)
+    assert ops.fp_prefill_attn_varlen(s, p, lens, FAKE, FAKE, FAKE, FAKE, None, None, FAKE,
+                                      None) == ops.STATUS_CODES[code]
+
+
+def test_varlen_nulls_and_workspace(L):
+    s = shape()
+    p = ops.make_params(0.9, 0.1, 0, 0)
+    P = ctypes.c_void_p
+    assert L.fp_prefill_attn_varlen(ctypes.byref(s), ctypes.byref(p), 1, None, P(FAKE), P(FAKE),
+                                    P(FAKE), P(FAKE), None, None, P(FAKE), 1 << 40,
+                                    None) == ops.STATUS_CODES["FP_ERR_NULL"]
+    lens = (ctypes.c_int32 * 1)(1024)
+    assert L.fp_prefill_attn_varlen(ctypes.byref(s), ctypes.byref(p), 1, lens, P(FAKE), P(FAKE),
+                                    P(FAKE), P(FAKE), None, None, P(FAKE), 16,
+                                    None) == ops.STATUS_CODES["FP_ERR_WORKSPACE"]
 
 
 def test_workspace_checks(L):

@@ -414,6 +414,27 @@ def test_prefill_pattern_aware_mixed_heads_bitwise(name, n):
     assert int(stats[0]) == int(counts.sum()) and int(stats[1]) == n_qa
 
 
+def test_varlen_batch_matches_separate_calls():
+    """Three sequences of different lengths in one fp_prefill_attn_varlen call:
+    every output and every per-sequence stats row is bitwise that of the
+    sequence's own fp_prefill_attn call."""
+    base = synth.WORKLOADS["llama8b_n8192"].replace(n_q_heads=8, n_kv_heads=2)
+    seqs = [synth.make_inputs(base.replace(seq_len=n, seed=40 + i))
+            for i, n in enumerate((2048, 256, 1024))]
+    qs = [x["q"].to(DEV) for x in seqs]
+    ks = [x["k"].to(DEV) for x in seqs]
+    vs = [x["v"].to(DEV) for x in seqs]
+    p = ops.make_params(base.gamma, base.tau, base.min_budget, base.max_budget)
+    outs, stats = ops.prefill_attn_varlen(qs, ks, vs, base.block_size, p)
+    torch.cuda.synchronize()
+    for i in range(3):
+        want, _, st = ops.prefill_attn(qs[i], ks[i], vs[i], base.block_size, p)
+        torch.cuda.synchronize()
+        assert torch.equal(outs[i], want), i
+        assert torch.equal(stats[i], st), i
+    assert ops.fp_last_device_status() == 0
+
+
 def test_edge_empty_rows_and_device_checks():
     for name in ("tiny_n1024", "llama8b_n8192"):
         w, inp, d = _inputs(name, seq_len=1024) if name != "tiny_n1024" else _inputs(name)
