@@ -562,3 +562,33 @@ def test_full_size_128k_vs_capped_sampled():
     min budget 2048 and max budget 8192 tokens."""
     _full_size_sampled("llama8b_n131072", heads=[2, 17], q_blocks=[1, 640, 1023], rows_every=61,
                        tau=0.0, gamma=0.9, min_budget=2048, max_budget=8192)
+
+
+def test_maximum_block_count_sampled():
+    """nb = 4096, the largest block count the library takes (N = 262144 at
+    block 64, bf16, two query heads on one kv head): one head's selection
+    against the oracle (a map of 8.4 M entries), the allocation-free
+    selection at this size, and sampled attention rows."""
+    w = synth.WORKLOADS["glm9b_n65536_b64"].replace(seq_len=262144, n_q_heads=2, n_kv_heads=1)
+    assert w.n_blocks == 4096
+    inp = synth.make_inputs(w)
+    d = {x: inp[x].to(DEV) for x in ("q", "k", "v")}
+    res = _pipeline(w, d)
+    assert ops.fp_last_device_status() == 0
+    h = 1
+    oc, oi = oracle.select(res["pattern"][:, h:h + 1].cpu().numpy(),
+                           _np(res["est"]["map"][:, h:h + 1]), _np(res["est"]["vert"][:, h:h + 1]),
+                           _np(res["est"]["slash"][:, h:h + 1]), w.n_blocks, w.block_size,
+                           w.gamma, w.min_budget, w.max_budget)
+    gc = res["counts"][:, h:h + 1].cpu().numpy()
+    gi = res["indices"][:, h:h + 1].cpu().numpy()
+    np.testing.assert_array_equal(gc, oc)
+    for i in (0, 1, 2047, 4094, 4095):
+        np.testing.assert_array_equal(gi[0, 0, i, :gc[0, 0, i]], oi[0, 0, i, :oc[0, 0, i]])
+    c2 = torch.empty_like(res["counts"])
+    i2 = torch.empty_like(res["indices"])
+    assert ops.fp_select_noalloc(res["shape"], res["params"], res["pattern"], res["est"]["map"],
+                                 res["est"]["vert"], res["est"]["slash"], c2, i2) == 0
+    torch.cuda.synchronize()
+    assert torch.equal(c2, res["counts"])
+    _attn_check(inp, res, w, 2e-2, 2e-3, heads=[0, 1], q_blocks=[0, 2048, 4095])
