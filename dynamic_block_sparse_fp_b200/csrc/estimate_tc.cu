@@ -242,30 +242,51 @@ __global__ void __launch_bounds__(kThreads, 1) last_block_tc_kernel(
         m = mnew;
       } else {
         // key r of the tile, query c of the last block: visible iff r <= c.
-        // Diagonal sums (query - key) by a register-systolic chain per warp:
+        // Diagonal sums (query - key) by register-systolic chains per warp:
         // at step c lane l holds the diagonal c - l and passes it one lane up;
-        // lane 31 completes one diagonal per step.  The vertical sum of the
-        // key runs in 4 independent chains.
+        // lane 31 completes one diagonal per step (bins[c] = diagonal c - 31).
+        // Two independent chains, over columns 0..63 (A) and 64..127 (B), run
+        // interleaved so that each shuffle's latency hides the other's.  A
+        // diagonal c - 31 with c in 64..94 takes its lanes whose column is
+        // >= 64 from B and the others from A, whose lane l still holds
+        // diagonal 63 - l when A ends: that part is added once after the loop
+        // (a fixed order).  The vertical sum of the key runs in 4 chains.
+        static_assert(BS == 128, "two 64-column chains");
         float v4[4] = {0.f, 0.f, 0.f, 0.f};
-        float lq[4];
-        float acc = 0.f;
+        float lqa[4], lqb[4];
+        float acc_a = 0.f, acc_b = 0.f;
         float *bins = sm.bins[hh][wq];
 #pragma unroll
-        for (int c = 0; c < BS; ++c) {
+        for (int c = 0; c < BS / 2; ++c) {
+          const int cb = c + BS / 2;
           if (c % 4 == 0) {
-            const float4 ls = *reinterpret_cast<const float4 *>(&sm.lse2[hh][c]);
-            lq[0] = ls.x;
-            lq[1] = ls.y;
-            lq[2] = ls.z;
-            lq[3] = ls.w;
+            const float4 la = *reinterpret_cast<const float4 *>(&sm.lse2[hh][c]);
+            const float4 lb = *reinterpret_cast<const float4 *>(&sm.lse2[hh][cb]);
+            lqa[0] = la.x;
+            lqa[1] = la.y;
+            lqa[2] = la.z;
+            lqa[3] = la.w;
+            lqb[0] = lb.x;
+            lqb[1] = lb.y;
+            lqb[2] = lb.z;
+            lqb[3] = lb.w;
           }
-          const float p = (diag && r > c) ? 0.f : ex2(fmaf(x[c], sl2, -lq[c % 4]));
-          v4[c % 4] += p;
-          float a = __shfl_up_sync(0xffffffffu, acc, 1);
-          acc = (lane == 0 ? 0.f : a) + p;
-          if (lane == 31) bins[c] = acc;  // diagonal c - 31 is complete
+          const float pa = (diag && r > c) ? 0.f : ex2(fmaf(x[c], sl2, -lqa[c % 4]));
+          const float pb = (diag && r > cb) ? 0.f : ex2(fmaf(x[cb], sl2, -lqb[c % 4]));
+          v4[c % 4] += pa;
+          v4[c % 4] += pb;
+          const float ua = __shfl_up_sync(0xffffffffu, acc_a, 1);
+          const float ub = __shfl_up_sync(0xffffffffu, acc_b, 1);
+          acc_a = (lane == 0 ? 0.f : ua) + pa;
+          acc_b = (lane == 0 ? 0.f : ub) + pb;
+          if (lane == 31) {
+            bins[c] = acc_a;   // diagonal c - 31 (only columns < 64 reach it)
+            bins[cb] = acc_b;  // diagonal cb - 31: its columns >= 64
+          }
         }
-        if (lane < 31) bins[BS + 30 - lane] = acc;  // diagonals 127 - lane
+        __syncwarp();
+        if (lane < 31) bins[BS / 2 + 30 - lane] += acc_a;  // diagonal 63 - lane: columns < 64
+        if (lane < 31) bins[BS + 30 - lane] = acc_b;        // diagonals 127 - lane
         const float v = (v4[0] + v4[1]) + (v4[2] + v4[3]);
         vert[bh * n_tok + size_t(j) * BS + r] = v;
         // tile mass, fixed order: lanes (xor tree), then warps
