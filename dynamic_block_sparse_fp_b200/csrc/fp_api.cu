@@ -158,7 +158,7 @@ struct Prefill {
   void *stage_ws;
 };
 
-constexpr int kHostUnits = 4;  // fp_prefill_attn_host: pipelined units per batch entry
+constexpr int kHostMidUnits = 3;  // fp_prefill_attn_host: middle units per batch entry
 
 size_t carve_prefill(const Dims &D, void *ws, Prefill *P) {
   Carver c{static_cast<char *>(ws), 0};
@@ -422,13 +422,26 @@ FP_API fp_status fp_prefill_attn_host(const fp_shape *shape, const fp_params *pa
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream), sin = nullptr, sout = nullptr;
   if (!copy_streams(&sin, &sout)) return FP_ERR_CUDA;
   // Every stage is independent per (batch, kv head) with its query heads, so
-  // the call runs as units of consecutive kv heads (about a quarter of them
-  // per batch entry): the inputs of unit u+1 are copied in while unit u
-  // computes on `stream`, and its output is copied out while unit u+1
-  // computes.  The caller's stream forks to the copy streams and joins them
-  // at the end through events, so `stream` still orders the whole call.
-  const int per_unit = (D.hkv + kHostUnits - 1) / kHostUnits;
-  const int units_per_batch = (D.hkv + per_unit - 1) / per_unit;
+  // the call runs as units of consecutive kv heads: the inputs of unit u+1
+  // are copied in while unit u computes on `stream`, and its output is copied
+  // out while unit u+1 computes.  Only the first unit's copy in and the last
+  // unit's copy out are not hidden, so those two units hold one kv head each
+  // and the rest of a batch entry's kv heads go in three middle units.  The
+  // caller's stream forks to the copy streams and joins them at the end
+  // through events, so `stream` still orders the whole call.
+  std::vector<int> plan;  // kv heads per unit, one batch entry
+  if (D.hkv >= 4) {
+    const int mid = D.hkv - 2;
+    plan.push_back(1);
+    for (int i = 0; i < kHostMidUnits; ++i) {
+      const int n = mid / kHostMidUnits + (i < mid % kHostMidUnits ? 1 : 0);
+      if (n > 0) plan.push_back(n);
+    }
+    plan.push_back(1);
+  } else {
+    plan.assign(D.hkv, 1);
+  }
+  const int units_per_batch = int(plan.size());
   const int nunits = D.bt * units_per_batch;
   std::vector<cudaEvent_t> ev;
   auto event = [&](cudaEvent_t *e) {
@@ -451,9 +464,10 @@ FP_API fp_status fp_prefill_attn_host(const fp_shape *shape, const fp_params *pa
   const char *vh = static_cast<const char *>(v_host);
   char *oh = static_cast<char *>(out_host);
   for (int u = 0; u < nunits; ++u) {
-    const int b = u / units_per_batch;
-    const int kv0 = (u % units_per_batch) * per_unit;
-    const int nk = std::min(per_unit, D.hkv - kv0);
+    const int b = u / units_per_batch, ui = u % units_per_batch;
+    int kv0 = 0;
+    for (int i = 0; i < ui; ++i) kv0 += plan[i];
+    const int nk = plan[ui];
     fp_shape us = *shape;
     us.batch = 1;
     us.n_kv_heads = nk;

@@ -297,8 +297,9 @@ fp_status fp_prefill_attn_varlen(const fp_shape *shape, const fp_params *params,
  * to device memory inside `ws` (fp_workspace_size(shape,
  * FP_CALL_PREFILL_HOST) bytes), runs the path and copies the output back to
  * out_host.  Every stage is independent per (batch entry, kv head), so the
- * call runs as units of about a quarter of the kv heads of one batch entry:
- * the inputs of a unit are copied in (one cudaMemcpyAsync per buffer slice)
+ * call runs as units of consecutive kv heads of one batch entry (one kv head
+ * in the first and last unit, whose copies cannot be hidden; the rest in
+ * three middle units): the inputs of a unit are copied in (one cudaMemcpyAsync per buffer slice)
  * while the previous unit computes on `stream`, and each unit's output is
  * copied out while the next one computes.  The copies run on two streams of
  * the library's own, created once per device on first use and kept until the
