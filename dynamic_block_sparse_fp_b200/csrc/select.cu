@@ -140,6 +140,7 @@ __device__ void histogram(const Ctx &cx, const float *__restrict__ s, uint32_t i
   // issues all their loads before using any, so the scan is not one load
   // latency per 32 entries
   constexpr uint32_t kHistU = 8;
+  constexpr int kHistAggMax = 8;
   for (uint32_t base = i0 + (threadIdx.x / 32) * 32 * kHistU; base < i1;
        base += kCThreads * kHistU) {
     uint32_t bits[kHistU];
@@ -158,11 +159,23 @@ __device__ void histogram(const Ctx &cx, const float *__restrict__ s, uint32_t i
         w = score_mass(bits[u]);
       }
       const unsigned peers = __match_any_sync(0xffffffffu, bin);
-      const unsigned lo = __reduce_add_sync(peers, unsigned(w & 0xFFFFFFull));
-      const unsigned hi = __reduce_add_sync(peers, unsigned(w >> 24));
-      if (bin != 0xFFFFFFFFu && lane == __ffs(peers) - 1) {
-        atomicAdd(&sm.hmass[bin], ((unsigned long long)hi << 24) + lo);
-        atomicAdd(&sm.hcnt[bin], unsigned(__popc(peers)));
+      const bool leader = lane == __ffs(peers) - 1;
+      // a reduction over one group of peers runs once per distinct group, so
+      // when the lanes spread over many bins (the levels below the exponent,
+      // where most scores differ) every lane adds its own entry instead; the
+      // sums are integers, so both ways give the same bins
+      if (__popc(__ballot_sync(0xffffffffu, leader)) > kHistAggMax) {
+        if (bin != 0xFFFFFFFFu) {
+          atomicAdd(&sm.hmass[bin], (unsigned long long)w);
+          atomicAdd(&sm.hcnt[bin], 1u);
+        }
+      } else {
+        const unsigned lo = __reduce_add_sync(peers, unsigned(w & 0xFFFFFFull));
+        const unsigned hi = __reduce_add_sync(peers, unsigned(w >> 24));
+        if (bin != 0xFFFFFFFFu && leader) {
+          atomicAdd(&sm.hmass[bin], ((unsigned long long)hi << 24) + lo);
+          atomicAdd(&sm.hcnt[bin], unsigned(__popc(peers)));
+        }
       }
     }
   }
