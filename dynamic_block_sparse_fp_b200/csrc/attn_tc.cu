@@ -246,13 +246,14 @@ __device__ __forceinline__ void tile_exp(const uint32_t (&u)[BN], int lim, float
   }
 }
 
-// One S tile of one row (TMEM lane): read out (then released); the row max
-// and the exponentials against the running max m are computed side by side
-// (independent instruction streams), and the exponentials are redone only
+// One S tile of one row (TMEM lane): read out (then released); the
+// exponentials are computed against the running max m first, and redone only
 // if some row of the warp needs a new max: the max grew by more than 2^8
 // (lazy rescale: p <= 256 is exact enough in fp32 and bf16, and the final
 // 1/l uses the same stale max, so the result is unchanged), or this is the
-// first tile.
+// first tile.  The tile max itself is computed only when that may be the
+// case (it costs a max per pair of scores, a fifth of the softmax's
+// instructions).
 template <bool MASK>
 __device__ __forceinline__ void softmax_tile(uint32_t s_addr, uint64_t *s_free, bool first,
                                              int lim, float sl2, float m, float &muse,
@@ -266,10 +267,18 @@ __device__ __forceinline__ void softmax_tile(uint32_t s_addr, uint64_t *s_free, 
   tc_fence_before();
   mbar_arrive(s_free);
   if (!first) tile_exp<MASK>(u, lim, sl2, m, acc, pk);
-  const float tmax = tile_max<MASK>(u, lim) * sl2;
   muse = m;
-  if (tmax > m + 8.0f || m == -INFINITY) muse = fmaxf(m, tmax);
-  if (muse == -INFINITY) muse = 0.f;  // every key so far masked
+  // the exact tile max is needed only where the lazy rule may move m: on the
+  // first tile, or when some key is more than 8 above m, i.e. some p > 2^8,
+  // which a tile sum <= 2^8 rules out (a NaN sum takes the exact path too)
+  const float ps0 = ((acc[0].x + acc[0].y) + (acc[1].x + acc[1].y)) +
+                    ((acc[2].x + acc[2].y) + (acc[3].x + acc[3].y));
+  const bool need = first || !(ps0 <= 256.f);
+  if (__any_sync(0xffffffffu, need)) {
+    const float tmax = tile_max<MASK>(u, lim) * sl2;
+    if (need && (tmax > m + 8.0f || m == -INFINITY)) muse = fmaxf(m, tmax);
+    if (muse == -INFINITY) muse = 0.f;  // every key so far masked
+  }
   if (__any_sync(0xffffffffu, first || muse != m)) {
 #pragma unroll
     for (int k = 0; k < 4; ++k) acc[k] = make_float2(0.f, 0.f);
