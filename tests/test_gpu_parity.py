@@ -464,6 +464,59 @@ def test_edge_empty_rows_and_device_checks():
         assert ops.fp_last_device_status() == 0
 
 
+def _staircase_inputs():
+    """bf16 Q/K/V (Bt 1, Hq 4, Hkv 2, N 1024, d 128) whose scores step from one
+    64-key tile to the next by a fixed amount: q = c e0 and k_j[0] = a_j (bf16
+    rounded; kernel and oracle read the same values), so
+    scale*log2(e)*q.k_j = 0.1275 c a_j.
+      head 0 (kv 0, c = 1):    +80 per tile, +10.3 in log2 units: the row max
+                               jumps by more than 2^8 on every tile;
+      head 1 (kv 0, c = -1):   the same keys falling: the max stays on the
+                               first tile, later p underflow towards 0;
+      head 2 (kv 1, c = 1):    +55 per tile, +7.1: tile sums above 2^8 with no
+                               move, then a move every second tile;
+      head 3 (kv 1, c = 0.5):  +3.6 per tile: a move every third tile.
+    A small within-tile ramp (j mod 7) keeps the rows from being flat."""
+    n, d = 1024, 128
+    j = torch.arange(n)
+    k = torch.zeros(1, 2, n, d)
+    k[0, 0, :, 0] = 80.0 * (j // 64) + (j % 7)
+    k[0, 1, :, 0] = 55.0 * (j // 64) + (j % 7)
+    k[:, :, :, 1:] = torch.randn(1, 2, n, d - 1, generator=torch.Generator().manual_seed(5))
+    q = torch.zeros(1, 4, n, d)
+    for h, c in enumerate((1.0, -1.0, 1.0, 0.5)):
+        q[0, h, :, 0] = c
+    v = torch.randn(1, 2, n, d, generator=torch.Generator().manual_seed(6))
+    return tuple(x.to(torch.bfloat16) for x in (q, k, v))
+
+
+def test_attention_lazy_rescale_paths():
+    """Rows whose running max moves by more than 2^8 on later tiles (O is
+    rescaled in TMEM), rows whose tile sums exceed 2^8 without a move, and
+    falling rows, dense and through sparse lists with gaps."""
+    q, k, v = _staircase_inputs()
+    qd, kd, vd = (x.to(DEV) for x in (q, k, v))
+    bs, nb = 128, 8
+    out, lse = ops.dense_attn(qd, kd, vd, bs)
+    torch.cuda.synchronize()
+    o, l = oracle.dense_attention(q, k, v, bs)
+    assert np.abs(_np(out) - o).max() <= 2e-2
+    assert np.abs(_np(lse) - l).max() <= 2e-3
+    # every other key block plus the diagonal: the max also jumps across gaps
+    counts = torch.zeros(1, 4, nb, dtype=torch.int32)
+    indices = torch.zeros(1, 4, nb, nb, dtype=torch.int32)
+    for qi in range(nb):
+        row = sorted(set(range(0, qi + 1, 2)) | {qi})
+        counts[0, :, qi] = len(row)
+        indices[0, :, qi, :len(row)] = torch.tensor(row, dtype=torch.int32)
+    out, lse = ops.sparse_attn(qd, kd, vd, counts.to(DEV), indices.to(DEV), bs)
+    torch.cuda.synchronize()
+    o, l = oracle.sparse_attention(q, k, v, counts.numpy(), indices.numpy(), bs)
+    assert np.abs(_np(out) - o).max() <= 2e-2
+    assert np.abs(_np(lse) - l).max() <= 2e-3
+    assert ops.fp_last_device_status() == 0
+
+
 def test_single_block_sequence():
     w, inp, d = _inputs("llama8b_n8192", seq_len=128, n_q_heads=8, n_kv_heads=2)
     res = _pipeline(w, d)
