@@ -277,7 +277,6 @@ __device__ __forceinline__ void softmax_tile(uint32_t s_addr, uint64_t *s_free, 
   if (__any_sync(0xffffffffu, need)) {
     const float tmax = tile_max<MASK>(u, lim) * sl2;
     if (need && (tmax > m + 8.0f || m == -INFINITY)) muse = fmaxf(m, tmax);
-    if (muse == -INFINITY) muse = 0.f;  // every key so far masked
   }
   if (__any_sync(0xffffffffu, first || muse != m)) {
 #pragma unroll
@@ -542,10 +541,14 @@ __global__ void __launch_bounds__(192, 2) attn_tc_kernel(
                        make_float2(0.f, 0.f)};
       uint32_t pk[BN / 2];
       const uint32_t s_addr = lane_base + S_COL;
+      // a row's first tile is its first with a key: until then every p is 0
+      // and m stays -inf (alpha 1), so m is taken from the row's own scores
+      // however low they are
+      const bool first = m == -INFINITY;
       if (masked)
-        softmax_tile<true>(s_addr, &sm.s_free, t == 0, lim, sl2, m, muse, alpha, acc, pk);
+        softmax_tile<true>(s_addr, &sm.s_free, first, lim, sl2, m, muse, alpha, acc, pk);
       else
-        softmax_tile<false>(s_addr, &sm.s_free, t == 0, lim, sl2, m, muse, alpha, acc, pk);
+        softmax_tile<false>(s_addr, &sm.s_free, first, lim, sl2, m, muse, alpha, acc, pk);
       const float ps = ((acc[0].x + acc[0].y) + (acc[1].x + acc[1].y)) +
                        ((acc[2].x + acc[2].y) + (acc[3].x + acc[3].y));
       l = l * alpha + ps;

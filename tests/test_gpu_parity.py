@@ -517,6 +517,36 @@ def test_attention_lazy_rescale_paths():
     assert ops.fp_last_device_status() == 0
 
 
+def test_attention_block64_masked_first_tiles_low_scores():
+    """Block size 64: a CTA's rows are two query blocks on the union of their
+    lists.  Rows of the odd block see the even block's tiles fully masked
+    first, then only their own diagonal block, whose scores are all about
+    -140 in log2 units; their softmax must still be the oracle's, not 0."""
+    n, d, bs = 512, 128, 64
+    nb = n // bs
+    j = torch.arange(n)
+    k = torch.zeros(1, 1, n, d)
+    k[0, 0, :, 0] = 1100.0 + (j % 7)
+    k[:, :, :, 1:] = torch.randn(1, 1, n, d - 1, generator=torch.Generator().manual_seed(7))
+    q = torch.zeros(1, 1, n, d)
+    q[0, 0, :, 0] = torch.where((j // bs) % 2 == 1, -1.0, 1.0)
+    v = torch.randn(1, 1, n, d, generator=torch.Generator().manual_seed(8))
+    q, k, v = (x.to(torch.bfloat16) for x in (q, k, v))
+    counts = torch.zeros(1, 1, nb, dtype=torch.int32)
+    indices = torch.zeros(1, 1, nb, nb, dtype=torch.int32)
+    for qi in range(nb):
+        row = list(range(qi + 1)) if qi % 2 == 0 else [qi]
+        counts[0, 0, qi] = len(row)
+        indices[0, 0, qi, :len(row)] = torch.tensor(row, dtype=torch.int32)
+    out, lse = ops.sparse_attn(q.to(DEV), k.to(DEV), v.to(DEV), counts.to(DEV),
+                               indices.to(DEV), bs)
+    torch.cuda.synchronize()
+    o, l = oracle.sparse_attention(q, k, v, counts.numpy(), indices.numpy(), bs)
+    assert np.abs(_np(out) - o).max() <= 2e-2
+    assert np.abs(_np(lse) - l).max() <= 2e-3
+    assert ops.fp_last_device_status() == 0
+
+
 def test_single_block_sequence():
     w, inp, d = _inputs("llama8b_n8192", seq_len=128, n_q_heads=8, n_kv_heads=2)
     res = _pipeline(w, d)
