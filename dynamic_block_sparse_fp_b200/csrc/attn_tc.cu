@@ -258,7 +258,7 @@ template <bool MASK>
 __device__ __forceinline__ void softmax_tile(uint32_t s_addr, uint64_t *s_free, bool first,
                                              int lim, float sl2, float m, float &muse,
                                              float &alpha, float2 (&acc)[4],
-                                             uint32_t (&pk)[BN / 2]) {
+                                             uint32_t (&pk)[BN / 2], float &ps) {
   uint32_t u[BN];
   tmem_ld32(s_addr, *reinterpret_cast<uint32_t(*)[32]>(&u[0]));
   tmem_ld32(s_addr + 32u, *reinterpret_cast<uint32_t(*)[32]>(&u[32]));
@@ -274,6 +274,7 @@ __device__ __forceinline__ void softmax_tile(uint32_t s_addr, uint64_t *s_free, 
   const float ps0 = ((acc[0].x + acc[0].y) + (acc[1].x + acc[1].y)) +
                     ((acc[2].x + acc[2].y) + (acc[3].x + acc[3].y));
   const bool need = first || !(ps0 <= 256.f);
+  ps = ps0;
   if (__any_sync(0xffffffffu, need)) {
     const float tmax = tile_max<MASK>(u, lim) * sl2;
     if (need && (tmax > m + 8.0f || m == -INFINITY)) muse = fmaxf(m, tmax);
@@ -282,6 +283,8 @@ __device__ __forceinline__ void softmax_tile(uint32_t s_addr, uint64_t *s_free, 
 #pragma unroll
     for (int k = 0; k < 4; ++k) acc[k] = make_float2(0.f, 0.f);
     tile_exp<MASK>(u, lim, sl2, muse, acc, pk);
+    ps = ((acc[0].x + acc[0].y) + (acc[1].x + acc[1].y)) +
+         ((acc[2].x + acc[2].y) + (acc[3].x + acc[3].y));
   }
   alpha = muse != m ? ex2(m - muse) : 1.f;  // 0 on the first tile
 }
@@ -536,7 +539,7 @@ __global__ void __launch_bounds__(192, 2) attn_tc_kernel(
       // row's list, or an invalid entry, hides all; other tiles are unmasked
       const bool masked = !valid || cur.j == qh;
       const int lim = valid ? rl - BN * cur.sub : -1;
-      float muse, alpha;
+      float muse, alpha, ps;
       float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
                        make_float2(0.f, 0.f)};
       uint32_t pk[BN / 2];
@@ -546,11 +549,9 @@ __global__ void __launch_bounds__(192, 2) attn_tc_kernel(
       // however low they are
       const bool first = m == -INFINITY;
       if (masked)
-        softmax_tile<true>(s_addr, &sm.s_free, first, lim, sl2, m, muse, alpha, acc, pk);
+        softmax_tile<true>(s_addr, &sm.s_free, first, lim, sl2, m, muse, alpha, acc, pk, ps);
       else
-        softmax_tile<false>(s_addr, &sm.s_free, first, lim, sl2, m, muse, alpha, acc, pk);
-      const float ps = ((acc[0].x + acc[0].y) + (acc[1].x + acc[1].y)) +
-                       ((acc[2].x + acc[2].y) + (acc[3].x + acc[3].y));
+        softmax_tile<false>(s_addr, &sm.s_free, first, lim, sl2, m, muse, alpha, acc, pk, ps);
       l = l * alpha + ps;
       // P(t) overwrites P(t-1), and O may be rescaled: both need P(t-1) V(t-1)
       // finished (for t = 0 the wait is on the phase before the first and
