@@ -421,25 +421,46 @@ FP_API fp_status fp_prefill_attn_host(const fp_shape *shape, const fp_params *pa
   char *pre = c.take<char>(carve_prefill(D, nullptr, &Pfull));
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream), sin = nullptr, sout = nullptr;
   if (!copy_streams(&sin, &sout)) return FP_ERR_CUDA;
-  // Every stage is independent per (batch, kv head) with its query heads, so
-  // the call runs as units of consecutive kv heads: the inputs of unit u+1
-  // are copied in while unit u computes on `stream`, and its output is copied
-  // out while unit u+1 computes.  Only the first unit's copy in and the last
-  // unit's copy out are not hidden, so those two units hold one kv head each
-  // and the rest of a batch entry's kv heads go in three middle units.  The
-  // caller's stream forks to the copy streams and joins them at the end
-  // through events, so `stream` still orders the whole call.
-  std::vector<int> plan;  // kv heads per unit, one batch entry
-  if (D.hkv >= 4) {
+  // Every stage is independent per query head (a query head reads only its
+  // kv head's K and V), so the call runs as units of consecutive heads: the
+  // inputs of unit u+1 are copied in while unit u computes on `stream`, and
+  // its output is copied out while unit u+1 computes.  Only the first unit's
+  // copy in and the last unit's copy out are not hidden, so those two units
+  // hold one query head each (with the first, its kv head's K and V come in;
+  // the second unit then brings only the rest of that kv head's Q), the next
+  // to them the rest of the first and last kv heads' query heads, and the
+  // kv heads between go in three middle units.  The caller's stream forks to
+  // the copy streams and joins them at the end through events, so `stream`
+  // still orders the whole call.
+  struct Unit {
+    int kv0, nk;  // kv heads [kv0, kv0 + nk)
+    int q0, nq;   // their query heads [kv0 g + q0, kv0 g + q0 + nq)
+    bool kv_in;   // this unit copies the kv heads' K and V in
+  };
+  std::vector<Unit> plan;  // one batch entry
+  auto whole = [&](int kv0, int nk) { plan.push_back({kv0, nk, 0, nk * D.g, true}); };
+  if (D.hkv >= 4 && D.g >= 2) {
+    plan.push_back({0, 1, 0, 1, true});
+    plan.push_back({0, 1, 1, D.g - 1, false});
     const int mid = D.hkv - 2;
-    plan.push_back(1);
-    for (int i = 0; i < kHostMidUnits; ++i) {
+    for (int i = 0, kv = 1; i < kHostMidUnits; ++i) {
       const int n = mid / kHostMidUnits + (i < mid % kHostMidUnits ? 1 : 0);
-      if (n > 0) plan.push_back(n);
+      if (n > 0) whole(kv, n);
+      kv += n;
     }
-    plan.push_back(1);
+    plan.push_back({D.hkv - 1, 1, 0, D.g - 1, true});
+    plan.push_back({D.hkv - 1, 1, D.g - 1, 1, false});
+  } else if (D.hkv >= 4) {
+    whole(0, 1);
+    const int mid = D.hkv - 2;
+    for (int i = 0, kv = 1; i < kHostMidUnits; ++i) {
+      const int n = mid / kHostMidUnits + (i < mid % kHostMidUnits ? 1 : 0);
+      if (n > 0) whole(kv, n);
+      kv += n;
+    }
+    whole(D.hkv - 1, 1);
   } else {
-    plan.assign(D.hkv, 1);
+    for (int kv = 0; kv < D.hkv; ++kv) whole(kv, 1);
   }
   const int units_per_batch = int(plan.size());
   const int nunits = D.bt * units_per_batch;
@@ -464,27 +485,28 @@ FP_API fp_status fp_prefill_attn_host(const fp_shape *shape, const fp_params *pa
   const char *vh = static_cast<const char *>(v_host);
   char *oh = static_cast<char *>(out_host);
   for (int u = 0; u < nunits; ++u) {
-    const int b = u / units_per_batch, ui = u % units_per_batch;
-    int kv0 = 0;
-    for (int i = 0; i < ui; ++i) kv0 += plan[i];
-    const int nk = plan[ui];
+    const int b = u / units_per_batch;
+    const Unit &un = plan[u % units_per_batch];
     fp_shape us = *shape;
     us.batch = 1;
-    us.n_kv_heads = nk;
-    us.n_q_heads = nk * D.g;
+    us.n_kv_heads = un.nk;
+    us.n_q_heads = un.nq;
     Dims Du;
     if (check_shape(&us, &Du) != FP_OK) return finish(FP_ERR_SHAPE);
-    const size_t qoff = (size_t(b) * D.hq + size_t(kv0) * D.g) * head_bytes;
-    const size_t kvoff = (size_t(b) * D.hkv + kv0) * head_bytes;
-    const size_t qlen = size_t(nk) * D.g * head_bytes, kvlen = size_t(nk) * head_bytes;
+    const size_t qoff = (size_t(b) * D.hq + size_t(un.kv0) * D.g + un.q0) * head_bytes;
+    const size_t kvoff = (size_t(b) * D.hkv + un.kv0) * head_bytes;
+    const size_t qlen = size_t(un.nq) * head_bytes, kvlen = size_t(un.nk) * head_bytes;
     cudaEvent_t e_in, e_comp;
     if (!event(&e_in) || !event(&e_comp) ||
-        cudaMemcpyAsync(qd + qoff, qh + qoff, qlen, cudaMemcpyHostToDevice, sin) != cudaSuccess ||
-        cudaMemcpyAsync(kd + kvoff, kh + kvoff, kvlen, cudaMemcpyHostToDevice, sin) !=
-            cudaSuccess ||
-        cudaMemcpyAsync(vd + kvoff, vh + kvoff, kvlen, cudaMemcpyHostToDevice, sin) !=
-            cudaSuccess ||
-        cudaEventRecord(e_in, sin) != cudaSuccess || cudaStreamWaitEvent(st, e_in, 0) != cudaSuccess)
+        cudaMemcpyAsync(qd + qoff, qh + qoff, qlen, cudaMemcpyHostToDevice, sin) != cudaSuccess)
+      return finish(FP_ERR_CUDA);
+    if (un.kv_in &&
+        (cudaMemcpyAsync(kd + kvoff, kh + kvoff, kvlen, cudaMemcpyHostToDevice, sin) !=
+             cudaSuccess ||
+         cudaMemcpyAsync(vd + kvoff, vh + kvoff, kvlen, cudaMemcpyHostToDevice, sin) !=
+             cudaSuccess))
+      return finish(FP_ERR_CUDA);
+    if (cudaEventRecord(e_in, sin) != cudaSuccess || cudaStreamWaitEvent(st, e_in, 0) != cudaSuccess)
       return finish(FP_ERR_CUDA);
     Prefill Pu;
     carve_prefill(Du, pre, &Pu);  // units run one after another on `stream`

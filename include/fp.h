@@ -296,12 +296,14 @@ fp_status fp_prefill_attn_varlen(const fp_shape *shape, const fp_params *params,
  * fp_prefill_attn_host -- fp_prefill_attn on HOST buffers: copies q, k, v
  * to device memory inside `ws` (fp_workspace_size(shape,
  * FP_CALL_PREFILL_HOST) bytes), runs the path and copies the output back to
- * out_host.  Every stage is independent per (batch entry, kv head), so the
- * call runs as units of consecutive kv heads of one batch entry (one kv head
- * in the first and last unit, whose copies cannot be hidden; the rest in
- * three middle units): the inputs of a unit are copied in (one cudaMemcpyAsync per buffer slice)
- * while the previous unit computes on `stream`, and each unit's output is
- * copied out while the next one computes.  The copies run on two streams of
+ * out_host.  Every stage is independent per query head, so the call runs as
+ * units of consecutive heads of one batch entry (one query head in the first
+ * and in the last unit, whose copies cannot be hidden; the rest of the first
+ * and last kv heads' query heads next to them; the kv heads between in three
+ * middle units): the inputs of a unit are copied in (one cudaMemcpyAsync per
+ * buffer slice; a kv head's K and V with its first unit) while the previous
+ * unit computes on `stream`, and each unit's output is copied out while the
+ * next one computes.  The copies run on two streams of
  * the library's own, created once per device on first use and kept until the
  * process exits; `stream` forks to them and joins them through events, so
  * work enqueued on `stream` after this call sees the finished output.
