@@ -375,6 +375,28 @@ def test_host_path_batch2_fp32_matches_device_path():
     assert ops.fp_last_device_status() == 0
 
 
+@pytest.mark.parametrize("batch,hq,hkv", [(1, 4, 4), (2, 8, 4)])
+def test_host_path_unit_plans_match_device_path(batch, hq, hkv):
+    """The host path's unit plans: one query head per kv head (whole kv heads
+    in every unit) and, with two query heads per kv head over two batch
+    entries, single-query-head first and last units whose kv heads' K and V
+    come in with the first; bitwise the device path's output."""
+    w = synth.WORKLOADS["llama8b_n8192"].replace(batch=batch, seq_len=1024, n_q_heads=hq,
+                                                 n_kv_heads=hkv)
+    inp = synth.make_inputs(w)
+    d = {x: inp[x].to(DEV) for x in ("q", "k", "v")}
+    s = ops.make_shape(d["q"], d["k"], w.block_size)
+    p = ops.make_params(w.gamma, w.tau, w.min_budget, w.max_budget)
+    out, _, _ = ops.prefill_attn(d["q"], d["k"], d["v"], w.block_size, p)
+    qh, kh, vh = (inp[x].contiguous().pin_memory() for x in ("q", "k", "v"))
+    oh = torch.empty_like(qh).pin_memory()
+    ws = ops.workspace(s, ops.FP_CALL_PREFILL_HOST, DEV)
+    assert ops.fp_prefill_attn_host(s, p, qh, kh, vh, oh, ws) == 0
+    torch.cuda.synchronize()
+    assert torch.equal(oh, out.cpu())
+    assert ops.fp_last_device_status() == 0
+
+
 def test_sharded_single_rank_is_the_whole_path():
     """With one rank the head-sharded entry is fp_prefill_attn, bitwise."""
     from dynamic_block_sparse_fp_b200 import sharded
