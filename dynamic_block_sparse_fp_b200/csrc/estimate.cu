@@ -448,9 +448,10 @@ cudaError_t run_true_last(const Dims &Dm, const T *q, const T *k, float *true_la
     float *sp = nullptr;
     cudaError_t e = launch_last_block_tc(Dm, q, k, true_last, vert, &sp, ws, st);
     if (e != cudaSuccess) return e;
+    // the passes' partials are per 128-key tile, whatever the block size
     const long long tot = (long long)Dm.bt * Dm.hq * Dm.n;
-    slash_combine_kernel<<<unsigned((tot + 255) / 256), 256, 0, st>>>(sp, slash, tot, Dm.n,
-                                                                      Dm.nb, Dm.bs);
+    slash_combine_kernel<<<unsigned((tot + 255) / 256), 256, 0, st>>>(
+        sp, slash, tot, Dm.n, last_block_tc_tiles(Dm), 128);
     return cudaGetLastError();
   }
   if (Dm.bs == 128 && Dm.d == 128)

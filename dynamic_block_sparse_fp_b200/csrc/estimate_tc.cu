@@ -64,10 +64,13 @@ __device__ __forceinline__ void wg_sync(int wg) {
   asm volatile("bar.sync %0, 128;" ::"r"(wg + 1) : "memory");
 }
 
+// nb counts 128-key tiles.  Block size 64 runs the same tiles: the queries are
+// the last 128 rows with the first q_lo = 64 left out of every sum, and each
+// tile holds two output blocks (nb_out = 2 nb).
 template <int PASS>
 __global__ void __launch_bounds__(kThreads, 1) last_block_tc_kernel(
     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-    int hq, int g, int n_tok, int nb, int n_chunks, float *__restrict__ pm,
+    int hq, int g, int n_tok, int nb, int q_lo, int nb_out, int n_chunks, float *__restrict__ pm,
     float *__restrict__ pl, const float *__restrict__ lse2g, float *__restrict__ vert,
     float *__restrict__ true_last, float *__restrict__ sp, int *status) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -271,8 +274,10 @@ __global__ void __launch_bounds__(kThreads, 1) last_block_tc_kernel(
             lqb[2] = lb.z;
             lqb[3] = lb.w;
           }
-          const float pa = (diag && r > c) ? 0.f : ex2(fmaf(x[c], sl2, -lqa[c % 4]));
-          const float pb = (diag && r > cb) ? 0.f : ex2(fmaf(x[cb], sl2, -lqb[c % 4]));
+          const float pa =
+              (c < q_lo || (diag && r > c)) ? 0.f : ex2(fmaf(x[c], sl2, -lqa[c % 4]));
+          const float pb =
+              (cb < q_lo || (diag && r > cb)) ? 0.f : ex2(fmaf(x[cb], sl2, -lqb[c % 4]));
           v4[c % 4] += pa;
           v4[c % 4] += pb;
           const float ua = __shfl_up_sync(0xffffffffu, acc_a, 1);
@@ -295,11 +300,16 @@ __global__ void __launch_bounds__(kThreads, 1) last_block_tc_kernel(
         for (int o = 16; o > 0; o >>= 1) wsum += __shfl_xor_sync(0xffffffffu, wsum, o);
         if (lane == 0) sm.warp_mass[hh][wq] = wsum;
         wg_sync(hh);
-        if (r == 0)
-          true_last[bh * nb + j] =
-              (sm.warp_mass[hh][0] + sm.warp_mass[hh][1] + sm.warp_mass[hh][2] +
-               sm.warp_mass[hh][3]) /
-              float(BS);
+        if (r == 0) {
+          const float *wm = sm.warp_mass[hh];
+          if (q_lo == 0) {
+            true_last[bh * nb_out + j] = (wm[0] + wm[1] + wm[2] + wm[3]) / float(BS);
+          } else {  // block 2j: keys 0-63 (warps 0, 1); block 2j + 1: keys 64-127
+            const float rows = float(BS - q_lo);
+            true_last[bh * nb_out + 2 * j] = (wm[0] + wm[1]) / rows;
+            true_last[bh * nb_out + 2 * j + 1] = (wm[2] + wm[3]) / rows;
+          }
+        }
         // tile diagonal D = query - key in [-127, 127] -> partial index D + 127;
         // warp w holds D = (bin - 31) - 32 w
         float *dst = sp + (bh * nb + j) * size_t(kBins);
@@ -370,22 +380,27 @@ bool encode_rows(CUtensorMap *map, const void *ptr, uint64_t rows) {
 }  // namespace
 
 bool last_block_tc_supported(const Dims &D) {
-  return D.dtype == FP_BF16 && D.bs == BS && D.d == HD;
+  return D.dtype == FP_BF16 && D.d == HD && (D.bs == BS || (D.bs == BS / 2 && D.n % BS == 0));
 }
+
+// 128-key tiles of the passes (block size 64 runs two blocks per tile)
+int last_block_tc_tiles(const Dims &D) { return D.n / BS; }
 
 size_t last_block_tc_ws_bytes(const Dims &D) {
   Carver c{nullptr, 0};
   const size_t heads = size_t(D.bt) * D.hq;
-  const int n_chunks = (D.nb + kChunk - 1) / kChunk;
+  const int nt = last_block_tc_tiles(D);
+  const int n_chunks = (nt + kChunk - 1) / kChunk;
   c.take<float>(heads * n_chunks * BS);
   c.take<float>(heads * n_chunks * BS);
   c.take<float>(heads * BS);
-  c.take<float>(heads * D.nb * size_t(kBins));
+  c.take<float>(heads * nt * size_t(kBins));
   return c.off + 256;
 }
 
-// Writes true_last and vert, and the diagonal partials sp [Bt,Hq,nb,2B-1]
-// (combined into slash by the caller's slash_combine step).
+// Writes true_last and vert, and the diagonal partials sp [Bt,Hq,n/128,255]
+// of the 128-key tiles (combined into slash by the caller's slash_combine
+// step with block size 128).
 cudaError_t launch_last_block_tc(const Dims &D, const void *q, const void *k, float *true_last,
                                  float *vert, float **sp_out, void *ws, cudaStream_t st) {
   CUtensorMap mq, mk;
@@ -394,11 +409,13 @@ cudaError_t launch_last_block_tc(const Dims &D, const void *q, const void *k, fl
     return cudaErrorInvalidValue;
   Carver c{static_cast<char *>(ws), 0};
   const size_t heads = size_t(D.bt) * D.hq;
-  const int n_chunks = (D.nb + kChunk - 1) / kChunk;
+  const int nt = last_block_tc_tiles(D);
+  const int q_lo = BS - D.bs;  // block 64: the last 128 rows minus the first 64
+  const int n_chunks = (nt + kChunk - 1) / kChunk;
   float *pm = c.take<float>(heads * n_chunks * BS);
   float *pl = c.take<float>(heads * n_chunks * BS);
   float *lse2 = c.take<float>(heads * BS);
-  float *sp = c.take<float>(heads * D.nb * size_t(kBins));
+  float *sp = c.take<float>(heads * nt * size_t(kBins));
   *sp_out = sp;
   cudaFuncSetAttribute(last_block_tc_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                        int(kSmemBytes));
@@ -407,13 +424,13 @@ cudaError_t launch_last_block_tc(const Dims &D, const void *q, const void *k, fl
   const dim3 grid(n_chunks, D.hkv * ((D.g + 1) / 2), D.bt);
   int *status = device_status_ptr();
   last_block_tc_kernel<1><<<grid, kThreads, kSmemBytes, st>>>(
-      mq, mk, D.hq, D.g, D.n, D.nb, n_chunks, pm, pl, nullptr, nullptr, nullptr, nullptr,
-      status);
+      mq, mk, D.hq, D.g, D.n, nt, q_lo, D.nb, n_chunks, pm, pl, nullptr, nullptr, nullptr,
+      nullptr, status);
   const int rows = int(heads * BS);
   lse2_combine_kernel<<<(rows + 127) / 128, 128, 0, st>>>(pm, pl, lse2, rows, n_chunks);
   last_block_tc_kernel<2><<<grid, kThreads, kSmemBytes, st>>>(
-      mq, mk, D.hq, D.g, D.n, D.nb, n_chunks, nullptr, nullptr, lse2, vert, true_last, sp,
-      status);
+      mq, mk, D.hq, D.g, D.n, nt, q_lo, D.nb, n_chunks, nullptr, nullptr, lse2, vert,
+      true_last, sp, status);
   return cudaGetLastError();
 }
 

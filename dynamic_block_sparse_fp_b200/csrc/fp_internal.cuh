@@ -59,6 +59,7 @@ cudaError_t launch_estimate_map_qa(const Dims &D, const void *q, float *qbar, co
 // Tensor-core passes over the last query block (estimate_tc.cu): bf16,
 // block 128, head dim 128.
 bool last_block_tc_supported(const Dims &D);
+int last_block_tc_tiles(const Dims &D);
 size_t last_block_tc_ws_bytes(const Dims &D);
 cudaError_t launch_last_block_tc(const Dims &D, const void *q, const void *k, float *true_last,
                                  float *vert, float **sp_out, void *ws, cudaStream_t st);

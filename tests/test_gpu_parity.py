@@ -63,6 +63,19 @@ def test_estimate_parity(name):
     assert ops.fp_last_device_status() == 0
 
 
+@pytest.mark.parametrize("n", [1024, 1088])
+def test_estimate_parity_block64_bf16(n):
+    """Block size 64, bf16: N a multiple of 128 runs the tensor-core last-block
+    passes on 128-key tiles with the first 64 of the last 128 queries left out;
+    N = 1088 (an odd number of blocks) takes the CUDA-core passes."""
+    w, inp, d = _inputs("glm9b_n65536_b64", seq_len=n, n_q_heads=8, n_kv_heads=2)
+    got = ops.estimate(d["q"], d["k"], 64)
+    torch.cuda.synchronize()
+    want = oracle.estimate(inp["q"], inp["k"], 64)
+    _estimate_close(got, want, f"b64bf16n{n}")
+    assert ops.fp_last_device_status() == 0
+
+
 def test_estimate_parity_block64_and_d128_fp32():
     w, inp, d = _inputs("tiny_n1024", head_dim=128, n_q_heads=4, n_kv_heads=2,
                         fixed_kinds=("qa", "vs"), seq_len=512)
