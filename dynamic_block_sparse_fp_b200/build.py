@@ -40,7 +40,9 @@ def build(force: bool = False, verbose: bool = False, extra: list[str] | None = 
     if not force and up_to_date():
         return LIB
     nvcc = os.environ.get("NVCC", "nvcc")
-    tmp = LIB + ".tmp"
+    # one temporary per process: ranks that find the library stale at the same
+    # time each build their own copy, and the atomic rename keeps a whole one
+    tmp = f"{LIB}.tmp.{os.getpid()}"
     cmd = [nvcc, *NVCC_FLAGS, *(extra or []), "-shared", "-o", tmp, *sources(),
            "-Xlinker", "--version-script=" + os.path.join(CSRC, "exports.map")]
     if verbose:
