@@ -64,13 +64,14 @@ __device__ __forceinline__ void wg_sync(int wg) {
   asm volatile("bar.sync %0, 128;" ::"r"(wg + 1) : "memory");
 }
 
-// nb counts 128-key tiles.  Block size 64 runs the same tiles: the queries are
-// the last 128 rows with the first q_lo = 64 left out of every sum, and each
-// tile holds two output blocks (nb_out = 2 nb).
-template <int PASS>
+// nb counts 128-key tiles.  Block size 64 (QLO = 64) runs the same tiles: the
+// queries are the last 128 rows with the first QLO left out of every sum, and
+// each tile holds two output blocks (nb_out = 2 nb).  QLO is a template
+// parameter so that block size 128 carries no extra compare per element.
+template <int PASS, int QLO>
 __global__ void __launch_bounds__(kThreads, 1) last_block_tc_kernel(
     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-    int hq, int g, int n_tok, int nb, int q_lo, int nb_out, int n_chunks, float *__restrict__ pm,
+    int hq, int g, int n_tok, int nb, int nb_out, int n_chunks, float *__restrict__ pm,
     float *__restrict__ pl, const float *__restrict__ lse2g, float *__restrict__ vert,
     float *__restrict__ true_last, float *__restrict__ sp, int *status) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -275,9 +276,9 @@ __global__ void __launch_bounds__(kThreads, 1) last_block_tc_kernel(
             lqb[3] = lb.w;
           }
           const float pa =
-              (c < q_lo || (diag && r > c)) ? 0.f : ex2(fmaf(x[c], sl2, -lqa[c % 4]));
+              (c < QLO || (diag && r > c)) ? 0.f : ex2(fmaf(x[c], sl2, -lqa[c % 4]));
           const float pb =
-              (cb < q_lo || (diag && r > cb)) ? 0.f : ex2(fmaf(x[cb], sl2, -lqb[c % 4]));
+              (cb < QLO || (diag && r > cb)) ? 0.f : ex2(fmaf(x[cb], sl2, -lqb[c % 4]));
           v4[c % 4] += pa;
           v4[c % 4] += pb;
           const float ua = __shfl_up_sync(0xffffffffu, acc_a, 1);
@@ -302,10 +303,10 @@ __global__ void __launch_bounds__(kThreads, 1) last_block_tc_kernel(
         wg_sync(hh);
         if (r == 0) {
           const float *wm = sm.warp_mass[hh];
-          if (q_lo == 0) {
+          if (QLO == 0) {
             true_last[bh * nb_out + j] = (wm[0] + wm[1] + wm[2] + wm[3]) / float(BS);
           } else {  // block 2j: keys 0-63 (warps 0, 1); block 2j + 1: keys 64-127
-            const float rows = float(BS - q_lo);
+            const float rows = float(BS - QLO);
             true_last[bh * nb_out + 2 * j] = (wm[0] + wm[1]) / rows;
             true_last[bh * nb_out + 2 * j + 1] = (wm[2] + wm[3]) / rows;
           }
@@ -417,20 +418,23 @@ cudaError_t launch_last_block_tc(const Dims &D, const void *q, const void *k, fl
   float *lse2 = c.take<float>(heads * BS);
   float *sp = c.take<float>(heads * nt * size_t(kBins));
   *sp_out = sp;
-  cudaFuncSetAttribute(last_block_tc_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                       int(kSmemBytes));
-  cudaFuncSetAttribute(last_block_tc_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                       int(kSmemBytes));
   const dim3 grid(n_chunks, D.hkv * ((D.g + 1) / 2), D.bt);
   int *status = device_status_ptr();
-  last_block_tc_kernel<1><<<grid, kThreads, kSmemBytes, st>>>(
-      mq, mk, D.hq, D.g, D.n, nt, q_lo, D.nb, n_chunks, pm, pl, nullptr, nullptr, nullptr,
-      nullptr, status);
   const int rows = int(heads * BS);
-  lse2_combine_kernel<<<(rows + 127) / 128, 128, 0, st>>>(pm, pl, lse2, rows, n_chunks);
-  last_block_tc_kernel<2><<<grid, kThreads, kSmemBytes, st>>>(
-      mq, mk, D.hq, D.g, D.n, nt, q_lo, D.nb, n_chunks, nullptr, nullptr, lse2, vert,
-      true_last, sp, status);
+  auto passes = [&](auto pass1, auto pass2) {
+    cudaFuncSetAttribute(pass1, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmemBytes));
+    cudaFuncSetAttribute(pass2, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmemBytes));
+    pass1<<<grid, kThreads, kSmemBytes, st>>>(mq, mk, D.hq, D.g, D.n, nt, D.nb, n_chunks, pm, pl,
+                                              nullptr, nullptr, nullptr, nullptr, status);
+    lse2_combine_kernel<<<(rows + 127) / 128, 128, 0, st>>>(pm, pl, lse2, rows, n_chunks);
+    pass2<<<grid, kThreads, kSmemBytes, st>>>(mq, mk, D.hq, D.g, D.n, nt, D.nb, n_chunks,
+                                              nullptr, nullptr, lse2, vert, true_last, sp,
+                                              status);
+  };
+  if (q_lo == 0)
+    passes(last_block_tc_kernel<1, 0>, last_block_tc_kernel<2, 0>);
+  else
+    passes(last_block_tc_kernel<1, BS / 2>, last_block_tc_kernel<2, BS / 2>);
   return cudaGetLastError();
 }
 
