@@ -197,9 +197,11 @@ fp_status run_attn(const Dims &D, const void *q, const void *k, const void *v,
 // head; then Q pooling and the block map only for the query-aware heads (the
 // vertical-slash heads' selection never reads them).  Every value is bitwise
 // the one the separate fp_estimate / fp_pattern / fp_select calls produce.
+// `v_ready` (may be null): an event the attention stage waits for, the only
+// stage that reads v (the host path's copy of v in lands behind it).
 fp_status run_prefill(const Dims &D, const fp_params &p, const void *q, const void *k,
                       const void *v, void *out, float *lse, int64_t *stats, const Prefill &P,
-                      cudaStream_t st) {
+                      cudaStream_t st, cudaEvent_t v_ready = nullptr) {
   cudaError_t e = launch_estimate_decision(D, q, k, P.qbar, P.kbar, P.map, P.est_last,
                                            P.true_last, P.vert, P.slash, P.stage_ws, st);
   if (e != cudaSuccess) return FP_ERR_CUDA;
@@ -212,6 +214,7 @@ fp_status run_prefill(const Dims &D, const fp_params &p, const void *q, const vo
   if (e != cudaSuccess) return FP_ERR_CUDA;
   if (stats && launch_stats(D, P.counts, P.pattern, stats, st) != cudaSuccess)
     return FP_ERR_CUDA;
+  if (v_ready && cudaStreamWaitEvent(st, v_ready, 0) != cudaSuccess) return FP_ERR_CUDA;
   return run_attn(D, q, k, v, P.counts, P.indices, out, lse, false, P.stage_ws, st);
 }
 
@@ -496,22 +499,27 @@ FP_API fp_status fp_prefill_attn_host(const fp_shape *shape, const fp_params *pa
     const size_t qoff = (size_t(b) * D.hq + size_t(un.kv0) * D.g + un.q0) * head_bytes;
     const size_t kvoff = (size_t(b) * D.hkv + un.kv0) * head_bytes;
     const size_t qlen = size_t(un.nq) * head_bytes, kvlen = size_t(un.nk) * head_bytes;
-    cudaEvent_t e_in, e_comp;
+    // Q and K first: the unit's estimate can start on them, while V (read only
+    // by the attention stage) is still coming in behind its own event
+    cudaEvent_t e_in, e_v = nullptr, e_comp;
     if (!event(&e_in) || !event(&e_comp) ||
         cudaMemcpyAsync(qd + qoff, qh + qoff, qlen, cudaMemcpyHostToDevice, sin) != cudaSuccess)
       return finish(FP_ERR_CUDA);
     if (un.kv_in &&
-        (cudaMemcpyAsync(kd + kvoff, kh + kvoff, kvlen, cudaMemcpyHostToDevice, sin) !=
-             cudaSuccess ||
-         cudaMemcpyAsync(vd + kvoff, vh + kvoff, kvlen, cudaMemcpyHostToDevice, sin) !=
-             cudaSuccess))
+        cudaMemcpyAsync(kd + kvoff, kh + kvoff, kvlen, cudaMemcpyHostToDevice, sin) != cudaSuccess)
       return finish(FP_ERR_CUDA);
     if (cudaEventRecord(e_in, sin) != cudaSuccess || cudaStreamWaitEvent(st, e_in, 0) != cudaSuccess)
+      return finish(FP_ERR_CUDA);
+    if (un.kv_in &&
+        (!event(&e_v) ||
+         cudaMemcpyAsync(vd + kvoff, vh + kvoff, kvlen, cudaMemcpyHostToDevice, sin) !=
+             cudaSuccess ||
+         cudaEventRecord(e_v, sin) != cudaSuccess))
       return finish(FP_ERR_CUDA);
     Prefill Pu;
     carve_prefill(Du, pre, &Pu);  // units run one after another on `stream`
     const fp_status r = run_prefill(Du, *params, qd + qoff, kd + kvoff, vd + kvoff, od + qoff,
-                                    nullptr, nullptr, Pu, st);
+                                    nullptr, nullptr, Pu, st, e_v);
     if (r != FP_OK) return finish(r);
     if (cudaEventRecord(e_comp, st) != cudaSuccess ||
         cudaStreamWaitEvent(sout, e_comp, 0) != cudaSuccess ||
