@@ -1,0 +1,52 @@
+"""Host-side checks of bench.py's roofline bookkeeping (no GPU).
+
+The `traffic` figure of the bench line comes from a committed one-pass ncu
+capture of the attention kernel; it may be used only while the kernel source
+is the one that was captured, and only for the workload it was captured on.
+"""
+import hashlib
+import json
+import os
+
+import bench
+
+
+def _tree(tmp_path, src_text: str, rec: dict | None):
+    csrc = tmp_path / "dynamic_block_sparse_fp_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    (csrc / "k.cu").write_text(src_text)
+    (tmp_path / "profiles").mkdir()
+    if rec is not None:
+        (tmp_path / "profiles" / "k_traffic.json").write_text(json.dumps(rec))
+    return tmp_path
+
+
+def _rec(src_text: str, workload="w1", nbytes=1234):
+    return {"source_sha256": hashlib.sha256(src_text.encode()).hexdigest(),
+            "workload": workload, "bytes_per_launch": nbytes}
+
+
+def test_traffic_used_only_for_the_captured_source_and_workload(tmp_path, monkeypatch):
+    src = "// kernel v1\n"
+    root = _tree(tmp_path, src, _rec(src))
+    monkeypatch.setattr(bench, "ROOT", str(root))
+    assert bench.kernel_traffic("k.cu", "w1") == 1234
+    assert bench.kernel_traffic("k.cu", "w2") is None          # another workload
+    (root / "dynamic_block_sparse_fp_b200" / "csrc" / "k.cu").write_text("// kernel v2\n")
+    assert bench.kernel_traffic("k.cu", "w1") is None          # the kernel changed
+
+
+def test_traffic_missing_record_or_source_is_none(tmp_path, monkeypatch):
+    root = _tree(tmp_path, "// kernel\n", None)
+    monkeypatch.setattr(bench, "ROOT", str(root))
+    assert bench.kernel_traffic("k.cu", "w1") is None
+    assert bench.kernel_traffic("absent.cu", "w1") is None
+
+
+def test_committed_record_names_a_real_kernel_and_the_bench_workload():
+    """The committed capture is of attn_tc.cu on the bench's default workload
+    and is a plausible DRAM figure (at least the algorithmic Q + K + V + O)."""
+    rec = json.load(open(os.path.join(bench.ROOT, "profiles", "attn_tc_traffic.json")))
+    assert rec["workload"] == "llama8b_n131072"
+    assert len(rec["source_sha256"]) == 64
+    assert rec["bytes_per_launch"] >= 2 * 1_073_741_824 + 2 * 268_435_456
