@@ -6,8 +6,10 @@ CUDA kernels behind the C ABI):
 * ``fp_*`` functions with the C names and the C argument order; tensors are
   passed as device pointers, the stream defaults to torch's current stream.
 * allocation helpers (``estimate``, ``pattern``, ``select``, ``sparse_attn``,
-  ``dense_attn``, ``prefill_attn``, ``prefill_attn_host``) that create the
-  output tensors and workspace with torch and call the ``fp_*`` function.
+  ``dense_attn``, ``prefill_attn``, ``prefill_attn_varlen``) that create the
+  output tensors and workspace with torch and call the ``fp_*`` function
+  (``fp_prefill_attn_host`` takes caller-made page-locked host tensors and a
+  ``workspace(shape, FP_CALL_PREFILL_HOST, device)``).
 
 The library is loaded on first use; if it is missing this raises instead of
 falling back to anything else.
@@ -237,6 +239,7 @@ def _nbytes(t) -> int:
 # ------------------------------------------------------- allocation helpers --
 
 def workspace(shape: fp_shape, which_call: int, device) -> torch.Tensor | None:
+    """A device byte buffer of fp_workspace_size(shape, which_call), or None if 0."""
     n = fp_workspace_size(shape, which_call)
     if n == 0:
         return None
@@ -244,6 +247,8 @@ def workspace(shape: fp_shape, which_call: int, device) -> torch.Tensor | None:
 
 
 def estimate(q, k, block_size: int, stream=None) -> dict:
+    """fp_estimate: dict of qbar, kbar, map (packed causal), est_last, true_last,
+    vert, slash (fp32 device tensors)."""
     s = make_shape(q, k, block_size)
     dev = q.device
     bt, hq, n, d = q.shape
@@ -260,6 +265,7 @@ def estimate(q, k, block_size: int, stream=None) -> dict:
 
 
 def pattern(shape: fp_shape, params: fp_params, est_last, true_last, stream=None):
+    """fp_pattern: (d_JS fp32 [Bt, Hq], pattern int32 [Bt, Hq])."""
     bt, hq = est_last.shape[:2]
     djs = torch.empty(bt, hq, dtype=torch.float32, device=est_last.device)
     pat = torch.empty(bt, hq, dtype=torch.int32, device=est_last.device)
@@ -268,6 +274,8 @@ def pattern(shape: fp_shape, params: fp_params, est_last, true_last, stream=None
 
 
 def select(shape: fp_shape, params: fp_params, pat, map_, vert, slash, stream=None):
+    """fp_select: (counts int32 [Bt, Hq, nb], indices int32 [Bt, Hq, nb, nb]),
+    each row's list ascending in its first counts entries."""
     bt, hq, nb = shape.batch, shape.n_q_heads, shape.seq_len // shape.block_size
     dev = map_.device
     counts = torch.empty(bt, hq, nb, dtype=torch.int32, device=dev)
@@ -280,6 +288,7 @@ def select(shape: fp_shape, params: fp_params, pat, map_, vert, slash, stream=No
 
 def sparse_attn(q, k, v, counts, indices, block_size: int, with_lse: bool = True,
                 stream=None):
+    """fp_sparse_attn: (out like q, lse fp32 [Bt, Hq, N] or None)."""
     s = make_shape(q, k, block_size)
     out = torch.empty_like(q)
     lse = torch.empty(q.shape[:3], dtype=torch.float32, device=q.device) if with_lse else None
@@ -289,6 +298,7 @@ def sparse_attn(q, k, v, counts, indices, block_size: int, with_lse: bool = True
 
 
 def dense_attn(q, k, v, block_size: int, with_lse: bool = True, stream=None):
+    """fp_dense_attn: causal attention over every block; (out, lse or None)."""
     s = make_shape(q, k, block_size)
     out = torch.empty_like(q)
     lse = torch.empty(q.shape[:3], dtype=torch.float32, device=q.device) if with_lse else None
@@ -327,6 +337,8 @@ def prefill_attn_varlen(seqs_q, seqs_k, seqs_v, block_size: int, params: fp_para
 
 def prefill_attn(q, k, v, block_size: int, params: fp_params, with_lse: bool = False,
                  ws=None, stream=None):
+    """fp_prefill_attn, the whole path on device tensors: (out, lse or None,
+    stats int64 [kept blocks, query-aware heads])."""
     s = make_shape(q, k, block_size)
     out = torch.empty_like(q)
     lse = torch.empty(q.shape[:3], dtype=torch.float32, device=q.device) if with_lse else None
