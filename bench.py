@@ -9,8 +9,11 @@ d = 128, block 128).  Prints ONE JSON line (rank 0).
 
 --impl reference times the CPU oracle (the plain fp64 restatement of the
 method) on a bounded sample of the same workload.  Multi-GPU runs (torchrun)
-give every rank its own layer (independent problems, weak scaling); there is
-no exchange on the data path.
+split the layer's kv heads over the ranks (every stage is per head, so the
+path itself has no exchange) and all-gather the outputs inside the step
+(strong scaling); --shard layers gives every rank its own layer instead
+(independent problems, weak scaling).  --sweep prints one line per point of
+the gamma x tau x min x max budget sweep instead of the headline line.
 """
 from __future__ import annotations
 
@@ -267,6 +270,159 @@ def run_reference(args, w, ws, rank):
 
 # --------------------------------------------------------------------- ours --
 
+# the config-3 sweep at 128k: gamma x tau x min budget x max budget (0 = uncapped)
+SWEEP = [(g, t, lo, hi) for g in (0.9, 0.95) for t in (0.0, 0.1, 0.3) for lo in (1024, 2048)
+         for hi in (0, 8192)]
+
+
+class Layer:
+    """Device buffers of one layer and the four-call step over them."""
+
+    def __init__(self, ops, q, k, v, bs, dev):
+        self.ops = ops
+        self.q, self.k, self.v = q, k, v
+        bt, hq, n, d = q.shape
+        hkv = k.shape[1]
+        nb = n // bs
+        self.bs, self.nb = bs, nb
+        self.s = ops.make_shape(q, k, bs)
+        f32 = dict(dtype=torch.float32, device=dev)
+        self.qbar = torch.empty(bt, hq, nb, d, **f32)
+        self.kbar = torch.empty(bt, hkv, nb, d, **f32)
+        self.amap = torch.empty(bt, hq, nb * (nb + 1) // 2, **f32)
+        self.est_last = torch.empty(bt, hq, nb, **f32)
+        self.true_last = torch.empty(bt, hq, nb, **f32)
+        self.vert = torch.empty(bt, hq, n, **f32)
+        self.slash = torch.empty(bt, hq, n, **f32)
+        self.djs = torch.empty(bt, hq, **f32)
+        self.pat = torch.empty(bt, hq, dtype=torch.int32, device=dev)
+        self.counts = torch.empty(bt, hq, nb, dtype=torch.int32, device=dev)
+        self.indices = torch.empty(bt, hq, nb, nb, dtype=torch.int32, device=dev)
+        self.out = torch.empty_like(q)
+        self.ws_est = ops.workspace(self.s, ops.FP_CALL_ESTIMATE, dev)
+        self.ws_sel = ops.workspace(self.s, ops.FP_CALL_SELECT, dev)
+
+    def step(self, p, e, stream, gather=None):
+        ops = self.ops
+        e[0].record(stream)
+        ops._check(ops.fp_estimate(self.s, self.q, self.k, self.qbar, self.kbar, self.amap,
+                                   self.est_last, self.true_last, self.vert, self.slash,
+                                   self.ws_est, stream), "fp_estimate")
+        e[1].record(stream)
+        ops._check(ops.fp_pattern(self.s, p, self.est_last, self.true_last, self.djs, self.pat,
+                                  stream), "fp_pattern")
+        e[2].record(stream)
+        ops._check(ops.fp_select(self.s, p, self.pat, self.amap, self.vert, self.slash,
+                                 self.counts, self.indices, self.ws_sel, stream), "fp_select")
+        e[3].record(stream)
+        ops._check(ops.fp_sparse_attn(self.s, self.q, self.k, self.v, self.counts, self.indices,
+                                      self.out, None, None, stream), "fp_sparse_attn")
+        e[4].record(stream)
+        if gather is not None:
+            gather(self.out)
+
+    def estimate_bytes(self) -> int:
+        """fp_estimate's algorithmic bytes: read Q and K once, write every output."""
+        return (self.q.numel() + self.k.numel()) * self.q.element_size() + 4 * sum(
+            x.numel() for x in (self.qbar, self.kbar, self.amap, self.est_last,
+                                self.true_last, self.vert, self.slash))
+
+    def select_bytes(self, qa_heads: int, kept: int) -> int:
+        """fp_select's algorithmic bytes: each query-aware head reads its map once,
+        each vertical-slash head its two line lists; every kept block and every
+        row count is written once."""
+        bt, hq, n, _ = self.q.shape
+        t_pairs = self.nb * (self.nb + 1) // 2
+        return 4 * (qa_heads * t_pairs + (bt * hq - qa_heads) * 2 * n + kept + bt * hq * self.nb)
+
+
+def measure(layer, p, args, stream, ws, local, gather=None) -> dict:
+    """W untimed steps, then K timed steps bracketed by barrier + synchronize."""
+    from dynamic_block_sparse_fp_b200 import ops
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)]
+          for _ in range(args.warmup + args.steps)]
+    for i in range(args.warmup):
+        layer.step(p, ev[i], stream, gather)
+    torch.cuda.synchronize()
+    assert ops.fp_last_device_status(stream) == 0
+    barrier(ws)
+    torch.cuda.synchronize()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        t_start.record(stream)
+        for i in range(args.warmup, args.warmup + args.steps):
+            layer.step(p, ev[i], stream, gather)
+        t_end.record(stream)
+        torch.cuda.synchronize()
+    barrier(ws)
+    status = ops.fp_last_device_status(stream)
+    if status != 0:
+        raise RuntimeError(f"device status {ops.STATUS.get(status, status)}")
+    total_ms = max_over_ranks(t_start.elapsed_time(t_end), ws, layer.q.device)
+    timed = ev[args.warmup:]
+    stage_ms = [statistics.mean(e[j].elapsed_time(e[j + 1]) for e in timed) for j in range(4)]
+    return {"ms_step": total_ms / args.steps, "stage_ms": stage_ms,
+            "kept": int(layer.counts.sum()),
+            "qa_heads": int((layer.pat == ops.FP_PATTERN_QA).sum()),
+            "clocks": clk.summary()}
+
+
+def dense_ms(layer, stream, reps: int = 2) -> float:
+    """fp_dense_attn (the same kernel over every causal block), CUDA events."""
+    from dynamic_block_sparse_fp_b200 import ops
+    dout = torch.empty_like(layer.q)
+    de = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    ops._check(ops.fp_dense_attn(layer.s, layer.q, layer.k, layer.v, dout, None, stream),
+               "fp_dense_attn")
+    de[0].record(stream)
+    for _ in range(reps):
+        ops._check(ops.fp_dense_attn(layer.s, layer.q, layer.k, layer.v, dout, None, stream),
+                   "fp_dense_attn")
+    de[1].record(stream)
+    torch.cuda.synchronize()
+    return de[0].elapsed_time(de[1]) / reps
+
+
+def path_fields(layer, m: dict, peaks: dict, dense: float | None) -> dict:
+    """Kept fraction, per-stage times and rooflines of one measured configuration."""
+    bt, hq, n, d = layer.q.shape
+    bs, nb = layer.bs, layer.nb
+    st = m["stage_ms"]
+    t_pairs = nb * (nb + 1) // 2
+    flop_block = 4.0 * bs * bs * d
+    attn_flops = flop_block * m["kept"]
+    attn_tflops = attn_flops / (st[3] * 1e-3) / 1e12
+    peak_t = peaks["bf16_tflops_sustained"]
+    eb = layer.estimate_bytes()
+    sb = layer.select_bytes(m["qa_heads"], m["kept"])
+    hbm = peaks["hbm_gbs"]
+    f = {
+        "roofline": {"bound": "tensor", "kernel": "fp_sparse_attn", "achieved": attn_tflops,
+                     "peak": peak_t, "unit": "TFLOP/s", "frac": attn_tflops / peak_t,
+                     "peak_kind": f"bf16 dense, sustained ({peaks['source']})",
+                     "algorithmic_flops_per_launch": attn_flops},
+        "stages_ms": {"estimate": st[0], "pattern": st[1], "select": st[2],
+                      "sparse_attn": st[3]},
+        "estimate_hbm": {"bytes": eb, "gbs": eb / (st[0] * 1e-3) / 1e9,
+                         "frac": eb / (st[0] * 1e-3) / 1e9 / hbm},
+        "select_hbm": {"bytes": sb, "gbs": sb / (st[2] * 1e-3) / 1e9,
+                       "frac": sb / (st[2] * 1e-3) / 1e9 / hbm},
+        "effective_tflops": {"sparse_attn": attn_tflops,
+                             "whole_step": attn_flops / (m["ms_step"] * 1e-3) / 1e12},
+        "kept_blocks": m["kept"], "causal_blocks": t_pairs * hq * bt,
+        "kept_fraction": m["kept"] / (t_pairs * hq * bt), "qa_heads": m["qa_heads"],
+        "sparsity_implied_ratio": t_pairs * hq * bt / m["kept"],
+    }
+    if dense is not None:
+        f["dense_attn_ms"] = dense
+        f["dense_tflops"] = flop_block * t_pairs * hq * bt / (dense * 1e-3) / 1e12
+        f["speedup_vs_dense"] = {"whole_step": dense / m["ms_step"],
+                                 "sparse_attn_only": dense / st[3]}
+        f["speedup_target"] = 0.8 * f["sparsity_implied_ratio"]
+    return f
+
+
 def run_ours(args, w, ws, rank, local):
     from dynamic_block_sparse_fp_b200 import build, ops, sharded
 
@@ -284,97 +440,21 @@ def run_ours(args, w, ws, rank, local):
         # every rank: its own independent layer
         inp = synth.make_inputs(rank_workload(w, rank))
     q, k, v = (inp[x].to(dev) for x in ("q", "k", "v"))
-    bt, hq, n, d = q.shape
-    hkv, bs = k.shape[1], w.block_size
-    nb = n // bs
-    s = ops.make_shape(q, k, bs)
-    p = ops.make_params(w.gamma, w.tau, w.min_budget, w.max_budget, w.qa_mode, w.vs_mode)
-    f32 = dict(dtype=torch.float32, device=dev)
-    qbar = torch.empty(bt, hq, nb, d, **f32)
-    kbar = torch.empty(bt, hkv, nb, d, **f32)
-    amap = torch.empty(bt, hq, nb * (nb + 1) // 2, **f32)
-    est_last = torch.empty(bt, hq, nb, **f32)
-    true_last = torch.empty(bt, hq, nb, **f32)
-    vert = torch.empty(bt, hq, n, **f32)
-    slash = torch.empty(bt, hq, n, **f32)
-    djs = torch.empty(bt, hq, **f32)
-    pat = torch.empty(bt, hq, dtype=torch.int32, device=dev)
-    counts = torch.empty(bt, hq, nb, dtype=torch.int32, device=dev)
-    indices = torch.empty(bt, hq, nb, nb, dtype=torch.int32, device=dev)
-    out = torch.empty_like(q)
-    ws_est = ops.workspace(s, ops.FP_CALL_ESTIMATE, dev)
-    ws_sel = ops.workspace(s, ops.FP_CALL_SELECT, dev)
+    layer = Layer(ops, q, k, v, w.block_size, dev)
     stream = torch.cuda.current_stream(dev)
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)]
-          for _ in range(args.warmup + args.steps)]
-
-    def step(e):
-        e[0].record(stream)
-        ops._check(ops.fp_estimate(s, q, k, qbar, kbar, amap, est_last, true_last, vert, slash,
-                                   ws_est, stream), "fp_estimate")
-        e[1].record(stream)
-        ops._check(ops.fp_pattern(s, p, est_last, true_last, djs, pat, stream), "fp_pattern")
-        e[2].record(stream)
-        ops._check(ops.fp_select(s, p, pat, amap, vert, slash, counts, indices, ws_sel, stream),
-                   "fp_select")
-        e[3].record(stream)
-        ops._check(ops.fp_sparse_attn(s, q, k, v, counts, indices, out, None, None, stream),
-                   "fp_sparse_attn")
-        e[4].record(stream)
-        if heads and ws > 1:
-            sharded.gather_heads(out, ws)  # the whole layer's output on every rank
-
-    for i in range(args.warmup):
-        step(ev[i])
-    torch.cuda.synchronize()
-    assert ops.fp_last_device_status(stream) == 0
-    barrier(ws)
-    torch.cuda.synchronize()
-    t_start = torch.cuda.Event(enable_timing=True)
-    t_end = torch.cuda.Event(enable_timing=True)
-    with ClockSampler(local) as clk:
-        t_start.record(stream)
-        for i in range(args.warmup, args.warmup + args.steps):
-            step(ev[i])
-        t_end.record(stream)
-        torch.cuda.synchronize()
-    barrier(ws)
-    status = ops.fp_last_device_status(stream)
-    if status != 0:
-        raise RuntimeError(f"device status {ops.STATUS.get(status, status)}")
-    total_ms = max_over_ranks(t_start.elapsed_time(t_end), ws, dev)
-    ms_step = total_ms / args.steps
-    timed = ev[args.warmup:]
-    stage_ms = [statistics.mean(e[j].elapsed_time(e[j + 1]) for e in timed) for j in range(4)]
-    kept = int(counts.sum())
-    qa_heads = int((pat == ops.FP_PATTERN_QA).sum())
-    t_pairs = nb * (nb + 1) // 2
-    flop_block = 4.0 * bs * bs * d
-    attn_flops = flop_block * kept
-    attn_tflops = attn_flops / (stage_ms[3] * 1e-3) / 1e12
-    tokens = n * bt
+    gather = (lambda out: sharded.gather_heads(out, ws)) if heads and ws > 1 else None
+    tokens = q.shape[2] * q.shape[0]
+    if args.sweep:
+        run_sweep(args, w, layer, ws, rank, local, stream, peaks, gather, heads)
+        return
+    p = ops.make_params(w.gamma, w.tau, w.min_budget, w.max_budget, w.qa_mode, w.vs_mode)
+    m = measure(layer, p, args, stream, ws, local, gather)
+    ms_step = m["ms_step"]
     # weak scaling: every rank's own layer; head sharding: one layer in all
     value = tokens / (ms_step * 1e-3) if heads else job_value(tokens, ws, ms_step)
-    # dense comparison at the same length (same kernel over every causal block)
-    dense_ms = None
-    if not args.no_dense:
-        dout = torch.empty_like(q)
-        de = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
-        ops._check(ops.fp_dense_attn(s, q, k, v, dout, None, stream), "fp_dense_attn")
-        de[0].record(stream)
-        reps = 2
-        for _ in range(reps):
-            ops._check(ops.fp_dense_attn(s, q, k, v, dout, None, stream), "fp_dense_attn")
-        de[1].record(stream)
-        torch.cuda.synchronize()
-        dense_ms = de[0].elapsed_time(de[1]) / reps
-        del dout
-    # estimate: algorithmic bytes = read Q and K once + write its outputs
-    eb = q.element_size()
-    est_bytes = (q.numel() + k.numel()) * eb + 4 * (qbar.numel() + kbar.numel() + amap.numel()
-                                                   + est_last.numel() + true_last.numel()
-                                                   + vert.numel() + slash.numel())
-    peak_t = peaks["bf16_tflops_sustained"]
+    dense = None if args.no_dense else dense_ms(layer, stream)
+    fields = path_fields(layer, m, peaks, dense)
+    fields["roofline"]["traffic"] = kernel_traffic("attn_tc.cu", w.name)
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
@@ -383,37 +463,20 @@ def run_ours(args, w, ws, rank, local):
         "data": "synthetic (seeded Q/K/V with planted query-aware / vertical-slash structure "
                 "and RoPE; no dataset or weights)",
         "config": workload_config(w, ws, heads),
-        "roofline": {"bound": "tensor", "kernel": "fp_sparse_attn", "achieved": attn_tflops,
-                     "peak": peak_t, "unit": "TFLOP/s", "frac": attn_tflops / peak_t,
-                     "traffic": kernel_traffic("attn_tc.cu", w.name),
-                     "peak_kind": f"bf16 dense, sustained ({peaks['source']})",
-                     "algorithmic_flops_per_launch": attn_flops},
         # the library's kernels per step: 12, plus the query-wise row
         # selection and the line pooling when those modes are on
         "gpu_launches": (LAUNCHES_PER_STEP + int(w.qa_mode == 1) + int(w.vs_mode == 1))
                         * args.steps,
-        "stages_ms": {"estimate": stage_ms[0], "pattern": stage_ms[1], "select": stage_ms[2],
-                      "sparse_attn": stage_ms[3]},
-        "estimate_hbm": {"bytes": est_bytes, "gbs": est_bytes / (stage_ms[0] * 1e-3) / 1e9,
-                         "frac": est_bytes / (stage_ms[0] * 1e-3) / 1e9 / peaks["hbm_gbs"]},
-        "effective_tflops": {"sparse_attn": attn_tflops,
-                             "whole_step": attn_flops / (ms_step * 1e-3) / 1e12},
-        "kept_blocks": kept, "causal_blocks": t_pairs * hq * bt,
-        "kept_fraction": kept / (t_pairs * hq * bt), "qa_heads": qa_heads,
-        "sparsity_implied_ratio": t_pairs * hq * bt / kept,
     }
-    if dense_ms is not None:
-        line["dense_attn_ms"] = dense_ms
-        line["dense_tflops"] = flop_block * t_pairs * hq * bt / (dense_ms * 1e-3) / 1e12
-        line["speedup_vs_dense"] = {"whole_step": dense_ms / ms_step,
-                                    "sparse_attn_only": dense_ms / stage_ms[3]}
-    line["clocks"] = clk.summary()
+    line.update(fields)
+    line["clocks"] = m["clocks"]
     # ---- end to end through the C ABI with host buffers ----
     if not args.no_e2e:
         qh, kh, vh = (inp[x].contiguous().pin_memory() for x in ("q", "k", "v"))
         oh = torch.empty_like(qh).pin_memory()
-        del out, indices
+        del layer
         torch.cuda.empty_cache()
+        s = ops.make_shape(q, k, w.block_size)
         wsh = ops.workspace(s, ops.FP_CALL_PREFILL_HOST, dev)
         ops._check(ops.fp_prefill_attn_host(s, p, qh, kh, vh, oh, wsh, stream), "host")
         torch.cuda.synchronize()
@@ -442,7 +505,29 @@ def run_ours(args, w, ws, rank, local):
         print(json.dumps(line), flush=True)
 
 
-def main():
+def run_sweep(args, w, layer, ws, rank, local, stream, peaks, gather, heads):
+    """One JSON line per (gamma, tau, min, max) point of SWEEP on the same inputs;
+    the dense comparison is measured once (it does not depend on the parameters)."""
+    from dynamic_block_sparse_fp_b200 import ops
+    dense = None if args.no_dense else dense_ms(layer, stream)
+    tokens = layer.q.shape[2] * layer.q.shape[0]
+    for g, t, lo, hi in SWEEP:
+        wp = w.replace(gamma=g, tau=t, min_budget=lo, max_budget=hi)
+        p = ops.make_params(g, t, lo, hi, w.qa_mode, w.vs_mode)
+        m = measure(layer, p, args, stream, ws, local, gather)
+        value = tokens / (m["ms_step"] * 1e-3) if heads else job_value(tokens, ws, m["ms_step"])
+        line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": m["ms_step"],
+                "higher_is_better": True, "scaling": "strong" if heads else "weak",
+                "sweep_point": {"gamma": g, "tau": t, "min_budget": lo, "max_budget": hi},
+                "dtype": "bf16", "data": "synthetic", "config": workload_config(wp, ws, heads)}
+        line.update(path_fields(layer, m, peaks, dense))
+        line["clocks"] = m["clocks"]
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+
+
+def parser() -> argparse.ArgumentParser:
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=10)
@@ -457,18 +542,26 @@ def main():
                     help="selection rule for query-aware heads (default: flattened)")
     ap.add_argument("--vs-mode", choices=["tokens", "blocks"],
                     help="line granularity for vertical-slash heads (default: tokens)")
+    ap.add_argument("--sweep", action="store_true",
+                    help="one line per point of the gamma x tau x min x max sweep (24 points) "
+                         "on the workload's inputs, instead of the single headline line")
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--shard", choices=["layers", "heads"], default="layers",
-                    help="N > 1: independent layers per rank (weak scaling, default) or one "
-                         "layer's kv heads split over the ranks (strong scaling)")
+    ap.add_argument("--shard", choices=["layers", "heads"], default="heads",
+                    help="N > 1: one layer's kv heads split over the ranks, outputs "
+                         "all-gathered (strong scaling, the default) or an independent layer "
+                         "per rank (weak scaling)")
     ap.add_argument("--cpu-baseline-s", type=float, default=12.0,
                     help="seconds of oracle work in the cpu_baseline sample")
     ap.add_argument("--reference-step-s", type=float, default=8.0,
                     help="seconds of oracle work per step of --impl reference")
-    args = ap.parse_args()
+    return ap
+
+
+def main():
+    args = parser().parse_args()
     w = synth.WORKLOADS[args.workload]
     over = {k: v for k, v in (("gamma", args.gamma), ("tau", args.tau),
                               ("min_budget", args.min_budget),

@@ -156,54 +156,11 @@ __device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
       : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
   return d;
 }
-__device__ __forceinline__ float2 fsub2(float2 a, float2 b) {
-  float2 d;
-  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
-      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
-      "sub.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
-      : "=f"(d.x), "=f"(d.y)
-      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
-  return d;
-}
 __device__ __forceinline__ float max3f(float a, float b, float c) {
   float d;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
   return d;
 }
-
-// 2^x on the FMA pipe (no MUFU), for the share of the exponentials that the
-// MUFU unit would otherwise queue: x = j + f with j the nearest integer (adding
-// 1.5 * 2^23 rounds x and leaves j in the low mantissa bits of the sum) and
-// |f| <= 1/2 (Cody-Waite range reduction); 2^f by a cubic whose coefficients
-// were fitted here by Remez exchange for least maximum relative error on
-// [-1/2, 1/2] (7.5e-5 evaluated in fp32: far below the bf16 rounding of P);
-// then j is added to the exponent field.  Inputs here are <= 8; x is clamped
-// below at -126 (the result there is < 2^-125, i.e. nothing next to the row
-// maximum's 1).
-constexpr float kPolyC0 = 0x1.fff692p-1f, kPolyC1 = 0x1.62f31ap-1f, kPolyC2 = 0x1.f0de1ap-3f,
-                kPolyC3 = 0x1.c3f76p-5f;
-__device__ __forceinline__ float2 exp2_poly2(float2 x) {
-  constexpr float kShift = 12582912.f;  // 1.5 * 2^23
-  x.x = fmaxf(x.x, -126.f);
-  x.y = fmaxf(x.y, -126.f);
-  const float2 t = fadd2(x, make_float2(kShift, kShift));
-  const float2 f = fsub2(x, fsub2(t, make_float2(kShift, kShift)));
-  float2 p = ffma2(make_float2(kPolyC3, kPolyC3), f, make_float2(kPolyC2, kPolyC2));
-  p = ffma2(p, f, make_float2(kPolyC1, kPolyC1));
-  p = ffma2(p, f, make_float2(kPolyC0, kPolyC0));
-  // t's bits are 0x4B400000 + j; shifted by 23 only j * 2^23 survives
-  return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
-                     __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
-}
-
-// Of every 4 column pairs of an S row, how many take exp2_poly2 rather than
-// the MUFU ex2 (the MUFU unit, 16 lanes per clock per SM, would otherwise be
-// as busy as the tensor cores).
-#ifndef FP_ATTN_POLY_PAIRS
-#define FP_ATTN_POLY_PAIRS 0
-#endif
-constexpr int kPolyPairs = FP_ATTN_POLY_PAIRS;
-static_assert(kPolyPairs >= 0 && kPolyPairs <= 4, "poly pairs per 4");
 
 // The maximum of one S row over a 64-key tile (raw scores); MASK: keys
 // c > lim are left out.
@@ -231,12 +188,8 @@ __device__ __forceinline__ void tile_exp(const uint32_t (&u)[BN], int lim, float
   for (int i = 0; i < BN; i += 2) {
     const float2 x = ffma2(make_float2(__uint_as_float(u[i]), __uint_as_float(u[i + 1])), sc, nm);
     float2 p;
-    if ((i / 2) % 4 < kPolyPairs) {
-      p = exp2_poly2(x);
-    } else {
-      p.x = ex2(x.x);
-      p.y = ex2(x.y);
-    }
+    p.x = ex2(x.x);
+    p.y = ex2(x.y);
     if (MASK) {
       p.x = i > lim ? 0.f : p.x;
       p.y = i + 1 > lim ? 0.f : p.y;

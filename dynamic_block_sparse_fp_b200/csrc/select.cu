@@ -34,6 +34,8 @@
 // with block size 1 (a column is a key block, an offset one block distance).
 #include <cooperative_groups.h>
 
+#include <mutex>
+
 #include "fp_internal.cuh"
 
 namespace cg = cooperative_groups;
@@ -739,12 +741,17 @@ static __device__ __align__(256) unsigned char g_select_scratch[FP_SELECT_NOALLO
 
 namespace {
 
+// The array's device address on the current device, looked up on the first
+// call made with that device current and cached (under a lock: two host
+// threads may make their first calls at the same time).
 cudaError_t select_scratch_address(void **out) {
+  static std::mutex mu;
   static void *addr[64] = {nullptr};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(mu);
   if (!addr[dev]) {
     void *p = nullptr;
     e = cudaGetSymbolAddress(&p, g_select_scratch);
@@ -757,6 +764,7 @@ cudaError_t select_scratch_address(void **out) {
 
 }  // namespace
 
+// The same launches as launch_select, with the fixed array as the workspace.
 cudaError_t launch_select_noalloc(const Dims &D, float gamma, const SelectBudgets &bud,
                                   const int32_t *pattern, const float *map, const float *vert,
                                   const float *slash, int32_t *counts, int32_t *indices,
@@ -766,37 +774,7 @@ cudaError_t launch_select_noalloc(const Dims &D, float gamma, const SelectBudget
   void *scratch = nullptr;
   cudaError_t e = select_scratch_address(&scratch);
   if (e != cudaSuccess) return e;
-  Carver c{static_cast<char *>(scratch), 0};
-  const size_t heads = size_t(D.bt) * D.hq;
-  HeadSel *sel = c.take<HeadSel>(2 * heads);
-  uint8_t *cf = c.take<uint8_t>(heads * D.nb);
-  uint8_t *df = c.take<uint8_t>(heads * D.nb);
-  const int smem = int(sizeof(SelSmem));
-  cudaFuncSetAttribute(select_head_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  if (bud.vs_mode == FP_VS_BLOCKS) {
-    // pooled lines live in the outputs until emit_rows_kernel overwrites them:
-    // vert sums in indices (>= Bt*Hq*nb entries), slash sums in counts
-    float *pv = reinterpret_cast<float *>(indices);
-    float *ps = reinterpret_cast<float *>(counts);
-    pool_lines_kernel<<<dim3((D.nb + 255) / 256, D.hq, D.bt), 256, 0, st>>>(
-        pattern, vert, slash, D.n, D.nb, D.bs, pv, ps);
-    select_head_kernel<<<dim3(kCluster * D.hq, D.bt), kCThreads, smem, st>>>(
-        pattern, map, pv, ps, D.nb, D.nb, 1, gamma, bud.qa_lo, bud.qa_hi, bud.vsb_lo,
-        bud.vsb_hi, bud.qa_mode, sel, cf, df);
-  } else {
-    select_head_kernel<<<dim3(kCluster * D.hq, D.bt), kCThreads, smem, st>>>(
-        pattern, map, vert, slash, D.n, D.nb, D.bs, gamma, bud.qa_lo, bud.qa_hi, bud.vs_lo,
-        bud.vs_hi, bud.qa_mode, sel, cf, df);
-  }
-  emit_rows_kernel<<<dim3((D.nb + 7) / 8, D.hq, D.bt), 256, 0, st>>>(
-      pattern, map, D.nb, sel, cf, df, bud.qa_mode, counts, indices);
-  if (bud.qa_mode == FP_QA_QUERYWISE) {
-    int pmax;
-    const size_t rsm = rows_qa_smem(D.nb, &pmax);
-    select_rows_qa_kernel<<<dim3(D.nb, D.hq, D.bt), kRowThreads, rsm, st>>>(
-        pattern, map, D.nb, pmax, gamma, bud.row_lo, bud.row_hi, counts, indices);
-  }
-  return cudaGetLastError();
+  return launch_select(D, gamma, bud, pattern, map, vert, slash, counts, indices, scratch, st);
 }
 
 }  // namespace fpi

@@ -48,11 +48,20 @@ def gather_heads(out_local: torch.Tensor, world: int, group=None) -> torch.Tenso
     if dist.get_backend(group) == "nccl":
         buf = torch.empty((world,) + tuple(x.shape), dtype=x.dtype, device=x.device)
         dist.all_gather_into_tensor(buf, x, group=group)
-        parts = buf.unbind(0)
+        return heads_of_gathered(buf)
     else:
         parts = [torch.empty_like(x) for _ in range(world)]
         dist.all_gather(parts, x, group=group)
     return torch.cat(parts, dim=1)
+
+
+def heads_of_gathered(buf: torch.Tensor) -> torch.Tensor:
+    """[world, Bt, h, N, d] (rank-major, as all_gather_into_tensor leaves it) ->
+    [Bt, world*h, N, d]; with Bt = 1 that is a view of the same memory (no copy)."""
+    world, bt, h = buf.shape[:3]
+    if bt == 1:
+        return buf.view((1, world * h) + tuple(buf.shape[3:]))
+    return torch.cat(buf.unbind(0), dim=1)
 
 
 def sharded_prefill_attn(q, k, v, block_size: int, params, group=None, gather: bool = True):

@@ -213,8 +213,10 @@ fp_status fp_select(const fp_shape *shape, const fp_params *params,
  *     with FP_ERR_WORKSPACE before anything is launched.
  *   * It allocates nothing (no cudaMalloc / cudaFree / allocating library
  *     routine).  The first call on a device looks up the array's device
- *     address for that device (cudaGetSymbolAddress); make that first call
- *     before capturing any stream.
+ *     address for that device (cudaGetSymbolAddress) and keeps it for the
+ *     life of the process; make that first call before capturing any
+ *     stream.  A cudaDeviceReset() ends the context that address belongs
+ *     to, so do not call this entry point on a device after resetting it.
  *   * Every call on a device uses the same array, which keeps the last
  *     call's contents (nothing in it needs clearing).  Two calls whose work
  *     can overlap on the GPU (different streams, several host threads) race

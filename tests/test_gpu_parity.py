@@ -301,6 +301,29 @@ def test_pipeline_glm_block64_bf16_parity(n, tau, hi):
     assert ops.fp_last_device_status() == 0
 
 
+@pytest.mark.parametrize("bs", [128, 64])
+def test_pipeline_fp32_llama_heads_parity(bs):
+    """The fp32 debug path on Llama-shaped heads (d = 128), block 128 and 64:
+    sparse attention under a capped budget (rows of different lengths) and
+    dense attention, both against the oracle at the fp32 bound."""
+    w, inp, d = _inputs("llama8b_n8192", dtype="f32", seq_len=2048, n_q_heads=4, n_kv_heads=2,
+                        block_size=bs)
+    res = _pipeline(w, d, hi=512)
+    nb = w.n_blocks
+    full = torch.arange(1, nb + 1, device=DEV, dtype=torch.int32)
+    assert res["counts"].min() >= 1 and (res["counts"] < full).any()  # some rows skip blocks
+    _attn_check(inp, res, w, 1e-4, 1e-4, heads=[0, 1, 2, 3], q_blocks=[0, 1, nb // 2, nb - 1])
+    out, lse = ops.dense_attn(d["q"], d["k"], d["v"], bs)
+    torch.cuda.synchronize()
+    o, l = oracle.dense_attention(inp["q"], inp["k"], inp["v"], bs, heads=[0, 3],
+                                  q_blocks=[0, nb // 2, nb - 1])
+    m = ~np.isnan(o)
+    assert np.abs(_np(out)[m] - o[m]).max() <= 1e-4
+    ml = ~np.isnan(l)
+    assert np.abs(_np(lse)[ml] - l[ml]).max() <= 1e-4
+    assert ops.fp_last_device_status() == 0
+
+
 def test_dense_parity():
     w, inp, d = _inputs("tiny_n1024")
     out, lse = ops.dense_attn(d["q"], d["k"], d["v"], w.block_size)
@@ -709,4 +732,8 @@ def test_maximum_block_count_sampled():
                                  res["est"]["vert"], res["est"]["slash"], c2, i2) == 0
     torch.cuda.synchronize()
     assert torch.equal(c2, res["counts"])
+    for hh in (0, 1):
+        for i in (0, 1, 2047, 4094, 4095):
+            n = int(res["counts"][0, hh, i])
+            assert torch.equal(i2[0, hh, i, :n], res["indices"][0, hh, i, :n]), (hh, i)
     _attn_check(inp, res, w, 2e-2, 2e-3, heads=[0, 1], q_blocks=[0, 2048, 4095])

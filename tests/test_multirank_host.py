@@ -1,8 +1,10 @@
 """World-size-2 checks of bench.py's multi-rank host logic on CPU (gloo).
 
-Ranks run independent layers (weak scaling, no exchange on the data path);
-the only collectives are the barrier and the max over ranks of the timed
-region, which these tests exercise without a GPU.
+By default the ranks split one layer's kv heads and all-gather the outputs
+(strong scaling); with --shard layers they run independent layers (weak
+scaling, no exchange on the data path).  The collectives are the barrier, the
+max over ranks of the timed region and the output gather, which these tests
+exercise without a GPU.
 """
 import os
 import socket
@@ -111,3 +113,23 @@ def test_head_shard_rule():
         sharded.head_shard(8, 3, 0)
     with pytest.raises(ValueError):
         sharded.head_shard(8, 2, 2)
+
+
+def test_bench_splits_heads_by_default():
+    import bench
+    assert bench.parser().parse_args([]).shard == "heads"
+    assert bench.parser().parse_args(["--shard", "layers"]).shard == "layers"
+
+
+@pytest.mark.parametrize("bt", [1, 3])
+def test_gathered_heads_layout(bt):
+    """all_gather_into_tensor leaves [world, Bt, h, N, d]; the gathered layer is
+    [Bt, world*h, N, d] in rank order (a view without a copy when Bt = 1)."""
+    from dynamic_block_sparse_fp_b200 import sharded
+    world, h = 4, 2
+    parts = [torch.randn(bt, h, 5, 3) for _ in range(world)]
+    buf = torch.stack(parts)
+    got = sharded.heads_of_gathered(buf)
+    assert torch.equal(got, torch.cat(parts, dim=1))
+    if bt == 1:
+        assert got.data_ptr() == buf.data_ptr()

@@ -44,8 +44,14 @@ def test_noalloc_select_matches_fp_select_twice():
     # half the heads query-aware, half vertical-slash: both scratch layouts
     pat = (torch.arange(w.n_q_heads, device=DEV, dtype=torch.int32) % 2).reshape(1, -1)
     nb = w.n_blocks
-    cases = [ops.make_params(0.95, 0.1, 1024, 0), ops.make_params(0.9, 0.1, 2048, 8192)]
-    for p in cases:  # two calls in a row; the second reuses the first's scratch
+    # two calls in a row per mode (the second reuses the first's scratch); the
+    # query-wise rows and the block-pooled lines both stage data in the outputs
+    cases = [ops.make_params(0.95, 0.1, 1024, 0), ops.make_params(0.9, 0.1, 2048, 8192),
+             ops.make_params(0.95, 0.1, 1024, 0, qa_mode=ops.FP_QA_QUERYWISE),
+             ops.make_params(0.9, 0.1, 2048, 8192, qa_mode=ops.FP_QA_QUERYWISE),
+             ops.make_params(0.95, 0.1, 1024, 0, vs_mode=ops.FP_VS_BLOCKS),
+             ops.make_params(0.9, 0.1, 2048, 8192, vs_mode=ops.FP_VS_BLOCKS)]
+    for p in cases:
         ref_c, ref_i = ops.select(s, p, pat, est["map"], est["vert"], est["slash"])
         counts = torch.full((1, w.n_q_heads, nb), -7, dtype=torch.int32, device=DEV)
         indices = torch.full((1, w.n_q_heads, nb, nb), -7, dtype=torch.int32, device=DEV)
