@@ -36,7 +36,7 @@ import torch  # noqa: E402
 from dynamic_block_sparse_fp_b200 import synth  # noqa: E402
 
 METRIC = "prefill-attn tokens/s and effective TFLOPS (% bf16 peak) at 128k; speedup vs dense"
-LAUNCHES_PER_STEP = 12  # estimate 8, pattern 1, select 2, attention 1
+LAUNCHES_PER_STEP = 16  # estimate 8, pattern 1, select 6, attention 1
 
 
 def kernel_traffic(source: str, workload: str):

@@ -15,11 +15,13 @@
 //   kept        the first k entries of the order.
 // Because non-negative fp32 scores order like their bit patterns, the kept
 // set is {bits_i > b} u {bits_i == b and i <= idx} for one threshold pair
-// (b, idx).  select_head_kernel finds it with a three-level radix descent on
-// the bit patterns (12 + 12 + 8 bits), weighted by mass to find k_gamma and by
-// count when the clamp moves k, and one ordered count for the tie rank.  All
-// of it is integer arithmetic, so the result does not depend on thread order.
-// emit_rows_kernel then writes every row's ascending block list.
+// (b, idx).  A radix select over the whole GPU finds it: two histogram passes
+// over every list (digits of 11 + 11 bits, weighted by mass to find k_gamma
+// and by count once the budget clamp decides k), one pass that gathers the
+// few entries sharing the crossing 22-bit prefix, and the last digit and the
+// tie rank on those.  All of it is integer arithmetic, so the result does not
+// depend on thread order.  emit_rows_kernel then writes every row's ascending
+// block list.
 //
 // Query-wise rule for query-aware heads ("Measured effects": query-wise index
 // selection instead of the flattened map): the same rule on each row
@@ -32,18 +34,15 @@
 // sums vert per key block and slash per block distance into nb-entry lists,
 // which select_head_kernel then selects as lines of a sequence of nb tokens
 // with block size 1 (a column is a key block, an offset one block distance).
-#include <cooperative_groups.h>
-
+#include <algorithm>
 #include <mutex>
 
 #include "fp_internal.cuh"
 
-namespace cg = cooperative_groups;
-
 namespace fpi {
 namespace {
 
-constexpr int kMaxBlocks = 4096;  // nb limit (flags live in shared memory)
+constexpr int kMaxBlocks = 4096;  // nb limit
 
 enum : int { SEL_THRESHOLD = 0, SEL_NONE = 1, SEL_ALL = 2 };
 
@@ -66,406 +65,695 @@ __device__ __forceinline__ bool kept(uint32_t bits, uint32_t i, const HeadSel &s
   return bits > s.bits || (bits == s.bits && i <= s.idx);
 }
 
-
 // ---------------------------------------------------------------------------
-// One selection problem per head, spread over a cluster of kCluster CTAs.
-// Rank r of the cluster owns the contiguous slice [r*ceil(n/C), ...) of the
-// list.  Each histogram level is built per slice, then every rank sums its
-// share of the bins over all ranks (distributed shared memory) into rank 0's
-// copy; rank 0 finds the crossing bin and the other ranks read the result.
-// Integer arithmetic throughout: the result does not depend on the split.
+// The flattened rule and the line lists, as a radix select over the whole GPU.
+// Every head owns two list slots: slot 2h is its map (query-aware) or its
+// vert list (vertical-slash), slot 2h+1 its slash list (vertical-slash only).
+// A score's bit pattern (bit 31 is 0 after score_bits) splits into three
+// digits: the exponent, bits 30..23 (level 1), bits 22..11 (level 2) and bits
+// 10..0 (level 3).
+//
+//   hist_kernel<1>   every CTA histograms (mass and count) the level-1 digit
+//                    of its chunks of one list in shared memory and adds its
+//                    non-empty bins to the list's global histogram; the last
+//                    CTA of a list to finish (a counter, no waiting) finds the
+//                    crossing digit and clears the histogram for level 2.
+//   hist_kernel<2>   the same for the level-2 digit of the entries whose
+//                    level-1 digit is the crossing one.
+//   compact_kernel   entries whose first two digits are the crossing ones go
+//                    to a short candidate list; the last CTA of a list finds
+//                    the level-3 digit and the tie rank among the candidates
+//                    (or, when more than kCand share the prefix, by scans of
+//                    the whole list).
+// At each level the crossing is found by mass (the gamma rule) until it is
+// clear that the budget clamp decides k; from then on by count.  The mass
+// crossing bin b bounds k_gamma to (A, A + C] (A entries above the bin, C in
+// it): hi <= A means k = hi, lo >= A + C means k = lo, and otherwise a clamped
+// k lies in the same bin, so one prefix serves both.  Integer sums
+// throughout: the result does not depend on the split into chunks.
+//
+// Shared-memory histograms of the scanning CTAs hold a mass as two 32-bit
+// sums, of its low 16 bits and of the rest (a mass is at most 2^32, so a CTA
+// may add up to kMaxCtaEntries entries to one bin): 32-bit shared atomics,
+// where 64-bit ones measured several times slower.
 
-constexpr int kCluster = 8;
-constexpr int kCThreads = 512;
-constexpr int kCWarps = kCThreads / 32;
+constexpr int kSelThreads = 256;
+constexpr int kChunk = 2048;         // entries per chunk (16-byte groups of 4)
+constexpr int kBins1 = 256;          // level-1 digit (8 bits)
+constexpr int kBins2 = 4096;         // level-2 digit (12 bits)
+constexpr int kBins3 = 2048;         // level-3 digit (11 bits)
+constexpr int kShift1 = 23, kShift2 = 11;
+constexpr int kBins = kBins2;        // global histogram bins per list (levels 1, 2)
+constexpr int kCand = 1024;          // candidate list length per list slot
+constexpr int kHistAggMax = 8;
+constexpr int kSelCtasPerSm = 6;     // scanning CTAs per SM (over every list)
+constexpr int kMaxCtaEntries = 32767;                   // 32767 * 2^17 < 2^32
+constexpr int kMaxCtaChunks = kMaxCtaEntries / kChunk;  // chunks a CTA may take
+constexpr int kRounds = 4;
 
-struct SelSmem {
-  unsigned long long hmass[4096];
-  unsigned int hcnt[4096];
-  unsigned long long warp_tot[32];
-  unsigned long long res[8];  // [0..2] crossing, [3] scan total, [4] slice count, [5] tie index
-  uint8_t colflag[kMaxBlocks];
-  uint8_t distflag[kMaxBlocks];
+struct ListState {
+  unsigned long long am, ac;  // mass / count of the entries above the prefix
+  unsigned long long target_c;
+  double target_m;
+  uint32_t prefix;            // digits fixed so far
+  int finished;               // the list's HeadSel is written
+  int by_mass;                // descending by mass (1) or by count (0)
+  int overflow;               // more than kCand entries share the 20-bit prefix
+  unsigned int done[3];       // CTAs finished in hist<1>, hist<2>, compact
+  unsigned int cand;          // candidates appended
 };
 
-struct Ctx {
-  cg::cluster_group cl;
-  unsigned rank;
-  SelSmem *sm;
-  __device__ SelSmem *peer(unsigned q) const { return cl.map_shared_rank(sm, int(q)); }
+struct ListView {
+  const float *p;
+  uint32_t len;
+  unsigned long long lo, hi;
 };
+
+struct SelArgs {
+  const int32_t *pattern;
+  const float *map, *vert, *slash;
+  int n, nb, bs;  // line lists: n entries, block size bs
+  float gamma;
+  long long qa_lo, qa_hi;
+  int vs_lo, vs_hi;
+  int qa_mode;
+  HeadSel *sel;
+  ListState *state;
+  unsigned long long *hm;  // [slots][kBins]
+  unsigned int *hc;        // [slots][kBins]
+  uint2 *cand;             // [slots][kCand] (bits, index)
+  int ctas;                // CTAs per list in the scanning kernels
+};
+
+// The list of `slot`, or false when the slot holds none (the second slot of a
+// query-aware head, or a query-aware head under the query-wise rule).
+__device__ __forceinline__ bool list_of(const SelArgs &a, int slot, ListView *lv) {
+  const size_t bh = size_t(slot) / 2;
+  const int which = slot % 2;
+  if (a.pattern[bh] == FP_PATTERN_QA) {
+    if (which == 1 || a.qa_mode == FP_QA_QUERYWISE) return false;
+    const size_t t_pairs = size_t(a.nb) * (a.nb + 1) / 2;
+    lv->p = a.map + bh * t_pairs;
+    lv->len = uint32_t(t_pairs);
+    lv->lo = (unsigned long long)a.qa_lo;
+    lv->hi = (unsigned long long)a.qa_hi;
+  } else {
+    lv->p = (which == 0 ? a.vert : a.slash) + bh * size_t(a.n);
+    lv->len = uint32_t(a.n);
+    lv->lo = (unsigned long long)a.vs_lo;
+    lv->hi = (unsigned long long)a.vs_hi;
+  }
+  return true;
+}
+
+// Element offset of a list inside its 16-byte group: chunks are cut on
+// 16-byte boundaries of memory, so every full group is one aligned float4.
+__device__ __forceinline__ int group_offset(const float *p) {
+  return int((reinterpret_cast<uintptr_t>(p) >> 2) & 3u);
+}
+__device__ __forceinline__ int list_chunks(const ListView &lv) {
+  return int((uint64_t(lv.len) + group_offset(lv.p) + kChunk - 1) / kChunk);
+}
+
+// The 4 entries of group g (elements 4g - off .. 4g - off + 3): bit patterns,
+// and which are inside the list.  A group that lies wholly inside is one
+// aligned 16-byte load; the first and last groups read only their valid
+// elements.
+__device__ __forceinline__ void load_group(const ListView &lv, int off, uint32_t g,
+                                           uint32_t (&bits)[4], bool (&valid)[4]) {
+  const long long i0 = (long long)g * 4 - off;
+  if (i0 >= 0 && i0 + 3 < (long long)lv.len) {
+    const float4 v = __ldg(reinterpret_cast<const float4 *>(lv.p + i0));
+    bits[0] = score_bits(v.x);
+    bits[1] = score_bits(v.y);
+    bits[2] = score_bits(v.z);
+    bits[3] = score_bits(v.w);
+    valid[0] = valid[1] = valid[2] = valid[3] = true;
+  } else {
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const long long i = i0 + e;
+      valid[e] = i >= 0 && i < (long long)lv.len;
+      bits[e] = valid[e] ? score_bits(__ldg(lv.p + i)) : 0u;
+    }
+  }
+}
+
+// Adds one entry per lane (bin 0xFFFFFFFF: none) to a shared histogram.  A
+// warp groups its lanes by bin; with at most kHistAggMax groups one lane per
+// group adds the group's sums (the mass from two 32-bit reductions of its low
+// 24 and high bits), with more every lane adds its own (a reduction over one
+// group runs once per distinct group).  Integer sums: both give the same bins.
+__device__ __forceinline__ void hist_add(unsigned long long *hm, unsigned int *hc, uint32_t bin,
+                                         uint64_t w, int lane) {
+  const unsigned peers = __match_any_sync(0xffffffffu, bin);
+  const bool leader = lane == __ffs(peers) - 1;
+  if (__popc(__ballot_sync(0xffffffffu, leader)) > kHistAggMax) {
+    if (bin != 0xFFFFFFFFu) {
+      atomicAdd(&hm[bin], (unsigned long long)w);
+      atomicAdd(&hc[bin], 1u);
+    }
+  } else {
+    const unsigned lo = __reduce_add_sync(peers, unsigned(w & 0xFFFFFFull));
+    const unsigned hi = __reduce_add_sync(peers, unsigned(w >> 24));
+    if (bin != 0xFFFFFFFFu && leader) {
+      atomicAdd(&hm[bin], ((unsigned long long)hi << 24) + lo);
+      atomicAdd(&hc[bin], unsigned(__popc(peers)));
+    }
+  }
+}
+
+// A CTA's shared histogram: mass as the sums of its low 16 bits (lo) and of
+// the rest (hi), and the count.
+struct SmemHist {
+  unsigned int *lo, *hi, *cnt;
+  __device__ __forceinline__ void add(uint32_t b, uint64_t w, unsigned n) {
+    atomicAdd(&lo[b], unsigned(w & 0xFFFFull));
+    atomicAdd(&hi[b], unsigned(w >> 16));
+    atomicAdd(&cnt[b], n);
+  }
+};
+
+// Level 1: adds the 4 entries of every lane (bin 0xFFFFFFFF: none).  The warp
+// takes its smallest pending bin (a whole-warp minimum), every lane sums its
+// entries in that bin, whole-warp reductions add the lanes' sums and one lane
+// adds them; neighbouring scores mostly share their exponent, so a round or
+// two take every entry.  After kRounds rounds the lanes add what is left one
+// entry at a time.  Integer sums: every way gives the same bins.
+__device__ __forceinline__ void hist_add4(SmemHist h, const uint32_t (&b)[4],
+                                          const uint64_t (&w)[4], int lane) {
+  bool pend[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) pend[e] = b[e] != 0xFFFFFFFFu;
+#pragma unroll 1
+  for (int r = 0; r < kRounds; ++r) {
+    uint32_t lmin = 0xFFFFFFFFu;
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+      if (pend[e]) lmin = min(lmin, b[e]);
+    const uint32_t t = __reduce_min_sync(0xffffffffu, lmin);
+    if (t == 0xFFFFFFFFu) return;
+    unsigned lo = 0, hi = 0, n = 0;  // 4 entries: lo < 2^18, hi < 2^19
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+      if (pend[e] && b[e] == t) {
+        lo += unsigned(w[e] & 0xFFFFull);
+        hi += unsigned(w[e] >> 16);
+        ++n;
+        pend[e] = false;
+      }
+    lo = __reduce_add_sync(0xffffffffu, lo);
+    hi = __reduce_add_sync(0xffffffffu, hi);
+    n = __reduce_add_sync(0xffffffffu, n);
+    if (lane == 0) {
+      atomicAdd(&h.lo[t], lo);
+      atomicAdd(&h.hi[t], hi);
+      atomicAdd(&h.cnt[t], n);
+    }
+  }
+#pragma unroll
+  for (int e = 0; e < 4; ++e)
+    if (pend[e]) h.add(b[e], w[e], 1u);
+}
 
 // Block-wide exclusive prefix sum (thread order) of one value per thread.
-__device__ unsigned long long block_excl_scan(unsigned long long v, SelSmem &sm,
+__device__ unsigned long long block_excl_scan(unsigned long long v, unsigned long long *warp_tot,
                                               unsigned long long *total) {
   const int lane = threadIdx.x % 32, w = threadIdx.x / 32;
+  constexpr int kWarps = kSelThreads / 32;
   unsigned long long x = v;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
-    unsigned long long y = __shfl_up_sync(0xffffffffu, x, o);
+    const unsigned long long y = __shfl_up_sync(0xffffffffu, x, o);
     if (lane >= o) x += y;
   }
   __syncthreads();
-  if (lane == 31) sm.warp_tot[w] = x;
+  if (lane == 31) warp_tot[w] = x;
   __syncthreads();
   if (w == 0) {
-    unsigned long long t = lane < kCWarps ? sm.warp_tot[lane] : 0ull;
+    const unsigned long long t = lane < kWarps ? warp_tot[lane] : 0ull;
     unsigned long long s = t;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-      unsigned long long y = __shfl_up_sync(0xffffffffu, s, o);
+      const unsigned long long y = __shfl_up_sync(0xffffffffu, s, o);
       if (lane >= o) s += y;
     }
-    if (lane < kCWarps) sm.warp_tot[lane] = s - t;  // exclusive over warps
-    if (lane == 31) sm.res[3] = s;
+    if (lane < kWarps) warp_tot[lane] = s - t;
+    if (lane == 31) warp_tot[kWarps] = s;
   }
   __syncthreads();
-  unsigned long long r = sm.warp_tot[w] + x - v;
-  *total = sm.res[3];
+  const unsigned long long r = warp_tot[w] + x - v;
+  *total = warp_tot[kWarps];
   __syncthreads();
   return r;
 }
 
-// Histogram of (bits >> shift) & (nbins-1) over the slice [i0, i1), entries
-// whose masked bits equal `prefix`; mass and count, warp-aggregated
-// shared-memory atomics.  Then the cluster-wide merge into rank 0.
-__device__ void histogram(const Ctx &cx, const float *__restrict__ s, uint32_t i0, uint32_t i1,
-                          uint32_t prefix, uint32_t pmask, int shift, uint32_t nbins) {
-  SelSmem &sm = *cx.sm;
-  for (uint32_t i = threadIdx.x; i < nbins; i += kCThreads) {
-    sm.hmass[i] = 0;
-    sm.hcnt[i] = 0;
+struct Crossing {
+  uint32_t bin;
+  unsigned long long above_m, above_c;  // sums of the bins above `bin`
+};
+
+// The first bin, scanning [0, nbins) from the top, at which the cumulative
+// mass (by_mass) reaches target_m - base_m, or the cumulative count reaches
+// target_c - base_c.  Run by the whole CTA; the result is in *out for every
+// thread.  With no crossing (not reached for valid targets) the lowest bin.
+__device__ void find_crossing(const unsigned long long *hm, const unsigned int *hc, int nbins,
+                              bool by_mass, double target_m, unsigned long long base_m,
+                              unsigned long long target_c, unsigned long long base_c,
+                              unsigned long long *warp_tot, Crossing *out) {
+  const int per = nbins / kSelThreads;
+  const int p0 = threadIdx.x * per;  // positions in descending-bin order
+  unsigned long long lm = 0, lc = 0;
+  for (int p = p0; p < p0 + per; ++p) {
+    lm += hm[nbins - 1 - p];
+    lc += hc[nbins - 1 - p];
   }
+  unsigned long long tm, tc;
+  const unsigned long long em = block_excl_scan(lm, warp_tot, &tm);
+  const unsigned long long ec = block_excl_scan(lc, warp_tot, &tc);
+  if (threadIdx.x == 0) *out = Crossing{0u, tm - hm[0], tc - hc[0]};
   __syncthreads();
-  const int lane = threadIdx.x % 32;
-  // each warp takes kHistU consecutive groups of 32 entries per round and
-  // issues all their loads before using any, so the scan is not one load
-  // latency per 32 entries
-  constexpr uint32_t kHistU = 8;
-  constexpr int kHistAggMax = 8;
-  for (uint32_t base = i0 + (threadIdx.x / 32) * 32 * kHistU; base < i1;
-       base += kCThreads * kHistU) {
-    uint32_t bits[kHistU];
-#pragma unroll
-    for (uint32_t u = 0; u < kHistU; ++u) {
-      const uint32_t i = base + u * 32 + lane;
-      bits[u] = i < i1 ? score_bits(s[i]) : 0u;
-    }
-#pragma unroll
-    for (uint32_t u = 0; u < kHistU; ++u) {
-      const uint32_t i = base + u * 32 + lane;
-      uint32_t bin = 0xFFFFFFFFu;
-      uint64_t w = 0;
-      if (i < i1 && (bits[u] & pmask) == prefix) {
-        bin = (bits[u] >> shift) & (nbins - 1);
-        w = score_mass(bits[u]);
-      }
-      const unsigned peers = __match_any_sync(0xffffffffu, bin);
-      const bool leader = lane == __ffs(peers) - 1;
-      // a reduction over one group of peers runs once per distinct group, so
-      // when the lanes spread over many bins (the levels below the exponent,
-      // where most scores differ) every lane adds its own entry instead; the
-      // sums are integers, so both ways give the same bins
-      if (__popc(__ballot_sync(0xffffffffu, leader)) > kHistAggMax) {
-        if (bin != 0xFFFFFFFFu) {
-          atomicAdd(&sm.hmass[bin], (unsigned long long)w);
-          atomicAdd(&sm.hcnt[bin], 1u);
-        }
-      } else {
-        const unsigned lo = __reduce_add_sync(peers, unsigned(w & 0xFFFFFFull));
-        const unsigned hi = __reduce_add_sync(peers, unsigned(w >> 24));
-        if (bin != 0xFFFFFFFFu && leader) {
-          atomicAdd(&sm.hmass[bin], ((unsigned long long)hi << 24) + lo);
-          atomicAdd(&sm.hcnt[bin], unsigned(__popc(peers)));
-        }
-      }
-    }
-  }
-  // merge: rank r sums bins [r*nbins/C, (r+1)*nbins/C) of every rank into rank 0
-  cx.cl.sync();
-  const uint32_t per = nbins / kCluster;
-  SelSmem *root = cx.peer(0);
-  for (uint32_t b = cx.rank * per + threadIdx.x; b < (cx.rank + 1) * per; b += kCThreads) {
-    unsigned long long m = 0;
-    unsigned int c = 0;
-#pragma unroll
-    for (unsigned q = 0; q < kCluster; ++q) {
-      const SelSmem *pq = cx.peer(q);
-      m += pq->hmass[b];
-      c += pq->hcnt[b];
-    }
-    root->hmass[b] = m;
-    root->hcnt[b] = c;
-  }
-  cx.cl.sync();
-}
-
-// Rank 0: scan the merged histogram from the highest bin down and find the
-// first bin at which above + (inclusive cumulative) reaches the target.  Every
-// rank then reads the bin and the mass / count of the bins strictly higher.
-__device__ uint32_t find_crossing(const Ctx &cx, uint32_t nbins, bool by_mass, double target_m,
-                                  unsigned long long target_c, unsigned long long *above_m,
-                                  unsigned long long *above_c) {
-  SelSmem &sm = *cx.sm;
-  if (cx.rank == 0) {
-    const uint32_t per = nbins >= kCThreads ? nbins / kCThreads : 1;
-    const uint32_t p0 = threadIdx.x * per;  // positions in descending-bin order
-    unsigned long long lm = 0, lc = 0;
-    if (p0 < nbins)
-      for (uint32_t p = p0; p < p0 + per; ++p) {
-        const uint32_t b = nbins - 1 - p;
-        lm += sm.hmass[b];
-        lc += sm.hcnt[b];
-      }
-    unsigned long long tm, tc;
-    const unsigned long long em = block_excl_scan(lm, sm, &tm);
-    const unsigned long long ec = block_excl_scan(lc, sm, &tc);
-    if (threadIdx.x == 0) {
-      sm.res[0] = 0;  // fallback: lowest bin (unreachable for valid targets)
-      sm.res[1] = tm - sm.hmass[0];
-      sm.res[2] = tc - sm.hcnt[0];
-    }
-    __syncthreads();
-    const unsigned long long am = *above_m, ac = *above_c;
-    auto reach = [&](unsigned long long m, unsigned long long c) {
-      return by_mass ? (double)(am + m) >= target_m : (ac + c) >= target_c;
-    };
-    if (p0 < nbins && !reach(em, ec) && reach(em + lm, ec + lc)) {
-      unsigned long long cm = em, cc = ec;
-      for (uint32_t p = p0; p < p0 + per; ++p) {
-        const uint32_t b = nbins - 1 - p;
-        if (reach(cm + sm.hmass[b], cc + sm.hcnt[b])) {
-          sm.res[0] = b;
-          sm.res[1] = cm;
-          sm.res[2] = cc;
-          break;
-        }
-        cm += sm.hmass[b];
-        cc += sm.hcnt[b];
-      }
-    }
-  }
-  cx.cl.sync();
-  const SelSmem *root = cx.peer(0);
-  const uint32_t bin = uint32_t(root->res[0]);
-  *above_m += root->res[1];
-  *above_c += root->res[2];
-  cx.cl.sync();  // rank 0 may reuse res afterwards
-  return bin;
-}
-
-// Rank 0 sums the merged level-1 histogram (every entry is in it): W.
-__device__ unsigned long long total_mass(const Ctx &cx, uint32_t nbins) {
-  SelSmem &sm = *cx.sm;
-  if (cx.rank == 0) {
-    unsigned long long part = 0;
-    for (uint32_t b = threadIdx.x; b < nbins; b += kCThreads) part += sm.hmass[b];
-    unsigned long long tot;
-    block_excl_scan(part, sm, &tot);
-    if (threadIdx.x == 0) sm.res[6] = tot;
-  }
-  cx.cl.sync();
-  const unsigned long long w = cx.peer(0)->res[6];
-  cx.cl.sync();
-  return w;
-}
-
-// Radix descent; returns the threshold bit pattern and the mass / count of
-// every entry with larger bits.  By mass the target is gamma * W.
-__device__ uint32_t descend(const Ctx &cx, const float *s, uint32_t i0, uint32_t i1,
-                            bool by_mass, float gamma, unsigned long long target_c,
-                            unsigned long long *above_m, unsigned long long *above_c,
-                            double *target_m_out) {
-  const int shifts[3] = {20, 8, 0};
-  const int widths[3] = {12, 12, 8};
-  uint32_t prefix = 0, pmask = 0;
-  *above_m = 0;
-  *above_c = 0;
-  double target_m = 0.0;
-  for (int lv = 0; lv < 3; ++lv) {
-    const uint32_t nbins = 1u << widths[lv];
-    histogram(cx, s, i0, i1, prefix, pmask, shifts[lv], nbins);
-    if (lv == 0 && by_mass) {
-      const unsigned long long tot = total_mass(cx, nbins);
-      target_m = (double)gamma * (double)tot;
-      *target_m_out = target_m;
-    }
-    const uint32_t bin = find_crossing(cx, nbins, by_mass, target_m, target_c, above_m, above_c);
-    prefix |= bin << shifts[lv];
-    pmask |= (nbins - 1) << shifts[lv];
-  }
-  return prefix;
-}
-
-// Index of the m-th (1-based) entry with bit pattern == b, in index order,
-// over the whole list (the slices are in index order across ranks).  Warp w
-// of a rank scans its contiguous chunk of the rank's slice 32 entries at a
-// time (coalesced, kTieU groups in flight) and counts matches by ballot; an
-// exclusive scan over the warps and the ranks' totals place the m-th match,
-// and the warp holding it rescans its chunk to find it.
-__device__ uint32_t tie_index(const Ctx &cx, const float *s, uint32_t n, uint32_t i0,
-                              uint32_t i1, uint32_t b, unsigned long long m) {
-  SelSmem &sm = *cx.sm;
-  constexpr uint32_t kTieU = 8;
-  const int lane = threadIdx.x % 32, warp = threadIdx.x / 32;
-  const uint32_t len = i1 > i0 ? i1 - i0 : 0;
-  const uint32_t per = ((len + kCWarps - 1) / kCWarps + 31u) & ~31u;
-  const uint32_t w0 = min(i1, i0 + uint32_t(warp) * per), w1 = min(i1, w0 + per);
-  auto matches = [&](uint32_t g) -> unsigned {  // ballot of group g (32 entries from w0)
-    const uint32_t i = w0 + g * 32 + lane;
-    return __ballot_sync(0xffffffffu, i < w1 && score_bits(s[i]) == b);
+  auto reach = [&](unsigned long long m, unsigned long long c) {
+    return by_mass ? (double)(base_m + m) >= target_m : (base_c + c) >= target_c;
   };
-  const uint32_t ngroups = (w1 - w0 + 31) / 32;
-  unsigned long long c = 0;
-  for (uint32_t g0 = 0; g0 < ngroups; g0 += kTieU) {
-    unsigned bal[kTieU];
-#pragma unroll
-    for (uint32_t u = 0; u < kTieU; ++u) bal[u] = g0 + u < ngroups ? matches(g0 + u) : 0u;
-#pragma unroll
-    for (uint32_t u = 0; u < kTieU; ++u) c += __popc(bal[u]);
-  }
-  unsigned long long tot;
-  const unsigned long long e = __shfl_sync(0xffffffffu,
-                                           block_excl_scan(lane == 0 ? c : 0ull, sm, &tot), 0);
-  if (threadIdx.x == 0) {
-    sm.res[4] = tot;
-    if (cx.rank == 0) sm.res[5] = n - 1;
-  }
-  cx.cl.sync();
-  unsigned long long off = 0;  // matches in the slices of lower ranks
-  for (unsigned q = 0; q < cx.rank; ++q) off += cx.peer(q)->res[4];
-  if (off + e < m && m <= off + e + c) {  // warp-uniform
-    unsigned long long r = off + e;
-    for (uint32_t g = 0; g < ngroups; ++g) {
-      const unsigned bal = matches(g);
-      const unsigned cnt = __popc(bal);
-      if (r + cnt >= m) {
-        // the (m - r)-th set bit of bal
-        unsigned x = bal;
-        for (unsigned long long k = r + 1; k < m; ++k) x &= x - 1;
-        if (lane == 0) cx.peer(0)->res[5] = w0 + g * 32 + uint32_t(__ffs(x) - 1);
+  if (!reach(em, ec) && reach(em + lm, ec + lc)) {
+    unsigned long long cm = em, cc = ec;
+    for (int p = p0; p < p0 + per; ++p) {
+      const int b = nbins - 1 - p;
+      if (reach(cm + hm[b], cc + hc[b])) {
+        *out = Crossing{uint32_t(b), cm, cc};
         break;
       }
-      r += cnt;
+      cm += hm[b];
+      cc += hc[b];
     }
-  }
-  cx.cl.sync();
-  const uint32_t idx = uint32_t(cx.peer(0)->res[5]);
-  cx.cl.sync();
-  return idx;
-}
-
-__device__ HeadSel select_list(const Ctx &cx, const float *s, uint32_t n, float gamma,
-                               unsigned long long lo, unsigned long long hi) {
-  HeadSel r{SEL_NONE, 0u, 0u, 0};
-  if (n == 0) return r;
-  const uint32_t chunk = (n + kCluster - 1) / kCluster;
-  const uint32_t i0 = min(n, cx.rank * chunk), i1 = min(n, i0 + chunk);
-  unsigned long long am = 0, ac = 0, k;
-  double target = 0.0;
-  uint32_t b = 0;
-  unsigned long long m = 0;
-  bool have_threshold = false;
-  if (gamma >= 1.f) {
-    k = n;
-  } else {
-    b = descend(cx, s, i0, i1, true, gamma, 0, &am, &ac, &target);
-    if (target <= 0.0) {
-      k = 0;
-    } else {
-      const unsigned long long w = score_mass(b);
-      // smallest m >= 1 with am + m * w >= target (w >= 1 here: a zero-mass
-      // bin cannot be the crossing one for a positive target)
-      unsigned long long mm = 1;
-      if (w > 0) {
-        double need = (target - (double)am) / (double)w;
-        mm = need <= 1.0 ? 1ull : (unsigned long long)ceil(need);
-        while (mm > 1 && (double)(am + (mm - 1) * w) >= target) --mm;
-        while ((double)(am + mm * w) < target) ++mm;
-      }
-      k = ac + mm;
-      m = mm;
-      have_threshold = true;
-    }
-  }
-  const unsigned long long kc = k < lo ? lo : (k > hi ? hi : k);
-  if (kc == 0) return r;
-  if (kc >= n) {
-    r.mode = SEL_ALL;
-    return r;
-  }
-  if (!(have_threshold && kc == k)) {
-    b = descend(cx, s, i0, i1, false, gamma, kc, &am, &ac, &target);
-    m = kc - ac;
-  }
-  r.mode = SEL_THRESHOLD;
-  r.bits = b;
-  r.idx = tie_index(cx, s, n, i0, i1, b, m);
-  return r;
-}
-
-// grid (kCluster * Hq, Bt), clusters of kCluster CTAs along x, kCThreads
-// threads, dynamic shared memory SelSmem.  Cluster h selects head h.
-__global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kCThreads)
-    select_head_kernel(const int32_t *__restrict__ pattern, const float *__restrict__ map,
-                       const float *__restrict__ vert, const float *__restrict__ slash, int n,
-                       int nb, int bs, float gamma, long long qa_lo, long long qa_hi, int vs_lo,
-                       int vs_hi, int qa_mode, HeadSel *__restrict__ sel,
-                       uint8_t *__restrict__ colflag, uint8_t *__restrict__ distflag) {
-  extern __shared__ __align__(16) unsigned char smem_raw[];
-  Ctx cx{cg::this_cluster(), 0u, reinterpret_cast<SelSmem *>(smem_raw)};
-  cx.rank = cx.cl.block_rank();
-  SelSmem &sm = *cx.sm;
-  const size_t heads_x = gridDim.x / kCluster;
-  const size_t bh = size_t(blockIdx.y) * heads_x + blockIdx.x / kCluster;
-  const size_t t_pairs = size_t(nb) * (nb + 1) / 2;
-  if (pattern[bh] == FP_PATTERN_QA) {  // uniform over the cluster
-    if (qa_mode == FP_QA_QUERYWISE) return;  // rows selected by select_rows_qa_kernel
-    HeadSel r = select_list(cx, map + bh * t_pairs, uint32_t(t_pairs), gamma, qa_lo, qa_hi);
-    if (cx.rank == 0 && threadIdx.x == 0) sel[2 * bh] = r;
-    return;
-  }
-  for (int i = threadIdx.x; i < nb; i += kCThreads) {
-    sm.colflag[i] = 0;
-    sm.distflag[i] = 0;
   }
   __syncthreads();
-  const float *vv = vert + bh * n;
-  const float *ss = slash + bh * n;
-  const uint32_t chunk = (uint32_t(n) + kCluster - 1) / kCluster;
-  const int s0 = int(min(uint32_t(n), cx.rank * chunk)), s1 = int(min(uint32_t(n), s0 + chunk));
-  HeadSel rv = select_list(cx, vv, uint32_t(n), gamma, vs_lo, vs_hi);
-  for (int t = s0 + threadIdx.x; t < s1; t += kCThreads)
-    if (kept(score_bits(vv[t]), uint32_t(t), rv)) sm.colflag[t / bs] = 1;
-  HeadSel rs = select_list(cx, ss, uint32_t(n), gamma, vs_lo, vs_hi);
-  for (int o = s0 + threadIdx.x; o < s1; o += kCThreads)
-    if (kept(score_bits(ss[o]), uint32_t(o), rs)) {
-      const int d0 = o / bs;
-      sm.distflag[d0] = 1;
-      if (o % bs != 0 && d0 + 1 < nb) sm.distflag[d0 + 1] = 1;
-    }
-  // OR the slices' flags: rank r writes blocks [r*per, (r+1)*per)
-  cx.cl.sync();
-  const int per = (nb + kCluster - 1) / kCluster;
-  for (int i = int(cx.rank) * per + threadIdx.x; i < min(nb, int(cx.rank + 1) * per);
-       i += kCThreads) {
-    uint8_t c = 0, d = 0;
-#pragma unroll
-    for (unsigned q = 0; q < kCluster; ++q) {
-      c |= cx.peer(q)->colflag[i];
-      d |= cx.peer(q)->distflag[i];
-    }
-    colflag[bh * nb + i] = c;
-    distflag[bh * nb + i] = d;
-  }
-  if (cx.rank == 0 && threadIdx.x == 0) {
-    sel[2 * bh] = rv;
-    sel[2 * bh + 1] = rs;
-  }
-  cx.cl.sync();  // peers' flags stay readable until every rank is done
 }
 
-// grid (ceil(nb/8), Hq, Bt), 256 threads: one warp per row.
+__device__ __forceinline__ void finish(ListState &st, HeadSel *sel, int mode, uint32_t bits,
+                                       uint32_t idx) {
+  st.finished = 1;
+  *sel = HeadSel{mode, bits, idx, 0};
+}
+
+// Switches to the count rule with target k; k = 0 keeps nothing and k >= len
+// everything.
+__device__ __forceinline__ void count_mode(ListState &st, HeadSel *sel, unsigned long long k,
+                                           uint32_t len) {
+  st.by_mass = 0;
+  st.target_c = k;
+  if (k == 0) finish(st, sel, SEL_NONE, 0u, 0u);
+  else if (k >= len) finish(st, sel, SEL_ALL, 0u, 0u);
+}
+
+// One level's decision (the whole CTA; st and the histogram in shared memory):
+// the crossing digit by mass, or by count once the clamp decides k, appended
+// to the prefix.  Returns the crossing bin's count.
+__device__ unsigned int decide_level(ListState &st, HeadSel *sel, const ListView &lv,
+                                     const unsigned long long *hm, const unsigned int *hc,
+                                     int nbins, int shift, unsigned long long *warp_tot,
+                                     Crossing *cr) {
+  if (st.by_mass) {
+    find_crossing(hm, hc, nbins, true, st.target_m, st.am, 0, 0, warp_tot, cr);
+    const unsigned long long A = st.ac + cr->above_c, C = hc[cr->bin];
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      if (lv.hi <= A) count_mode(st, sel, lv.hi, lv.len);
+      else if (lv.lo >= A + C) count_mode(st, sel, lv.lo, lv.len);
+    }
+    __syncthreads();
+    if (st.finished) return 0;
+  }
+  if (!st.by_mass) find_crossing(hm, hc, nbins, false, 0.0, 0, st.target_c, st.ac, warp_tot, cr);
+  const unsigned int cnt = hc[cr->bin];
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    st.am += cr->above_m;
+    st.ac += cr->above_c;
+    st.prefix |= cr->bin << shift;
+  }
+  __syncthreads();
+  return cnt;
+}
+
+// Clears the histograms and states of every slot and the VS flags; grid
+// (slots), kSelThreads threads.
+__global__ void __launch_bounds__(kSelThreads) sel_prep_kernel(SelArgs a, uint8_t *colflag,
+                                                               uint8_t *distflag) {
+  const int slot = blockIdx.x;
+  for (int b = threadIdx.x; b < kBins; b += kSelThreads) {
+    a.hm[size_t(slot) * kBins + b] = 0ull;
+    a.hc[size_t(slot) * kBins + b] = 0u;
+  }
+  uint8_t *flags = (slot % 2 == 0 ? colflag : distflag) + size_t(slot / 2) * a.nb;
+  for (int i = threadIdx.x; i < a.nb; i += kSelThreads) flags[i] = 0;
+  if (threadIdx.x == 0) a.state[slot] = ListState{};
+}
+
+// Levels 1 and 2: grid (CTAs per list, slots), kSelThreads threads, dynamic
+// shared memory hist_smem<LEVEL>(); CTA x of a list takes its chunks x,
+// x + nct, ... (at most kMaxCtaChunks of them), the next one's loads issued
+// before the current one is added.
+template <int LEVEL>
+constexpr size_t hist_smem() {
+  return (LEVEL == 1 ? kBins1 : kBins2) * 12;
+}
+
+template <int LEVEL>
+__global__ void __launch_bounds__(kSelThreads) sel_hist_kernel(SelArgs a) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  constexpr int NB = LEVEL == 1 ? kBins1 : kBins2;
+  __shared__ unsigned long long warp_tot[kSelThreads / 32 + 1];
+  __shared__ ListState st;
+  __shared__ Crossing cr;
+  __shared__ int is_last;
+  const int slot = blockIdx.y, lane = threadIdx.x % 32;
+  ListView lv;
+  if (!list_of(a, slot, &lv)) return;
+  const int nch = list_chunks(lv);
+  const int nct = min(nch, a.ctas);  // CTAs on this list, each taking every nct-th chunk
+  if (int(blockIdx.x) >= nct) return;
+  ListState *gst = a.state + slot;
+  uint32_t want = 0;  // level 2: the level-1 digit
+  if (LEVEL == 2) {
+    if (gst->finished) return;
+    want = gst->prefix >> kShift1;
+  }
+  SmemHist h{reinterpret_cast<unsigned int *>(smem_raw),
+             reinterpret_cast<unsigned int *>(smem_raw) + NB,
+             reinterpret_cast<unsigned int *>(smem_raw) + 2 * NB};
+  for (int b = threadIdx.x; b < 3 * NB; b += kSelThreads) h.lo[b] = 0u;
+  __syncthreads();
+  const int off = group_offset(lv.p);
+  constexpr int kG = kChunk / 4 / kSelThreads;  // groups per thread per chunk
+  uint32_t bits[kG][4], nbits[kG][4];
+  bool valid[kG][4], nvalid[kG][4];
+  int chunk = blockIdx.x;
+#pragma unroll
+  for (int u = 0; u < kG; ++u)
+    load_group(lv, off, uint32_t(chunk) * (kChunk / 4) + u * kSelThreads + threadIdx.x, bits[u],
+               valid[u]);
+  for (; chunk < nch; chunk += nct) {
+    const int next = chunk + nct;
+    if (next < nch) {
+#pragma unroll
+      for (int u = 0; u < kG; ++u)
+        load_group(lv, off, uint32_t(next) * (kChunk / 4) + u * kSelThreads + threadIdx.x,
+                   nbits[u], nvalid[u]);
+    }
+#pragma unroll
+    for (int u = 0; u < kG; ++u) {
+      uint32_t bin[4];
+      uint64_t w[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const uint32_t x = bits[u][e];
+        bin[e] = 0xFFFFFFFFu;
+        w[e] = 0;
+        if (valid[u][e] && (LEVEL == 1 || (x >> kShift1) == want)) {
+          bin[e] = LEVEL == 1 ? (x >> kShift1) : ((x >> kShift2) & (kBins2 - 1));
+          w[e] = score_mass(x);
+        }
+      }
+      if (LEVEL == 1) {
+        hist_add4(h, bin, w, lane);
+      } else {  // below the exponent nearly every entry has its own bin
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          if (bin[e] != 0xFFFFFFFFu) h.add(bin[e], w[e], 1u);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kG; ++u)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        bits[u][e] = nbits[u][e];
+        valid[u][e] = nvalid[u][e];
+      }
+  }
+  __syncthreads();
+  unsigned long long *ghm = a.hm + size_t(slot) * kBins;
+  unsigned int *ghc = a.hc + size_t(slot) * kBins;
+  for (int b = threadIdx.x; b < NB; b += kSelThreads)
+    if (h.cnt[b]) {
+      atomicAdd(&ghm[b], (unsigned long long)h.lo[b] + ((unsigned long long)h.hi[b] << 16));
+      atomicAdd(&ghc[b], h.cnt[b]);
+    }
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) is_last = atomicAdd(&gst->done[LEVEL - 1], 1u) == unsigned(nct - 1);
+  __syncthreads();
+  if (!is_last) return;
+  // the last CTA of this list: every other CTA's bins are in the global
+  // histogram; it is read into this CTA's shared memory (NB * 12 bytes)
+  __threadfence();
+  unsigned long long *hm = reinterpret_cast<unsigned long long *>(smem_raw);
+  unsigned int *hc = reinterpret_cast<unsigned int *>(smem_raw + size_t(NB) * 8);
+  for (int b = threadIdx.x; b < NB; b += kSelThreads) {
+    hm[b] = __ldcg(&ghm[b]);
+    hc[b] = __ldcg(&ghc[b]);
+  }
+  if (threadIdx.x == 0) st = *gst;
+  __syncthreads();
+  HeadSel *sel = a.sel + slot;
+  if (LEVEL == 1) {
+    unsigned long long part = 0, tot;
+    for (int b = threadIdx.x; b < NB; b += kSelThreads) part += hm[b];
+    block_excl_scan(part, warp_tot, &tot);  // tot = W, the list's total mass
+    if (threadIdx.x == 0) {
+      st.by_mass = 0;
+      if (a.gamma >= 1.f) {
+        count_mode(st, sel, lv.hi < lv.len ? lv.hi : lv.len, lv.len);  // k_gamma = len
+      } else {
+        st.target_m = (double)a.gamma * (double)tot;
+        if (st.target_m <= 0.0) count_mode(st, sel, lv.lo, lv.len);  // k_gamma = 0
+        else st.by_mass = 1;
+      }
+    }
+    __syncthreads();
+  }
+  if (!st.finished) {
+    const unsigned int cnt = decide_level(st, sel, lv, hm, hc, NB,
+                                          LEVEL == 1 ? kShift1 : kShift2, warp_tot, &cr);
+    if (LEVEL == 2 && threadIdx.x == 0 && !st.finished) st.overflow = cnt > unsigned(kCand);
+  }
+  // level 1: the global histogram is reused for level 2
+  if (LEVEL == 1)
+    for (int b = threadIdx.x; b < NB; b += kSelThreads) {
+      ghm[b] = 0ull;
+      ghc[b] = 0u;
+    }
+  if (threadIdx.x == 0) {
+    st.done[LEVEL - 1] = gst->done[LEVEL - 1];
+    *gst = st;
+  }
+}
+
+// The m-th (1-based) smallest of the n indices in idx[] (shared memory, n <=
+// kCand): a bitonic sort of the padded power of two.
+__device__ uint32_t mth_smallest(uint32_t *idx, int n, unsigned long long m) {
+  if (m < 1) m = 1;  // (1 <= m <= n by construction)
+  if (m > (unsigned long long)n) m = n > 0 ? n : 1;
+  int P = 1;
+  while (P < n) P <<= 1;
+  for (int i = n + threadIdx.x; i < P; i += kSelThreads) idx[i] = 0xFFFFFFFFu;
+  __syncthreads();
+  for (int k = 2; k <= P; k <<= 1)
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      for (int i = threadIdx.x; i < P; i += kSelThreads) {
+        const int ixj = i ^ j;
+        if (ixj > i) {
+          const uint32_t x = idx[i], y = idx[ixj];
+          if ((i & k) == 0 ? x > y : x < y) {
+            idx[i] = y;
+            idx[ixj] = x;
+          }
+        }
+      }
+      __syncthreads();
+    }
+  return idx[m - 1];
+}
+
+// Level 3 and the tie rank: grid (CTAs per list, slots), chunks as above.
+__global__ void __launch_bounds__(kSelThreads) sel_compact_kernel(SelArgs a) {
+  __shared__ unsigned long long hm[kBins3];
+  __shared__ unsigned int hc[kBins3];
+  __shared__ uint2 cand[kCand];
+  __shared__ uint32_t ties[kCand];
+  __shared__ unsigned long long warp_tot[kSelThreads / 32 + 1];
+  __shared__ ListState st;
+  __shared__ Crossing cr;
+  __shared__ int is_last, nties;
+  __shared__ unsigned long long found;
+  const int slot = blockIdx.y, lane = threadIdx.x % 32;
+  ListView lv;
+  if (!list_of(a, slot, &lv)) return;
+  const int nch = list_chunks(lv);
+  const int nct = min(nch, a.ctas);
+  if (int(blockIdx.x) >= nct) return;
+  ListState *gst = a.state + slot;
+  if (gst->finished) return;
+  const uint32_t want = gst->prefix >> kShift2;  // the first two digits
+  const int off = group_offset(lv.p);
+  uint2 *gc = a.cand + size_t(slot) * kCand;
+  if (!gst->overflow) {
+    constexpr int kG = kChunk / 4 / kSelThreads;
+    for (int chunk = blockIdx.x; chunk < nch; chunk += nct) {
+      const uint32_t g0 = uint32_t(chunk) * (kChunk / 4);
+      uint32_t bits[kG][4];
+      bool valid[kG][4];
+#pragma unroll
+      for (int u = 0; u < kG; ++u)
+        load_group(lv, off, g0 + u * kSelThreads + threadIdx.x, bits[u], valid[u]);
+#pragma unroll
+      for (int u = 0; u < kG; ++u)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const bool hit = valid[u][e] && (bits[u][e] >> kShift2) == want;
+          const unsigned bal = __ballot_sync(0xffffffffu, hit);
+          if (bal) {
+            unsigned base = 0;
+            if (lane == __ffs(bal) - 1) base = atomicAdd(&gst->cand, unsigned(__popc(bal)));
+            base = __shfl_sync(0xffffffffu, base, __ffs(bal) - 1);
+            if (hit) {
+              const uint32_t i = (g0 + u * kSelThreads + threadIdx.x) * 4 + e - off;
+              gc[base + __popc(bal & ((1u << lane) - 1u))] = make_uint2(bits[u][e], i);
+            }
+          }
+        }
+    }
+  }
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) is_last = atomicAdd(&gst->done[2], 1u) == unsigned(nct - 1);
+  __syncthreads();
+  if (!is_last) return;
+  __threadfence();
+  if (threadIdx.x == 0) st = *gst;
+  for (int b = threadIdx.x; b < kBins3; b += kSelThreads) {
+    hm[b] = 0ull;
+    hc[b] = 0u;
+  }
+  __syncthreads();
+  HeadSel *sel = a.sel + slot;
+  // level 3 over the entries that share the first two digits
+  const int nc = st.overflow ? 0 : int(__ldcg(&gst->cand));
+  if (!st.overflow) {
+    for (int c = threadIdx.x; c < nc; c += kSelThreads) cand[c] = __ldcg(&gc[c]);
+    __syncthreads();
+    for (int c0 = 0; c0 < nc; c0 += kSelThreads) {
+      const int c = c0 + threadIdx.x;
+      uint32_t bin = 0xFFFFFFFFu;
+      uint64_t w = 0;
+      if (c < nc) {
+        bin = cand[c].x & (kBins3 - 1);  // (the third digit)
+        w = score_mass(cand[c].x);
+      }
+      hist_add(hm, hc, bin, w, lane);
+    }
+  } else {  // too many entries share the prefix: scan the whole list
+    for (uint32_t i0 = 0; i0 < lv.len; i0 += kSelThreads) {
+      const uint32_t i = i0 + threadIdx.x;
+      uint32_t bin = 0xFFFFFFFFu;
+      uint64_t w = 0;
+      if (i < lv.len) {
+        const uint32_t x = score_bits(lv.p[i]);
+        if ((x >> kShift2) == want) {
+          bin = x & (kBins3 - 1);
+          w = score_mass(x);
+        }
+      }
+      hist_add(hm, hc, bin, w, lane);
+    }
+  }
+  __syncthreads();
+  decide_level(st, sel, lv, hm, hc, kBins3, 0, warp_tot, &cr);
+  if (st.finished) {  // (the clamp with k = 0 or k >= len, decided here)
+    if (threadIdx.x == 0) *gst = st;
+    return;
+  }
+  const uint32_t b = st.prefix;  // the full threshold pattern
+  unsigned long long m;
+  if (st.by_mass) {
+    // smallest m >= 1 with am + m w >= target (w >= 1: a zero-mass bin cannot
+    // be the crossing one for a positive target), then the clamp, which by
+    // construction keeps k inside this pattern's entries
+    const unsigned long long w = score_mass(b);
+    unsigned long long mm = 1;
+    if (w > 0) {
+      const double need = (st.target_m - (double)st.am) / (double)w;
+      mm = need <= 1.0 ? 1ull : (unsigned long long)ceil(need);
+      while (mm > 1 && (double)(st.am + (mm - 1) * w) >= st.target_m) --mm;
+      while ((double)(st.am + mm * w) < st.target_m) ++mm;
+    }
+    unsigned long long k = st.ac + mm;
+    k = k < lv.lo ? lv.lo : (k > lv.hi ? lv.hi : k);
+    m = k - st.ac;
+  } else {
+    m = st.target_c - st.ac;
+  }
+  // the m-th entry with pattern b, in index order
+  if (!st.overflow) {
+    if (threadIdx.x == 0) nties = 0;
+    __syncthreads();
+    for (int c = threadIdx.x; c < nc; c += kSelThreads)
+      if (cand[c].x == b) ties[atomicAdd(&nties, 1)] = cand[c].y;
+    __syncthreads();
+    const uint32_t idx = mth_smallest(ties, nties, m);
+    if (threadIdx.x == 0) finish(st, sel, SEL_THRESHOLD, b, idx);
+  } else {
+    // ordered count over the whole list, kSelThreads entries at a time
+    if (threadIdx.x == 0) found = 0xFFFFFFFFull;
+    __syncthreads();
+    unsigned long long before = 0;
+    for (uint32_t i0 = 0; i0 < lv.len && found == 0xFFFFFFFFull; i0 += kSelThreads) {
+      const uint32_t i = i0 + threadIdx.x;
+      const bool hit = i < lv.len && score_bits(lv.p[i]) == b;
+      unsigned long long tot;
+      const unsigned long long e = block_excl_scan(hit ? 1ull : 0ull, warp_tot, &tot);
+      if (hit && before + e + 1 == m) found = i;
+      before += tot;
+      __syncthreads();
+    }
+    if (threadIdx.x == 0) finish(st, sel, SEL_THRESHOLD, b, uint32_t(found));
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) *gst = st;
+}
+
+// Column and distance flags of the vertical-slash heads from their kept
+// lines: grid (ceil(n / (256 * kFlagU)), slots), 256 threads, kFlagU lines a
+// thread (strided by 256).
+constexpr int kFlagU = 16;
+__global__ void __launch_bounds__(256) sel_flags_kernel(SelArgs a, uint8_t *__restrict__ colflag,
+                                                        uint8_t *__restrict__ distflag) {
+  const int slot = blockIdx.y;
+  const size_t bh = size_t(slot) / 2;
+  if (a.pattern[bh] == FP_PATTERN_QA) return;
+  const HeadSel s = a.sel[slot];
+  if (s.mode == SEL_NONE) return;
+  const float *line = (slot % 2 == 0 ? a.vert : a.slash) + bh * a.n;
+  uint8_t *cf = colflag + bh * a.nb;
+  uint8_t *df = distflag + bh * a.nb;
+#pragma unroll 4
+  for (int u = 0; u < kFlagU; ++u) {
+    const int t = (blockIdx.x * kFlagU + u) * 256 + threadIdx.x;
+    if (t >= a.n || !kept(score_bits(line[t]), uint32_t(t), s)) continue;
+    if (slot % 2 == 0) {
+      cf[t / a.bs] = 1;
+    } else {
+      const int d0 = t / a.bs;
+      df[d0] = 1;
+      if (t % a.bs != 0 && d0 + 1 < a.nb) df[d0 + 1] = 1;
+    }
+  }
+}
+
+// grid (ceil(nb/8), Hq, Bt), 256 threads: one warp per row, kEmitU groups of
+// 32 entries in flight.
+constexpr int kEmitU = 8;
 __global__ void __launch_bounds__(256) emit_rows_kernel(
     const int32_t *__restrict__ pattern, const float *__restrict__ map, int nb,
     const HeadSel *__restrict__ sel, const uint8_t *__restrict__ colflag,
@@ -484,20 +772,28 @@ __global__ void __launch_bounds__(256) emit_rows_kernel(
   const uint8_t *df = distflag + bh * nb;
   int32_t *out = indices + (bh * nb + qi) * size_t(nb);
   int cnt = 0;
-  for (int j0 = 0; j0 <= qi; j0 += 32) {
-    const int j = j0 + lane;
-    bool keep = false;
-    if (j <= qi) {
-      if (j == qi)
-        keep = true;
-      else if (qa)
-        keep = kept(score_bits(mrow[j]), uint32_t(rowbase + j), s);
-      else
-        keep = cf[j] || df[qi - j];
+  constexpr int kU = kEmitU;
+  for (int j0 = 0; j0 <= qi; j0 += 32 * kU) {
+    bool keep[kU];
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const int j = j0 + u * 32 + lane;
+      keep[u] = false;
+      if (j <= qi) {
+        if (j == qi)
+          keep[u] = true;
+        else if (qa)
+          keep[u] = kept(score_bits(mrow[j]), uint32_t(rowbase + j), s);
+        else
+          keep[u] = cf[j] || df[qi - j];
+      }
     }
-    const unsigned bal = __ballot_sync(0xffffffffu, keep);
-    if (keep) out[cnt + __popc(bal & ((1u << lane) - 1u))] = j;
-    cnt += __popc(bal);
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const unsigned bal = __ballot_sync(0xffffffffu, keep[u]);
+      if (keep[u]) out[cnt + __popc(bal & ((1u << lane) - 1u))] = j0 + u * 32 + lane;
+      cnt += __popc(bal);
+    }
   }
   if (lane == 0) counts[bh * nb + qi] = cnt;
 }
@@ -671,12 +967,30 @@ __global__ void stats_kernel(const int32_t *__restrict__ counts,
 
 }  // namespace
 
+// Streaming multiprocessors of the current device (cached per device).
+int sm_count() {
+  static int cache[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (cache[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1)
+      n = 148;
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
 size_t select_ws_bytes(const Dims &D) {
   Carver c{nullptr, 0};
-  const size_t heads = size_t(D.bt) * D.hq;
-  c.take<HeadSel>(2 * heads);
+  const size_t heads = size_t(D.bt) * D.hq, slots = 2 * heads;
+  c.take<HeadSel>(slots);
   c.take<uint8_t>(heads * D.nb);
   c.take<uint8_t>(heads * D.nb);
+  c.take<ListState>(slots);
+  c.take<unsigned long long>(slots * kBins);
+  c.take<unsigned int>(slots * kBins);
+  c.take<uint2>(slots * kCand);
   return c.off + 256;
 }
 
@@ -687,28 +1001,61 @@ cudaError_t launch_select(const Dims &D, float gamma, const SelectBudgets &bud,
   if (D.nb > kMaxBlocks) return cudaErrorInvalidValue;
   Carver c{static_cast<char *>(ws), 0};
   const size_t heads = size_t(D.bt) * D.hq;
-  HeadSel *sel = c.take<HeadSel>(2 * heads);
+  const int slots = int(2 * heads);
+  SelArgs a;
+  a.sel = c.take<HeadSel>(slots);
   uint8_t *cf = c.take<uint8_t>(heads * D.nb);
   uint8_t *df = c.take<uint8_t>(heads * D.nb);
-  const int smem = int(sizeof(SelSmem));
-  cudaFuncSetAttribute(select_head_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  a.state = c.take<ListState>(slots);
+  a.hm = c.take<unsigned long long>(size_t(slots) * kBins);
+  a.hc = c.take<unsigned int>(size_t(slots) * kBins);
+  a.cand = c.take<uint2>(size_t(slots) * kCand);
+  a.pattern = pattern;
+  a.map = map;
+  a.vert = vert;
+  a.slash = slash;
+  a.n = D.n;
+  a.nb = D.nb;
+  a.bs = D.bs;
+  a.gamma = gamma;
+  a.qa_lo = bud.qa_lo;
+  a.qa_hi = bud.qa_hi;
+  a.vs_lo = bud.vs_lo;
+  a.vs_hi = bud.vs_hi;
+  a.qa_mode = bud.qa_mode;
   if (bud.vs_mode == FP_VS_BLOCKS) {
     // pooled lines live in the outputs until emit_rows_kernel overwrites them:
-    // vert sums in indices (>= Bt*Hq*nb entries), slash sums in counts
+    // vert sums in indices (>= Bt*Hq*nb entries), slash sums in counts; they
+    // are then lines of nb tokens with block size 1
     float *pv = reinterpret_cast<float *>(indices);
     float *ps = reinterpret_cast<float *>(counts);
     pool_lines_kernel<<<dim3((D.nb + 255) / 256, D.hq, D.bt), 256, 0, st>>>(
         pattern, vert, slash, D.n, D.nb, D.bs, pv, ps);
-    select_head_kernel<<<dim3(kCluster * D.hq, D.bt), kCThreads, smem, st>>>(
-        pattern, map, pv, ps, D.nb, D.nb, 1, gamma, bud.qa_lo, bud.qa_hi, bud.vsb_lo,
-        bud.vsb_hi, bud.qa_mode, sel, cf, df);
-  } else {
-    select_head_kernel<<<dim3(kCluster * D.hq, D.bt), kCThreads, smem, st>>>(
-        pattern, map, vert, slash, D.n, D.nb, D.bs, gamma, bud.qa_lo, bud.qa_hi, bud.vs_lo,
-        bud.vs_hi, bud.qa_mode, sel, cf, df);
+    a.vert = pv;
+    a.slash = ps;
+    a.n = D.nb;
+    a.bs = 1;
+    a.vs_lo = bud.vsb_lo;
+    a.vs_hi = bud.vsb_hi;
   }
+  long long maxlen = a.n;
+  if (bud.qa_mode == FP_QA_FLATTENED && D.t_pairs > maxlen) maxlen = D.t_pairs;
+  const int max_chunks = int((maxlen + 3 + kChunk - 1) / kChunk);
+  // about kSelCtasPerSm CTAs per SM over all slots, each looping over chunks,
+  // and enough of them that no CTA takes more than kMaxCtaChunks
+  a.ctas = std::max(1, std::min(max_chunks, sm_count() * kSelCtasPerSm / slots));
+  a.ctas = std::max(a.ctas, (max_chunks + kMaxCtaChunks - 1) / kMaxCtaChunks);
+  const unsigned chunks = unsigned(a.ctas);
+  cudaFuncSetAttribute(sel_hist_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                       int(hist_smem<2>()));
+  sel_prep_kernel<<<slots, kSelThreads, 0, st>>>(a, cf, df);
+  sel_hist_kernel<1><<<dim3(chunks, slots), kSelThreads, hist_smem<1>(), st>>>(a);
+  sel_hist_kernel<2><<<dim3(chunks, slots), kSelThreads, hist_smem<2>(), st>>>(a);
+  sel_compact_kernel<<<dim3(chunks, slots), kSelThreads, 0, st>>>(a);
+  sel_flags_kernel<<<dim3((a.n + 256 * kFlagU - 1) / (256 * kFlagU), slots), 256, 0, st>>>(
+      a, cf, df);
   emit_rows_kernel<<<dim3((D.nb + 7) / 8, D.hq, D.bt), 256, 0, st>>>(
-      pattern, map, D.nb, sel, cf, df, bud.qa_mode, counts, indices);
+      pattern, map, D.nb, a.sel, cf, df, bud.qa_mode, counts, indices);
   if (bud.qa_mode == FP_QA_QUERYWISE) {
     int pmax;
     const size_t rsm = rows_qa_smem(D.nb, &pmax);
@@ -732,9 +1079,9 @@ cudaError_t launch_stats(const Dims &D, const int32_t *counts, const int32_t *pa
 // select_ws_bytes describes) is one fixed array compiled into the library.
 // The array's name is only a host-side stand-in in host code, so the device
 // address is looked up with cudaGetSymbolAddress once per device (on the
-// first call made with that device current) and cached.  Nothing in the
-// scratch has to start at zero: select_head_kernel writes every record and
-// flag that emit_rows_kernel later reads.
+// first call made with that device current) and cached.  What must start at
+// zero (histograms, counters, flags) is cleared by sel_prep_kernel, the
+// first launch of every call.
 namespace fpi {
 
 static __device__ __align__(256) unsigned char g_select_scratch[FP_SELECT_NOALLOC_SCRATCH_BYTES];

@@ -218,11 +218,12 @@ fp_status fp_select(const fp_shape *shape, const fp_params *params,
  *     stream.  A cudaDeviceReset() ends the context that address belongs
  *     to, so do not call this entry point on a device after resetting it.
  *   * Every call on a device uses the same array, which keeps the last
- *     call's contents (nothing in it needs clearing).  Two calls whose work
- *     can overlap on the GPU (different streams, several host threads) race
- *     on it: the caller must order them.
+ *     call's contents; each call first clears the histograms, counters and
+ *     flags it accumulates into, so no call depends on the one before it.
+ *     Two calls whose work can overlap on the GPU (different streams,
+ *     several host threads) race on it: the caller must order them.
  */
-#define FP_SELECT_NOALLOC_SCRATCH_BYTES (1u << 20)
+#define FP_SELECT_NOALLOC_SCRATCH_BYTES (4u << 20)
 fp_status fp_select_noalloc(const fp_shape *shape, const fp_params *params,
                             const int32_t *pattern, const float *map,
                             const float *vert, const float *slash,
