@@ -1,9 +1,12 @@
 """Benchmark of the FlexPrefill prefill-attention hot path on B200.
 
-One step = one pass of the whole path over one attention layer (all heads):
-fp_estimate -> fp_pattern -> fp_select -> fp_sparse_attn, on seeded synthetic
-Q/K/V shaped like a Llama-3.1-8B layer at 128k tokens (32 q / 8 kv heads,
-d = 128, block 128).  Prints ONE JSON line (rank 0).
+One step = one pass of the whole path over one attention layer (all heads)
+in one fp_prefill_attn call (estimate -> pattern -> select -> sparse
+attention, each head's estimate limited to what its pattern reads), on seeded
+synthetic Q/K/V shaped like a Llama-3.1-8B layer at 128k tokens (32 q / 8 kv
+heads, d = 128, block 128).  The same layer then runs as the four staged calls
+(fp_estimate, fp_pattern, fp_select, fp_sparse_attn) for the per-stage times
+and the attention roofline.  Prints ONE JSON line (rank 0).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -36,7 +39,10 @@ import torch  # noqa: E402
 from dynamic_block_sparse_fp_b200 import synth  # noqa: E402
 
 METRIC = "prefill-attn tokens/s and effective TFLOPS (% bf16 peak) at 128k; speedup vs dense"
-LAUNCHES_PER_STEP = 16  # estimate 8, pattern 1, select 6, attention 1
+# the library's kernels per step of fp_prefill_attn: estimate 11 (6 for the
+# pattern's inputs, 3 for the query-aware heads' map, 2 for the vertical-slash
+# heads' lines), pattern 1, select 6, attention 1
+LAUNCHES_PER_STEP = 19
 
 
 def kernel_traffic(source: str, workload: str):
@@ -228,10 +234,12 @@ def cores() -> int:
 
 
 def workload_config(w: synth.Workload, ws: int, heads: bool = False) -> dict:
-    if heads:
+    if ws == 1:
+        par = "single GPU"
+    elif heads:
         par = f"kv heads split over {ws} ranks, outputs all-gathered (NCCL)"
     else:
-        par = f"independent layers x{ws}" if ws > 1 else "single GPU"
+        par = f"independent layers x{ws}"
     return {"workload": w.name, "batch_per_gpu": w.batch,
             "global_batch": w.batch if heads else w.batch * ws,
             "seq_len": w.seq_len, "n_q_heads": w.n_q_heads, "n_kv_heads": w.n_kv_heads,
@@ -368,6 +376,45 @@ def measure(layer, p, args, stream, ws, local, gather=None) -> dict:
             "clocks": clk.summary()}
 
 
+def measure_prefill(layer, p, args, stream, ws, local, gather=None) -> dict:
+    """The whole path in one fp_prefill_attn call per step: W untimed steps,
+    then K timed steps bracketed by barrier + synchronize."""
+    from dynamic_block_sparse_fp_b200 import ops
+    wsp = ops.workspace(layer.s, ops.FP_CALL_PREFILL, layer.q.device)
+    stats = torch.zeros(2, dtype=torch.int64, device=layer.q.device)
+
+    def step(st=None):
+        ops._check(ops.fp_prefill_attn(layer.s, p, layer.q, layer.k, layer.v, layer.out, None,
+                                       st, wsp, stream), "fp_prefill_attn")
+        if gather is not None:
+            gather(layer.out)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert ops.fp_last_device_status(stream) == 0
+    barrier(ws)
+    torch.cuda.synchronize()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        t_start.record(stream)
+        for _ in range(args.steps):
+            step()
+        t_end.record(stream)
+        torch.cuda.synchronize()
+    barrier(ws)
+    status = ops.fp_last_device_status(stream)
+    if status != 0:
+        raise RuntimeError(f"device status {ops.STATUS.get(status, status)}")
+    total_ms = max_over_ranks(t_start.elapsed_time(t_end), ws, layer.q.device)
+    step(stats)  # (untimed) the kept blocks and query-aware heads of this layer
+    torch.cuda.synchronize()
+    del wsp
+    return {"ms_step": total_ms / args.steps, "kept": int(stats[0]), "qa_heads": int(stats[1]),
+            "clocks": clk.summary()}
+
+
 def dense_ms(layer, stream, reps: int = 2) -> float:
     """fp_dense_attn (the same kernel over every causal block), CUDA events."""
     from dynamic_block_sparse_fp_b200 import ops
@@ -384,11 +431,13 @@ def dense_ms(layer, stream, reps: int = 2) -> float:
     return de[0].elapsed_time(de[1]) / reps
 
 
-def path_fields(layer, m: dict, peaks: dict, dense: float | None) -> dict:
-    """Kept fraction, per-stage times and rooflines of one measured configuration."""
+def path_fields(layer, m: dict, peaks: dict, dense: float | None, whole: dict) -> dict:
+    """Kept fraction, per-stage times and rooflines of one measured configuration:
+    `whole` is the timed fp_prefill_attn loop, `m` the staged calls' loop."""
     bt, hq, n, d = layer.q.shape
     bs, nb = layer.bs, layer.nb
     st = m["stage_ms"]
+    assert whole["kept"] == m["kept"] and whole["qa_heads"] == m["qa_heads"]
     t_pairs = nb * (nb + 1) // 2
     flop_block = 4.0 * bs * bs * d
     attn_flops = flop_block * m["kept"]
@@ -402,14 +451,17 @@ def path_fields(layer, m: dict, peaks: dict, dense: float | None) -> dict:
                      "peak": peak_t, "unit": "TFLOP/s", "frac": attn_tflops / peak_t,
                      "peak_kind": f"bf16 dense, sustained ({peaks['source']})",
                      "algorithmic_flops_per_launch": attn_flops},
+        # the four staged calls (fp_estimate computes every output for every
+        # head; the whole-path call skips what each head's pattern does not read)
         "stages_ms": {"estimate": st[0], "pattern": st[1], "select": st[2],
-                      "sparse_attn": st[3]},
+                      "sparse_attn": st[3], "staged_step": m["ms_step"],
+                      "whole_path_before_attention": whole["ms_step"] - st[3]},
         "estimate_hbm": {"bytes": eb, "gbs": eb / (st[0] * 1e-3) / 1e9,
                          "frac": eb / (st[0] * 1e-3) / 1e9 / hbm},
         "select_hbm": {"bytes": sb, "gbs": sb / (st[2] * 1e-3) / 1e9,
                        "frac": sb / (st[2] * 1e-3) / 1e9 / hbm},
         "effective_tflops": {"sparse_attn": attn_tflops,
-                             "whole_step": attn_flops / (m["ms_step"] * 1e-3) / 1e12},
+                             "whole_step": attn_flops / (whole["ms_step"] * 1e-3) / 1e12},
         "kept_blocks": m["kept"], "causal_blocks": t_pairs * hq * bt,
         "kept_fraction": m["kept"] / (t_pairs * hq * bt), "qa_heads": m["qa_heads"],
         "sparsity_implied_ratio": t_pairs * hq * bt / m["kept"],
@@ -417,7 +469,8 @@ def path_fields(layer, m: dict, peaks: dict, dense: float | None) -> dict:
     if dense is not None:
         f["dense_attn_ms"] = dense
         f["dense_tflops"] = flop_block * t_pairs * hq * bt / (dense * 1e-3) / 1e12
-        f["speedup_vs_dense"] = {"whole_step": dense / m["ms_step"],
+        f["speedup_vs_dense"] = {"whole_step": dense / whole["ms_step"],
+                                 "staged_step": dense / m["ms_step"],
                                  "sparse_attn_only": dense / st[3]}
         f["speedup_target"] = 0.8 * f["sparsity_implied_ratio"]
     return f
@@ -448,12 +501,13 @@ def run_ours(args, w, ws, rank, local):
         run_sweep(args, w, layer, ws, rank, local, stream, peaks, gather, heads)
         return
     p = ops.make_params(w.gamma, w.tau, w.min_budget, w.max_budget, w.qa_mode, w.vs_mode)
+    whole = measure_prefill(layer, p, args, stream, ws, local, gather)
     m = measure(layer, p, args, stream, ws, local, gather)
-    ms_step = m["ms_step"]
+    ms_step = whole["ms_step"]
     # weak scaling: every rank's own layer; head sharding: one layer in all
     value = tokens / (ms_step * 1e-3) if heads else job_value(tokens, ws, ms_step)
     dense = None if args.no_dense else dense_ms(layer, stream)
-    fields = path_fields(layer, m, peaks, dense)
+    fields = path_fields(layer, m, peaks, dense, whole)
     fields["roofline"]["traffic"] = kernel_traffic("attn_tc.cu", w.name)
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws,
@@ -463,13 +517,16 @@ def run_ours(args, w, ws, rank, local):
         "data": "synthetic (seeded Q/K/V with planted query-aware / vertical-slash structure "
                 "and RoPE; no dataset or weights)",
         "config": workload_config(w, ws, heads),
-        # the library's kernels per step: 12, plus the query-wise row
+        "step": "fp_prefill_attn (the whole path in one call); stages_ms and the roofline "
+                "come from the same layer run as the four staged calls",
+        # the library's kernels per timed step, plus the query-wise row
         # selection and the line pooling when those modes are on
         "gpu_launches": (LAUNCHES_PER_STEP + int(w.qa_mode == 1) + int(w.vs_mode == 1))
                         * args.steps,
     }
     line.update(fields)
-    line["clocks"] = m["clocks"]
+    line["clocks"] = whole["clocks"]
+    line["clocks_staged"] = m["clocks"]
     # ---- end to end through the C ABI with host buffers ----
     if not args.no_e2e:
         qh, kh, vh = (inp[x].contiguous().pin_memory() for x in ("q", "k", "v"))
@@ -514,15 +571,17 @@ def run_sweep(args, w, layer, ws, rank, local, stream, peaks, gather, heads):
     for g, t, lo, hi in SWEEP:
         wp = w.replace(gamma=g, tau=t, min_budget=lo, max_budget=hi)
         p = ops.make_params(g, t, lo, hi, w.qa_mode, w.vs_mode)
+        whole = measure_prefill(layer, p, args, stream, ws, local, gather)
         m = measure(layer, p, args, stream, ws, local, gather)
-        value = tokens / (m["ms_step"] * 1e-3) if heads else job_value(tokens, ws, m["ms_step"])
+        ms = whole["ms_step"]
+        value = tokens / (ms * 1e-3) if heads else job_value(tokens, ws, ms)
         line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws,
-                "steps": args.steps, "warmup": args.warmup, "ms_per_step": m["ms_step"],
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
                 "higher_is_better": True, "scaling": "strong" if heads else "weak",
                 "sweep_point": {"gamma": g, "tau": t, "min_budget": lo, "max_budget": hi},
                 "dtype": "bf16", "data": "synthetic", "config": workload_config(wp, ws, heads)}
-        line.update(path_fields(layer, m, peaks, dense))
-        line["clocks"] = m["clocks"]
+        line.update(path_fields(layer, m, peaks, dense, whole))
+        line["clocks"] = whole["clocks"]
         if rank == 0:
             print(json.dumps(line), flush=True)
 

@@ -13,9 +13,14 @@
 //   last_pass1_kernel    per (head, key block): row max / sum of exp of the
 //                        last query block's logits (online-softmax partials)
 //   last_lse_kernel      combine partials -> log-sum-exp of each last-block row
+//   block_mass_kernel    the partials scaled by exp(max - lse), summed over the
+//                        rows: the pooled true distribution (true_last)
 //   last_pass2_kernel    per (head, key block): P = exp(logit - lse); column
-//                        sums (vert), block mass (true_last), diagonal partials
+//                        sums (vert) and diagonal partials
 //   slash_combine_kernel diagonal partials of neighbouring key blocks -> slash
+// The line sums (pass 2 and the slash combine) are read only by the
+// selection of vertical-slash heads, so the whole-path call runs them after
+// the pattern test, for those heads alone.
 #include <math.h>
 
 #include "fp_internal.cuh"
@@ -332,17 +337,42 @@ __global__ void last_lse_kernel(const float *__restrict__ pm, const float *__res
   lse[t] = mx + logf(s);
 }
 
+// grid (ceil(nb/8), Bt*Hq), 256 threads, one warp per key block j:
+// true_last[j] = (1/BS) sum over rows r of pl[j][r] * exp(pm[j][r] - lse[r]),
+// the rows summed in a fixed order (BS/32 per lane, then a xor tree).
+template <int BS>
+__global__ void __launch_bounds__(256) block_mass_kernel(const float *__restrict__ pm,
+                                                         const float *__restrict__ pl,
+                                                         const float *__restrict__ lse,
+                                                         float *__restrict__ true_last, int nb) {
+  const int j = blockIdx.x * 8 + threadIdx.x / 32, lane = threadIdx.x % 32;
+  if (j >= nb) return;
+  const size_t bh = blockIdx.y;
+  float s = 0.f;
+#pragma unroll
+  for (int k = 0; k < BS / 32; ++k) {
+    const int r = lane + 32 * k;
+    const size_t o = (bh * nb + j) * BS + r;
+    s = fmaf(pl[o], expf(pm[o] - lse[bh * BS + r]), s);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  if (lane == 0) true_last[bh * nb + j] = s / float(BS);
+}
+
+// grid (nb, Hq, Bt), 256 threads; with `vs_only` (a pattern array) heads
+// whose pattern is not vertical-slash are skipped.
 template <int BS, int D, class T>
 __global__ void __launch_bounds__(256) last_pass2_kernel(
     const T *__restrict__ q, const T *__restrict__ k, int hq, int g, int n, float scale,
-    const float *__restrict__ lse, float *__restrict__ vert, float *__restrict__ true_last,
-    float *__restrict__ sp) {
+    const float *__restrict__ lse, float *__restrict__ vert, float *__restrict__ sp,
+    const int32_t *__restrict__ vs_only) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   auto &sm = *reinterpret_cast<LastTile<BS, D, T> *>(smem_raw);
-  __shared__ float colsum[BS];
   const int j = blockIdx.x, h = blockIdx.y, b = blockIdx.z, nb = gridDim.x;
   const int kv = h / g, hkv = hq / g;
   const size_t bh = size_t(b) * hq + h;
+  if (vs_only && vs_only[bh] != FP_PATTERN_VS) return;
   const T *qlast = q + (bh * n + (n - BS)) * D;
   const T *kt = k + ((size_t(b) * hkv + kv) * n + size_t(j) * BS) * D;
   last_tile_scores<BS, D, T>(sm, qlast, kt, scale, j == nb - 1);
@@ -356,7 +386,6 @@ __global__ void __launch_bounds__(256) last_pass2_kernel(
     const int c = threadIdx.x;
     float s = 0.f;
     for (int r = 0; r < BS; ++r) s += sm.S[r][c];
-    colsum[c] = s;
     vert[bh * n + size_t(j) * BS + c] = s;
   }
   // diagonal partials: delta = r - c + BS - 1 in [0, 2BS-2]
@@ -368,21 +397,17 @@ __global__ void __launch_bounds__(256) last_pass2_kernel(
     for (int r = r0; r <= r1; ++r) s += sm.S[r][r - delta + BS - 1];
     sp[(bh * nb + j) * (2 * BS - 1) + delta] = s;
   }
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    float s = 0.f;
-    for (int c = 0; c < BS; ++c) s += colsum[c];
-    true_last[bh * nb + j] = s / float(BS);
-  }
 }
 
 // one thread per (b, h, o): slash[o] from the (at most two) key blocks whose
-// diagonal partials hold offset o.
+// diagonal partials hold offset o; with `vs_only`, vertical-slash heads only.
 __global__ void slash_combine_kernel(const float *__restrict__ sp, float *__restrict__ slash,
-                                     long long total, int n, int nb, int bs) {
+                                     long long total, int n, int nb, int bs,
+                                     const int32_t *__restrict__ vs_only) {
   const long long t = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (t >= total) return;
   const long long bh = t / n;
+  if (vs_only && vs_only[bh] != FP_PATTERN_VS) return;
   const int o = int(t % n);
   // tile j holds o at delta = o - n + (j + 2) * bs - 1, valid in [0, 2bs-2]
   int jlo = (n - o + 1 + bs - 1) / bs - 2;
@@ -397,30 +422,60 @@ __global__ void slash_combine_kernel(const float *__restrict__ sp, float *__rest
   slash[t] = s;
 }
 
-template <int BS, int D, class T>
-cudaError_t run_last(const Dims &Dm, const T *q, const T *k, float *true_last, float *vert,
-                     float *slash, void *ws, cudaStream_t st) {
+// CUDA-core workspace: pass-1 partials per (row, key block), the rows'
+// log-sum-exps and the diagonal partials.
+struct CoreWs {
+  float *pm, *pl, *lse, *sp;
+  size_t bytes;
+};
+CoreWs carve_core(const Dims &Dm, void *ws) {
   Carver c{static_cast<char *>(ws), 0};
   const size_t rows = size_t(Dm.bt) * Dm.hq;
-  float *pm = c.take<float>(rows * Dm.nb * BS);
-  float *pl = c.take<float>(rows * Dm.nb * BS);
-  float *lse = c.take<float>(rows * BS);
-  float *sp = c.take<float>(rows * Dm.nb * (2 * BS - 1));
+  CoreWs w;
+  w.pm = c.take<float>(rows * Dm.nb * Dm.bs);
+  w.pl = c.take<float>(rows * Dm.nb * Dm.bs);
+  w.lse = c.take<float>(rows * Dm.bs);
+  w.sp = c.take<float>(rows * Dm.nb * (2 * Dm.bs - 1));
+  w.bytes = c.off + 256;
+  return w;
+}
+
+// Pass 1, the log-sum-exps and true_last (every head).
+template <int BS, int D, class T>
+cudaError_t run_last_rows(const Dims &Dm, const T *q, const T *k, float *true_last, void *ws,
+                          cudaStream_t st) {
+  const CoreWs w = carve_core(Dm, ws);
+  const size_t rows = size_t(Dm.bt) * Dm.hq;
   const float scale = 1.f / sqrtf(float(D));
   const size_t smem = sizeof(LastTile<BS, D, T>);
   cudaFuncSetAttribute(last_pass1_kernel<BS, D, T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                        int(smem));
+  last_pass1_kernel<BS, D, T><<<dim3(Dm.nb, Dm.hq, Dm.bt), 256, smem, st>>>(q, k, Dm.hq, Dm.g,
+                                                                            Dm.n, scale, w.pm,
+                                                                            w.pl);
+  const int lrows = int(rows * BS);
+  last_lse_kernel<<<(lrows + 127) / 128, 128, 0, st>>>(w.pm, w.pl, w.lse, lrows, Dm.nb, BS);
+  block_mass_kernel<BS><<<dim3((Dm.nb + 7) / 8, unsigned(rows)), 256, 0, st>>>(
+      w.pm, w.pl, w.lse, true_last, Dm.nb);
+  return cudaGetLastError();
+}
+
+// Pass 2 and the slash combine (after run_last_rows on the same workspace);
+// with `vs_only`, vertical-slash heads only.
+template <int BS, int D, class T>
+cudaError_t run_last_lines(const Dims &Dm, const T *q, const T *k, float *vert, float *slash,
+                           const int32_t *vs_only, void *ws, cudaStream_t st) {
+  const CoreWs w = carve_core(Dm, ws);
+  const size_t rows = size_t(Dm.bt) * Dm.hq;
+  const float scale = 1.f / sqrtf(float(D));
+  const size_t smem = sizeof(LastTile<BS, D, T>);
   cudaFuncSetAttribute(last_pass2_kernel<BS, D, T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                        int(smem));
-  dim3 grid(Dm.nb, Dm.hq, Dm.bt);
-  last_pass1_kernel<BS, D, T><<<grid, 256, smem, st>>>(q, k, Dm.hq, Dm.g, Dm.n, scale, pm, pl);
-  const int lrows = int(rows * BS);
-  last_lse_kernel<<<(lrows + 127) / 128, 128, 0, st>>>(pm, pl, lse, lrows, Dm.nb, BS);
-  last_pass2_kernel<BS, D, T><<<grid, 256, smem, st>>>(q, k, Dm.hq, Dm.g, Dm.n, scale, lse, vert,
-                                                       true_last, sp);
+  last_pass2_kernel<BS, D, T><<<dim3(Dm.nb, Dm.hq, Dm.bt), 256, smem, st>>>(
+      q, k, Dm.hq, Dm.g, Dm.n, scale, w.lse, vert, w.sp, vs_only);
   const long long tot = (long long)rows * Dm.n;
-  slash_combine_kernel<<<unsigned((tot + 255) / 256), 256, 0, st>>>(sp, slash, tot, Dm.n, Dm.nb,
-                                                                    BS);
+  slash_combine_kernel<<<unsigned((tot + 255) / 256), 256, 0, st>>>(w.sp, slash, tot, Dm.n,
+                                                                    Dm.nb, BS, vs_only);
   return cudaGetLastError();
 }
 
@@ -440,27 +495,39 @@ cudaError_t run_map(const Dims &Dm, const T *q, float *qbar, const float *kbar, 
   return cudaGetLastError();
 }
 
-// The true last-block distribution, vertical and slash sums.
+// The true last-block distribution (every head).
 template <class T>
-cudaError_t run_true_last(const Dims &Dm, const T *q, const T *k, float *true_last,
-                          float *vert, float *slash, void *ws, cudaStream_t st) {
+cudaError_t run_true_last(const Dims &Dm, const T *q, const T *k, float *true_last, void *ws,
+                          cudaStream_t st) {
+  if (last_block_tc_supported(Dm)) return launch_last_block_rows_tc(Dm, q, k, true_last, ws, st);
+  if (Dm.bs == 128 && Dm.d == 128) return run_last_rows<128, 128, T>(Dm, q, k, true_last, ws, st);
+  if (Dm.bs == 128 && Dm.d == 64) return run_last_rows<128, 64, T>(Dm, q, k, true_last, ws, st);
+  if (Dm.bs == 64 && Dm.d == 128) return run_last_rows<64, 128, T>(Dm, q, k, true_last, ws, st);
+  return run_last_rows<64, 64, T>(Dm, q, k, true_last, ws, st);
+}
+
+// The vertical and slash sums (after run_true_last on the same workspace); with
+// `vs_only`, for the vertical-slash heads of that pattern array only.
+template <class T>
+cudaError_t run_lines(const Dims &Dm, const T *q, const T *k, float *vert, float *slash,
+                      const int32_t *vs_only, void *ws, cudaStream_t st) {
   if (last_block_tc_supported(Dm)) {
     float *sp = nullptr;
-    cudaError_t e = launch_last_block_tc(Dm, q, k, true_last, vert, &sp, ws, st);
+    cudaError_t e = launch_last_block_lines_tc(Dm, q, k, vert, vs_only, &sp, ws, st);
     if (e != cudaSuccess) return e;
     // the passes' partials are per 128-key tile, whatever the block size
     const long long tot = (long long)Dm.bt * Dm.hq * Dm.n;
     slash_combine_kernel<<<unsigned((tot + 255) / 256), 256, 0, st>>>(
-        sp, slash, tot, Dm.n, last_block_tc_tiles(Dm), 128);
+        sp, slash, tot, Dm.n, last_block_tc_tiles(Dm), 128, vs_only);
     return cudaGetLastError();
   }
   if (Dm.bs == 128 && Dm.d == 128)
-    return run_last<128, 128, T>(Dm, q, k, true_last, vert, slash, ws, st);
+    return run_last_lines<128, 128, T>(Dm, q, k, vert, slash, vs_only, ws, st);
   if (Dm.bs == 128 && Dm.d == 64)
-    return run_last<128, 64, T>(Dm, q, k, true_last, vert, slash, ws, st);
+    return run_last_lines<128, 64, T>(Dm, q, k, vert, slash, vs_only, ws, st);
   if (Dm.bs == 64 && Dm.d == 128)
-    return run_last<64, 128, T>(Dm, q, k, true_last, vert, slash, ws, st);
-  return run_last<64, 64, T>(Dm, q, k, true_last, vert, slash, ws, st);
+    return run_last_lines<64, 128, T>(Dm, q, k, vert, slash, vs_only, ws, st);
+  return run_last_lines<64, 64, T>(Dm, q, k, vert, slash, vs_only, ws, st);
 }
 
 template <class T>
@@ -471,16 +538,18 @@ cudaError_t run_estimate(const Dims &Dm, const T *q, const T *k, float *qbar, fl
                                                               0, nullptr);
   cudaError_t e = run_map<T>(Dm, q, qbar, kbar, map, est_last, nullptr, st);
   if (e != cudaSuccess) return e;
-  return run_true_last<T>(Dm, q, k, true_last, vert, slash, ws, st);
+  e = run_true_last<T>(Dm, q, k, true_last, ws, st);
+  if (e != cudaSuccess) return e;
+  return run_lines<T>(Dm, q, k, vert, slash, nullptr, ws, st);
 }
 
-// Pattern-aware first half: everything the pattern test reads, for every head
-// (K pooled, Q pooled over the last block only, the map's last row, the true
-// last-block distribution and the line sums), but not the rest of the map.
+// Pattern-aware first part: everything the pattern test reads, for every head
+// (K pooled, Q pooled over the last block only, the map's last row and the
+// true last-block distribution), and nothing else.
 template <class T>
 cudaError_t run_decision(const Dims &Dm, const T *q, const T *k, float *qbar, float *kbar,
-                         float *map, float *est_last, float *true_last, float *vert,
-                         float *slash, void *ws, cudaStream_t st) {
+                         float *map, float *est_last, float *true_last, void *ws,
+                         cudaStream_t st) {
   pool_kernel<T><<<dim3(Dm.nb, Dm.hkv, Dm.bt), 256, 0, st>>>(k, kbar, Dm.n, Dm.d, Dm.bs, Dm.nb,
                                                               0, nullptr);
   pool_kernel<T><<<dim3(1, Dm.hq, Dm.bt), 256, 0, st>>>(q, qbar, Dm.n, Dm.d, Dm.bs, Dm.nb,
@@ -490,32 +559,36 @@ cudaError_t run_decision(const Dims &Dm, const T *q, const T *k, float *qbar, fl
                                                            1.f / sqrtf(float(Dm.d)));
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  return run_true_last<T>(Dm, q, k, true_last, vert, slash, ws, st);
+  return run_true_last<T>(Dm, q, k, true_last, ws, st);
 }
 
 }  // namespace
 
 size_t estimate_ws_bytes(const Dims &D) {
   if (last_block_tc_supported(D)) return last_block_tc_ws_bytes(D);
-  Carver c{nullptr, 0};
-  const size_t rows = size_t(D.bt) * D.hq;
-  c.take<float>(rows * D.nb * D.bs);
-  c.take<float>(rows * D.nb * D.bs);
-  c.take<float>(rows * D.bs);
-  c.take<float>(rows * D.nb * (2 * D.bs - 1));
-  return c.off + 256;
+  return carve_core(D, nullptr).bytes;
 }
 
 cudaError_t launch_estimate_decision(const Dims &D, const void *q, const void *k, float *qbar,
                                      float *kbar, float *map, float *est_last,
-                                     float *true_last, float *vert, float *slash, void *ws,
-                                     cudaStream_t st) {
+                                     float *true_last, void *ws, cudaStream_t st) {
   if (D.dtype == FP_F32)
     return run_decision<float>(D, static_cast<const float *>(q), static_cast<const float *>(k),
-                               qbar, kbar, map, est_last, true_last, vert, slash, ws, st);
+                               qbar, kbar, map, est_last, true_last, ws, st);
   return run_decision<__nv_bfloat16>(D, static_cast<const __nv_bfloat16 *>(q),
                                      static_cast<const __nv_bfloat16 *>(k), qbar, kbar, map,
-                                     est_last, true_last, vert, slash, ws, st);
+                                     est_last, true_last, ws, st);
+}
+
+cudaError_t launch_estimate_lines_vs(const Dims &D, const void *q, const void *k, float *vert,
+                                     float *slash, const int32_t *pattern, void *ws,
+                                     cudaStream_t st) {
+  if (D.dtype == FP_F32)
+    return run_lines<float>(D, static_cast<const float *>(q), static_cast<const float *>(k),
+                            vert, slash, pattern, ws, st);
+  return run_lines<__nv_bfloat16>(D, static_cast<const __nv_bfloat16 *>(q),
+                                  static_cast<const __nv_bfloat16 *>(k), vert, slash, pattern,
+                                  ws, st);
 }
 
 cudaError_t launch_estimate_map_qa(const Dims &D, const void *q, float *qbar, const float *kbar,

@@ -9,14 +9,19 @@
 //
 // Pass 1 (row statistics): S = Q_last K^T per key tile, thread = query row
 //   (= TMEM lane); every CTA keeps an online max / sum of 2^(S*scale*log2e)
-//   per row over its chunk of key tiles and writes one partial per row.
-// Combine: partials -> log-sum-exp of every last-block row (log2 units).
-// Pass 2 (sums): S^T = K Q_last^T per key tile, thread = key (= TMEM lane),
-//   so P = 2^(S^T*scale*log2e - lse2[query]) is summed per thread into the
-//   vertical score of its key; the tile's mass goes to the pooled true
-//   distribution; diagonal (query - key) sums of the tile are formed by a
-//   register-systolic shuffle within each warp and combined across warps in
-//   a fixed order, giving the slash partials of the tile.
+//   per row over its chunk of key tiles and writes one partial per row, and
+//   for every tile the row's running max and the sums over the tile's two
+//   64-key halves against it.
+// Combine: partials -> log-sum-exp of every last-block row (log2 units); the
+//   tile partials scaled by 2^(max - lse) and summed over the rows give the
+//   pooled true distribution (no second pass needed for it).
+// Pass 2 (line sums): S^T = K Q_last^T per key tile, thread = key (= TMEM
+//   lane), so P = 2^(S^T*scale*log2e - lse2[query]) is summed per thread into
+//   the vertical score of its key; diagonal (query - key) sums of the tile
+//   are formed by a register-systolic shuffle within each warp and combined
+//   across warps in a fixed order, giving the slash partials of the tile.
+//   Only vertical-slash heads read the line sums, so the whole-path call runs
+//   this pass for those heads alone (after the pattern test).
 // Every reduction has a fixed order, so results are reproducible.
 //
 // CTA: one kv head, a pair of its query heads (A, B), a chunk of key tiles.
@@ -46,7 +51,6 @@ struct EstSmem {
   uint8_t ring[RING][TILE_BYTES];
   float lse2[2][BS];               // pass 2: per-query log2-sum-exp
   float bins[2][4][kWarpBins];     // pass 2: per-warp diagonal sums
-  float warp_mass[2][4];
   uint64_t q_full, ring_full[RING], ring_empty[RING], s_full[2], s_free[2];
   uint32_t tmem_base;
   int abort_flag;
@@ -66,14 +70,16 @@ __device__ __forceinline__ void wg_sync(int wg) {
 
 // nb counts 128-key tiles.  Block size 64 (QLO = 64) runs the same tiles: the
 // queries are the last 128 rows with the first QLO left out of every sum, and
-// each tile holds two output blocks (nb_out = 2 nb).  QLO is a template
-// parameter so that block size 128 carries no extra compare per element.
+// each tile holds two output blocks.  QLO is a template parameter so that
+// block size 128 carries no extra compare per element.  ptile [Bt,Hq,nb,3,128]
+// (pass 1): per tile and row the running max and the two halves' sums.
 template <int PASS, int QLO>
 __global__ void __launch_bounds__(kThreads, 1) last_block_tc_kernel(
     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-    int hq, int g, int n_tok, int nb, int nb_out, int n_chunks, float *__restrict__ pm,
-    float *__restrict__ pl, const float *__restrict__ lse2g, float *__restrict__ vert,
-    float *__restrict__ true_last, float *__restrict__ sp, int *status) {
+    int hq, int g, int n_tok, int nb, int n_chunks, float *__restrict__ pm,
+    float *__restrict__ pl, float *__restrict__ ptile, const float *__restrict__ lse2g,
+    float *__restrict__ vert, float *__restrict__ sp, const int32_t *__restrict__ vs_only,
+    int *status) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   EstSmem &sm = *reinterpret_cast<EstSmem *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -82,8 +88,16 @@ __global__ void __launch_bounds__(kThreads, 1) last_block_tc_kernel(
   const int pairs = (g + 1) / 2;
   const int chunk = blockIdx.x;
   const int kv = blockIdx.y / pairs, pair = blockIdx.y % pairs, b = blockIdx.z;
-  const int h0 = kv * g + 2 * pair;
-  const int nheads = (2 * pair + 1 < g) ? 2 : 1;
+  // the pair's query heads, or (pass 2 with vs_only) those of them whose
+  // pattern is vertical-slash; a CTA left with none returns at once
+  int hs[2] = {0, 0};
+  int nheads = 0;
+  for (int hh = 0; hh < 2; ++hh) {
+    const int h = kv * g + 2 * pair + hh;
+    if (2 * pair + hh < g && (!vs_only || vs_only[size_t(b) * hq + h] == FP_PATTERN_VS))
+      hs[nheads++] = h;
+  }
+  if (nheads == 0) return;
   const int j0 = chunk * kChunk;
   const int j1 = min(nb, j0 + kChunk);
   const int ntiles = j1 - j0;
@@ -103,7 +117,7 @@ __global__ void __launch_bounds__(kThreads, 1) last_block_tc_kernel(
   }
   if (PASS == 2 && threadIdx.x < 2 * BS) {
     const int hh = threadIdx.x / BS, r = threadIdx.x % BS;
-    sm.lse2[hh][r] = hh < nheads ? lse2g[(size_t(b) * hq + h0 + hh) * BS + r] : 0.f;
+    sm.lse2[hh][r] = hh < nheads ? lse2g[(size_t(b) * hq + hs[hh]) * BS + r] : 0.f;
   }
   if (warp == 9) {
     tmem_alloc(&sm.tmem_base, 512);
@@ -122,7 +136,7 @@ __global__ void __launch_bounds__(kThreads, 1) last_block_tc_kernel(
       prefetch_tmap(&tm_k);
       mbar_arrive_expect_tx(&sm.q_full, TILE_BYTES * nheads);
       for (int hh = 0; hh < nheads; ++hh) {
-        const int qrow = int((size_t(b) * hq + h0 + hh) * n_tok + (n_tok - BS));
+        const int qrow = int((size_t(b) * hq + hs[hh]) * n_tok + (n_tok - BS));
         tma_load_2d(sm.q[hh], &tm_q, &sm.q_full, 0, qrow);
         tma_load_2d(sm.q[hh] + HALF_BYTES, &tm_q, &sm.q_full, 64, qrow);
       }
@@ -190,7 +204,7 @@ __global__ void __launch_bounds__(kThreads, 1) last_block_tc_kernel(
     const uint32_t lane_base = tmem + (uint32_t(wq * 32) << 16) + uint32_t(hh * 256);
     const float sl2 = 1.4426950408889634f / sqrtf(float(HD));
     const bool active = hh < nheads;
-    const size_t bh = size_t(b) * hq + h0 + hh;
+    const size_t bh = size_t(b) * hq + (hh == 1 && active ? hs[1] : hs[0]);
     float m = -INFINITY, l = 0.f;  // pass 1
     bool ok = true;
     for (int t = 0; t < ntiles; ++t) {
@@ -226,12 +240,14 @@ __global__ void __launch_bounds__(kThreads, 1) last_block_tc_kernel(
           for (int c = 0; c < BS; ++c)
             if (c > r) x[c] = -INFINITY;
         }
-        // 8 independent chains for the max and the sum, then trees
-        float mx[8], sm8[8];
+        // 8 independent chains for the max and the sums (one set per 64-key
+        // half), then trees
+        float mx[8], sa[8], sb[8];
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
           mx[k] = x[k];
-          sm8[k] = 0.f;
+          sa[k] = 0.f;
+          sb[k] = 0.f;
         }
 #pragma unroll
         for (int c = 8; c < BS; ++c) mx[c % 8] = fmaxf(mx[c % 8], x[c]);
@@ -239,11 +255,18 @@ __global__ void __launch_bounds__(kThreads, 1) last_block_tc_kernel(
                                  fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
         const float mnew = fmaxf(m, tmax * sl2);
 #pragma unroll
-        for (int c = 0; c < BS; ++c) sm8[c % 8] += ex2(fmaf(x[c], sl2, -mnew));
-        const float s = ((sm8[0] + sm8[1]) + (sm8[2] + sm8[3])) +
-                        ((sm8[4] + sm8[5]) + (sm8[6] + sm8[7]));
-        l = l * ex2(m - mnew) + s;
+        for (int c = 0; c < BS / 2; ++c) sa[c % 8] += ex2(fmaf(x[c], sl2, -mnew));
+#pragma unroll
+        for (int c = BS / 2; c < BS; ++c) sb[c % 8] += ex2(fmaf(x[c], sl2, -mnew));
+        const float s0 = ((sa[0] + sa[1]) + (sa[2] + sa[3])) + ((sa[4] + sa[5]) + (sa[6] + sa[7]));
+        const float s1 = ((sb[0] + sb[1]) + (sb[2] + sb[3])) + ((sb[4] + sb[5]) + (sb[6] + sb[7]));
+        l = l * ex2(m - mnew) + (s0 + s1);
         m = mnew;
+        // this tile's mass for row r is (s0 + s1) * 2^(mnew - lse2[r])
+        float *pt = ptile + ((bh * nb + j) * 3) * BS + r;
+        pt[0] = mnew;
+        pt[BS] = s0;
+        pt[2 * BS] = s1;
       } else {
         // key r of the tile, query c of the last block: visible iff r <= c.
         // Diagonal sums (query - key) by register-systolic chains per warp:
@@ -295,22 +318,7 @@ __global__ void __launch_bounds__(kThreads, 1) last_block_tc_kernel(
         if (lane < 31) bins[BS + 30 - lane] = acc_b;        // diagonals 127 - lane
         const float v = (v4[0] + v4[1]) + (v4[2] + v4[3]);
         vert[bh * n_tok + size_t(j) * BS + r] = v;
-        // tile mass, fixed order: lanes (xor tree), then warps
-        float wsum = v;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) wsum += __shfl_xor_sync(0xffffffffu, wsum, o);
-        if (lane == 0) sm.warp_mass[hh][wq] = wsum;
-        wg_sync(hh);
-        if (r == 0) {
-          const float *wm = sm.warp_mass[hh];
-          if (QLO == 0) {
-            true_last[bh * nb_out + j] = (wm[0] + wm[1] + wm[2] + wm[3]) / float(BS);
-          } else {  // block 2j: keys 0-63 (warps 0, 1); block 2j + 1: keys 64-127
-            const float rows = float(BS - QLO);
-            true_last[bh * nb_out + 2 * j] = (wm[0] + wm[1]) / rows;
-            true_last[bh * nb_out + 2 * j + 1] = (wm[2] + wm[3]) / rows;
-          }
-        }
+        wg_sync(hh);  // every warp's diagonal bins are written
         // tile diagonal D = query - key in [-127, 127] -> partial index D + 127;
         // warp w holds D = (bin - 31) - 32 w
         float *dst = sp + (bh * nb + j) * size_t(kBins);
@@ -357,6 +365,43 @@ __global__ void lse2_combine_kernel(const float *__restrict__ pm, const float *_
   lse2[t] = mx + log2f(s);
 }
 
+// The pooled true distribution from pass 1's tile partials: grid (ceil(nt/8),
+// Bt*Hq), 256 threads, one warp per 128-key tile.  Row r's mass on the tile's
+// key half is s * 2^(m - lse2[r]); the rows' masses are summed in a fixed
+// order (4 per lane, then a xor tree) and averaged over the rows.  Block size
+// 64 (QLO = 64): rows below QLO are not in the last block, and each half is a
+// block of its own.
+template <int QLO>
+__global__ void __launch_bounds__(256) tile_mass_kernel(const float *__restrict__ ptile,
+                                                        const float *__restrict__ lse2,
+                                                        float *__restrict__ true_last, int nt) {
+  const int j = blockIdx.x * 8 + threadIdx.x / 32, lane = threadIdx.x % 32;
+  if (j >= nt) return;
+  const size_t bh = blockIdx.y;
+  const float *pt = ptile + (bh * nt + j) * 3 * BS;
+  float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+  for (int k = QLO / 32; k < BS / 32; ++k) {
+    const int r = lane + 32 * k;
+    const float f = ex2(pt[r] - lse2[bh * BS + r]);
+    s0 = fmaf(pt[BS + r], f, s0);
+    s1 = fmaf(pt[2 * BS + r], f, s1);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    s0 += __shfl_xor_sync(0xffffffffu, s0, o);
+    s1 += __shfl_xor_sync(0xffffffffu, s1, o);
+  }
+  if (lane == 0) {
+    if (QLO == 0) {
+      true_last[bh * nt + j] = (s0 + s1) / float(BS);
+    } else {
+      true_last[bh * 2 * nt + 2 * j] = s0 / float(BS - QLO);
+      true_last[bh * 2 * nt + 2 * j + 1] = s1 / float(BS - QLO);
+    }
+  }
+}
+
 bool encode_rows(CUtensorMap *map, const void *ptr, uint64_t rows) {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   if (!fn) {
@@ -387,54 +432,90 @@ bool last_block_tc_supported(const Dims &D) {
 // 128-key tiles of the passes (block size 64 runs two blocks per tile)
 int last_block_tc_tiles(const Dims &D) { return D.n / BS; }
 
-size_t last_block_tc_ws_bytes(const Dims &D) {
-  Carver c{nullptr, 0};
-  const size_t heads = size_t(D.bt) * D.hq;
-  const int nt = last_block_tc_tiles(D);
-  const int n_chunks = (nt + kChunk - 1) / kChunk;
-  c.take<float>(heads * n_chunks * BS);
-  c.take<float>(heads * n_chunks * BS);
-  c.take<float>(heads * BS);
-  c.take<float>(heads * nt * size_t(kBins));
-  return c.off + 256;
-}
+namespace {
 
-// Writes true_last and vert, and the diagonal partials sp [Bt,Hq,n/128,255]
-// of the 128-key tiles (combined into slash by the caller's slash_combine
-// step with block size 128).
-cudaError_t launch_last_block_tc(const Dims &D, const void *q, const void *k, float *true_last,
-                                 float *vert, float **sp_out, void *ws, cudaStream_t st) {
-  CUtensorMap mq, mk;
-  if (!encode_rows(&mq, q, uint64_t(D.bt) * D.hq * D.n) ||
-      !encode_rows(&mk, k, uint64_t(D.bt) * D.hkv * D.n))
-    return cudaErrorInvalidValue;
+struct TcWs {
+  float *pm, *pl, *lse2, *sp, *ptile;
+  size_t bytes;
+};
+
+TcWs carve_tc(const Dims &D, void *ws) {
   Carver c{static_cast<char *>(ws), 0};
   const size_t heads = size_t(D.bt) * D.hq;
   const int nt = last_block_tc_tiles(D);
-  const int q_lo = BS - D.bs;  // block 64: the last 128 rows minus the first 64
   const int n_chunks = (nt + kChunk - 1) / kChunk;
-  float *pm = c.take<float>(heads * n_chunks * BS);
-  float *pl = c.take<float>(heads * n_chunks * BS);
-  float *lse2 = c.take<float>(heads * BS);
-  float *sp = c.take<float>(heads * nt * size_t(kBins));
-  *sp_out = sp;
+  TcWs w;
+  w.pm = c.take<float>(heads * n_chunks * BS);
+  w.pl = c.take<float>(heads * n_chunks * BS);
+  w.lse2 = c.take<float>(heads * BS);
+  w.sp = c.take<float>(heads * nt * size_t(kBins));
+  w.ptile = c.take<float>(heads * nt * size_t(3 * BS));
+  w.bytes = c.off + 256;
+  return w;
+}
+
+bool encode_qk(const Dims &D, const void *q, const void *k, CUtensorMap *mq, CUtensorMap *mk) {
+  return encode_rows(mq, q, uint64_t(D.bt) * D.hq * D.n) &&
+         encode_rows(mk, k, uint64_t(D.bt) * D.hkv * D.n);
+}
+
+}  // namespace
+
+size_t last_block_tc_ws_bytes(const Dims &D) { return carve_tc(D, nullptr).bytes; }
+
+// Pass 1, the log-sum-exps and the pooled true distribution, for every head.
+cudaError_t launch_last_block_rows_tc(const Dims &D, const void *q, const void *k,
+                                      float *true_last, void *ws, cudaStream_t st) {
+  CUtensorMap mq, mk;
+  if (!encode_qk(D, q, k, &mq, &mk)) return cudaErrorInvalidValue;
+  const TcWs w = carve_tc(D, ws);
+  const size_t heads = size_t(D.bt) * D.hq;
+  const int nt = last_block_tc_tiles(D);
+  const int n_chunks = (nt + kChunk - 1) / kChunk;
   const dim3 grid(n_chunks, D.hkv * ((D.g + 1) / 2), D.bt);
   int *status = device_status_ptr();
   const int rows = int(heads * BS);
-  auto passes = [&](auto pass1, auto pass2) {
+  auto run = [&](auto pass1, auto mass) {
     cudaFuncSetAttribute(pass1, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmemBytes));
+    pass1<<<grid, kThreads, kSmemBytes, st>>>(mq, mk, D.hq, D.g, D.n, nt, n_chunks, w.pm, w.pl,
+                                              w.ptile, nullptr, nullptr, nullptr, nullptr,
+                                              status);
+    lse2_combine_kernel<<<(rows + 127) / 128, 128, 0, st>>>(w.pm, w.pl, w.lse2, rows, n_chunks);
+    mass<<<dim3((nt + 7) / 8, unsigned(heads)), 256, 0, st>>>(w.ptile, w.lse2, true_last, nt);
+  };
+  if (D.bs == BS)
+    run(last_block_tc_kernel<1, 0>, tile_mass_kernel<0>);
+  else  // block 64: the last 128 rows minus the first 64
+    run(last_block_tc_kernel<1, BS / 2>, tile_mass_kernel<BS / 2>);
+  return cudaGetLastError();
+}
+
+// Pass 2 (after launch_last_block_rows_tc on the same workspace): vert and
+// the diagonal partials sp [Bt,Hq,n/128,255] of the 128-key tiles (combined
+// into slash by the caller's slash_combine step with block size 128), for
+// every head, or with `vs_only` (a pattern array) for its vertical-slash
+// heads only.
+cudaError_t launch_last_block_lines_tc(const Dims &D, const void *q, const void *k, float *vert,
+                                       const int32_t *vs_only, float **sp_out, void *ws,
+                                       cudaStream_t st) {
+  CUtensorMap mq, mk;
+  if (!encode_qk(D, q, k, &mq, &mk)) return cudaErrorInvalidValue;
+  const TcWs w = carve_tc(D, ws);
+  *sp_out = w.sp;
+  const int nt = last_block_tc_tiles(D);
+  const int n_chunks = (nt + kChunk - 1) / kChunk;
+  const dim3 grid(n_chunks, D.hkv * ((D.g + 1) / 2), D.bt);
+  int *status = device_status_ptr();
+  auto run = [&](auto pass2) {
     cudaFuncSetAttribute(pass2, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmemBytes));
-    pass1<<<grid, kThreads, kSmemBytes, st>>>(mq, mk, D.hq, D.g, D.n, nt, D.nb, n_chunks, pm, pl,
-                                              nullptr, nullptr, nullptr, nullptr, status);
-    lse2_combine_kernel<<<(rows + 127) / 128, 128, 0, st>>>(pm, pl, lse2, rows, n_chunks);
-    pass2<<<grid, kThreads, kSmemBytes, st>>>(mq, mk, D.hq, D.g, D.n, nt, D.nb, n_chunks,
-                                              nullptr, nullptr, lse2, vert, true_last, sp,
+    pass2<<<grid, kThreads, kSmemBytes, st>>>(mq, mk, D.hq, D.g, D.n, nt, n_chunks, nullptr,
+                                              nullptr, nullptr, w.lse2, vert, w.sp, vs_only,
                                               status);
   };
-  if (q_lo == 0)
-    passes(last_block_tc_kernel<1, 0>, last_block_tc_kernel<2, 0>);
+  if (D.bs == BS)
+    run(last_block_tc_kernel<2, 0>);
   else
-    passes(last_block_tc_kernel<1, BS / 2>, last_block_tc_kernel<2, BS / 2>);
+    run(last_block_tc_kernel<2, BS / 2>);
   return cudaGetLastError();
 }
 

@@ -194,20 +194,24 @@ fp_status run_attn(const Dims &D, const void *q, const void *k, const void *v,
 }
 
 // The whole path, pattern-aware: the inputs of the pattern test first, for every
-// head; then Q pooling and the block map only for the query-aware heads (the
-// vertical-slash heads' selection never reads them).  Every value is bitwise
-// the one the separate fp_estimate / fp_pattern / fp_select calls produce.
-// `v_ready` (may be null): an event the attention stage waits for, the only
-// stage that reads v (the host path's copy of v in lands behind it).
+// head; then Q pooling and the block map only for the query-aware heads, and
+// the vertical / slash line sums only for the vertical-slash heads (each
+// head's selection reads one or the other).  Every value a head's selection
+// reads is bitwise the one the separate fp_estimate / fp_pattern / fp_select
+// calls produce.  `v_ready` (may be null): an event the attention stage waits
+// for, the only stage that reads v (the host path's copy of v in lands
+// behind it).
 fp_status run_prefill(const Dims &D, const fp_params &p, const void *q, const void *k,
                       const void *v, void *out, float *lse, int64_t *stats, const Prefill &P,
                       cudaStream_t st, cudaEvent_t v_ready = nullptr) {
   cudaError_t e = launch_estimate_decision(D, q, k, P.qbar, P.kbar, P.map, P.est_last,
-                                           P.true_last, P.vert, P.slash, P.stage_ws, st);
+                                           P.true_last, P.stage_ws, st);
   if (e != cudaSuccess) return FP_ERR_CUDA;
   e = launch_pattern(D, p.tau, P.est_last, P.true_last, P.djs, P.pattern, st);
   if (e != cudaSuccess) return FP_ERR_CUDA;
   e = launch_estimate_map_qa(D, q, P.qbar, P.kbar, P.map, P.est_last, P.pattern, st);
+  if (e != cudaSuccess) return FP_ERR_CUDA;
+  e = launch_estimate_lines_vs(D, q, k, P.vert, P.slash, P.pattern, P.stage_ws, st);
   if (e != cudaSuccess) return FP_ERR_CUDA;
   e = launch_select(D, p.gamma, budgets(D, p), P.pattern, P.map, P.vert, P.slash, P.counts,
                     P.indices, P.stage_ws, st);

@@ -44,25 +44,32 @@ size_t estimate_ws_bytes(const Dims &D);
 cudaError_t launch_estimate(const Dims &D, const void *q, const void *k, float *qbar,
                             float *kbar, float *map, float *est_last, float *true_last,
                             float *vert, float *slash, void *ws, cudaStream_t st);
-// Pattern-aware halves of launch_estimate (fp_prefill_attn): everything the
-// pattern test reads for every head (K pooled, Q pooled over the last block,
-// the map's last row, true_last, vert, slash) ...
+// Pattern-aware parts of launch_estimate (fp_prefill_attn): everything the
+// pattern test reads, for every head (K pooled, Q pooled over the last block,
+// the map's last row, true_last) ...
 cudaError_t launch_estimate_decision(const Dims &D, const void *q, const void *k, float *qbar,
                                      float *kbar, float *map, float *est_last,
-                                     float *true_last, float *vert, float *slash, void *ws,
-                                     cudaStream_t st);
-// ... and then Q pooling and the map for the query-aware heads of `pattern`.
+                                     float *true_last, void *ws, cudaStream_t st);
+// ... then Q pooling and the map for the query-aware heads of `pattern` ...
 cudaError_t launch_estimate_map_qa(const Dims &D, const void *q, float *qbar, const float *kbar,
                                    float *map, float *est_last, const int32_t *pattern,
                                    cudaStream_t st);
+// ... and vert and slash for its vertical-slash heads (on the workspace the
+// decision part left).
+cudaError_t launch_estimate_lines_vs(const Dims &D, const void *q, const void *k, float *vert,
+                                     float *slash, const int32_t *pattern, void *ws,
+                                     cudaStream_t st);
 
 // Tensor-core passes over the last query block (estimate_tc.cu): bf16,
 // block 128, head dim 128.
 bool last_block_tc_supported(const Dims &D);
 int last_block_tc_tiles(const Dims &D);
 size_t last_block_tc_ws_bytes(const Dims &D);
-cudaError_t launch_last_block_tc(const Dims &D, const void *q, const void *k, float *true_last,
-                                 float *vert, float **sp_out, void *ws, cudaStream_t st);
+cudaError_t launch_last_block_rows_tc(const Dims &D, const void *q, const void *k,
+                                      float *true_last, void *ws, cudaStream_t st);
+cudaError_t launch_last_block_lines_tc(const Dims &D, const void *q, const void *k, float *vert,
+                                       const int32_t *vs_only, float **sp_out, void *ws,
+                                       cudaStream_t st);
 
 cudaError_t launch_pattern(const Dims &D, float tau, const float *est_last,
                            const float *true_last, float *djs, int32_t *pattern,
