@@ -1,6 +1,7 @@
 """CPU oracle (test infrastructure only; see flexprefill.py's header)."""
 from .flexprefill import *  # noqa: F401,F403
 from .flexprefill import (PATTERN_QA, PATTERN_VS, QA_FLATTENED, QA_QUERYWISE,  # noqa: F401
+                          n_blocks_of,
                           VS_BLOCKS, VS_TOKENS, pool_lines, select_head_vs_blocks,
                           vs_block_budget,
                           block_pool, cumulative_count,

@@ -36,7 +36,11 @@ force; none is "parity unpinned".
 
 Layouts (all C-contiguous):
   q [Bt, Hq, N, d];  k, v [Bt, Hkv, N, d];  g = Hq // Hkv;  kv head of h = h // g
-  nb = N // B;  T = nb (nb + 1) / 2 (causal block pairs)
+  nb = ceil(N / B);  T = nb (nb + 1) / 2 (causal block pairs).  When B does not
+  divide N the last block is partial: it holds the N - (nb - 1) B tokens left
+  (reading of a sequence of any length: the pages define the method per
+  sequence and never tie N to B), and every block-level step uses that
+  block's real tokens only.
   map   [Bt, Hq, T]: row i of the block map stored at i(i+1)/2 .. i(i+1)/2 + i
   counts [Bt, Hq, nb] int32; indices [Bt, Hq, nb, nb] int32, first counts[...]
   entries of each row ascending, the rest unspecified.
@@ -76,15 +80,25 @@ def tri_offset(i: int) -> int:
 
 # ---------------------------------------------------------------- estimate --
 
+def n_blocks_of(n: int, block: int) -> int:
+    """ceil(N / B): the blocks of a sequence of N tokens (the last may be partial)."""
+    return -(-n // block)
+
+
 def block_pool(x, block: int) -> np.ndarray:
-    """Mean over each run of ``block`` tokens: [..., N, d] -> [..., N/B, d].
+    """Mean over each run of ``block`` tokens: [..., N, d] -> [..., nb, d].
 
     [approach] says the estimate is "block-pooled"; the operator is not
-    named.  Reading: arithmetic mean.
+    named.  Reading: arithmetic mean, over the real tokens of a partial last
+    block.
     """
     x = _f64(x)
     *lead, n, d = x.shape
-    return x.reshape(*lead, n // block, block, d).mean(axis=-2)
+    nb = n_blocks_of(n, block)
+    out = np.empty((*lead, nb, d))
+    for c in range(nb):
+        out[..., c, :] = x[..., c * block: min((c + 1) * block, n), :].mean(axis=-2)
+    return out
 
 
 def estimated_block_map(qbar: np.ndarray, kbar: np.ndarray, scale: float):
@@ -109,10 +123,11 @@ def estimated_block_map(qbar: np.ndarray, kbar: np.ndarray, scale: float):
 def last_block_attention(q_last: np.ndarray, k: np.ndarray, n_total: int, scale: float):
     """True causal attention probabilities of the last query block, one head.
 
-    q_last [B, d] holds the queries at positions N-B .. N-1; k [N, d].
-    Returns P [B, N] with P[r, t] = softmax over t <= N-B+r of scale*q.k, and
-    0 for t > N-B+r.  [approach] "the true distribution" of the last query
-    block ([ablations]: last, not middle, representative queries).
+    q_last [R, d] holds the queries at positions N-R .. N-1 (R = B, or the
+    partial last block's length); k [N, d].  Returns P [R, N] with P[r, t] =
+    softmax over t <= N-R+r of scale*q.k, and 0 for t > N-R+r.  [approach]
+    "the true distribution" of the last query block ([ablations]: last, not
+    middle, representative queries).
     """
     bsz = q_last.shape[0]
     logits = scale * (q_last @ k.T)
@@ -134,11 +149,12 @@ def estimate(q, k, block: int):
       est_last [Bt,Hq,nb]    last row of the map (the estimate a-hat)
       true_last [Bt,Hq,nb]   true pooled distribution a-bar of the last block:
                              P summed over the keys of each block and averaged
-                             over the B query rows (sums to 1).  Reading of
-                             "true distribution" [approach].
+                             over the last block's R query rows (sums to 1).
+                             Reading of "true distribution" [approach].
       vert [Bt,Hq,N]         column sums  vert[t]  = sum_r P[r, t]
-      slash [Bt,Hq,N]        diagonal sums slash[o] = sum_r P[r, N-B+r-o]
+      slash [Bt,Hq,N]        diagonal sums slash[o] = sum_r P[r, N-R+r-o]
                              (o = query position - key position >= 0)
+    R = B, or the partial last block's length when B does not divide N.
     vert and slash are the vertical and slash line scores of the
     vertical-slash pattern [approach], read off the same last-block P.
     """
@@ -146,7 +162,9 @@ def estimate(q, k, block: int):
     bt, hq, n, d = qf.shape
     hkv = kf.shape[1]
     g = hq // hkv
-    nb = n // block
+    nb = n_blocks_of(n, block)
+    q0 = (nb - 1) * block  # first query of the last block
+    rows = n - q0
     t_pairs = nb * (nb + 1) // 2
     scale = 1.0 / math.sqrt(d)
     qbar = block_pool(qf, block)
@@ -163,11 +181,12 @@ def estimate(q, k, block: int):
             for i in range(nb):
                 amap[b, h, tri_offset(i): tri_offset(i) + i + 1] = a[i, : i + 1]
             est_last[b, h] = a[nb - 1]
-            p = last_block_attention(qf[b, h, n - block:], kf[b, kv], n, scale)
-            true_last[b, h] = p.reshape(block, nb, block).sum(axis=2).sum(axis=0) / block
+            p = last_block_attention(qf[b, h, q0:], kf[b, kv], n, scale)
+            for j in range(nb):
+                true_last[b, h, j] = p[:, j * block: min((j + 1) * block, n)].sum() / rows
             vert[b, h] = p.sum(axis=0)
-            for r in range(block):
-                pos = n - block + r
+            for r in range(rows):
+                pos = q0 + r
                 # key t = pos - o for o = 0..pos
                 slash[b, h, : pos + 1] += p[r, pos::-1]
     return {"qbar": qbar, "kbar": kbar, "map": amap, "est_last": est_last,
@@ -464,7 +483,7 @@ def sparse_attention(q, k, v, counts, indices, block: int, heads=None, q_blocks=
     qf, kf, vf = _f64(q), _f64(k), _f64(v)
     bt, hq, n, d = qf.shape
     g = hq // kf.shape[1]
-    nb = n // block
+    nb = n_blocks_of(n, block)
     scale = 1.0 / math.sqrt(d)
     out = np.full((bt, hq, n, d), np.nan)
     lse = np.full((bt, hq, n), np.nan)
@@ -477,16 +496,18 @@ def sparse_attention(q, k, v, counts, indices, block: int, heads=None, q_blocks=
             kv = h // g
             for qi in qbs:
                 blocks = [int(j) for j in idx[b, h, qi, : cnt[b, h, qi]]]
-                keys = np.concatenate([np.arange(j * block, (j + 1) * block) for j in blocks])
-                qrows = qf[b, h, qi * block:(qi + 1) * block]
+                keys = np.concatenate([np.arange(j * block, min((j + 1) * block, n))
+                                       for j in blocks])
+                q1 = min((qi + 1) * block, n)  # (a partial last block ends at N)
+                qrows = qf[b, h, qi * block:q1]
                 logits = scale * (qrows @ kf[b, kv, keys].T)
-                qpos = np.arange(qi * block, (qi + 1) * block)
+                qpos = np.arange(qi * block, q1)
                 logits = np.where(keys[None, :] <= qpos[:, None], logits, -np.inf)
                 mx = logits.max(axis=1, keepdims=True)
                 e = np.exp(logits - mx)
                 s = e.sum(axis=1, keepdims=True)
-                out[b, h, qi * block:(qi + 1) * block] = (e / s) @ vf[b, kv, keys]
-                lse[b, h, qi * block:(qi + 1) * block] = (mx + np.log(s))[:, 0]
+                out[b, h, qi * block:q1] = (e / s) @ vf[b, kv, keys]
+                lse[b, h, qi * block:q1] = (mx + np.log(s))[:, 0]
     return out, lse
 
 
@@ -503,7 +524,7 @@ def dense_attention(q, k, v, block: int, heads=None, q_blocks=None):
     """Dense causal attention: sparse_attention over the full causal lists."""
     qf = _f64(q)
     bt, hq, n, _ = qf.shape
-    counts, indices = dense_lists(bt, hq, n // block)
+    counts, indices = dense_lists(bt, hq, n_blocks_of(n, block))
     return sparse_attention(qf, k, v, counts, indices, block, heads, q_blocks)
 
 
@@ -521,7 +542,7 @@ def flexprefill(q, k, v, block: int, gamma: float, tau: float, min_budget: int,
     e32 = {key: est[key].astype(np.float32) for key in ("map", "est_last", "true_last",
                                                          "vert", "slash")}
     djs, pat = pattern(e32["est_last"], e32["true_last"], tau)
-    nb = _f64(q).shape[2] // block
+    nb = n_blocks_of(_f64(q).shape[2], block)
     counts, indices = select(pat, e32["map"], e32["vert"], e32["slash"], nb, block, gamma,
                              min_budget, max_budget, qa_mode, vs_mode)
     res = dict(est)
