@@ -291,7 +291,7 @@ class Layer:
         self.q, self.k, self.v = q, k, v
         bt, hq, n, d = q.shape
         hkv = k.shape[1]
-        nb = n // bs
+        nb = -(-n // bs)
         self.bs, self.nb = bs, nb
         self.s = ops.make_shape(q, k, bs)
         f32 = dict(dtype=torch.float32, device=dev)

@@ -38,11 +38,15 @@ __global__ void __launch_bounds__(BS * 4) attn_f32_kernel(
   const size_t bh = size_t(b) * hq + h;
   const int r = threadIdx.x / 4, part = threadIdx.x % 4;
   const float scale = 1.f / sqrtf(float(D));
+  // a partial last block (N not a multiple of BS): rows and keys at or past
+  // N are not read or written (their keys come in as zeros, which the causal
+  // mask hides from every real row)
+  const bool row_ok = size_t(qi) * BS + r < size_t(n);
   const float *qrow = q + (bh * n + size_t(qi) * BS + r) * D;
   float qv[DP], acc[DP];
 #pragma unroll
   for (int i = 0; i < DP; ++i) {
-    qv[i] = qrow[part + 4 * i];
+    qv[i] = row_ok ? qrow[part + 4 * i] : 0.f;
     acc[i] = 0.f;
   }
   const float *kbase = k + (size_t(b) * hkv + kv) * n * D;
@@ -62,9 +66,11 @@ __global__ void __launch_bounds__(BS * 4) attn_f32_kernel(
     const float4 *vs = reinterpret_cast<const float4 *>(vbase + size_t(j) * BS * D);
     float4 *kd = reinterpret_cast<float4 *>(&sm.K[0][0]);
     float4 *vd = reinterpret_cast<float4 *>(&sm.V[0][0]);
+    const int keys = min(BS, n - j * BS);  // real keys of block j
     for (int e = threadIdx.x; e < BS * D / 4; e += BS * 4) {
-      kd[e] = ks[e];
-      vd[e] = vs[e];
+      const bool in = e / (D / 4) < keys;
+      kd[e] = in ? ks[e] : make_float4(0.f, 0.f, 0.f, 0.f);
+      vd[e] = in ? vs[e] : make_float4(0.f, 0.f, 0.f, 0.f);
     }
     __syncthreads();
     const bool diag = j == qi;
@@ -103,6 +109,7 @@ __global__ void __launch_bounds__(BS * 4) attn_f32_kernel(
     }
     m = mnew;
   }
+  if (!row_ok) return;
   float *orow = out + (bh * n + size_t(qi) * BS + r) * D;
   const float inv = l > 0.f ? 1.f / l : 0.f;
 #pragma unroll

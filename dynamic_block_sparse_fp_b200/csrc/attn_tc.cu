@@ -453,7 +453,9 @@ __global__ void __launch_bounds__(192, 2) attn_tc_kernel(
     const int half = PAIR ? r / 64 : 0;
     const int qh = PAIR ? qa + half : qa;
     const int rl = r - 64 * half;  // row inside its block
-    const bool row_exists = !PAIR || half == 0 || has_b;
+    // (a partial last block: rows at or past N are not read or written)
+    const bool row_exists =
+        (!PAIR || half == 0 || has_b) && size_t(qa) * KB + size_t(r) < size_t(n_tok);
     {
       // the first 64 d of this row's query -> TMEM (A operand of Q K^T);
       // 32-bit column c holds d 2c (low half) and 2c + 1

@@ -57,8 +57,9 @@ __device__ __forceinline__ void ld8(const __nv_bfloat16 *p, float (&x)[8]) {
 
 // ------------------------------------------------------------------ pooling --
 // grid (blocks, heads, Bt), 256 threads.  x [Bt, heads, N, d] -> out [Bt, heads,
-// nb, d], blocks blk0 .. blk0 + gridDim.x - 1.  With `qa_only` (a pattern
-// array, or null), heads whose pattern is not query-aware are skipped.
+// nb, d], blocks blk0 .. blk0 + gridDim.x - 1; a partial last block is the
+// mean of its real tokens.  With `qa_only` (a pattern array, or null), heads
+// whose pattern is not query-aware are skipped.
 template <class T>
 __global__ void __launch_bounds__(256) pool_kernel(const T *__restrict__ x, float *__restrict__ out,
                                                    int n, int d, int bs, int nb, int blk0,
@@ -71,8 +72,9 @@ __global__ void __launch_bounds__(256) pool_kernel(const T *__restrict__ x, floa
   const int rows_per_it = 256 / vec_per_row;
   const int tv = threadIdx.x % vec_per_row, tr = threadIdx.x / vec_per_row;
   const T *base = x + ((size_t(b) * heads + head) * n + size_t(blk) * bs) * d;
+  const int rows = min(bs, n - blk * bs);  // a partial last block: its real tokens
   float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-  for (int r = tr; r < bs; r += rows_per_it) {
+  for (int r = tr; r < rows; r += rows_per_it) {
     float v[8];
     ld8(base + size_t(r) * d + tv * 8, v);
 #pragma unroll
@@ -84,7 +86,7 @@ __global__ void __launch_bounds__(256) pool_kernel(const T *__restrict__ x, floa
   if (threadIdx.x < d) {
     float s = 0.f;
     for (int r = 0; r < rows_per_it; ++r) s += part[r][threadIdx.x];
-    out[((size_t(b) * heads + head) * nb + blk) * d + threadIdx.x] = s / float(bs);
+    out[((size_t(b) * heads + head) * nb + blk) * d + threadIdx.x] = s / float(rows);
   }
 }
 
@@ -246,9 +248,13 @@ struct LastTile {
   float S[BS][BS + 1];
 };
 
+// Rows of q_last at or past qrows and keys at or past krows (a partial last
+// block) are read as zeros; the causal mask hides such keys from every real
+// query row.
 template <int BS, int D, class T>
 __device__ void last_tile_scores(LastTile<BS, D, T> &sm, const T *__restrict__ qlast,
-                                 const T *__restrict__ ktile, float scale, bool diagonal) {
+                                 const T *__restrict__ ktile, float scale, bool diagonal,
+                                 int qrows, int krows) {
   constexpr int KC = LastTile<BS, D, T>::KC;
   constexpr int TPR = LastTile<BS, D, T>::TPR;
   const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
@@ -260,8 +266,8 @@ __device__ void last_tile_scores(LastTile<BS, D, T> &sm, const T *__restrict__ q
   for (int k0 = 0; k0 < D; k0 += KC) {
     for (int e = threadIdx.x; e < BS * KC; e += 256) {
       int r = e / KC, c = e % KC;
-      sm.A[c][r] = ld_f(qlast + size_t(r) * D + k0 + c);
-      sm.Bm[c][r] = ld_f(ktile + size_t(r) * D + k0 + c);
+      sm.A[c][r] = r < qrows ? ld_f(qlast + size_t(r) * D + k0 + c) : 0.f;
+      sm.Bm[c][r] = r < krows ? ld_f(ktile + size_t(r) * D + k0 + c) : 0.f;
     }
     __syncthreads();
 #pragma unroll 4
@@ -299,9 +305,10 @@ __global__ void __launch_bounds__(256) last_pass1_kernel(const T *__restrict__ q
   auto &sm = *reinterpret_cast<LastTile<BS, D, T> *>(smem_raw);
   const int j = blockIdx.x, h = blockIdx.y, b = blockIdx.z, nb = gridDim.x;
   const int kv = h / g, hkv = hq / g;
-  const T *qlast = q + ((size_t(b) * hq + h) * n + (n - BS)) * D;
+  const int q0 = (nb - 1) * BS;  // the last block's first query
+  const T *qlast = q + ((size_t(b) * hq + h) * n + q0) * D;
   const T *kt = k + ((size_t(b) * hkv + kv) * n + size_t(j) * BS) * D;
-  last_tile_scores<BS, D, T>(sm, qlast, kt, scale, j == nb - 1);
+  last_tile_scores<BS, D, T>(sm, qlast, kt, scale, j == nb - 1, n - q0, min(BS, n - j * BS));
   // 256 threads, BS rows: 256/BS threads per row
   constexpr int TPRW = 256 / BS;
   const int r = threadIdx.x / TPRW, part = threadIdx.x % TPRW;
@@ -338,13 +345,15 @@ __global__ void last_lse_kernel(const float *__restrict__ pm, const float *__res
 }
 
 // grid (ceil(nb/8), Bt*Hq), 256 threads, one warp per key block j:
-// true_last[j] = (1/BS) sum over rows r of pl[j][r] * exp(pm[j][r] - lse[r]),
-// the rows summed in a fixed order (BS/32 per lane, then a xor tree).
+// true_last[j] = (1/R) sum over the last block's R rows r of pl[j][r] *
+// exp(pm[j][r] - lse[r]), the rows summed in a fixed order (BS/32 per lane,
+// then a xor tree).
 template <int BS>
 __global__ void __launch_bounds__(256) block_mass_kernel(const float *__restrict__ pm,
                                                          const float *__restrict__ pl,
                                                          const float *__restrict__ lse,
-                                                         float *__restrict__ true_last, int nb) {
+                                                         float *__restrict__ true_last, int nb,
+                                                         int rows) {
   const int j = blockIdx.x * 8 + threadIdx.x / 32, lane = threadIdx.x % 32;
   if (j >= nb) return;
   const size_t bh = blockIdx.y;
@@ -353,11 +362,11 @@ __global__ void __launch_bounds__(256) block_mass_kernel(const float *__restrict
   for (int k = 0; k < BS / 32; ++k) {
     const int r = lane + 32 * k;
     const size_t o = (bh * nb + j) * BS + r;
-    s = fmaf(pl[o], expf(pm[o] - lse[bh * BS + r]), s);
+    if (r < rows) s = fmaf(pl[o], expf(pm[o] - lse[bh * BS + r]), s);
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-  if (lane == 0) true_last[bh * nb + j] = s / float(BS);
+  if (lane == 0) true_last[bh * nb + j] = s / float(rows);
 }
 
 // grid (nb, Hq, Bt), 256 threads; with `vs_only` (a pattern array) heads
@@ -373,16 +382,18 @@ __global__ void __launch_bounds__(256) last_pass2_kernel(
   const int kv = h / g, hkv = hq / g;
   const size_t bh = size_t(b) * hq + h;
   if (vs_only && vs_only[bh] != FP_PATTERN_VS) return;
-  const T *qlast = q + (bh * n + (n - BS)) * D;
+  const int q0 = (nb - 1) * BS, rows = n - q0;  // the last block's queries
+  const T *qlast = q + (bh * n + q0) * D;
   const T *kt = k + ((size_t(b) * hkv + kv) * n + size_t(j) * BS) * D;
-  last_tile_scores<BS, D, T>(sm, qlast, kt, scale, j == nb - 1);
+  const int keys = min(BS, n - j * BS);
+  last_tile_scores<BS, D, T>(sm, qlast, kt, scale, j == nb - 1, rows, keys);
   for (int e = threadIdx.x; e < BS * BS; e += 256) {
     int r = e / BS, c = e % BS;
     float s = sm.S[r][c];
-    sm.S[r][c] = (s == -INFINITY) ? 0.f : expf(s - lse[bh * BS + r]);
+    sm.S[r][c] = (s == -INFINITY || r >= rows) ? 0.f : expf(s - lse[bh * BS + r]);
   }
   __syncthreads();
-  if (threadIdx.x < BS) {
+  if (threadIdx.x < keys) {
     const int c = threadIdx.x;
     float s = 0.f;
     for (int r = 0; r < BS; ++r) s += sm.S[r][c];
@@ -400,23 +411,26 @@ __global__ void __launch_bounds__(256) last_pass2_kernel(
 }
 
 // one thread per (b, h, o): slash[o] from the (at most two) key blocks whose
-// diagonal partials hold offset o; with `vs_only`, vertical-slash heads only.
+// diagonal partials hold offset o (q0: the first query of the partials'
+// query rows); with `vs_only`, vertical-slash heads only.
 __global__ void slash_combine_kernel(const float *__restrict__ sp, float *__restrict__ slash,
-                                     long long total, int n, int nb, int bs,
+                                     long long total, int n, int q0, int nb, int bs,
                                      const int32_t *__restrict__ vs_only) {
   const long long t = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (t >= total) return;
   const long long bh = t / n;
   if (vs_only && vs_only[bh] != FP_PATTERN_VS) return;
   const int o = int(t % n);
-  // tile j holds o at delta = o - n + (j + 2) * bs - 1, valid in [0, 2bs-2]
-  int jlo = (n - o + 1 + bs - 1) / bs - 2;
-  if (jlo < 0) jlo = 0;
-  int jhi = (n - o - 1) / bs;
-  if (jhi > nb - 1) jhi = nb - 1;
+  // query row c (position q0 + c) and key r of tile j (position j bs + r) sit
+  // at delta = c - r + bs - 1 = (j + 1) bs - 1 - u with u = q0 - o, valid in
+  // [0, 2bs-2]: (j + 1) bs in [u + 1, u + 2bs - 1], i.e. j + 1 = m1 or m1 + 1
+  // with m1 = ceil((u + 1) / bs) (u + 2bs > 0 keeps the division positive)
+  const long long u = (long long)q0 - o;
+  const long long m1 = (u + 2ll * bs) / bs - 1;
   float s = 0.f;
-  for (int j = jlo; j <= jhi; ++j) {
-    int delta = o - n + (j + 2) * bs - 1;
+  for (long long j = m1 - 1; j <= m1; ++j) {  // ascending, a fixed order
+    if (j < 0 || j >= nb) continue;
+    const long long delta = (j + 1) * bs - 1 - u;
     if (delta >= 0 && delta <= 2 * bs - 2) s += sp[(bh * nb + j) * (2 * bs - 1) + delta];
   }
   slash[t] = s;
@@ -456,7 +470,7 @@ cudaError_t run_last_rows(const Dims &Dm, const T *q, const T *k, float *true_la
   const int lrows = int(rows * BS);
   last_lse_kernel<<<(lrows + 127) / 128, 128, 0, st>>>(w.pm, w.pl, w.lse, lrows, Dm.nb, BS);
   block_mass_kernel<BS><<<dim3((Dm.nb + 7) / 8, unsigned(rows)), 256, 0, st>>>(
-      w.pm, w.pl, w.lse, true_last, Dm.nb);
+      w.pm, w.pl, w.lse, true_last, Dm.nb, Dm.n - (Dm.nb - 1) * BS);
   return cudaGetLastError();
 }
 
@@ -474,8 +488,8 @@ cudaError_t run_last_lines(const Dims &Dm, const T *q, const T *k, float *vert, 
   last_pass2_kernel<BS, D, T><<<dim3(Dm.nb, Dm.hq, Dm.bt), 256, smem, st>>>(
       q, k, Dm.hq, Dm.g, Dm.n, scale, w.lse, vert, w.sp, vs_only);
   const long long tot = (long long)rows * Dm.n;
-  slash_combine_kernel<<<unsigned((tot + 255) / 256), 256, 0, st>>>(w.sp, slash, tot, Dm.n,
-                                                                    Dm.nb, BS, vs_only);
+  slash_combine_kernel<<<unsigned((tot + 255) / 256), 256, 0, st>>>(
+      w.sp, slash, tot, Dm.n, (Dm.nb - 1) * BS, Dm.nb, BS, vs_only);
   return cudaGetLastError();
 }
 
@@ -517,8 +531,9 @@ cudaError_t run_lines(const Dims &Dm, const T *q, const T *k, float *vert, float
     if (e != cudaSuccess) return e;
     // the passes' partials are per 128-key tile, whatever the block size
     const long long tot = (long long)Dm.bt * Dm.hq * Dm.n;
+    const int nt = last_block_tc_tiles(Dm);
     slash_combine_kernel<<<unsigned((tot + 255) / 256), 256, 0, st>>>(
-        sp, slash, tot, Dm.n, last_block_tc_tiles(Dm), 128, vs_only);
+        sp, slash, tot, Dm.n, (nt - 1) * 128, nt, 128, vs_only);
     return cudaGetLastError();
   }
   if (Dm.bs == 128 && Dm.d == 128)

@@ -68,15 +68,19 @@ __device__ __forceinline__ void wg_sync(int wg) {
   asm volatile("bar.sync %0, 128;" ::"r"(wg + 1) : "memory");
 }
 
-// nb counts 128-key tiles.  Block size 64 (QLO = 64) runs the same tiles: the
-// queries are the last 128 rows with the first QLO left out of every sum, and
-// each tile holds two output blocks.  QLO is a template parameter so that
-// block size 128 carries no extra compare per element.  ptile [Bt,Hq,nb,3,128]
-// (pass 1): per tile and row the running max and the two halves' sums.
-template <int PASS, int QLO>
+// nb counts 128-key tiles; the query rows are the 128 from q0 = (nb - 1) 128.
+// Block size 64 (QLO = 64) runs the same tiles: the queries are the last 128
+// rows with the first QLO left out of every sum, and each tile holds two
+// output blocks.  RAG (block 128, N not a multiple of 128): only the first
+// qrows = N - q0 query rows are the last block's, and keys at or past N (in
+// the last tile) are hidden from them by the causal mask.  QLO and RAG are
+// template parameters so that the common case carries no extra compare per
+// element.  ptile [Bt,Hq,nb,3,128] (pass 1): per tile and row the running max
+// and the two halves' sums.
+template <int PASS, int QLO, bool RAG>
 __global__ void __launch_bounds__(kThreads, 1) last_block_tc_kernel(
     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-    int hq, int g, int n_tok, int nb, int n_chunks, float *__restrict__ pm,
+    int hq, int g, int n_tok, int nb, int q0, int qrows, int n_chunks, float *__restrict__ pm,
     float *__restrict__ pl, float *__restrict__ ptile, const float *__restrict__ lse2g,
     float *__restrict__ vert, float *__restrict__ sp, const int32_t *__restrict__ vs_only,
     int *status) {
@@ -136,7 +140,7 @@ __global__ void __launch_bounds__(kThreads, 1) last_block_tc_kernel(
       prefetch_tmap(&tm_k);
       mbar_arrive_expect_tx(&sm.q_full, TILE_BYTES * nheads);
       for (int hh = 0; hh < nheads; ++hh) {
-        const int qrow = int((size_t(b) * hq + hs[hh]) * n_tok + (n_tok - BS));
+        const int qrow = int((size_t(b) * hq + hs[hh]) * n_tok + q0);
         tma_load_2d(sm.q[hh], &tm_q, &sm.q_full, 0, qrow);
         tma_load_2d(sm.q[hh] + HALF_BYTES, &tm_q, &sm.q_full, 64, qrow);
       }
@@ -298,10 +302,12 @@ __global__ void __launch_bounds__(kThreads, 1) last_block_tc_kernel(
             lqb[2] = lb.z;
             lqb[3] = lb.w;
           }
-          const float pa =
-              (c < QLO || (diag && r > c)) ? 0.f : ex2(fmaf(x[c], sl2, -lqa[c % 4]));
-          const float pb =
-              (cb < QLO || (diag && r > cb)) ? 0.f : ex2(fmaf(x[cb], sl2, -lqb[c % 4]));
+          const float pa = (c < QLO || (RAG && c >= qrows) || (diag && r > c))
+                               ? 0.f
+                               : ex2(fmaf(x[c], sl2, -lqa[c % 4]));
+          const float pb = (cb < QLO || (RAG && cb >= qrows) || (diag && r > cb))
+                               ? 0.f
+                               : ex2(fmaf(x[cb], sl2, -lqb[c % 4]));
           v4[c % 4] += pa;
           v4[c % 4] += pb;
           const float ua = __shfl_up_sync(0xffffffffu, acc_a, 1);
@@ -317,7 +323,7 @@ __global__ void __launch_bounds__(kThreads, 1) last_block_tc_kernel(
         if (lane < 31) bins[BS / 2 + 30 - lane] += acc_a;  // diagonal 63 - lane: columns < 64
         if (lane < 31) bins[BS + 30 - lane] = acc_b;        // diagonals 127 - lane
         const float v = (v4[0] + v4[1]) + (v4[2] + v4[3]);
-        vert[bh * n_tok + size_t(j) * BS + r] = v;
+        if (!RAG || size_t(j) * BS + r < size_t(n_tok)) vert[bh * n_tok + size_t(j) * BS + r] = v;
         wg_sync(hh);  // every warp's diagonal bins are written
         // tile diagonal D = query - key in [-127, 127] -> partial index D + 127;
         // warp w holds D = (bin - 31) - 32 w
@@ -368,13 +374,14 @@ __global__ void lse2_combine_kernel(const float *__restrict__ pm, const float *_
 // The pooled true distribution from pass 1's tile partials: grid (ceil(nt/8),
 // Bt*Hq), 256 threads, one warp per 128-key tile.  Row r's mass on the tile's
 // key half is s * 2^(m - lse2[r]); the rows' masses are summed in a fixed
-// order (4 per lane, then a xor tree) and averaged over the rows.  Block size
-// 64 (QLO = 64): rows below QLO are not in the last block, and each half is a
-// block of its own.
+// order (4 per lane, then a xor tree) and averaged over the last block's
+// rows (the first qrows).  Block size 64 (QLO = 64): rows below QLO are not
+// in the last block, and each half is a block of its own.
 template <int QLO>
 __global__ void __launch_bounds__(256) tile_mass_kernel(const float *__restrict__ ptile,
                                                         const float *__restrict__ lse2,
-                                                        float *__restrict__ true_last, int nt) {
+                                                        float *__restrict__ true_last, int nt,
+                                                        int qrows) {
   const int j = blockIdx.x * 8 + threadIdx.x / 32, lane = threadIdx.x % 32;
   if (j >= nt) return;
   const size_t bh = blockIdx.y;
@@ -383,6 +390,7 @@ __global__ void __launch_bounds__(256) tile_mass_kernel(const float *__restrict_
 #pragma unroll
   for (int k = QLO / 32; k < BS / 32; ++k) {
     const int r = lane + 32 * k;
+    if (r >= qrows) continue;  // (block 128, N not a multiple of 128)
     const float f = ex2(pt[r] - lse2[bh * BS + r]);
     s0 = fmaf(pt[BS + r], f, s0);
     s1 = fmaf(pt[2 * BS + r], f, s1);
@@ -394,7 +402,7 @@ __global__ void __launch_bounds__(256) tile_mass_kernel(const float *__restrict_
   }
   if (lane == 0) {
     if (QLO == 0) {
-      true_last[bh * nt + j] = (s0 + s1) / float(BS);
+      true_last[bh * nt + j] = (s0 + s1) / float(qrows);
     } else {
       true_last[bh * 2 * nt + 2 * j] = s0 / float(BS - QLO);
       true_last[bh * 2 * nt + 2 * j + 1] = s1 / float(BS - QLO);
@@ -429,8 +437,9 @@ bool last_block_tc_supported(const Dims &D) {
   return D.dtype == FP_BF16 && D.d == HD && (D.bs == BS || (D.bs == BS / 2 && D.n % BS == 0));
 }
 
-// 128-key tiles of the passes (block size 64 runs two blocks per tile)
-int last_block_tc_tiles(const Dims &D) { return D.n / BS; }
+// 128-key tiles of the passes (block size 64 runs two blocks per tile; a
+// partial last block of block size 128 is a partial last tile)
+int last_block_tc_tiles(const Dims &D) { return (D.n + BS - 1) / BS; }
 
 namespace {
 
@@ -475,18 +484,22 @@ cudaError_t launch_last_block_rows_tc(const Dims &D, const void *q, const void *
   const dim3 grid(n_chunks, D.hkv * ((D.g + 1) / 2), D.bt);
   int *status = device_status_ptr();
   const int rows = int(heads * BS);
+  const int q0 = (nt - 1) * BS, qrows = D.n - q0;
   auto run = [&](auto pass1, auto mass) {
     cudaFuncSetAttribute(pass1, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmemBytes));
-    pass1<<<grid, kThreads, kSmemBytes, st>>>(mq, mk, D.hq, D.g, D.n, nt, n_chunks, w.pm, w.pl,
-                                              w.ptile, nullptr, nullptr, nullptr, nullptr,
-                                              status);
+    pass1<<<grid, kThreads, kSmemBytes, st>>>(mq, mk, D.hq, D.g, D.n, nt, q0, qrows, n_chunks,
+                                              w.pm, w.pl, w.ptile, nullptr, nullptr, nullptr,
+                                              nullptr, status);
     lse2_combine_kernel<<<(rows + 127) / 128, 128, 0, st>>>(w.pm, w.pl, w.lse2, rows, n_chunks);
-    mass<<<dim3((nt + 7) / 8, unsigned(heads)), 256, 0, st>>>(w.ptile, w.lse2, true_last, nt);
+    mass<<<dim3((nt + 7) / 8, unsigned(heads)), 256, 0, st>>>(w.ptile, w.lse2, true_last, nt,
+                                                              qrows);
   };
-  if (D.bs == BS)
-    run(last_block_tc_kernel<1, 0>, tile_mass_kernel<0>);
+  if (D.bs == BS && qrows == BS)
+    run(last_block_tc_kernel<1, 0, false>, tile_mass_kernel<0>);
+  else if (D.bs == BS)  // N not a multiple of 128: a partial last block
+    run(last_block_tc_kernel<1, 0, true>, tile_mass_kernel<0>);
   else  // block 64: the last 128 rows minus the first 64
-    run(last_block_tc_kernel<1, BS / 2>, tile_mass_kernel<BS / 2>);
+    run(last_block_tc_kernel<1, BS / 2, false>, tile_mass_kernel<BS / 2>);
   return cudaGetLastError();
 }
 
@@ -506,16 +519,19 @@ cudaError_t launch_last_block_lines_tc(const Dims &D, const void *q, const void 
   const int n_chunks = (nt + kChunk - 1) / kChunk;
   const dim3 grid(n_chunks, D.hkv * ((D.g + 1) / 2), D.bt);
   int *status = device_status_ptr();
+  const int q0 = (nt - 1) * BS, qrows = D.n - q0;
   auto run = [&](auto pass2) {
     cudaFuncSetAttribute(pass2, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmemBytes));
-    pass2<<<grid, kThreads, kSmemBytes, st>>>(mq, mk, D.hq, D.g, D.n, nt, n_chunks, nullptr,
-                                              nullptr, nullptr, w.lse2, vert, w.sp, vs_only,
-                                              status);
+    pass2<<<grid, kThreads, kSmemBytes, st>>>(mq, mk, D.hq, D.g, D.n, nt, q0, qrows, n_chunks,
+                                              nullptr, nullptr, nullptr, w.lse2, vert, w.sp,
+                                              vs_only, status);
   };
-  if (D.bs == BS)
-    run(last_block_tc_kernel<2, 0>);
+  if (D.bs == BS && qrows == BS)
+    run(last_block_tc_kernel<2, 0, false>);
+  else if (D.bs == BS)
+    run(last_block_tc_kernel<2, 0, true>);
   else
-    run(last_block_tc_kernel<2, BS / 2>);
+    run(last_block_tc_kernel<2, BS / 2, false>);
   return cudaGetLastError();
 }
 

@@ -54,8 +54,8 @@ fp_status check_shape(const fp_shape *s, Dims *D) {
   if (s->n_q_heads % s->n_kv_heads != 0) return FP_ERR_SHAPE;
   if (s->block_size != 64 && s->block_size != 128) return FP_ERR_SHAPE;
   if (s->head_dim != 64 && s->head_dim != 128) return FP_ERR_SHAPE;
-  if (s->seq_len % s->block_size != 0) return FP_ERR_SHAPE;
-  const long long nb = s->seq_len / s->block_size;
+  // a partial last block holds the seq_len - (nb - 1) * block_size tokens left
+  const long long nb = (s->seq_len + s->block_size - 1) / s->block_size;
   if (nb > 4096) return FP_ERR_SHAPE;
   // row coordinates of every (batch, head, token) must fit in int32
   if ((long long)s->batch * s->n_q_heads * s->seq_len >= (1ll << 31)) return FP_ERR_SHAPE;
@@ -378,7 +378,7 @@ FP_API fp_status fp_prefill_attn_varlen(const fp_shape *shape, const fp_params *
   if (!q || !k || !v || !out || !seq_lens) return FP_ERR_NULL;
   if (n_seqs < 1) return FP_ERR_SHAPE;
   for (int i = 0; i < n_seqs; ++i)
-    if (seq_lens[i] <= 0 || seq_lens[i] > D.n || seq_lens[i] % D.bs != 0) return FP_ERR_SHAPE;
+    if (seq_lens[i] <= 0 || seq_lens[i] > D.n) return FP_ERR_SHAPE;
   Prefill Pmax;
   if ((s = check_ws(ws, ws_bytes, carve_prefill(D, nullptr, &Pmax))) != FP_OK) return s;
   if ((s = check_device()) != FP_OK) return s;

@@ -812,8 +812,9 @@ __global__ void __launch_bounds__(256) pool_lines_kernel(
   if (c >= nb || pattern[bh] == FP_PATTERN_QA) return;
   const float *v = vert + bh * n + size_t(c) * bs;
   const float *s = slash + bh * n + size_t(c) * bs;
+  const int len = min(bs, n - c * bs);  // a partial last block: its real lines
   double av = 0.0, as = 0.0;
-  for (int t = 0; t < bs; ++t) {
+  for (int t = 0; t < len; ++t) {
     av += (double)v[t];
     as += (double)s[t];
   }

@@ -252,7 +252,7 @@ def estimate(q, k, block_size: int, stream=None) -> dict:
     s = make_shape(q, k, block_size)
     dev = q.device
     bt, hq, n, d = q.shape
-    hkv, nb = k.shape[1], n // block_size
+    hkv, nb = k.shape[1], -(-n // block_size)  # a partial last block counts
     f = dict(dtype=torch.float32, device=dev)
     r = {"qbar": torch.empty(bt, hq, nb, d, **f), "kbar": torch.empty(bt, hkv, nb, d, **f),
          "map": torch.empty(bt, hq, nb * (nb + 1) // 2, **f),
@@ -276,7 +276,7 @@ def pattern(shape: fp_shape, params: fp_params, est_last, true_last, stream=None
 def select(shape: fp_shape, params: fp_params, pat, map_, vert, slash, stream=None):
     """fp_select: (counts int32 [Bt, Hq, nb], indices int32 [Bt, Hq, nb, nb]),
     each row's list ascending in its first counts entries."""
-    bt, hq, nb = shape.batch, shape.n_q_heads, shape.seq_len // shape.block_size
+    bt, hq, nb = shape.batch, shape.n_q_heads, -(-shape.seq_len // shape.block_size)
     dev = map_.device
     counts = torch.empty(bt, hq, nb, dtype=torch.int32, device=dev)
     indices = torch.empty(bt, hq, nb, nb, dtype=torch.int32, device=dev)

@@ -69,7 +69,7 @@ class Workload:
 
     @property
     def n_blocks(self) -> int:
-        return self.seq_len // self.block_size
+        return -(-self.seq_len // self.block_size)  # ceil: a partial last block counts
 
 
 WORKLOADS: dict[str, Workload] = {
@@ -147,7 +147,7 @@ def make_group(w: Workload, b: int, kv: int):
     """Q [g,N,d], K [N,d], V [N,d] (fp32, before the dtype cast) for one kv group."""
     g = w.n_q_heads // w.n_kv_heads
     n, d, bs = w.seq_len, w.head_dim, w.block_size
-    nb = n // bs
+    nb = -(-n // bs)  # a partial last block is planted like the others
     gen = torch.Generator().manual_seed(_group_seed(w, b, kv))
     q = torch.randn(g, n, d, generator=gen, dtype=torch.float32)
     k = torch.randn(n, d, generator=gen, dtype=torch.float32)

@@ -19,8 +19,12 @@
  *      q            [Bt, Hq,  N, d]   (fp_shape.dtype: bf16 or fp32)
  *      k, v         [Bt, Hkv, N, d]
  *      out          [Bt, Hq,  N, d]   (same dtype as q)
- *    with N = seq_len, d = head_dim, B = block_size, nb = N / B,
+ *    with N = seq_len, d = head_dim, B = block_size, nb = ceil(N / B),
  *    T = nb (nb + 1) / 2 and g = Hq / Hkv; query head h reads kv head h / g.
+ *    When B does not divide N the last block is partial: it holds the
+ *    N - (nb - 1) B tokens left, is pooled over those tokens, is the last
+ *    query block of the estimate (its queries are the representative ones),
+ *    and attention reads no key or query position at or past N.
  *  * Every data pointer is DEVICE memory owned by the caller, except the
  *    *_host pointers of fp_prefill_attn_host.  The library allocates no
  *    device memory; scratch space is the caller's workspace (`ws`, at least
@@ -35,9 +39,10 @@
  *    fp_last_device_status().
  *  * No C++ exception crosses this ABI.  Calls on distinct streams with
  *    distinct workspaces may run from several host threads.
- *  * Supported shapes: N % B == 0, Hq % Hkv == 0, B in {64, 128},
- *    d in {64, 128}.  The bf16 attention (tensor cores) needs d == 128;
- *    fp32 (the debug path, CUDA cores) takes every listed shape.
+ *  * Supported shapes: N >= 1 (any length), nb <= 4096, Hq % Hkv == 0,
+ *    B in {64, 128}, d in {64, 128}.  The bf16 attention (tensor cores)
+ *    needs d == 128; fp32 (the debug path, CUDA cores) takes every listed
+ *    shape.
  */
 #ifndef FP_H_
 #define FP_H_
@@ -143,10 +148,11 @@ size_t fp_workspace_size(const fp_shape *shape, int which_call);
  *             qbar[i].kbar[j] / sqrt(d)
  *   est_last  [Bt,Hq,nb]    fp32  the last row of map (the estimate a-hat)
  *   true_last [Bt,Hq,nb]    fp32  true attention of the last query block,
- *             summed over the keys of each block and averaged over its B rows
- *   vert      [Bt,Hq,N]     fp32  vert[t]  = sum over the last B queries of P[r,t]
- *   slash     [Bt,Hq,N]     fp32  slash[o] = sum over r of P[r, N-B+r-o]
- * where P is the causal softmax of q.k/sqrt(d) for the last B queries.
+ *             summed over the keys of each block and averaged over its R rows
+ *   vert      [Bt,Hq,N]     fp32  vert[t]  = sum over the last R queries of P[r,t]
+ *   slash     [Bt,Hq,N]     fp32  slash[o] = sum over r of P[r, N-R+r-o]
+ * where P is the causal softmax of q.k/sqrt(d) for the last block's R
+ * queries (R = B, or the partial last block's length).
  * Workspace: fp_workspace_size(shape, FP_CALL_ESTIMATE).
  */
 fp_status fp_estimate(const fp_shape *shape, const void *q, const void *k,
@@ -276,8 +282,7 @@ fp_status fp_prefill_attn(const fp_shape *shape, const fp_params *params,
  *   shape     batch must be 1 and seq_len the longest allowed length N_max;
  *             the other fields as for fp_prefill_attn
  *   n_seqs    number of sequences, >= 1
- *   seq_lens  HOST int32[n_seqs]: N_s, each a positive multiple of
- *             block_size and <= N_max
+ *   seq_lens  HOST int32[n_seqs]: N_s, each in 1 .. N_max (any length)
  *   q, out    the sequences' [Hq, N_s, d] tensors back to back (sequence s
  *             starts Hq * d * (N_0 + ... + N_{s-1}) elements in);
  *   k, v      likewise [Hkv, N_s, d]

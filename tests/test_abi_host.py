@@ -51,7 +51,7 @@ def test_workspace_sizes(L):
     host = ops.fp_workspace_size(s, ops.FP_CALL_PREFILL_HOST)
     io = (2 * 4 + 2 * 2) * 1024 * 128 * 2  # q, out (4 heads) + k, v (2 heads), bf16
     assert host >= pre + io
-    assert ops.fp_workspace_size(shape(seq_len=1000), ops.FP_CALL_PREFILL) == 0
+    assert ops.fp_workspace_size(shape(seq_len=0), ops.FP_CALL_PREFILL) == 0
     assert ops.fp_workspace_size(s, 17) == 0
     # larger problems need more
     assert ops.fp_workspace_size(shape(seq_len=4096), ops.FP_CALL_ESTIMATE) > \
@@ -59,7 +59,7 @@ def test_workspace_sizes(L):
 
 
 @pytest.mark.parametrize("bad,code", [
-    (dict(seq_len=1000), 2), (dict(block_size=32), 2), (dict(head_dim=96), 2),
+    (dict(seq_len=0), 2), (dict(block_size=32), 2), (dict(head_dim=96), 2),
     (dict(n_q_heads=3), 2), (dict(n_kv_heads=0), 2), (dict(dtype=7), 3),
     (dict(seq_len=128 * 4097), 2),
 ])
@@ -119,8 +119,8 @@ def test_bad_vs_mode_rejected(L, vs_mode):
 
 
 @pytest.mark.parametrize("lens,batch,code", [
-    ([1024, 1000], 1, "FP_ERR_SHAPE"),   # not a multiple of the block size
     ([1024, 0], 1, "FP_ERR_SHAPE"),      # empty sequence
+    ([1024, -3], 1, "FP_ERR_SHAPE"),     # negative length
     ([2048], 1, "FP_ERR_SHAPE"),         # longer than shape.seq_len (1024)
     ([], 1, "FP_ERR_SHAPE"),             # no sequence
     ([1024], 2, "FP_ERR_SHAPE"),         # the shape's batch must be 1
@@ -175,3 +175,18 @@ def test_missing_library_fails_loudly(monkeypatch):
     monkeypatch.setenv("FP_LIBRARY", "/nonexistent/libfp.so")
     with pytest.raises(RuntimeError, match="no fallback"):
         ops.lib()
+
+
+@pytest.mark.parametrize("n,bs", [(1000, 128), (1105, 64), (1, 64), (8256, 128)])
+def test_ragged_lengths_accepted(L, n, bs):
+    """N need not be a multiple of the block size: nb = ceil(N / B), the last
+    block partial.  Validation passes (a NULL pointer is what fails here) and
+    the workspaces are sized for nb blocks."""
+    s = shape(seq_len=n, block_size=bs)
+    assert L.fp_estimate(ctypes.byref(s), FAKE, None, *([FAKE] * 7), FAKE, 1 << 40,
+                         None) == ops.STATUS_CODES["FP_ERR_NULL"]
+    for call in (ops.FP_CALL_ESTIMATE, ops.FP_CALL_SELECT, ops.FP_CALL_PREFILL):
+        assert ops.fp_workspace_size(s, call) > 0
+    whole = shape(seq_len=-(-n // bs) * bs, block_size=bs)
+    assert ops.fp_workspace_size(s, ops.FP_CALL_SELECT) == ops.fp_workspace_size(
+        whole, ops.FP_CALL_SELECT)
