@@ -410,17 +410,18 @@ __global__ void __launch_bounds__(256) last_pass2_kernel(
   }
 }
 
-// one thread per (b, h, o): slash[o] from the (at most two) key blocks whose
-// diagonal partials hold offset o (q0: the first query of the partials'
-// query rows); with `vs_only`, vertical-slash heads only.
+// grid (ceil(n/256), Bt*Hq), one thread per (b, h, o): slash[o] from the (at
+// most two) key blocks whose diagonal partials hold offset o (q0: the first
+// query of the partials' query rows); with `vs_only`, vertical-slash heads
+// only.
 __global__ void slash_combine_kernel(const float *__restrict__ sp, float *__restrict__ slash,
-                                     long long total, int n, int q0, int nb, int bs,
+                                     int n, int q0, int nb, int bs,
                                      const int32_t *__restrict__ vs_only) {
-  const long long t = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  if (t >= total) return;
-  const long long bh = t / n;
+  const size_t bh = blockIdx.y;  // (a head whose pattern skips the lines exits at once)
   if (vs_only && vs_only[bh] != FP_PATTERN_VS) return;
-  const int o = int(t % n);
+  const int o = blockIdx.x * blockDim.x + threadIdx.x;
+  if (o >= n) return;
+  const size_t t = bh * n + o;
   // query row c (position q0 + c) and key r of tile j (position j bs + r) sit
   // at delta = c - r + bs - 1 = (j + 1) bs - 1 - u with u = q0 - o, valid in
   // [0, 2bs-2]: (j + 1) bs in [u + 1, u + 2bs - 1], i.e. j + 1 = m1 or m1 + 1
@@ -487,9 +488,8 @@ cudaError_t run_last_lines(const Dims &Dm, const T *q, const T *k, float *vert, 
                        int(smem));
   last_pass2_kernel<BS, D, T><<<dim3(Dm.nb, Dm.hq, Dm.bt), 256, smem, st>>>(
       q, k, Dm.hq, Dm.g, Dm.n, scale, w.lse, vert, w.sp, vs_only);
-  const long long tot = (long long)rows * Dm.n;
-  slash_combine_kernel<<<unsigned((tot + 255) / 256), 256, 0, st>>>(
-      w.sp, slash, tot, Dm.n, (Dm.nb - 1) * BS, Dm.nb, BS, vs_only);
+  slash_combine_kernel<<<dim3((Dm.n + 255) / 256, unsigned(rows)), 256, 0, st>>>(
+      w.sp, slash, Dm.n, (Dm.nb - 1) * BS, Dm.nb, BS, vs_only);
   return cudaGetLastError();
 }
 
@@ -530,10 +530,9 @@ cudaError_t run_lines(const Dims &Dm, const T *q, const T *k, float *vert, float
     cudaError_t e = launch_last_block_lines_tc(Dm, q, k, vert, vs_only, &sp, ws, st);
     if (e != cudaSuccess) return e;
     // the passes' partials are per 128-key tile, whatever the block size
-    const long long tot = (long long)Dm.bt * Dm.hq * Dm.n;
     const int nt = last_block_tc_tiles(Dm);
-    slash_combine_kernel<<<unsigned((tot + 255) / 256), 256, 0, st>>>(
-        sp, slash, tot, Dm.n, (nt - 1) * 128, nt, 128, vs_only);
+    slash_combine_kernel<<<dim3((Dm.n + 255) / 256, unsigned(Dm.bt * Dm.hq)), 256, 0, st>>>(
+        sp, slash, Dm.n, (nt - 1) * 128, nt, 128, vs_only);
     return cudaGetLastError();
   }
   if (Dm.bs == 128 && Dm.d == 128)

@@ -470,6 +470,11 @@ def test_prefill_pattern_aware_mixed_heads_bitwise(name, n):
     torch.cuda.synchronize()
     assert torch.equal(out2, out)
     assert int(stats[0]) == int(counts.sum()) and int(stats[1]) == n_qa
+    # the whole-path call's kept blocks against the oracle's rule on the same scores
+    oc, _ = oracle.select(pat.cpu().numpy(), _np(est["map"]), _np(est["vert"]),
+                          _np(est["slash"]), w.n_blocks, w.block_size, w.gamma, w.min_budget,
+                          w.max_budget)
+    assert int(stats[0]) == int(oc.sum())
 
 
 def test_varlen_batch_matches_separate_calls():
@@ -703,6 +708,22 @@ def test_full_size_128k_vs_capped_sampled():
     min budget 2048 and max budget 8192 tokens."""
     _full_size_sampled("llama8b_n131072", heads=[2, 17], q_blocks=[1, 640, 1023], rows_every=61,
                        tau=0.0, gamma=0.9, min_budget=2048, max_budget=8192)
+
+
+def test_full_size_128k_qa_capped_sampled():
+    """The 128k sweep's sparse regime with query-aware heads: gamma = 0.9,
+    tau = 0.1 (every head query-aware on this data), min budget 1024 and max
+    budget 8192 tokens (12.6 % of the causal blocks kept); the whole-path
+    call's output is bitwise the staged calls'."""
+    res = _full_size_sampled("llama8b_n131072", heads=[0, 21], q_blocks=[0, 511, 1023],
+                             rows_every=53, tau=0.1, gamma=0.9, min_budget=1024,
+                             max_budget=8192)
+    assert int((res["pattern"] == ops.FP_PATTERN_QA).sum()) > 0
+    w, _, d = _inputs("llama8b_n131072")
+    out, _, stats = ops.prefill_attn(d["q"], d["k"], d["v"], w.block_size, res["params"])
+    torch.cuda.synchronize()
+    assert torch.equal(out, res["out"])
+    assert int(stats[0]) == int(res["counts"].sum())
 
 
 def test_maximum_block_count_sampled():
