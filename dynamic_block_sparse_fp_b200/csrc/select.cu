@@ -26,9 +26,9 @@
 // Query-wise rule for query-aware heads ("Measured effects": query-wise index
 // selection instead of the flattened map): the same rule on each row
 // A[i, 0..i] of the map with the row's own total and per-row budgets.
-// select_rows_qa_kernel gives each (row, head) one CTA, which sorts the row's
-// (bit pattern, index) keys in shared memory, finds k by an exact uint64
-// prefix sum of the masses, and writes the row's list itself.
+// select_rows_qa_kernel gives each (row, head) one warp, which runs the same
+// radix select on the row (four digits, warp-private histograms, warp-scan
+// decisions) and writes the row's list itself.
 //
 // Block-pooled lines for vertical-slash heads (FP_VS_BLOCKS): pool_lines_kernel
 // sums vert per key block and slash per block distance into nb-entry lists,
@@ -822,123 +822,210 @@ __global__ void __launch_bounds__(256) pool_lines_kernel(
   ps[bh * nb + c] = __double2float_rn(as);
 }
 
-// Query-wise rule: grid (nb, Hq, Bt), kRowThreads threads, dynamic shared
-// memory for P = (smallest power of two >= nb) 64-bit keys and P flags.
-// Query-aware heads only (others return at once); row qi of head bh:
-//   key_j = (bit pattern of score j) << 32 | (0xFFFFFFFF - j), so a descending
-//   sort is the rule's order (score descending, then j ascending), with the
-//   padding keys (0) last;
-//   k_gamma = smallest k whose exact uint64 mass prefix reaches
-//   (double)gamma * (double)W; k = clamp(k_gamma, lo, hi) with the row's
-//   budgets; the row keeps the first k sorted entries and its diagonal.
-constexpr int kRowThreads = 256;
+// Query-wise rule: grid (ceil(nb / kRowWarps), Hq, Bt), kRowWarps warps; warp
+// w selects row qi = blockIdx.x * kRowWarps + w of a query-aware head (others
+// return at once).  The row A[qi, 0..qi] takes the same radix select as the
+// flattened lists, on four digits of its scores' bit patterns (bits 30..23,
+// 22..15, 14..7, 6..0), with a warp-private shared histogram per digit and
+// the decisions (by mass, or by count once the row's budget clamp decides k)
+// taken by the whole warp from warp scans; then the tie rank by an ordered
+// count, and the row's ascending list with its diagonal.  Integer sums, so
+// the result does not depend on thread order.
+constexpr int kRowWarps = 8;
+constexpr int kRowLevels = 4;  // digits: bits 30..23, 22..15, 14..7, 6..0
 
-__global__ void __launch_bounds__(kRowThreads) select_rows_qa_kernel(
-    const int32_t *__restrict__ pattern, const float *__restrict__ map, int nb, int pmax,
-    float gamma, int row_lo, int row_hi, int32_t *__restrict__ counts,
-    int32_t *__restrict__ indices) {
-  extern __shared__ __align__(16) unsigned char smem_raw[];
-  unsigned long long *keys = reinterpret_cast<unsigned long long *>(smem_raw);
-  uint8_t *flag = smem_raw + size_t(pmax) * 8;
-  __shared__ unsigned long long part[kRowThreads];
-  __shared__ int kmin;
-  __shared__ int wcount[kRowThreads / 32];
-  const int qi = blockIdx.x, tid = threadIdx.x;
-  const size_t bh = size_t(blockIdx.z) * gridDim.y + blockIdx.y;
-  if (pattern[bh] != FP_PATTERN_QA) return;
-  const int n = qi + 1;
-  int P = 1;
-  while (P < n) P <<= 1;
-  const float *mrow = map + bh * (size_t(nb) * (nb + 1) / 2) + size_t(qi) * (qi + 1) / 2;
-  for (int i = tid; i < P; i += kRowThreads) {
-    keys[i] = i < n ? ((unsigned long long)score_bits(mrow[i]) << 32) | (0xFFFFFFFFu - uint32_t(i))
-                    : 0ull;
-    flag[i] = 0;
+struct RowHist {
+  unsigned lo[256], hi[256], cnt[256];  // mass as its low 16 bits and the rest
+};
+
+// Warp-inclusive scan of a 64-bit value (lane order).
+__device__ __forceinline__ unsigned long long warp_incl_scan(unsigned long long x, int lane) {
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const unsigned long long y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
   }
-  if (tid == 0) kmin = n;
-  __syncthreads();
-  // bitonic sort, descending
-  for (int k = 2; k <= P; k <<= 1)
-    for (int j = k >> 1; j > 0; j >>= 1) {
-      for (int i = tid; i < P; i += kRowThreads) {
-        const int ixj = i ^ j;
-        if (ixj > i) {
-          const unsigned long long x = keys[i], y = keys[ixj];
-          const bool desc = (i & k) == 0;
-          if (desc ? (x < y) : (x > y)) {
-            keys[i] = y;
-            keys[ixj] = x;
-          }
-        }
-      }
-      __syncthreads();
-    }
-  // exact mass prefix: thread t owns sorted entries [t*per, (t+1)*per)
-  const int per = (n + kRowThreads - 1) / kRowThreads;
-  const int e0 = min(n, tid * per), e1 = min(n, e0 + per);
-  unsigned long long loc = 0;
-  for (int e = e0; e < e1; ++e) loc += score_mass(uint32_t(keys[e] >> 32));
-  part[tid] = loc;
-  __syncthreads();
-  // inclusive scan of the thread sums (fixed order)
-  for (int off = 1; off < kRowThreads; off <<= 1) {
-    const unsigned long long v = tid >= off ? part[tid - off] : 0ull;
-    __syncthreads();
-    part[tid] += v;
-    __syncthreads();
-  }
-  const unsigned long long total = part[kRowThreads - 1];
-  int kg;
-  if (gamma >= 1.f) {
-    kg = n;
-  } else {
-    const double target = (double)gamma * (double)total;
-    if (target <= 0.0) {
-      kg = 0;
-    } else {
-      unsigned long long cum = tid > 0 ? part[tid - 1] : 0ull;
-      for (int e = e0; e < e1; ++e) {
-        cum += score_mass(uint32_t(keys[e] >> 32));
-        if ((double)cum >= target) {
-          atomicMin(&kmin, e + 1);
-          break;
-        }
-      }
-      __syncthreads();
-      kg = kmin;
-    }
-  }
-  int lo = row_lo < n ? row_lo : n;
-  const int hi = row_hi < 0 ? n : (row_hi < n ? row_hi : n);
-  lo = lo < hi ? lo : hi;
-  const int kc = kg < lo ? lo : (kg > hi ? hi : kg);
-  for (int e = tid; e < kc; e += kRowThreads) flag[0xFFFFFFFFu - uint32_t(keys[e])] = 1;
-  if (tid == 0) flag[qi] = 1;
-  __syncthreads();
-  // ascending compaction of the flags
-  int32_t *out = indices + (bh * nb + qi) * size_t(nb);
-  const int warp = tid / 32, lane = tid % 32;
-  int base = 0;
-  for (int j0 = 0; j0 < n; j0 += kRowThreads) {
-    const int j = j0 + tid;
-    const bool keep = j < n && flag[j];
-    const unsigned bal = __ballot_sync(0xffffffffu, keep);
-    if (lane == 0) wcount[warp] = __popc(bal);
-    __syncthreads();
-    int before = base;
-    for (int w = 0; w < warp; ++w) before += wcount[w];
-    if (keep) out[before + __popc(bal & ((1u << lane) - 1u))] = j;
-    for (int w = 0; w < kRowThreads / 32; ++w) base += wcount[w];
-    __syncthreads();
-  }
-  if (tid == 0) counts[bh * nb + qi] = base;
+  return x;
 }
 
-size_t rows_qa_smem(int nb, int *pmax) {
-  int p = 1;
-  while (p < nb) p <<= 1;
-  *pmax = p;
-  return size_t(p) * 9;
+// The first bin of h[0, nbins), scanning from the top, at which base + the
+// cumulative mass reaches target_m (by_mass) or base_c + the cumulative count
+// reaches target_c; the sums of the bins above it.  Whole warp; lane l takes
+// bins nbins-1-l*per .. nbins-per-l*per.  With no crossing (not reached for
+// valid targets) the lowest bin.
+__device__ Crossing row_crossing(const RowHist &h, int nbins, bool by_mass, double target_m,
+                                 unsigned long long base_m, unsigned long long target_c,
+                                 unsigned long long base_c, int lane) {
+  const int per = nbins / 32;
+  unsigned long long lm = 0, lc = 0;
+  for (int k = 0; k < per; ++k) {
+    const int b = nbins - 1 - lane * per - k;
+    lm += (unsigned long long)h.lo[b] + ((unsigned long long)h.hi[b] << 16);
+    lc += h.cnt[b];
+  }
+  const unsigned long long im = warp_incl_scan(lm, lane), ic = warp_incl_scan(lc, lane);
+  const unsigned long long em = im - lm, ec = ic - lc;
+  auto reach = [&](unsigned long long m, unsigned long long c) {
+    return by_mass ? (double)(base_m + m) >= target_m : (base_c + c) >= target_c;
+  };
+  const unsigned hit = __ballot_sync(0xffffffffu, !reach(em, ec) && reach(im, ic));
+  Crossing cr;
+  if (hit == 0u) {  // fallback: the lowest bin, everything else above it
+    const unsigned long long tm = __shfl_sync(0xffffffffu, im, 31);
+    const unsigned long long tc = __shfl_sync(0xffffffffu, ic, 31);
+    cr.bin = 0u;
+    cr.above_m = tm - ((unsigned long long)h.lo[0] + ((unsigned long long)h.hi[0] << 16));
+    cr.above_c = tc - h.cnt[0];
+    return cr;
+  }
+  const int src = __ffs(hit) - 1;
+  uint32_t bin = 0u;
+  unsigned long long am = 0, ac = 0;
+  if (lane == src) {
+    unsigned long long cm = em, cc = ec;
+    for (int k = 0; k < per; ++k) {
+      const int b = nbins - 1 - lane * per - k;
+      const unsigned long long m = (unsigned long long)h.lo[b] + ((unsigned long long)h.hi[b] << 16);
+      if (reach(cm + m, cc + h.cnt[b])) {
+        bin = uint32_t(b);
+        am = cm;
+        ac = cc;
+        break;
+      }
+      cm += m;
+      cc += h.cnt[b];
+    }
+  }
+  cr.bin = __shfl_sync(0xffffffffu, bin, src);
+  cr.above_m = __shfl_sync(0xffffffffu, am, src);
+  cr.above_c = __shfl_sync(0xffffffffu, ac, src);
+  return cr;
+}
+
+__global__ void __launch_bounds__(kRowWarps * 32) select_rows_qa_kernel(
+    const int32_t *__restrict__ pattern, const float *__restrict__ map, int nb, float gamma,
+    int row_lo, int row_hi, int32_t *__restrict__ counts, int32_t *__restrict__ indices) {
+  __shared__ RowHist hist[kRowWarps];
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const size_t bh = size_t(blockIdx.z) * gridDim.y + blockIdx.y;
+  if (pattern[bh] != FP_PATTERN_QA) return;
+  const int qi = blockIdx.x * kRowWarps + warp;
+  if (qi >= nb) return;  // (no CTA-wide barrier below)
+  RowHist &h = hist[warp];
+  const int n = qi + 1;
+  const float *mrow = map + bh * (size_t(nb) * (nb + 1) / 2) + size_t(qi) * (qi + 1) / 2;
+  const unsigned long long lo = (unsigned long long)(row_lo < n ? row_lo : n);
+  const unsigned long long hi0 = row_hi < 0 ? n : (row_hi < n ? row_hi : n);
+  const unsigned long long blo = lo < hi0 ? lo : hi0, bhi = hi0;
+  // the rule's state (warp-uniform)
+  int mode = -1;  // SEL_* once decided by the clamp alone
+  bool by_mass = false;
+  double target_m = 0.0;
+  unsigned long long target_c = 0, am = 0, ac = 0;
+  uint32_t prefix = 0;
+  auto count_mode = [&](unsigned long long k) {
+    by_mass = false;
+    target_c = k;
+    if (k == 0) mode = SEL_NONE;
+    else if (k >= (unsigned long long)n) mode = SEL_ALL;
+  };
+  {
+    unsigned long long w = 0;
+    for (int j = lane; j < n; j += 32) w += score_mass(score_bits(mrow[j]));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) w += __shfl_xor_sync(0xffffffffu, w, o);
+    if (gamma >= 1.f) {
+      count_mode(bhi);  // k_gamma = n, clamped
+    } else {
+      target_m = (double)gamma * (double)w;
+      if (target_m <= 0.0) count_mode(blo);  // k_gamma = 0
+      else by_mass = true;
+    }
+  }
+  for (int lv = 0; lv < kRowLevels && mode < 0; ++lv) {
+    const int width = lv < 3 ? 8 : 7;
+    const int shift = lv < 3 ? 23 - 8 * lv : 0, nbins = 1 << width;
+    const int top = shift + width;  // the bits above this digit are fixed
+    for (int b = lane; b < 256; b += 32) {
+      h.lo[b] = 0u;
+      h.hi[b] = 0u;
+      h.cnt[b] = 0u;
+    }
+    __syncwarp();
+    for (int j = lane; j < n; j += 32) {
+      const uint32_t x = score_bits(mrow[j]);
+      if (top >= 31 || (x >> top) == (prefix >> top)) {
+        const uint32_t b = (x >> shift) & uint32_t(nbins - 1);
+        const uint64_t w = score_mass(x);
+        atomicAdd(&h.lo[b], unsigned(w & 0xFFFFull));
+        atomicAdd(&h.hi[b], unsigned(w >> 16));
+        atomicAdd(&h.cnt[b], 1u);
+      }
+    }
+    __syncwarp();
+    Crossing cr;
+    if (by_mass) {
+      cr = row_crossing(h, nbins, true, target_m, am, 0, 0, lane);
+      const unsigned long long A = ac + cr.above_c, C = h.cnt[cr.bin];
+      if (bhi <= A) count_mode(bhi);
+      else if (blo >= A + C) count_mode(blo);
+      if (mode >= 0) break;
+    }
+    if (!by_mass) cr = row_crossing(h, nbins, false, 0.0, 0, target_c, ac, lane);
+    am += cr.above_m;
+    ac += cr.above_c;
+    prefix |= cr.bin << shift;
+    __syncwarp();  // the histogram is cleared for the next digit
+  }
+  uint32_t tb = 0u, tidx = 0u;  // kept: bits > tb, or bits == tb and j <= tidx
+  if (mode < 0) {
+    const uint32_t b = prefix;
+    unsigned long long m;
+    if (by_mass) {
+      const unsigned long long w = score_mass(b);
+      unsigned long long mm = 1;
+      if (w > 0) {
+        const double need = (target_m - (double)am) / (double)w;
+        mm = need <= 1.0 ? 1ull : (unsigned long long)ceil(need);
+        while (mm > 1 && (double)(am + (mm - 1) * w) >= target_m) --mm;
+        while ((double)(am + mm * w) < target_m) ++mm;
+      }
+      unsigned long long k = ac + mm;
+      k = k < blo ? blo : (k > bhi ? bhi : k);
+      m = k - ac;
+    } else {
+      m = target_c - ac;
+    }
+    // the m-th (1-based) entry with pattern b, in index order
+    unsigned long long seen = 0;
+    uint32_t idx = uint32_t(n - 1);
+    for (int j0 = 0; j0 < n; j0 += 32) {
+      const int j = j0 + lane;
+      const bool hit = j < n && score_bits(mrow[j]) == b;
+      const unsigned bal = __ballot_sync(0xffffffffu, hit);
+      const unsigned c = __popc(bal);
+      if (seen + c >= m) {
+        unsigned x = bal;
+        for (unsigned long long r = seen + 1; r < m; ++r) x &= x - 1;
+        idx = uint32_t(j0 + __ffs(x) - 1);
+        break;
+      }
+      seen += c;
+    }
+    tb = b;
+    tidx = idx;
+  }
+  const HeadSel s{mode < 0 ? SEL_THRESHOLD : mode, tb, tidx, 0};
+  int32_t *out = indices + (bh * nb + qi) * size_t(nb);
+  int cnt = 0;
+  for (int j0 = 0; j0 < n; j0 += 32) {
+    const int j = j0 + lane;
+    const bool keep = j < n && (j == qi || kept(score_bits(mrow[j]), uint32_t(j), s));
+    const unsigned bal = __ballot_sync(0xffffffffu, keep);
+    if (keep) out[cnt + __popc(bal & ((1u << lane) - 1u))] = j;
+    cnt += __popc(bal);
+  }
+  if (lane == 0) counts[bh * nb + qi] = cnt;
 }
 
 __global__ void stats_kernel(const int32_t *__restrict__ counts,
@@ -1057,12 +1144,10 @@ cudaError_t launch_select(const Dims &D, float gamma, const SelectBudgets &bud,
       a, cf, df);
   emit_rows_kernel<<<dim3((D.nb + 7) / 8, D.hq, D.bt), 256, 0, st>>>(
       pattern, map, D.nb, a.sel, cf, df, bud.qa_mode, counts, indices);
-  if (bud.qa_mode == FP_QA_QUERYWISE) {
-    int pmax;
-    const size_t rsm = rows_qa_smem(D.nb, &pmax);
-    select_rows_qa_kernel<<<dim3(D.nb, D.hq, D.bt), kRowThreads, rsm, st>>>(
-        pattern, map, D.nb, pmax, gamma, bud.row_lo, bud.row_hi, counts, indices);
-  }
+  if (bud.qa_mode == FP_QA_QUERYWISE)
+    select_rows_qa_kernel<<<dim3((D.nb + kRowWarps - 1) / kRowWarps, D.hq, D.bt),
+                            kRowWarps * 32, 0, st>>>(pattern, map, D.nb, gamma, bud.row_lo,
+                                                     bud.row_hi, counts, indices);
   return cudaGetLastError();
 }
 
