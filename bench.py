@@ -454,8 +454,7 @@ def path_fields(layer, m: dict, peaks: dict, dense: float | None, whole: dict) -
         # the four staged calls (fp_estimate computes every output for every
         # head; the whole-path call skips what each head's pattern does not read)
         "stages_ms": {"estimate": st[0], "pattern": st[1], "select": st[2],
-                      "sparse_attn": st[3], "staged_step": m["ms_step"],
-                      "whole_path_before_attention": whole["ms_step"] - st[3]},
+                      "sparse_attn": st[3], "staged_step": m["ms_step"]},
         "estimate_hbm": {"bytes": eb, "gbs": eb / (st[0] * 1e-3) / 1e9,
                          "frac": eb / (st[0] * 1e-3) / 1e9 / hbm},
         "select_hbm": {"bytes": sb, "gbs": sb / (st[2] * 1e-3) / 1e9,

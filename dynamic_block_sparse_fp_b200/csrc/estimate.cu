@@ -94,8 +94,11 @@ __global__ void __launch_bounds__(256) pool_kernel(const T *__restrict__ x, floa
 // grid (tiles, tiles, Bt*Hq), 256 threads; a 128x128 tile of the nb x nb
 // logit matrix of one q head (tiles above the diagonal exit at once).  Each
 // thread accumulates an 8x8 register block (rows ty*4+{0..3} and 64+ty*4+..,
-// columns likewise) over d in steps of 8; fp32 fused multiply-adds.
-__global__ void __launch_bounds__(256) map_logits_kernel(const float *__restrict__ qbar,
+// columns likewise) with one fp32 fused multiply-add per element of d, in
+// order.  d is taken in slices of kMapK through two shared-memory buffers:
+// the next slice's loads are issued before the current slice's products.
+constexpr int kMapK = 16;
+__global__ void __launch_bounds__(256, 2) map_logits_kernel(const float *__restrict__ qbar,
                                                          const float *__restrict__ kbar,
                                                          float *__restrict__ map, int hq, int g,
                                                          int nb, int d, float scale,
@@ -105,46 +108,67 @@ __global__ void __launch_bounds__(256) map_logits_kernel(const float *__restrict
   const int bh = blockIdx.z, b = bh / hq, h = bh % hq, kv = h / g;
   if (qa_only && qa_only[bh] != FP_PATTERN_QA) return;
   const int hkv = hq / g;
-  __shared__ __align__(16) float As[8][128];
-  __shared__ __align__(16) float Bs[8][128];
+  __shared__ __align__(16) float As[2][kMapK][128];
+  __shared__ __align__(16) float Bs[2][kMapK][128];
   const float *qa = qbar + (size_t(b) * hq + h) * nb * d;
   const float *kb = kbar + (size_t(b) * hkv + kv) * nb * d;
   const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
-  // loader: thread -> (row, 4 consecutive k of the 8-wide chunk)
-  const int lr = threadIdx.x / 2, lk = (threadIdx.x % 2) * 4;
-  const int gi = ti * 128 + lr, gj = tj * 128 + lr;
+  // loader: thread -> rows lr and lr + 64, 4 consecutive k of the slice
+  const int lr = threadIdx.x / 4, lk = (threadIdx.x % 4) * 4;
+  float4 na[2], nbv[2];
+  auto load = [&](int k0) {
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const int gi = ti * 128 + lr + 64 * i, gj = tj * 128 + lr + 64 * i;
+      na[i] = gi < nb ? *reinterpret_cast<const float4 *>(qa + size_t(gi) * d + k0 + lk)
+                      : make_float4(0.f, 0.f, 0.f, 0.f);
+      nbv[i] = gj < nb ? *reinterpret_cast<const float4 *>(kb + size_t(gj) * d + k0 + lk)
+                       : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  };
+  auto store = [&](int buf) {
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const int r = lr + 64 * i;
+      As[buf][lk + 0][r] = na[i].x;
+      As[buf][lk + 1][r] = na[i].y;
+      As[buf][lk + 2][r] = na[i].z;
+      As[buf][lk + 3][r] = na[i].w;
+      Bs[buf][lk + 0][r] = nbv[i].x;
+      Bs[buf][lk + 1][r] = nbv[i].y;
+      Bs[buf][lk + 2][r] = nbv[i].z;
+      Bs[buf][lk + 3][r] = nbv[i].w;
+    }
+  };
   float acc[8][8];
 #pragma unroll
   for (int u = 0; u < 8; ++u)
 #pragma unroll
     for (int w = 0; w < 8; ++w) acc[u][w] = 0.f;
-  for (int k0 = 0; k0 < d; k0 += 8) {
-    const float4 av = gi < nb ? *reinterpret_cast<const float4 *>(qa + size_t(gi) * d + k0 + lk)
-                              : make_float4(0.f, 0.f, 0.f, 0.f);
-    const float4 bv = gj < nb ? *reinterpret_cast<const float4 *>(kb + size_t(gj) * d + k0 + lk)
-                              : make_float4(0.f, 0.f, 0.f, 0.f);
-    __syncthreads();
-    As[lk + 0][lr] = av.x;
-    As[lk + 1][lr] = av.y;
-    As[lk + 2][lr] = av.z;
-    As[lk + 3][lr] = av.w;
-    Bs[lk + 0][lr] = bv.x;
-    Bs[lk + 1][lr] = bv.y;
-    Bs[lk + 2][lr] = bv.z;
-    Bs[lk + 3][lr] = bv.w;
-    __syncthreads();
+  load(0);
+  store(0);
+  __syncthreads();
+  int buf = 0;
+  for (int k0 = 0; k0 < d; k0 += kMapK) {
+    const bool more = k0 + kMapK < d;
+    if (more) load(k0 + kMapK);
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const float4 a0 = *reinterpret_cast<const float4 *>(&As[k][ty * 4]);
-      const float4 a1 = *reinterpret_cast<const float4 *>(&As[k][64 + ty * 4]);
-      const float4 b0 = *reinterpret_cast<const float4 *>(&Bs[k][tx * 4]);
-      const float4 b1 = *reinterpret_cast<const float4 *>(&Bs[k][64 + tx * 4]);
+    for (int k = 0; k < kMapK; ++k) {
+      const float4 a0 = *reinterpret_cast<const float4 *>(&As[buf][k][ty * 4]);
+      const float4 a1 = *reinterpret_cast<const float4 *>(&As[buf][k][64 + ty * 4]);
+      const float4 b0 = *reinterpret_cast<const float4 *>(&Bs[buf][k][tx * 4]);
+      const float4 b1 = *reinterpret_cast<const float4 *>(&Bs[buf][k][64 + tx * 4]);
       const float a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
       const float bb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
 #pragma unroll
       for (int u = 0; u < 8; ++u)
 #pragma unroll
         for (int w = 0; w < 8; ++w) acc[u][w] = fmaf(a[u], bb[w], acc[u][w]);
+    }
+    if (more) {
+      store(buf ^ 1);  // the other buffer: its last readers passed the barrier below
+      __syncthreads();
+      buf ^= 1;
     }
   }
   float *m = map + (size_t(b) * hq + h) * (size_t(nb) * (nb + 1) / 2);
@@ -196,10 +220,11 @@ __global__ void __launch_bounds__(256) map_softmax_kernel(float *__restrict__ ma
 }
 
 // The last row of the map alone (the estimate a-hat that the pattern test
-// needs), for every head: grid (Hq, Bt), 256 threads.  Logit j is the same
-// fmaf chain over d, in order, times scale, that map_logits_kernel forms, and
-// the softmax is map_row_softmax, so the row is bitwise the full map's.
-__global__ void __launch_bounds__(256) map_last_row_kernel(const float *__restrict__ qbar,
+// needs), for every head: grid (Hq, Bt), 1024 threads (a key each, up to 4 at
+// nb = 4096).  Logit j is the same fmaf chain over d, in order, times scale,
+// that map_logits_kernel forms, and the softmax is map_row_softmax, so the
+// row is bitwise the full map's.
+__global__ void __launch_bounds__(1024) map_last_row_kernel(const float *__restrict__ qbar,
                                                            const float *__restrict__ kbar,
                                                            float *__restrict__ map,
                                                            float *__restrict__ est_last, int hq,
@@ -212,7 +237,7 @@ __global__ void __launch_bounds__(256) map_last_row_kernel(const float *__restri
   float *r = map + bh * (size_t(nb) * (nb + 1) / 2) + size_t(nb - 1) * nb / 2;
   if (threadIdx.x < d) qs[threadIdx.x] = qa[threadIdx.x];
   __syncthreads();
-  for (int j = threadIdx.x; j < nb; j += 256) {
+  for (int j = threadIdx.x; j < nb; j += 1024) {
     // k-bar row j in chunks of 8 float4 loads issued together; the fmaf
     // chain itself runs over d in order
     const float4 *kr = reinterpret_cast<const float4 *>(kb + size_t(j) * d);
@@ -568,7 +593,7 @@ cudaError_t run_decision(const Dims &Dm, const T *q, const T *k, float *qbar, fl
                                                               0, nullptr);
   pool_kernel<T><<<dim3(1, Dm.hq, Dm.bt), 256, 0, st>>>(q, qbar, Dm.n, Dm.d, Dm.bs, Dm.nb,
                                                          Dm.nb - 1, nullptr);
-  map_last_row_kernel<<<dim3(Dm.hq, Dm.bt), 256, 0, st>>>(qbar, kbar, map, est_last, Dm.hq,
+  map_last_row_kernel<<<dim3(Dm.hq, Dm.bt), 1024, 0, st>>>(qbar, kbar, map, est_last, Dm.hq,
                                                            Dm.g, Dm.nb, Dm.d,
                                                            1.f / sqrtf(float(Dm.d)));
   cudaError_t e = cudaGetLastError();
