@@ -26,21 +26,21 @@ int *device_status_ptr() {
   return ptrs[dev];
 }
 
-// The two copy streams fp_prefill_attn_host overlaps its transfers on (host to
-// device, device to host), created once per device on first use and kept
-// for the life of the process, like the status word.
-bool copy_streams(cudaStream_t *in, cudaStream_t *out) {
+// The streams of fp_prefill_attn_host besides the caller's: host-to-device
+// copies, device-to-host copies, and a second compute stream for every other
+// unit; created once per device on first use and kept for the life of the
+// process, like the status word.
+bool host_streams(cudaStream_t *in, cudaStream_t *out, cudaStream_t *comp) {
   static std::mutex mu;
-  static cudaStream_t s_in[64] = {nullptr}, s_out[64] = {nullptr};
+  static cudaStream_t s_in[64] = {nullptr}, s_out[64] = {nullptr}, s_comp[64] = {nullptr};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
   std::lock_guard<std::mutex> lock(mu);
-  if (!s_in[dev] && cudaStreamCreateWithFlags(&s_in[dev], cudaStreamNonBlocking) != cudaSuccess)
-    return false;
-  if (!s_out[dev] && cudaStreamCreateWithFlags(&s_out[dev], cudaStreamNonBlocking) != cudaSuccess)
-    return false;
+  for (cudaStream_t *s : {&s_in[dev], &s_out[dev], &s_comp[dev]})
+    if (!*s && cudaStreamCreateWithFlags(s, cudaStreamNonBlocking) != cudaSuccess) return false;
   *in = s_in[dev];
   *out = s_out[dev];
+  *comp = s_comp[dev];
   return true;
 }
 
@@ -160,6 +160,49 @@ struct Prefill {
 
 constexpr int kHostMidUnits = 3;  // fp_prefill_attn_host: middle units per batch entry
 
+// One unit of fp_prefill_attn_host: consecutive heads of one batch entry.
+struct Unit {
+  int kv0, nk;  // kv heads [kv0, kv0 + nk)
+  int q0, nq;   // their query heads [kv0 g + q0, kv0 g + q0 + nq)
+  bool kv_in;   // this unit copies the kv heads' K and V in
+};
+
+// The units of one batch entry.  Only the first unit's copy in and the last
+// unit's copy out are not hidden, so those two units hold one query head each
+// (with the first, its kv head's K and V come in; the second unit then brings
+// only the rest of that kv head's Q), the next to them the rest of the first
+// and last kv heads' query heads, and the kv heads between go in three middle
+// units.
+std::vector<Unit> host_plan(const Dims &D) {
+  std::vector<Unit> plan;
+  auto whole = [&](int kv0, int nk) { plan.push_back({kv0, nk, 0, nk * D.g, true}); };
+  auto middle = [&]() {
+    const int mid = D.hkv - 2;
+    for (int i = 0, kv = 1; i < kHostMidUnits; ++i) {
+      const int n = mid / kHostMidUnits + (i < mid % kHostMidUnits ? 1 : 0);
+      if (n > 0) whole(kv, n);
+      kv += n;
+    }
+  };
+  if (D.hkv >= 4 && D.g >= 2) {
+    plan.push_back({0, 1, 0, 1, true});
+    plan.push_back({0, 1, 1, D.g - 1, false});
+    middle();
+    plan.push_back({D.hkv - 1, 1, 0, D.g - 1, true});
+    plan.push_back({D.hkv - 1, 1, D.g - 1, 1, false});
+  } else if (D.hkv >= 4) {
+    whole(0, 1);
+    middle();
+    whole(D.hkv - 1, 1);
+  } else {
+    for (int kv = 0; kv < D.hkv; ++kv) whole(kv, 1);
+  }
+  return plan;
+}
+
+// The shape of one unit (batch 1, the unit's heads).
+bool unit_dims(const fp_shape &shape, const Unit &un, Dims *Du);
+
 size_t carve_prefill(const Dims &D, void *ws, Prefill *P) {
   Carver c{static_cast<char *>(ws), 0};
   const size_t heads = size_t(D.bt) * D.hq;
@@ -178,6 +221,41 @@ size_t carve_prefill(const Dims &D, void *ws, Prefill *P) {
                                                                attn_ws_bytes(D)));
   P->stage_ws = c.take<char>(stage);
   return c.off + 256;
+}
+
+bool unit_dims(const fp_shape &shape, const Unit &un, Dims *Du) {
+  fp_shape us = shape;
+  us.batch = 1;
+  us.n_kv_heads = un.nk;
+  us.n_q_heads = un.nq;
+  return check_shape(&us, Du) == FP_OK;
+}
+
+// Workspace of fp_prefill_attn_host: device copies of q, k, v and out, and two
+// unit regions (units alternate between two compute streams), each sized for
+// the largest unit.
+struct HostWs {
+  char *q, *k, *v, *out, *unit[2];
+  size_t bytes;
+};
+HostWs carve_host(const fp_shape &shape, const Dims &D, void *ws) {
+  const size_t eb = D.dtype == FP_BF16 ? 2 : 4;
+  Carver c{static_cast<char *>(ws), 0};
+  HostWs h;
+  h.q = c.take<char>(size_t(D.bt) * D.hq * D.n * D.d * eb);
+  h.k = c.take<char>(size_t(D.bt) * D.hkv * D.n * D.d * eb);
+  h.v = c.take<char>(size_t(D.bt) * D.hkv * D.n * D.d * eb);
+  h.out = c.take<char>(size_t(D.bt) * D.hq * D.n * D.d * eb);
+  size_t unit_bytes = 0;
+  for (const Unit &un : host_plan(D)) {
+    Dims Du;
+    Prefill P;
+    if (unit_dims(shape, un, &Du)) unit_bytes = std::max(unit_bytes, carve_prefill(Du, nullptr, &P));
+  }
+  h.unit[0] = c.take<char>(unit_bytes);
+  h.unit[1] = c.take<char>(unit_bytes);
+  h.bytes = c.off + 256;
+  return h;
 }
 
 size_t elem_bytes(const Dims &D) { return D.dtype == FP_BF16 ? 2 : 4; }
@@ -241,17 +319,8 @@ FP_API size_t fp_workspace_size(const fp_shape *shape, int which_call) {
       Prefill P;
       return carve_prefill(D, nullptr, &P);
     }
-    case FP_CALL_PREFILL_HOST: {
-      Prefill P;
-      Carver c{nullptr, 0};
-      const size_t eb = elem_bytes(D);
-      c.take<char>(size_t(D.bt) * D.hq * D.n * D.d * eb);
-      c.take<char>(size_t(D.bt) * D.hkv * D.n * D.d * eb);
-      c.take<char>(size_t(D.bt) * D.hkv * D.n * D.d * eb);
-      c.take<char>(size_t(D.bt) * D.hq * D.n * D.d * eb);
-      c.take<char>(carve_prefill(D, nullptr, &P));
-      return c.off + 256;
-    }
+    case FP_CALL_PREFILL_HOST:
+      return carve_host(*shape, D, nullptr).bytes;
     default:
       return 0;
   }
@@ -417,58 +486,20 @@ FP_API fp_status fp_prefill_attn_host(const fp_shape *shape, const fp_params *pa
     return s;
   if ((s = check_device()) != FP_OK) return s;
   const size_t eb = elem_bytes(D);
-  const size_t qbytes = size_t(D.bt) * D.hq * D.n * D.d * eb;
-  const size_t kvbytes = size_t(D.bt) * D.hkv * D.n * D.d * eb;
-  Carver c{static_cast<char *>(ws), 0};
-  char *qd = c.take<char>(qbytes);
-  char *kd = c.take<char>(kvbytes);
-  char *vd = c.take<char>(kvbytes);
-  char *od = c.take<char>(qbytes);
-  Prefill Pfull;
-  char *pre = c.take<char>(carve_prefill(D, nullptr, &Pfull));
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream), sin = nullptr, sout = nullptr;
-  if (!copy_streams(&sin, &sout)) return FP_ERR_CUDA;
+  const HostWs hw = carve_host(*shape, D, ws);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream), sin = nullptr, sout = nullptr,
+               scomp = nullptr;
+  if (!host_streams(&sin, &sout, &scomp)) return FP_ERR_CUDA;
   // Every stage is independent per query head (a query head reads only its
-  // kv head's K and V), so the call runs as units of consecutive heads: the
-  // inputs of unit u+1 are copied in while unit u computes on `stream`, and
-  // its output is copied out while unit u+1 computes.  Only the first unit's
-  // copy in and the last unit's copy out are not hidden, so those two units
-  // hold one query head each (with the first, its kv head's K and V come in;
-  // the second unit then brings only the rest of that kv head's Q), the next
-  // to them the rest of the first and last kv heads' query heads, and the
-  // kv heads between go in three middle units.  The caller's stream forks to
-  // the copy streams and joins them at the end through events, so `stream`
-  // still orders the whole call.
-  struct Unit {
-    int kv0, nk;  // kv heads [kv0, kv0 + nk)
-    int q0, nq;   // their query heads [kv0 g + q0, kv0 g + q0 + nq)
-    bool kv_in;   // this unit copies the kv heads' K and V in
-  };
-  std::vector<Unit> plan;  // one batch entry
-  auto whole = [&](int kv0, int nk) { plan.push_back({kv0, nk, 0, nk * D.g, true}); };
-  if (D.hkv >= 4 && D.g >= 2) {
-    plan.push_back({0, 1, 0, 1, true});
-    plan.push_back({0, 1, 1, D.g - 1, false});
-    const int mid = D.hkv - 2;
-    for (int i = 0, kv = 1; i < kHostMidUnits; ++i) {
-      const int n = mid / kHostMidUnits + (i < mid % kHostMidUnits ? 1 : 0);
-      if (n > 0) whole(kv, n);
-      kv += n;
-    }
-    plan.push_back({D.hkv - 1, 1, 0, D.g - 1, true});
-    plan.push_back({D.hkv - 1, 1, D.g - 1, 1, false});
-  } else if (D.hkv >= 4) {
-    whole(0, 1);
-    const int mid = D.hkv - 2;
-    for (int i = 0, kv = 1; i < kHostMidUnits; ++i) {
-      const int n = mid / kHostMidUnits + (i < mid % kHostMidUnits ? 1 : 0);
-      if (n > 0) whole(kv, n);
-      kv += n;
-    }
-    whole(D.hkv - 1, 1);
-  } else {
-    for (int kv = 0; kv < D.hkv; ++kv) whole(kv, 1);
-  }
+  // kv head's K and V), so the call runs as units of consecutive heads
+  // (host_plan): the inputs of unit u+1 are copied in while unit u computes,
+  // and each unit's output is copied out while the next one computes.  Units
+  // alternate between `stream` and a second compute stream, each with its own
+  // workspace region, so that one unit's latency-bound estimate and selection
+  // overlap the other's attention.  `stream` forks to the library's streams
+  // and joins them at the end through events, so it still orders the whole
+  // call.
+  const std::vector<Unit> plan = host_plan(D);
   const int units_per_batch = int(plan.size());
   const int nunits = D.bt * units_per_batch;
   std::vector<cudaEvent_t> ev;
@@ -484,52 +515,57 @@ FP_API fp_status fp_prefill_attn_host(const fp_shape *shape, const fp_params *pa
   cudaEvent_t e_start, e_end;
   if (!event(&e_start) || cudaEventRecord(e_start, st) != cudaSuccess ||
       cudaStreamWaitEvent(sin, e_start, 0) != cudaSuccess ||
-      cudaStreamWaitEvent(sout, e_start, 0) != cudaSuccess)
+      cudaStreamWaitEvent(sout, e_start, 0) != cudaSuccess ||
+      cudaStreamWaitEvent(scomp, e_start, 0) != cudaSuccess)
     return finish(FP_ERR_CUDA);
+  const cudaStream_t comp[2] = {st, scomp};
   const size_t head_bytes = size_t(D.n) * D.d * eb;
   const char *qh = static_cast<const char *>(q_host);
   const char *kh = static_cast<const char *>(k_host);
   const char *vh = static_cast<const char *>(v_host);
   char *oh = static_cast<char *>(out_host);
+  cudaEvent_t e_v = nullptr;  // the current kv head's V is in
   for (int u = 0; u < nunits; ++u) {
     const int b = u / units_per_batch;
     const Unit &un = plan[u % units_per_batch];
-    fp_shape us = *shape;
-    us.batch = 1;
-    us.n_kv_heads = un.nk;
-    us.n_q_heads = un.nq;
     Dims Du;
-    if (check_shape(&us, &Du) != FP_OK) return finish(FP_ERR_SHAPE);
+    if (!unit_dims(*shape, un, &Du)) return finish(FP_ERR_SHAPE);
+    const cudaStream_t cs = comp[u % 2];
     const size_t qoff = (size_t(b) * D.hq + size_t(un.kv0) * D.g + un.q0) * head_bytes;
     const size_t kvoff = (size_t(b) * D.hkv + un.kv0) * head_bytes;
     const size_t qlen = size_t(un.nq) * head_bytes, kvlen = size_t(un.nk) * head_bytes;
     // Q and K first: the unit's estimate can start on them, while V (read only
-    // by the attention stage) is still coming in behind its own event
-    cudaEvent_t e_in, e_v = nullptr, e_comp;
+    // by the attention stage) is still coming in behind its own event, which
+    // the kv heads' later units wait for too
+    cudaEvent_t e_in, e_comp;
     if (!event(&e_in) || !event(&e_comp) ||
-        cudaMemcpyAsync(qd + qoff, qh + qoff, qlen, cudaMemcpyHostToDevice, sin) != cudaSuccess)
+        cudaMemcpyAsync(hw.q + qoff, qh + qoff, qlen, cudaMemcpyHostToDevice, sin) != cudaSuccess)
       return finish(FP_ERR_CUDA);
     if (un.kv_in &&
-        cudaMemcpyAsync(kd + kvoff, kh + kvoff, kvlen, cudaMemcpyHostToDevice, sin) != cudaSuccess)
+        cudaMemcpyAsync(hw.k + kvoff, kh + kvoff, kvlen, cudaMemcpyHostToDevice, sin) !=
+            cudaSuccess)
       return finish(FP_ERR_CUDA);
-    if (cudaEventRecord(e_in, sin) != cudaSuccess || cudaStreamWaitEvent(st, e_in, 0) != cudaSuccess)
+    if (cudaEventRecord(e_in, sin) != cudaSuccess || cudaStreamWaitEvent(cs, e_in, 0) != cudaSuccess)
       return finish(FP_ERR_CUDA);
     if (un.kv_in &&
         (!event(&e_v) ||
-         cudaMemcpyAsync(vd + kvoff, vh + kvoff, kvlen, cudaMemcpyHostToDevice, sin) !=
+         cudaMemcpyAsync(hw.v + kvoff, vh + kvoff, kvlen, cudaMemcpyHostToDevice, sin) !=
              cudaSuccess ||
          cudaEventRecord(e_v, sin) != cudaSuccess))
       return finish(FP_ERR_CUDA);
     Prefill Pu;
-    carve_prefill(Du, pre, &Pu);  // units run one after another on `stream`
-    const fp_status r = run_prefill(Du, *params, qd + qoff, kd + kvoff, vd + kvoff, od + qoff,
-                                    nullptr, nullptr, Pu, st, e_v);
+    carve_prefill(Du, hw.unit[u % 2], &Pu);  // a region's units run in order on one stream
+    const fp_status r = run_prefill(Du, *params, hw.q + qoff, hw.k + kvoff, hw.v + kvoff,
+                                    hw.out + qoff, nullptr, nullptr, Pu, cs, e_v);
     if (r != FP_OK) return finish(r);
-    if (cudaEventRecord(e_comp, st) != cudaSuccess ||
+    if (cudaEventRecord(e_comp, cs) != cudaSuccess ||
         cudaStreamWaitEvent(sout, e_comp, 0) != cudaSuccess ||
-        cudaMemcpyAsync(oh + qoff, od + qoff, qlen, cudaMemcpyDeviceToHost, sout) != cudaSuccess)
+        cudaMemcpyAsync(oh + qoff, hw.out + qoff, qlen, cudaMemcpyDeviceToHost, sout) !=
+            cudaSuccess)
       return finish(FP_ERR_CUDA);
   }
+  // every unit's copy out follows its compute on the copy-out stream, so its
+  // last event covers both compute streams
   if (!event(&e_end) || cudaEventRecord(e_end, sout) != cudaSuccess ||
       cudaStreamWaitEvent(st, e_end, 0) != cudaSuccess)
     return finish(FP_ERR_CUDA);

@@ -310,11 +310,13 @@ fp_status fp_prefill_attn_varlen(const fp_shape *shape, const fp_params *params,
  * and last kv heads' query heads next to them; the kv heads between in three
  * middle units): the inputs of a unit are copied in (one cudaMemcpyAsync per
  * buffer slice; a kv head's K and V with its first unit) while the previous
- * unit computes on `stream`, and each unit's output is copied out while the
- * next one computes.  The copies run on two streams of
- * the library's own, created once per device on first use and kept until the
- * process exits; `stream` forks to them and joins them through events, so
- * work enqueued on `stream` after this call sees the finished output.
+ * unit computes, and each unit's output is copied out while the next one
+ * computes.  Units compute alternately on `stream` and on a compute stream of
+ * the library's own, each with its own part of `ws`.  The copies run on two
+ * more library streams; the library's streams are created once per device on
+ * first use and kept until the process exits; `stream` forks to them and
+ * joins them through events, so work enqueued on `stream` after this call
+ * sees the finished output.
  * Page-locked host memory makes the copies asynchronous and lets them
  * overlap.  The host buffers must stay valid until `stream` reaches the end
  * of the call.  The result is bitwise that of fp_prefill_attn.
