@@ -267,7 +267,7 @@ def run_reference(args, w, ws, rank):
     line = {"impl": "reference", "metric": METRIC, "value": tps, "unit": "tokens/s",
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1000.0 * w.seq_len * w.batch / tps, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "scaling": "strong", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": workload_config(w, 1),
             "cpu_baseline": {"value": tps, "unit": "tokens/s", "cores": cores(),
                              "kind": "oracle", "sample": steps[0]["sample"]},
