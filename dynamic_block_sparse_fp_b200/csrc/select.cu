@@ -32,7 +32,7 @@
 //
 // Block-pooled lines for vertical-slash heads (FP_VS_BLOCKS): pool_lines_kernel
 // sums vert per key block and slash per block distance into nb-entry lists,
-// which select_head_kernel then selects as lines of a sequence of nb tokens
+// which the radix select then takes as lines of a sequence of nb tokens
 // with block size 1 (a column is a key block, an offset one block distance).
 #include <algorithm>
 #include <mutex>
