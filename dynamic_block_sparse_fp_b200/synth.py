@@ -164,9 +164,10 @@ def make_group(w: Workload, b: int, kv: int):
                 k[j * bs:(j + 1) * bs, :] += w.amp_qa * u
     if kind == "vs" or w.sink_boost_all:
         vv = _unit(gen, d)
-        sinks = [0, 1, 2, 3]
+        sinks = list(range(min(4, n)))
         if kind == "vs":
-            extra = (torch.randperm(n - 4, generator=gen)[: w.n_random_vs_keys] + 4).tolist()
+            extra = (torch.randperm(max(n - 4, 0), generator=gen)[: w.n_random_vs_keys]
+                     + 4).tolist()
             sinks = sinks + extra
         for t in sinks:
             k[t, :] += w.amp_vs * vv

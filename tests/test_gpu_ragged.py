@@ -151,3 +151,43 @@ def test_ragged_varlen_and_host_paths():
     torch.cuda.synchronize()
     assert torch.equal(oh, want.cpu())
     assert ops.fp_last_device_status() == 0
+
+
+@pytest.mark.parametrize("n,base,kw", [
+    (1, "llama8b_n8192", dict(n_q_heads=4, n_kv_heads=2)),
+    (100, "llama8b_n8192", dict(n_q_heads=4, n_kv_heads=2)),
+    (129, "llama8b_n8192", dict(n_q_heads=4, n_kv_heads=2)),
+    (1, "tiny_n1024", {}),
+    (65, "tiny_n1024", {}),
+])
+def test_shortest_sequences(n, base, kw):
+    """A single token, fewer tokens than one block, and one token past a
+    block: the whole path against the oracle (estimate 1e-4, lists bit-exact,
+    every row of attention) and the whole-path call against the staged calls."""
+    w = synth.WORKLOADS[base].replace(seq_len=n, **kw)
+    inp = synth.make_inputs(w)
+    d = {x: inp[x].to(DEV) for x in ("q", "k", "v")}
+    bf16 = w.dtype == "bf16"
+    s = ops.make_shape(d["q"], d["k"], w.block_size)
+    p = ops.make_params(w.gamma, w.tau, w.min_budget, w.max_budget)
+    est = ops.estimate(d["q"], d["k"], w.block_size)
+    torch.cuda.synchronize()
+    want = oracle.estimate(inp["q"], inp["k"], w.block_size)
+    for key in ("qbar", "kbar", "map", "est_last", "true_last", "vert", "slash"):
+        np.testing.assert_allclose(_np(est[key]), want[key], rtol=1e-4, atol=1e-7, err_msg=key)
+    _, pat = ops.pattern(s, p, est["est_last"], est["true_last"])
+    counts, indices = ops.select(s, p, pat, est["map"], est["vert"], est["slash"])
+    out, lse = ops.sparse_attn(d["q"], d["k"], d["v"], counts, indices, w.block_size)
+    torch.cuda.synchronize()
+    nb = w.n_blocks
+    oc, oi = oracle.select(pat.cpu().numpy(), _np(est["map"]), _np(est["vert"]),
+                           _np(est["slash"]), nb, w.block_size, w.gamma, w.min_budget,
+                           w.max_budget)
+    np.testing.assert_array_equal(counts.cpu().numpy(), oc)
+    o, l = oracle.sparse_attention(inp["q"], inp["k"], inp["v"], oc, oi, w.block_size)
+    assert np.abs(_np(out) - o).max() <= (2e-2 if bf16 else 1e-4)
+    assert np.abs(_np(lse) - l).max() <= (2e-3 if bf16 else 1e-4)
+    out2, _, _ = ops.prefill_attn(d["q"], d["k"], d["v"], w.block_size, p)
+    torch.cuda.synchronize()
+    assert torch.equal(out2, out)
+    assert ops.fp_last_device_status() == 0

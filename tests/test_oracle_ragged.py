@@ -182,3 +182,32 @@ def test_ragged_pipeline_gamma_one_is_dense():
     kk, vv = k.repeat_interleave(2, dim=1), v.repeat_interleave(2, dim=1)
     ref = torch.nn.functional.scaled_dot_product_attention(q, kk, vv, is_causal=True).numpy()
     np.testing.assert_allclose(res["out"], ref, rtol=0, atol=1e-12)
+
+
+def test_single_token_sequence_closed_form():
+    """N = 1: one partial block, one key.  Whatever the pattern, each head keeps
+    that block; the output is V's only row and the log-sum-exp is the single
+    scaled logit q.k / sqrt(d)."""
+    g = torch.Generator().manual_seed(11)
+    q = torch.randn(1, 4, 1, 8, generator=g, dtype=torch.float64)
+    k = torch.randn(1, 2, 1, 8, generator=g, dtype=torch.float64)
+    v = torch.randn(1, 2, 1, 8, generator=g, dtype=torch.float64)
+    for gamma in (0.5, 0.95):
+        res = oracle.flexprefill(q, k, v, 16, gamma, 0.1, 0, 0)
+        assert (res["counts"] == 1).all()
+        assert (res["indices"][..., 0] == 0).all()
+        kk, vv = k.repeat_interleave(2, dim=1), v.repeat_interleave(2, dim=1)
+        np.testing.assert_allclose(res["out"], vv.numpy(), rtol=0, atol=0)
+        ref_lse = ((q * kk).sum(-1) / math.sqrt(8)).numpy()
+        np.testing.assert_allclose(res["lse"], ref_lse, rtol=0, atol=1e-14)
+
+
+@pytest.mark.parametrize("n", [1, 2, 3, 4])
+def test_synthetic_inputs_for_sequences_shorter_than_the_sinks(n):
+    """The generator plants up to four sink keys; a shorter sequence plants
+    the ones it has and still yields finite inputs of the asked shape."""
+    from dynamic_block_sparse_fp_b200 import synth
+    w = synth.WORKLOADS["tiny_n1024"].replace(seq_len=n)
+    inp = synth.make_inputs(w)
+    assert inp["q"].shape[2] == n and inp["k"].shape[2] == n
+    assert all(torch.isfinite(inp[x]).all() for x in ("q", "k", "v"))

@@ -63,6 +63,30 @@ def test_noalloc_select_matches_fp_select_twice():
     assert ops.fp_last_device_status() == 0
 
 
+def test_noalloc_select_ragged_length():
+    """A sequence whose length is not a multiple of the block size (a partial
+    last block): the same lists as fp_select, two calls in a row."""
+    build.build()
+    w = synth.WORKLOADS["llama8b_n8192"].replace(seq_len=8192 + 64 + 5, n_q_heads=8,
+                                                 n_kv_heads=2)
+    inp = synth.make_inputs(w)
+    q, k = inp["q"].to(DEV), inp["k"].to(DEV)
+    s = ops.make_shape(q, k, w.block_size)
+    est = ops.estimate(q, k, w.block_size)
+    pat = (torch.arange(w.n_q_heads, device=DEV, dtype=torch.int32) % 2).reshape(1, -1)
+    nb = w.n_blocks
+    for p in (ops.make_params(0.95, 0.1, 1024, 0), ops.make_params(0.9, 0.1, 512, 2048)):
+        ref_c, ref_i = ops.select(s, p, pat, est["map"], est["vert"], est["slash"])
+        counts = torch.full((1, w.n_q_heads, nb), -7, dtype=torch.int32, device=DEV)
+        indices = torch.full((1, w.n_q_heads, nb, nb), -7, dtype=torch.int32, device=DEV)
+        rc = ops.fp_select_noalloc(s, p, pat, est["map"], est["vert"], est["slash"], counts,
+                                   indices)
+        assert rc == 0, ops.STATUS.get(rc, rc)
+        torch.cuda.synchronize()
+        _same_lists(counts, indices, ref_c, ref_i)
+    assert ops.fp_last_device_status() == 0
+
+
 def test_noalloc_select_rejects_problems_beyond_its_scratch():
     L = ops.lib()
     # 16 x 32 heads at nb = 4096 needs ~36 MiB of scratch, above the fixed 4 MiB
