@@ -136,6 +136,15 @@ fp_status check_device() {
 
 fp_status cuda_status(cudaError_t e) { return e == cudaSuccess ? FP_OK : FP_ERR_CUDA; }
 
+// q, k, v, out, qbar and kbar are moved with 16-byte vector accesses and
+// tensor-map copies (whose base must be 16-byte aligned); the other arrays
+// with accesses of their element size.  A null pointer passes (the null
+// checks come first, and optional outputs may be null).
+bool al(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+bool qkvo_aligned(const void *q, const void *k, const void *v, const void *out) {
+  return al(q, 16) && al(k, 16) && al(v, 16) && al(out, 16);
+}
+
 // One thread waits on an mbarrier that nothing arrives at, with the bounded
 // wait of the pipelined kernels, and records FP_ERR_TIMEOUT when it gives up.
 __global__ void watchdog_selftest_kernel(int *status, unsigned long long limit_ns) {
@@ -335,6 +344,9 @@ FP_API fp_status fp_estimate(const fp_shape *shape, const void *q, const void *k
   if (s != FP_OK) return s;
   if (!q || !k || !qbar || !kbar || !map || !est_last || !true_last || !vert || !slash)
     return FP_ERR_NULL;
+  if (!al(q, 16) || !al(k, 16) || !al(qbar, 16) || !al(kbar, 16) || !al(map, 4) ||
+      !al(est_last, 4) || !al(true_last, 4) || !al(vert, 4) || !al(slash, 4))
+    return FP_ERR_ALIGN;
   if ((s = check_ws(ws, ws_bytes, estimate_ws_bytes(D))) != FP_OK) return s;
   if ((s = check_device()) != FP_OK) return s;
   return cuda_status(launch_estimate(D, q, k, qbar, kbar, map, est_last, true_last, vert, slash,
@@ -349,6 +361,8 @@ FP_API fp_status fp_pattern(const fp_shape *shape, const fp_params *params,
   if (s != FP_OK) return s;
   if ((s = check_params(params)) != FP_OK) return s;
   if (!est_last || !true_last || !djs || !pattern) return FP_ERR_NULL;
+  if (!al(est_last, 4) || !al(true_last, 4) || !al(djs, 4) || !al(pattern, 4))
+    return FP_ERR_ALIGN;
   if ((s = check_device()) != FP_OK) return s;
   return cuda_status(launch_pattern(D, params->tau, est_last, true_last, djs, pattern,
                                     reinterpret_cast<cudaStream_t>(stream)));
@@ -363,6 +377,9 @@ FP_API fp_status fp_select(const fp_shape *shape, const fp_params *params,
   if (s != FP_OK) return s;
   if ((s = check_params(params)) != FP_OK) return s;
   if (!pattern || !map || !vert || !slash || !counts || !indices) return FP_ERR_NULL;
+  if (!al(pattern, 4) || !al(map, 4) || !al(vert, 4) || !al(slash, 4) || !al(counts, 4) ||
+      !al(indices, 4))
+    return FP_ERR_ALIGN;
   if ((s = check_ws(ws, ws_bytes, select_ws_bytes(D))) != FP_OK) return s;
   if ((s = check_device()) != FP_OK) return s;
   return cuda_status(launch_select(D, params->gamma, budgets(D, *params), pattern, map, vert,
@@ -379,6 +396,9 @@ FP_API fp_status fp_select_noalloc(const fp_shape *shape, const fp_params *param
   if (s != FP_OK) return s;
   if ((s = check_params(params)) != FP_OK) return s;
   if (!pattern || !map || !vert || !slash || !counts || !indices) return FP_ERR_NULL;
+  if (!al(pattern, 4) || !al(map, 4) || !al(vert, 4) || !al(slash, 4) || !al(counts, 4) ||
+      !al(indices, 4))
+    return FP_ERR_ALIGN;
   if (select_ws_bytes(D) > FP_SELECT_NOALLOC_SCRATCH_BYTES) return FP_ERR_WORKSPACE;
   if ((s = check_device()) != FP_OK) return s;
   return cuda_status(launch_select_noalloc(D, params->gamma, budgets(D, *params), pattern, map,
@@ -395,6 +415,8 @@ FP_API fp_status fp_sparse_attn(const fp_shape *shape, const void *q, const void
   if (s != FP_OK) return s;
   if ((s = check_attn_shape(D)) != FP_OK) return s;
   if (!q || !k || !v || !counts || !indices || !out) return FP_ERR_NULL;
+  if (!qkvo_aligned(q, k, v, out) || !al(counts, 4) || !al(indices, 4) || !al(lse, 4))
+    return FP_ERR_ALIGN;
   if ((s = check_ws(ws, ws_bytes, attn_ws_bytes(D))) != FP_OK) return s;
   if ((s = check_device()) != FP_OK) return s;
   return run_attn(D, q, k, v, counts, indices, out, lse, false, ws,
@@ -408,6 +430,7 @@ FP_API fp_status fp_dense_attn(const fp_shape *shape, const void *q, const void 
   if (s != FP_OK) return s;
   if ((s = check_attn_shape(D)) != FP_OK) return s;
   if (!q || !k || !v || !out) return FP_ERR_NULL;
+  if (!qkvo_aligned(q, k, v, out) || !al(lse, 4)) return FP_ERR_ALIGN;
   if ((s = check_device()) != FP_OK) return s;
   // dense lists are implicit: counts / indices are never read
   static const int32_t dummy = 0;
@@ -425,6 +448,7 @@ FP_API fp_status fp_prefill_attn(const fp_shape *shape, const fp_params *params,
   if ((s = check_attn_shape(D)) != FP_OK) return s;
   if ((s = check_params(params)) != FP_OK) return s;
   if (!q || !k || !v || !out) return FP_ERR_NULL;
+  if (!qkvo_aligned(q, k, v, out) || !al(lse, 4) || !al(stats, 8)) return FP_ERR_ALIGN;
   Prefill P;
   if ((s = check_ws(ws, ws_bytes, carve_prefill(D, nullptr, &P))) != FP_OK) return s;
   if ((s = check_device()) != FP_OK) return s;
@@ -445,6 +469,8 @@ FP_API fp_status fp_prefill_attn_varlen(const fp_shape *shape, const fp_params *
   if ((s = check_attn_shape(D)) != FP_OK) return s;
   if ((s = check_params(params)) != FP_OK) return s;
   if (!q || !k || !v || !out || !seq_lens) return FP_ERR_NULL;
+  // a sequence starts at a multiple of Hq d (or Hkv d) elements: aligned with the base
+  if (!qkvo_aligned(q, k, v, out) || !al(lse, 4) || !al(stats, 8)) return FP_ERR_ALIGN;
   if (n_seqs < 1) return FP_ERR_SHAPE;
   for (int i = 0; i < n_seqs; ++i)
     if (seq_lens[i] <= 0 || seq_lens[i] > D.n) return FP_ERR_SHAPE;
@@ -606,6 +632,7 @@ FP_API const char *fp_status_string(fp_status status) {
     case FP_ERR_TIMEOUT: return "FP_ERR_TIMEOUT: a device pipeline wait ran out of time";
     case FP_ERR_DEVICE_CHECK: return "FP_ERR_DEVICE_CHECK: an argument failed a device check";
     case FP_ERR_UNSUPPORTED: return "FP_ERR_UNSUPPORTED: the device is not sm_100";
+    case FP_ERR_ALIGN: return "FP_ERR_ALIGN: a data pointer is not aligned as required";
   }
   return "unknown fp_status";
 }

@@ -32,7 +32,7 @@ FP_CALL_ESTIMATE, FP_CALL_SELECT, FP_CALL_SPARSE_ATTN, FP_CALL_PREFILL, FP_CALL_
     0, 1, 2, 3, 4)
 STATUS = {0: "FP_OK", 1: "FP_ERR_NULL", 2: "FP_ERR_SHAPE", 3: "FP_ERR_DTYPE", 4: "FP_ERR_PARAM",
           5: "FP_ERR_WORKSPACE", 6: "FP_ERR_CUDA", 7: "FP_ERR_TIMEOUT",
-          8: "FP_ERR_DEVICE_CHECK", 9: "FP_ERR_UNSUPPORTED"}
+          8: "FP_ERR_DEVICE_CHECK", 9: "FP_ERR_UNSUPPORTED", 10: "FP_ERR_ALIGN"}
 STATUS_CODES = {v: k for k, v in STATUS.items()}
 HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include",
                       "fp.h")

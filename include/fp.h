@@ -30,6 +30,11 @@
  *    device memory; scratch space is the caller's workspace (`ws`, at least
  *    fp_workspace_size() bytes, 256-byte aligned).  A workspace must not be
  *    shared by calls that may run concurrently.
+ *  * Device data pointers must be aligned: q, k, v, out, qbar and kbar to
+ *    16 bytes (they are moved with 16-byte vector accesses and tensor-map
+ *    copies), every other array to its element size (4 bytes; stats 8).
+ *    torch allocations and views that start on such a boundary qualify; a
+ *    misaligned pointer returns FP_ERR_ALIGN.
  *  * Arguments are validated on the host before anything is launched; a
  *    failed check returns an error code and launches nothing.
  *  * Kernels run asynchronously on `stream` (NULL = the legacy default
@@ -67,7 +72,8 @@ typedef enum {
   FP_ERR_CUDA = 6,          /* a CUDA runtime call or launch failed              */
   FP_ERR_TIMEOUT = 7,       /* device: a pipeline wait ran out of time           */
   FP_ERR_DEVICE_CHECK = 8,  /* device: an argument failed an on-device check     */
-  FP_ERR_UNSUPPORTED = 9    /* the current device is not sm_100                  */
+  FP_ERR_UNSUPPORTED = 9,   /* the current device is not sm_100                  */
+  FP_ERR_ALIGN = 10         /* a data pointer is not aligned as required         */
 } fp_status;
 
 typedef enum { FP_BF16 = 0, FP_F32 = 1 } fp_dtype;
@@ -76,7 +82,7 @@ typedef struct {
   int batch;       /* Bt                                    */
   int n_q_heads;   /* Hq                                    */
   int n_kv_heads;  /* Hkv, divides Hq (grouped-query heads) */
-  int seq_len;     /* N, a multiple of block_size           */
+  int seq_len;     /* N >= 1; need not be a multiple of B   */
   int head_dim;    /* d                                     */
   int block_size;  /* B                                     */
   fp_dtype dtype;  /* element type of q, k, v and out       */

@@ -158,6 +158,52 @@ def test_workspace_checks(L):
                              None, FAKE, need - 256, None) == 5
 
 
+def test_misaligned_pointers_rejected(L):
+    """q, k, v, out, qbar and kbar need 16-byte alignment, the other arrays
+    their element size: a misaligned pointer returns FP_ERR_ALIGN before any
+    device call; an aligned set gets past the check (to the device check,
+    which fails without a GPU, or to the workspace check)."""
+    ALIGN = ops.STATUS_CODES["FP_ERR_ALIGN"]
+    s = shape()
+    p = ops.make_params(0.9, 0.1, 0, 0)
+    P = ctypes.c_void_p
+    est = [FAKE] * 9
+    for i, off in [(0, 8), (1, 2), (2, 4), (3, 12), (4, 2), (5, 1), (6, 2), (7, 3), (8, 2)]:
+        args = list(est)
+        args[i] = FAKE + off
+        assert L.fp_estimate(ctypes.byref(s), *args, FAKE, 1 << 40, None) == ALIGN, (i, off)
+    # 4-byte aligned fp32 arrays (map, est_last, ..., slash) pass the check
+    args = est[:4] + [FAKE + 4] * 5
+    assert L.fp_estimate(ctypes.byref(s), *args, FAKE, 1 << 40, None) != ALIGN
+    assert L.fp_pattern(ctypes.byref(s), ctypes.byref(p), FAKE + 2, FAKE, FAKE, FAKE,
+                        None) == ALIGN
+    assert L.fp_select(ctypes.byref(s), ctypes.byref(p), FAKE, FAKE + 2, FAKE, FAKE, FAKE, FAKE,
+                       FAKE, 1 << 40, None) == ALIGN
+    assert L.fp_select_noalloc(ctypes.byref(s), ctypes.byref(p), FAKE, FAKE, FAKE, FAKE, FAKE,
+                               FAKE + 1, None) == ALIGN
+    for qkvo in range(4):
+        a = [FAKE] * 4
+        a[qkvo] += 8
+        assert L.fp_sparse_attn(ctypes.byref(s), a[0], a[1], a[2], FAKE, FAKE, a[3], None, None,
+                                0, None) == ALIGN
+        assert L.fp_dense_attn(ctypes.byref(s), *a, None, None) == ALIGN
+        assert L.fp_prefill_attn(ctypes.byref(s), ctypes.byref(p), *a, None, None, FAKE,
+                                 1 << 40, None) == ALIGN
+    assert L.fp_sparse_attn(ctypes.byref(s), FAKE, FAKE, FAKE, FAKE + 2, FAKE, FAKE, None, None,
+                            0, None) == ALIGN
+    assert L.fp_dense_attn(ctypes.byref(s), FAKE, FAKE, FAKE, FAKE, P(FAKE + 2), None) == ALIGN
+    assert L.fp_prefill_attn(ctypes.byref(s), ctypes.byref(p), FAKE, FAKE, FAKE, FAKE, None,
+                             P(FAKE + 4), FAKE, 1 << 40, None) == ALIGN
+    lens = (ctypes.c_int32 * 1)(1024)
+    assert L.fp_prefill_attn_varlen(ctypes.byref(s), ctypes.byref(p), 1, lens, P(FAKE + 8),
+                                    P(FAKE), P(FAKE), P(FAKE), None, None, P(FAKE), 1 << 40,
+                                    None) == ALIGN
+    # aligned: past the alignment check
+    assert L.fp_prefill_attn(ctypes.byref(s), ctypes.byref(p), FAKE, FAKE, FAKE, FAKE,
+                             P(FAKE + 4), P(FAKE + 8), FAKE, 16, None) == \
+        ops.STATUS_CODES["FP_ERR_WORKSPACE"]
+
+
 def test_bf16_attention_shape_limits(L):
     # the tensor-core path takes d == 128 (B 64 or 128); fp32 takes all four
     for bs, d in [(128, 64), (64, 64)]:
