@@ -7,9 +7,12 @@
 // attention sums of the same last block.
 //
 // Kernels (all reductions in a fixed order, so results are reproducible):
-//   pool_kernel          mean of each B-token block of q and k (HBM stream)
-//   map_logits_kernel    scaled qbar.kbar^T for the causal block pairs
+//   pool_kernel          mean of each B-token block of q and k (HBM stream);
+//                        for k also its tf32 halves
+//   (map_tc.cu)          scaled qbar.kbar^T for the causal block pairs, on the
+//                        tensor cores
 //   map_softmax_kernel   in-place row softmax of the packed map, + est_last
+//   map_last_softmax_kernel  the same for the last row alone
 //   last_pass1_kernel    per (head, key block): row max / sum of exp of the
 //                        last query block's logits (online-softmax partials)
 //   last_lse_kernel      combine partials -> log-sum-exp of each last-block row
@@ -22,6 +25,8 @@
 // selection of vertical-slash heads, so the whole-path call runs them after
 // the pattern test, for those heads alone.
 #include <math.h>
+
+#include <algorithm>
 
 #include "fp_internal.cuh"
 
@@ -59,11 +64,15 @@ __device__ __forceinline__ void ld8(const __nv_bfloat16 *p, float (&x)[8]) {
 // grid (blocks, heads, Bt), 256 threads.  x [Bt, heads, N, d] -> out [Bt, heads,
 // nb, d], blocks blk0 .. blk0 + gridDim.x - 1; a partial last block is the
 // mean of its real tokens.  With `qa_only` (a pattern array, or null), heads
-// whose pattern is not query-aware are skipped.
+// whose pattern is not query-aware are skipped.  With `hi_out` / `lo_out`
+// (both or neither), each mean is also written split into its tf32 high half
+// and the fp32 rest (the operands of the tensor-core map).
 template <class T>
 __global__ void __launch_bounds__(256) pool_kernel(const T *__restrict__ x, float *__restrict__ out,
                                                    int n, int d, int bs, int nb, int blk0,
-                                                   const int32_t *__restrict__ qa_only) {
+                                                   const int32_t *__restrict__ qa_only,
+                                                   float *__restrict__ hi_out = nullptr,
+                                                   float *__restrict__ lo_out = nullptr) {
   __shared__ float part[32][128];
   const int blk = blk0 + int(blockIdx.x), head = blockIdx.y, b = blockIdx.z;
   const int heads = gridDim.y;
@@ -86,104 +95,18 @@ __global__ void __launch_bounds__(256) pool_kernel(const T *__restrict__ x, floa
   if (threadIdx.x < d) {
     float s = 0.f;
     for (int r = 0; r < rows_per_it; ++r) s += part[r][threadIdx.x];
-    out[((size_t(b) * heads + head) * nb + blk) * d + threadIdx.x] = s / float(rows);
+    const size_t o = ((size_t(b) * heads + head) * nb + blk) * d + threadIdx.x;
+    const float mean = s / float(rows);
+    out[o] = mean;
+    if (hi_out) {
+      const float hi = tf32_hi(mean);
+      hi_out[o] = hi;
+      lo_out[o] = mean - hi;
+    }
   }
 }
 
 // ------------------------------------------------------------ block map --
-// grid (tiles, tiles, Bt*Hq), 256 threads; a 128x128 tile of the nb x nb
-// logit matrix of one q head (tiles above the diagonal exit at once).  Each
-// thread accumulates an 8x8 register block (rows ty*4+{0..3} and 64+ty*4+..,
-// columns likewise) with one fp32 fused multiply-add per element of d, in
-// order.  d is taken in slices of kMapK through two shared-memory buffers:
-// the next slice's loads are issued before the current slice's products.
-constexpr int kMapK = 16;
-__global__ void __launch_bounds__(256, 2) map_logits_kernel(const float *__restrict__ qbar,
-                                                         const float *__restrict__ kbar,
-                                                         float *__restrict__ map, int hq, int g,
-                                                         int nb, int d, float scale,
-                                                         const int32_t *__restrict__ qa_only) {
-  const int ti = blockIdx.x, tj = blockIdx.y;
-  if (tj > ti) return;
-  const int bh = blockIdx.z, b = bh / hq, h = bh % hq, kv = h / g;
-  if (qa_only && qa_only[bh] != FP_PATTERN_QA) return;
-  const int hkv = hq / g;
-  __shared__ __align__(16) float As[2][kMapK][128];
-  __shared__ __align__(16) float Bs[2][kMapK][128];
-  const float *qa = qbar + (size_t(b) * hq + h) * nb * d;
-  const float *kb = kbar + (size_t(b) * hkv + kv) * nb * d;
-  const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
-  // loader: thread -> rows lr and lr + 64, 4 consecutive k of the slice
-  const int lr = threadIdx.x / 4, lk = (threadIdx.x % 4) * 4;
-  float4 na[2], nbv[2];
-  auto load = [&](int k0) {
-#pragma unroll
-    for (int i = 0; i < 2; ++i) {
-      const int gi = ti * 128 + lr + 64 * i, gj = tj * 128 + lr + 64 * i;
-      na[i] = gi < nb ? *reinterpret_cast<const float4 *>(qa + size_t(gi) * d + k0 + lk)
-                      : make_float4(0.f, 0.f, 0.f, 0.f);
-      nbv[i] = gj < nb ? *reinterpret_cast<const float4 *>(kb + size_t(gj) * d + k0 + lk)
-                       : make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-  };
-  auto store = [&](int buf) {
-#pragma unroll
-    for (int i = 0; i < 2; ++i) {
-      const int r = lr + 64 * i;
-      As[buf][lk + 0][r] = na[i].x;
-      As[buf][lk + 1][r] = na[i].y;
-      As[buf][lk + 2][r] = na[i].z;
-      As[buf][lk + 3][r] = na[i].w;
-      Bs[buf][lk + 0][r] = nbv[i].x;
-      Bs[buf][lk + 1][r] = nbv[i].y;
-      Bs[buf][lk + 2][r] = nbv[i].z;
-      Bs[buf][lk + 3][r] = nbv[i].w;
-    }
-  };
-  float acc[8][8];
-#pragma unroll
-  for (int u = 0; u < 8; ++u)
-#pragma unroll
-    for (int w = 0; w < 8; ++w) acc[u][w] = 0.f;
-  load(0);
-  store(0);
-  __syncthreads();
-  int buf = 0;
-  for (int k0 = 0; k0 < d; k0 += kMapK) {
-    const bool more = k0 + kMapK < d;
-    if (more) load(k0 + kMapK);
-#pragma unroll
-    for (int k = 0; k < kMapK; ++k) {
-      const float4 a0 = *reinterpret_cast<const float4 *>(&As[buf][k][ty * 4]);
-      const float4 a1 = *reinterpret_cast<const float4 *>(&As[buf][k][64 + ty * 4]);
-      const float4 b0 = *reinterpret_cast<const float4 *>(&Bs[buf][k][tx * 4]);
-      const float4 b1 = *reinterpret_cast<const float4 *>(&Bs[buf][k][64 + tx * 4]);
-      const float a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-      const float bb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
-#pragma unroll
-      for (int u = 0; u < 8; ++u)
-#pragma unroll
-        for (int w = 0; w < 8; ++w) acc[u][w] = fmaf(a[u], bb[w], acc[u][w]);
-    }
-    if (more) {
-      store(buf ^ 1);  // the other buffer: its last readers passed the barrier below
-      __syncthreads();
-      buf ^= 1;
-    }
-  }
-  float *m = map + (size_t(b) * hq + h) * (size_t(nb) * (nb + 1) / 2);
-#pragma unroll
-  for (int u = 0; u < 8; ++u) {
-    const int i = ti * 128 + (u < 4 ? ty * 4 + u : 64 + ty * 4 + u - 4);
-    if (i >= nb) continue;
-#pragma unroll
-    for (int w = 0; w < 8; ++w) {
-      const int j = tj * 128 + (w < 4 ? tx * 4 + w : 64 + tx * 4 + w - 4);
-      if (j <= i) m[size_t(i) * (i + 1) / 2 + j] = acc[u][w] * scale;
-    }
-  }
-}
-
 // Softmax of one map row in place (one warp; the same steps for every row,
 // whichever kernel runs them); the last row also goes to est_last.
 __device__ __forceinline__ void map_row_softmax(float *r, int len, float *est_last_row,
@@ -219,46 +142,16 @@ __global__ void __launch_bounds__(256) map_softmax_kernel(float *__restrict__ ma
   map_row_softmax(r, i + 1, i == nb - 1 ? est_last + bh * nb : nullptr, lane);
 }
 
-// The last row of the map alone (the estimate a-hat that the pattern test
-// needs), for every head: grid (Hq, Bt), 1024 threads (a key each, up to 4 at
-// nb = 4096).  Logit j is the same fmaf chain over d, in order, times scale,
-// that map_logits_kernel forms, and the softmax is map_row_softmax, so the
-// row is bitwise the full map's.
-__global__ void __launch_bounds__(1024) map_last_row_kernel(const float *__restrict__ qbar,
-                                                           const float *__restrict__ kbar,
-                                                           float *__restrict__ map,
-                                                           float *__restrict__ est_last, int hq,
-                                                           int g, int nb, int d, float scale) {
-  const int h = blockIdx.x, b = blockIdx.y, kv = h / g, hkv = hq / g;
-  const size_t bh = size_t(b) * hq + h;
-  __shared__ __align__(16) float qs[128];
-  const float *qa = qbar + (bh * nb + (nb - 1)) * d;
-  const float *kb = kbar + (size_t(b) * hkv + kv) * nb * d;
+// The softmax of the map's last row alone (the estimate a-hat that the
+// pattern test needs; its logits from launch_map_logits_tc with last_only),
+// for every head: grid (Bt*Hq), one warp.  The same map_row_softmax as every
+// row of map_softmax_kernel, so the row is bitwise the full map's.
+__global__ void __launch_bounds__(32) map_last_softmax_kernel(float *__restrict__ map,
+                                                              float *__restrict__ est_last,
+                                                              int nb) {
+  const size_t bh = blockIdx.x;
   float *r = map + bh * (size_t(nb) * (nb + 1) / 2) + size_t(nb - 1) * nb / 2;
-  if (threadIdx.x < d) qs[threadIdx.x] = qa[threadIdx.x];
-  __syncthreads();
-  for (int j = threadIdx.x; j < nb; j += 1024) {
-    // k-bar row j in chunks of 8 float4 loads issued together; the fmaf
-    // chain itself runs over d in order
-    const float4 *kr = reinterpret_cast<const float4 *>(kb + size_t(j) * d);
-    float acc = 0.f;
-    for (int c = 0; c < d / 4; c += 8) {
-      float4 t[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) t[u] = kr[c + u];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const float *x = &qs[4 * (c + u)];
-        acc = fmaf(x[0], t[u].x, acc);
-        acc = fmaf(x[1], t[u].y, acc);
-        acc = fmaf(x[2], t[u].z, acc);
-        acc = fmaf(x[3], t[u].w, acc);
-      }
-    }
-    r[j] = acc * scale;
-  }
-  __syncthreads();
-  if (threadIdx.x < 32) map_row_softmax(r, nb, est_last + bh * nb, threadIdx.x);
+  map_row_softmax(r, nb, est_last + bh * nb, threadIdx.x);
 }
 
 // ---------------------------------------------------- last query block --
@@ -518,16 +411,16 @@ cudaError_t run_last_lines(const Dims &Dm, const T *q, const T *k, float *vert, 
   return cudaGetLastError();
 }
 
-// Q pooling and the block map; with `qa_only`, for query-aware heads only.
+// Q pooling and the block map (logits on the tensor cores, then the row
+// softmax); with `qa_only`, for query-aware heads only.
 template <class T>
-cudaError_t run_map(const Dims &Dm, const T *q, float *qbar, const float *kbar, float *map,
-                    float *est_last, const int32_t *qa_only, cudaStream_t st) {
+cudaError_t run_map(const Dims &Dm, const T *q, float *qbar, const float *kbar_hi,
+                    const float *kbar_lo, float *map, float *est_last, const int32_t *qa_only,
+                    cudaStream_t st) {
   pool_kernel<T><<<dim3(Dm.nb, Dm.hq, Dm.bt), 256, 0, st>>>(q, qbar, Dm.n, Dm.d, Dm.bs, Dm.nb,
                                                              0, qa_only);
-  const int tiles = (Dm.nb + 127) / 128;
-  const float scale = 1.f / sqrtf(float(Dm.d));
-  map_logits_kernel<<<dim3(tiles, tiles, Dm.bt * Dm.hq), 256, 0, st>>>(
-      qbar, kbar, map, Dm.hq, Dm.g, Dm.nb, Dm.d, scale, qa_only);
+  cudaError_t e = launch_map_logits_tc(Dm, qbar, kbar_hi, kbar_lo, map, qa_only, false, st);
+  if (e != cudaSuccess) return e;
   const long long rows = (long long)Dm.bt * Dm.hq * Dm.nb;
   map_softmax_kernel<<<unsigned((rows + 7) / 8), 256, 0, st>>>(map, est_last, rows, Dm.nb,
                                                                qa_only);
@@ -569,13 +462,28 @@ cudaError_t run_lines(const Dims &Dm, const T *q, const T *k, float *vert, float
   return run_last_lines<64, 64, T>(Dm, q, k, vert, slash, vs_only, ws, st);
 }
 
+// The pooled keys' tf32 halves, carved from the start of a workspace (the
+// staged estimate: they are dead before the last-block passes reuse it).
+struct Split {
+  float *hi, *lo;
+};
+Split carve_split(const Dims &Dm, void *ws) {
+  Carver c{static_cast<char *>(ws), 0};
+  const size_t n = size_t(Dm.bt) * Dm.hkv * Dm.nb * Dm.d;
+  Split sp;
+  sp.hi = c.take<float>(n);
+  sp.lo = c.take<float>(n);
+  return sp;
+}
+
 template <class T>
 cudaError_t run_estimate(const Dims &Dm, const T *q, const T *k, float *qbar, float *kbar,
                          float *map, float *est_last, float *true_last, float *vert,
                          float *slash, void *ws, cudaStream_t st) {
+  const Split sp = carve_split(Dm, ws);
   pool_kernel<T><<<dim3(Dm.nb, Dm.hkv, Dm.bt), 256, 0, st>>>(k, kbar, Dm.n, Dm.d, Dm.bs, Dm.nb,
-                                                              0, nullptr);
-  cudaError_t e = run_map<T>(Dm, q, qbar, kbar, map, est_last, nullptr, st);
+                                                              0, nullptr, sp.hi, sp.lo);
+  cudaError_t e = run_map<T>(Dm, q, qbar, sp.hi, sp.lo, map, est_last, nullptr, st);
   if (e != cudaSuccess) return e;
   e = run_true_last<T>(Dm, q, k, true_last, ws, st);
   if (e != cudaSuccess) return e;
@@ -587,16 +495,16 @@ cudaError_t run_estimate(const Dims &Dm, const T *q, const T *k, float *qbar, fl
 // true last-block distribution), and nothing else.
 template <class T>
 cudaError_t run_decision(const Dims &Dm, const T *q, const T *k, float *qbar, float *kbar,
-                         float *map, float *est_last, float *true_last, void *ws,
-                         cudaStream_t st) {
+                         float *kbar_hi, float *kbar_lo, float *map, float *est_last,
+                         float *true_last, void *ws, cudaStream_t st) {
   pool_kernel<T><<<dim3(Dm.nb, Dm.hkv, Dm.bt), 256, 0, st>>>(k, kbar, Dm.n, Dm.d, Dm.bs, Dm.nb,
-                                                              0, nullptr);
+                                                              0, nullptr, kbar_hi, kbar_lo);
   pool_kernel<T><<<dim3(1, Dm.hq, Dm.bt), 256, 0, st>>>(q, qbar, Dm.n, Dm.d, Dm.bs, Dm.nb,
                                                          Dm.nb - 1, nullptr);
-  map_last_row_kernel<<<dim3(Dm.hq, Dm.bt), 1024, 0, st>>>(qbar, kbar, map, est_last, Dm.hq,
-                                                           Dm.g, Dm.nb, Dm.d,
-                                                           1.f / sqrtf(float(Dm.d)));
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_map_logits_tc(Dm, qbar, kbar_hi, kbar_lo, map, nullptr, true, st);
+  if (e != cudaSuccess) return e;
+  map_last_softmax_kernel<<<unsigned(Dm.bt * Dm.hq), 32, 0, st>>>(map, est_last, Dm.nb);
+  e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   return run_true_last<T>(Dm, q, k, true_last, ws, st);
 }
@@ -604,19 +512,21 @@ cudaError_t run_decision(const Dims &Dm, const T *q, const T *k, float *qbar, fl
 }  // namespace
 
 size_t estimate_ws_bytes(const Dims &D) {
-  if (last_block_tc_supported(D)) return last_block_tc_ws_bytes(D);
-  return carve_core(D, nullptr).bytes;
+  const size_t passes =
+      last_block_tc_supported(D) ? last_block_tc_ws_bytes(D) : carve_core(D, nullptr).bytes;
+  return std::max(passes, map_split_bytes(D));
 }
 
 cudaError_t launch_estimate_decision(const Dims &D, const void *q, const void *k, float *qbar,
-                                     float *kbar, float *map, float *est_last,
-                                     float *true_last, void *ws, cudaStream_t st) {
+                                     float *kbar, float *kbar_hi, float *kbar_lo, float *map,
+                                     float *est_last, float *true_last, void *ws,
+                                     cudaStream_t st) {
   if (D.dtype == FP_F32)
     return run_decision<float>(D, static_cast<const float *>(q), static_cast<const float *>(k),
-                               qbar, kbar, map, est_last, true_last, ws, st);
+                               qbar, kbar, kbar_hi, kbar_lo, map, est_last, true_last, ws, st);
   return run_decision<__nv_bfloat16>(D, static_cast<const __nv_bfloat16 *>(q),
-                                     static_cast<const __nv_bfloat16 *>(k), qbar, kbar, map,
-                                     est_last, true_last, ws, st);
+                                     static_cast<const __nv_bfloat16 *>(k), qbar, kbar, kbar_hi,
+                                     kbar_lo, map, est_last, true_last, ws, st);
 }
 
 cudaError_t launch_estimate_lines_vs(const Dims &D, const void *q, const void *k, float *vert,
@@ -630,14 +540,14 @@ cudaError_t launch_estimate_lines_vs(const Dims &D, const void *q, const void *k
                                   ws, st);
 }
 
-cudaError_t launch_estimate_map_qa(const Dims &D, const void *q, float *qbar, const float *kbar,
-                                   float *map, float *est_last, const int32_t *pattern,
-                                   cudaStream_t st) {
+cudaError_t launch_estimate_map_qa(const Dims &D, const void *q, float *qbar,
+                                   const float *kbar_hi, const float *kbar_lo, float *map,
+                                   float *est_last, const int32_t *pattern, cudaStream_t st) {
   if (D.dtype == FP_F32)
-    return run_map<float>(D, static_cast<const float *>(q), qbar, kbar, map, est_last, pattern,
-                          st);
-  return run_map<__nv_bfloat16>(D, static_cast<const __nv_bfloat16 *>(q), qbar, kbar, map,
-                                est_last, pattern, st);
+    return run_map<float>(D, static_cast<const float *>(q), qbar, kbar_hi, kbar_lo, map,
+                          est_last, pattern, st);
+  return run_map<__nv_bfloat16>(D, static_cast<const __nv_bfloat16 *>(q), qbar, kbar_hi,
+                                kbar_lo, map, est_last, pattern, st);
 }
 
 cudaError_t launch_estimate(const Dims &D, const void *q, const void *k, float *qbar,

@@ -162,7 +162,7 @@ __global__ void watchdog_selftest_kernel(int *status, unsigned long long limit_n
 
 // Intermediates of the whole path, carved from a workspace.
 struct Prefill {
-  float *qbar, *kbar, *map, *est_last, *true_last, *vert, *slash, *djs;
+  float *qbar, *kbar, *kbar_hi, *kbar_lo, *map, *est_last, *true_last, *vert, *slash, *djs;
   int32_t *pattern, *counts, *indices;
   void *stage_ws;
 };
@@ -217,6 +217,8 @@ size_t carve_prefill(const Dims &D, void *ws, Prefill *P) {
   const size_t heads = size_t(D.bt) * D.hq;
   P->qbar = c.take<float>(heads * D.nb * D.d);
   P->kbar = c.take<float>(size_t(D.bt) * D.hkv * D.nb * D.d);
+  P->kbar_hi = c.take<float>(size_t(D.bt) * D.hkv * D.nb * D.d);
+  P->kbar_lo = c.take<float>(size_t(D.bt) * D.hkv * D.nb * D.d);
   P->map = c.take<float>(heads * D.t_pairs);
   P->est_last = c.take<float>(heads * D.nb);
   P->true_last = c.take<float>(heads * D.nb);
@@ -291,12 +293,13 @@ fp_status run_attn(const Dims &D, const void *q, const void *k, const void *v,
 fp_status run_prefill(const Dims &D, const fp_params &p, const void *q, const void *k,
                       const void *v, void *out, float *lse, int64_t *stats, const Prefill &P,
                       cudaStream_t st, cudaEvent_t v_ready = nullptr) {
-  cudaError_t e = launch_estimate_decision(D, q, k, P.qbar, P.kbar, P.map, P.est_last,
-                                           P.true_last, P.stage_ws, st);
+  cudaError_t e = launch_estimate_decision(D, q, k, P.qbar, P.kbar, P.kbar_hi, P.kbar_lo, P.map,
+                                           P.est_last, P.true_last, P.stage_ws, st);
   if (e != cudaSuccess) return FP_ERR_CUDA;
   e = launch_pattern(D, p.tau, P.est_last, P.true_last, P.djs, P.pattern, st);
   if (e != cudaSuccess) return FP_ERR_CUDA;
-  e = launch_estimate_map_qa(D, q, P.qbar, P.kbar, P.map, P.est_last, P.pattern, st);
+  e = launch_estimate_map_qa(D, q, P.qbar, P.kbar_hi, P.kbar_lo, P.map, P.est_last, P.pattern,
+                             st);
   if (e != cudaSuccess) return FP_ERR_CUDA;
   e = launch_estimate_lines_vs(D, q, k, P.vert, P.slash, P.pattern, P.stage_ws, st);
   if (e != cudaSuccess) return FP_ERR_CUDA;

@@ -45,15 +45,26 @@ cudaError_t launch_estimate(const Dims &D, const void *q, const void *k, float *
                             float *kbar, float *map, float *est_last, float *true_last,
                             float *vert, float *slash, void *ws, cudaStream_t st);
 // Pattern-aware parts of launch_estimate (fp_prefill_attn): everything the
-// pattern test reads, for every head (K pooled, Q pooled over the last block,
-// the map's last row, true_last) ...
+// pattern test reads, for every head (K pooled, with its tf32 halves in
+// kbar_hi / kbar_lo, map_split_bytes() / 2 each; Q pooled over the last block;
+// the map's last row; true_last) ...
 cudaError_t launch_estimate_decision(const Dims &D, const void *q, const void *k, float *qbar,
-                                     float *kbar, float *map, float *est_last,
-                                     float *true_last, void *ws, cudaStream_t st);
+                                     float *kbar, float *kbar_hi, float *kbar_lo, float *map,
+                                     float *est_last, float *true_last, void *ws,
+                                     cudaStream_t st);
 // ... then Q pooling and the map for the query-aware heads of `pattern` ...
-cudaError_t launch_estimate_map_qa(const Dims &D, const void *q, float *qbar, const float *kbar,
-                                   float *map, float *est_last, const int32_t *pattern,
-                                   cudaStream_t st);
+cudaError_t launch_estimate_map_qa(const Dims &D, const void *q, float *qbar,
+                                   const float *kbar_hi, const float *kbar_lo, float *map,
+                                   float *est_last, const int32_t *pattern, cudaStream_t st);
+
+// The map's logits on the tensor cores (map_tc.cu), 3xTF32 products of the
+// pooled vectors: for every causal block pair (or, with `last_only`, the last
+// row only) of every head (or the query-aware heads of `qa_only`).
+// kbar_hi / kbar_lo: the pooled keys split as tf32_hi(x) and x - tf32_hi(x).
+size_t map_split_bytes(const Dims &D);  // both halves, with carving slack
+cudaError_t launch_map_logits_tc(const Dims &D, const float *qbar, const float *kbar_hi,
+                                 const float *kbar_lo, float *map, const int32_t *qa_only,
+                                 bool last_only, cudaStream_t st);
 // ... and vert and slash for its vertical-slash heads (on the workspace the
 // decision part left).
 cudaError_t launch_estimate_lines_vs(const Dims &D, const void *q, const void *k, float *vert,
@@ -108,6 +119,12 @@ cudaError_t launch_attn_bf16(const Dims &D, const void *q, const void *k, const 
 
 __device__ __forceinline__ void report(int *status, int code) {
   if (status) atomicCAS(status, 0, code);
+}
+
+// x with its low 13 mantissa bits cleared: exact in tf32, the high half of a
+// 3xTF32 split (x - tf32_hi(x) is exact in fp32).
+__device__ __forceinline__ float tf32_hi(float x) {
+  return __uint_as_float(__float_as_uint(x) & 0xFFFFE000u);
 }
 
 __device__ __forceinline__ uint64_t globaltimer_ns() {
