@@ -245,25 +245,36 @@ __global__ void __launch_bounds__(kThreads, 1) last_block_tc_kernel(
             if (c > r) x[c] = -INFINITY;
         }
         // 8 independent chains for the max and the sums (one set per 64-key
-        // half), then trees
-        float mx[8], sa[8], sb[8];
+        // half), then trees.  Two scores an instruction: a three-input max,
+        // and the exponent arguments and the sums as two-lane FMAs and adds
+        // (sum chain k, the keys c = k mod 8 in order, is lane k % 2 of pair
+        // k / 2), so every lane does what the scalar chains would.
+        float mx[8];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          mx[k] = x[k];
-          sa[k] = 0.f;
-          sb[k] = 0.f;
-        }
+        for (int k = 0; k < 8; ++k) mx[k] = x[k];
 #pragma unroll
-        for (int c = 8; c < BS; ++c) mx[c % 8] = fmaxf(mx[c % 8], x[c]);
+        for (int c = 8; c < BS; c += 2) mx[(c / 2) % 8] = max3f(mx[(c / 2) % 8], x[c], x[c + 1]);
         const float tmax = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
                                  fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
         const float mnew = fmaxf(m, tmax * sl2);
+        const float2 sc2 = make_float2(sl2, sl2), nm2 = make_float2(-mnew, -mnew);
+        float2 sa[4], sb[4];
 #pragma unroll
-        for (int c = 0; c < BS / 2; ++c) sa[c % 8] += ex2(fmaf(x[c], sl2, -mnew));
+        for (int k = 0; k < 4; ++k) sa[k] = sb[k] = make_float2(0.f, 0.f);
 #pragma unroll
-        for (int c = BS / 2; c < BS; ++c) sb[c % 8] += ex2(fmaf(x[c], sl2, -mnew));
-        const float s0 = ((sa[0] + sa[1]) + (sa[2] + sa[3])) + ((sa[4] + sa[5]) + (sa[6] + sa[7]));
-        const float s1 = ((sb[0] + sb[1]) + (sb[2] + sb[3])) + ((sb[4] + sb[5]) + (sb[6] + sb[7]));
+        for (int c = 0; c < BS / 2; c += 2) {
+          const float2 e = ffma2(make_float2(x[c], x[c + 1]), sc2, nm2);
+          sa[(c % 8) / 2] = fadd2(sa[(c % 8) / 2], make_float2(ex2(e.x), ex2(e.y)));
+        }
+#pragma unroll
+        for (int c = BS / 2; c < BS; c += 2) {
+          const float2 e = ffma2(make_float2(x[c], x[c + 1]), sc2, nm2);
+          sb[(c % 8) / 2] = fadd2(sb[(c % 8) / 2], make_float2(ex2(e.x), ex2(e.y)));
+        }
+        const float s0 = ((sa[0].x + sa[0].y) + (sa[1].x + sa[1].y)) +
+                         ((sa[2].x + sa[2].y) + (sa[3].x + sa[3].y));
+        const float s1 = ((sb[0].x + sb[0].y) + (sb[1].x + sb[1].y)) +
+                         ((sb[2].x + sb[2].y) + (sb[3].x + sb[3].y));
         l = l * ex2(m - mnew) + (s0 + s1);
         m = mnew;
         // this tile's mass for row r is (s0 + s1) * 2^(mnew - lse2[r])
