@@ -728,15 +728,21 @@ def test_full_size_128k_qa_capped_sampled():
 
 def test_maximum_block_count_sampled():
     """nb = 4096, the largest block count the library takes (N = 262144 at
-    block 64, bf16, two query heads on one kv head): one head's selection
-    against the oracle (a map of 8.4 M entries), the allocation-free
-    selection at this size, and sampled attention rows."""
+    block 64, bf16, two query heads on one kv head): the estimate and one
+    head's selection against the oracle (a map of 8.4 M entries), the
+    allocation-free selection at this size, and sampled attention rows."""
     w = synth.WORKLOADS["glm9b_n65536_b64"].replace(seq_len=262144, n_q_heads=2, n_kv_heads=1)
     assert w.n_blocks == 4096
     inp = synth.make_inputs(w)
     d = {x: inp[x].to(DEV) for x in ("q", "k", "v")}
     res = _pipeline(w, d)
     assert ops.fp_last_device_status() == 0
+    # the whole estimate at this size (32 row tiles of 128 query blocks in
+    # the tensor-core map) against the oracle
+    want = oracle.estimate(inp["q"], inp["k"], w.block_size)
+    for key in ("map", "est_last", "true_last", "vert", "slash"):
+        np.testing.assert_allclose(_np(res["est"][key]), want[key], rtol=1e-4, atol=1e-7,
+                                   err_msg=key)
     h = 1
     oc, oi = oracle.select(res["pattern"][:, h:h + 1].cpu().numpy(),
                            _np(res["est"]["map"][:, h:h + 1]), _np(res["est"]["vert"][:, h:h + 1]),
