@@ -17,8 +17,10 @@ __device__ int g_fp_status;  // first device-side error since the last read
 
 int *device_status_ptr() {
   static int *ptrs[64] = {nullptr};
+  static std::mutex mu;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
   if (!ptrs[dev]) {
     void *p = nullptr;
     if (cudaGetSymbolAddress(&p, g_fp_status) == cudaSuccess) ptrs[dev] = static_cast<int *>(p);

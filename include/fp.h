@@ -44,6 +44,11 @@
  *    fp_last_device_status().
  *  * No C++ exception crosses this ABI.  Calls on distinct streams with
  *    distinct workspaces may run from several host threads.
+ *  * The device-memory calls (all but fp_prefill_attn_host) launch only on
+ *    `stream` and do not synchronise, so they may be captured into a CUDA
+ *    graph; make one eager call on the device first (it caches the device's
+ *    status word and properties).  A replay reads the current contents of
+ *    the captured buffers.
  *  * Supported shapes: N >= 1 (any length), nb <= 4096, Hq % Hkv == 0,
  *    B in {64, 128}, d in {64, 128}.  The bf16 attention (tensor cores)
  *    needs d == 128; fp32 (the debug path, CUDA cores) takes every listed
