@@ -8,7 +8,8 @@
 // operand is split as x = hi + lo, hi = x with its low 13 mantissa bits
 // cleared (exact in tf32) and lo = x - hi (exact in fp32), and the product is
 // hi.hi + hi.lo + lo.hi accumulated in fp32 (the dropped lo.lo term and lo's
-// own tf32 rounding are below 2^-19 of |x| |y|).  The keys' halves come from
+// own tf32 rounding are below 2^-19 of |x| |y|, so a logit is off by at most
+// about 2^-19 of sum_k |qbar_k kbar_k| times the scale).  The keys' halves come from
 // the K pooling (pool_kernel writes them beside kbar); the queries' are formed
 // here on the way into TMEM.
 //
@@ -24,8 +25,11 @@
 // lo, 128-B swizzled, by TMA) and a 128 x 128 staging tile through which a
 // warp writes 128 consecutive floats of one map row.
 // Warps: 0-7 epilogue (thread = tile row = TMEM lane of its quarter, each
-// warp of a quarter taking half of the columns), 8 TMA producer, 9 MMA issuer.  Every wait is bounded; on expiry the kernel records
-// FP_ERR_TIMEOUT, raises a CTA abort flag, drains its loads and frees TMEM.
+// warp of a quarter taking half of the columns), 8 TMA producer, 9 MMA
+// issuer.  Every wait is bounded; on expiry the kernel records FP_ERR_TIMEOUT,
+// raises a CTA abort flag, drains its loads and frees TMEM.
+// The kernel is held by the key-tile stream (128 KB of hi and lo per 128 x 128
+// tile, from L2), not by the tensor pipe: at 128k the pipe is busy about 40 %.
 #include "fp_internal.cuh"
 
 namespace fpi {
