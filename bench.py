@@ -50,19 +50,33 @@ def kernel_traffic(source: str, workload: str):
 
     profiles/<name>_traffic.json holds {"source_sha256", "workload",
     "bytes_per_launch", ...}; the figure is used only while the kernel source
-    still hashes to the captured one (else None: the counters are stale).
+    and the device header it includes (csrc/fp_internal.cuh) still hash to the
+    captured ones (else None: the counters are stale).
     """
-    import hashlib
     name = os.path.splitext(os.path.basename(source))[0]
     rec_path = os.path.join(ROOT, "profiles", f"{name}_traffic.json")
-    src_path = os.path.join(ROOT, "dynamic_block_sparse_fp_b200", "csrc", source)
-    if not (os.path.exists(rec_path) and os.path.exists(src_path)):
+    if not os.path.exists(rec_path):
+        return None
+    sha = kernel_source_sha(source)
+    if sha is None:
         return None
     rec = json.load(open(rec_path))
-    sha = hashlib.sha256(open(src_path, "rb").read()).hexdigest()
     if rec.get("source_sha256") != sha or rec.get("workload") != workload:
         return None
     return rec.get("bytes_per_launch")
+
+
+def kernel_source_sha(source: str):
+    """sha256 over csrc/<source> followed by csrc/fp_internal.cuh."""
+    import hashlib
+    csrc = os.path.join(ROOT, "dynamic_block_sparse_fp_b200", "csrc")
+    h = hashlib.sha256()
+    for f in (source, "fp_internal.cuh"):
+        p = os.path.join(csrc, f)
+        if not os.path.exists(p):
+            return None
+        h.update(open(p, "rb").read())
+    return h.hexdigest()
 
 
 def load_peaks() -> dict:

@@ -11,10 +11,14 @@ import os
 import bench
 
 
+HEADER = "// device helpers v1\n"
+
+
 def _tree(tmp_path, src_text: str, rec: dict | None):
     csrc = tmp_path / "dynamic_block_sparse_fp_b200" / "csrc"
     csrc.mkdir(parents=True)
     (csrc / "k.cu").write_text(src_text)
+    (csrc / "fp_internal.cuh").write_text(HEADER)
     (tmp_path / "profiles").mkdir()
     if rec is not None:
         (tmp_path / "profiles" / "k_traffic.json").write_text(json.dumps(rec))
@@ -22,8 +26,8 @@ def _tree(tmp_path, src_text: str, rec: dict | None):
 
 
 def _rec(src_text: str, workload="w1", nbytes=1234):
-    return {"source_sha256": hashlib.sha256(src_text.encode()).hexdigest(),
-            "workload": workload, "bytes_per_launch": nbytes}
+    sha = hashlib.sha256((src_text + HEADER).encode()).hexdigest()
+    return {"source_sha256": sha, "workload": workload, "bytes_per_launch": nbytes}
 
 
 def test_traffic_used_only_for_the_captured_source_and_workload(tmp_path, monkeypatch):
@@ -32,7 +36,12 @@ def test_traffic_used_only_for_the_captured_source_and_workload(tmp_path, monkey
     monkeypatch.setattr(bench, "ROOT", str(root))
     assert bench.kernel_traffic("k.cu", "w1") == 1234
     assert bench.kernel_traffic("k.cu", "w2") is None          # another workload
-    (root / "dynamic_block_sparse_fp_b200" / "csrc" / "k.cu").write_text("// kernel v2\n")
+    csrc = root / "dynamic_block_sparse_fp_b200" / "csrc"
+    (csrc / "fp_internal.cuh").write_text("// device helpers v2\n")
+    assert bench.kernel_traffic("k.cu", "w1") is None          # the shared header changed
+    (csrc / "fp_internal.cuh").write_text(HEADER)
+    assert bench.kernel_traffic("k.cu", "w1") == 1234
+    (csrc / "k.cu").write_text("// kernel v2\n")
     assert bench.kernel_traffic("k.cu", "w1") is None          # the kernel changed
 
 
