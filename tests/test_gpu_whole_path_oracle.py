@@ -26,7 +26,7 @@ DEV = "cuda:0"
 # at tau 0.1), a ragged fp32 length at tau 0 (every head vertical-slash), bf16
 # Llama heads with tau in the widest gap between the heads' d_JS values (both
 # patterns) under both selection variants, and bf16 block 64 with a 512-token
-# cap, all vertical-slash and all query-aware (ragged)
+# cap, all vertical-slash and all query-aware (ragged); two batch entries
 CASES = {
     "f32_b64_flat_tokens": ("tiny_n1024", {}, 0, 0, None),
     "f32_b64_ragged_all_vs": ("tiny_n1024", dict(seq_len=1000), 0, 0, 0.0),
@@ -38,6 +38,8 @@ CASES = {
                                                         n_kv_heads=2, max_budget=512), 0, 0, 0.0),
     "bf16_b64_all_qa_capped": ("glm9b_n65536_b64", dict(seq_len=2048 + 40, n_q_heads=8,
                                                         n_kv_heads=2, max_budget=512), 0, 0, None),
+    "bf16_b128_batch2": ("llama8b_n8192", dict(batch=2, seq_len=2048 + 40, n_q_heads=8,
+                                               n_kv_heads=2), 0, 0, "split"),
 }
 
 
@@ -95,24 +97,26 @@ def test_whole_path_against_oracle_whole_path(name):
     gc, gi = counts.cpu().numpy(), indices.cpu().numpy()
     oc, oi = res["counts"], res["indices"]
     same = np.zeros(gc.shape, dtype=bool)
-    for h in range(w.n_q_heads):
-        for i in range(nb):
-            same[0, h, i] = gc[0, h, i] == oc[0, h, i] and np.array_equal(
-                gi[0, h, i, :gc[0, h, i]], oi[0, h, i, :oc[0, h, i]])
+    for b in range(w.batch):
+        for h in range(w.n_q_heads):
+            for i in range(nb):
+                same[b, h, i] = gc[b, h, i] == oc[b, h, i] and np.array_equal(
+                    gi[b, h, i, :gc[b, h, i]], oi[b, h, i, :oc[b, h, i]])
     assert same.mean() >= 0.95, f"lists agree on {same.mean():.3f} of the rows"
     # output and log-sum-exp on the sampled rows whose lists agree
     o_g, l_g = _np(out), _np(lse)
     tol, ltol = (2e-2, 2e-3) if bf16 else (1e-4, 1e-4)
     checked = 0
-    for h in heads:
-        for i in q_blocks:
-            if not same[0, h, i]:
-                continue
-            r0, r1 = i * w.block_size, min((i + 1) * w.block_size, w.seq_len)
-            o_o = res["out"][0, h, r0:r1]
-            l_o = res["lse"][0, h, r0:r1]
-            assert not np.isnan(o_o).any()
-            assert np.abs(o_g[0, h, r0:r1] - o_o).max() <= tol, (h, i)
-            assert np.abs(l_g[0, h, r0:r1] - l_o).max() <= ltol, (h, i)
-            checked += 1
-    assert checked >= len(heads) * len(q_blocks) // 2
+    for b in range(w.batch):
+        for h in heads:
+            for i in q_blocks:
+                if not same[b, h, i]:
+                    continue
+                r0, r1 = i * w.block_size, min((i + 1) * w.block_size, w.seq_len)
+                o_o = res["out"][b, h, r0:r1]
+                l_o = res["lse"][b, h, r0:r1]
+                assert not np.isnan(o_o).any()
+                assert np.abs(o_g[b, h, r0:r1] - o_o).max() <= tol, (b, h, i)
+                assert np.abs(l_g[b, h, r0:r1] - l_o).max() <= ltol, (b, h, i)
+                checked += 1
+    assert checked >= w.batch * len(heads) * len(q_blocks) // 2
