@@ -753,7 +753,7 @@ __global__ void __launch_bounds__(256) sel_flags_kernel(SelArgs a, uint8_t *__re
 
 // grid (ceil(nb/8), Hq, Bt), 256 threads: one warp per row, kEmitU groups of
 // 32 entries in flight.
-constexpr int kEmitU = 8;
+constexpr int kEmitU = 4;
 __global__ void __launch_bounds__(256) emit_rows_kernel(
     const int32_t *__restrict__ pattern, const float *__restrict__ map, int nb,
     const HeadSel *__restrict__ sel, const uint8_t *__restrict__ colflag,
