@@ -127,7 +127,8 @@ __device__ __forceinline__ void map_row_softmax(float *r, int len, float *est_la
   }
 }
 
-// One warp per map row; 8 rows per CTA.  `qa_only`: as for pool_kernel.
+// One warp per map row; 8 rows per CTA, every head's longest rows first (the
+// short rows fill the tail).  `qa_only`: as for pool_kernel.
 __global__ void __launch_bounds__(256) map_softmax_kernel(float *__restrict__ map,
                                                           float *__restrict__ est_last,
                                                           long long rows_total, int nb,
@@ -135,9 +136,10 @@ __global__ void __launch_bounds__(256) map_softmax_kernel(float *__restrict__ ma
   const long long row = (long long)blockIdx.x * 8 + threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
   if (row >= rows_total) return;
-  const long long bh = row / nb;
+  const long long heads = rows_total / nb;
+  const long long bh = row % heads;
   if (qa_only && qa_only[bh] != FP_PATTERN_QA) return;
-  const int i = int(row % nb);
+  const int i = nb - 1 - int(row / heads);
   float *r = map + bh * ((long long)nb * (nb + 1) / 2) + (long long)i * (i + 1) / 2;
   map_row_softmax(r, i + 1, i == nb - 1 ? est_last + bh * nb : nullptr, lane);
 }
