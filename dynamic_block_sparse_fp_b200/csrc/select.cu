@@ -106,7 +106,10 @@ constexpr int kShift1 = 23, kShift2 = 11;
 constexpr int kBins = kBins2;        // global histogram bins per list (levels 1, 2)
 constexpr int kCand = 1024;          // candidate list length per list slot
 constexpr int kHistAggMax = 8;
-constexpr int kSelCtasPerSm = 6;     // scanning CTAs per SM (over every list)
+// scanning CTAs per SM (over every list), per kernel: the first digit's
+// 256-bin histograms merge cheaply and gain from more CTAs, the second
+// digit's 4096-bin ones pay a merge per CTA (measured at 128k: 24 / 6 / 12)
+constexpr int kHist1CtasPerSm = 24, kHist2CtasPerSm = 6, kCompactCtasPerSm = 12;
 constexpr int kMaxCtaEntries = 32767;                   // 32767 * 2^17 < 2^32
 constexpr int kMaxCtaChunks = kMaxCtaEntries / kChunk;  // chunks a CTA may take
 constexpr int kRounds = 4;
@@ -1129,17 +1132,24 @@ cudaError_t launch_select(const Dims &D, float gamma, const SelectBudgets &bud,
   long long maxlen = a.n;
   if (bud.qa_mode == FP_QA_FLATTENED && D.t_pairs > maxlen) maxlen = D.t_pairs;
   const int max_chunks = int((maxlen + 3 + kChunk - 1) / kChunk);
-  // about kSelCtasPerSm CTAs per SM over all slots, each looping over chunks,
-  // and enough of them that no CTA takes more than kMaxCtaChunks
-  a.ctas = std::max(1, std::min(max_chunks, sm_count() * kSelCtasPerSm / slots));
-  a.ctas = std::max(a.ctas, (max_chunks + kMaxCtaChunks - 1) / kMaxCtaChunks);
-  const unsigned chunks = unsigned(a.ctas);
+  // about `per_sm` CTAs per SM over all slots, each looping over chunks, and
+  // enough of them that no CTA takes more than kMaxCtaChunks; every scanning
+  // kernel derives its CTAs per list from its own args (the decisions are
+  // integer sums, the same for any count)
+  auto with_ctas = [&](int per_sm) {
+    SelArgs x = a;
+    x.ctas = std::max(1, std::min(max_chunks, sm_count() * per_sm / slots));
+    x.ctas = std::max(x.ctas, (max_chunks + kMaxCtaChunks - 1) / kMaxCtaChunks);
+    return x;
+  };
+  const SelArgs a1 = with_ctas(kHist1CtasPerSm), a2 = with_ctas(kHist2CtasPerSm),
+                a3 = with_ctas(kCompactCtasPerSm);
   cudaFuncSetAttribute(sel_hist_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                        int(hist_smem<2>()));
-  sel_prep_kernel<<<slots, kSelThreads, 0, st>>>(a, cf, df);
-  sel_hist_kernel<1><<<dim3(chunks, slots), kSelThreads, hist_smem<1>(), st>>>(a);
-  sel_hist_kernel<2><<<dim3(chunks, slots), kSelThreads, hist_smem<2>(), st>>>(a);
-  sel_compact_kernel<<<dim3(chunks, slots), kSelThreads, 0, st>>>(a);
+  sel_prep_kernel<<<slots, kSelThreads, 0, st>>>(a1, cf, df);
+  sel_hist_kernel<1><<<dim3(unsigned(a1.ctas), slots), kSelThreads, hist_smem<1>(), st>>>(a1);
+  sel_hist_kernel<2><<<dim3(unsigned(a2.ctas), slots), kSelThreads, hist_smem<2>(), st>>>(a2);
+  sel_compact_kernel<<<dim3(unsigned(a3.ctas), slots), kSelThreads, 0, st>>>(a3);
   sel_flags_kernel<<<dim3((a.n + 256 * kFlagU - 1) / (256 * kFlagU), slots), 256, 0, st>>>(
       a, cf, df);
   emit_rows_kernel<<<dim3((D.nb + 7) / 8, D.hq, D.bt), 256, 0, st>>>(
