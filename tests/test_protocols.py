@@ -1,5 +1,5 @@
-"""CPU model checks of the mbarrier protocols of the two pipelined tensor-core
-kernels (csrc/attn_tc.cu and csrc/map_tc.cu).
+"""CPU model checks of the mbarrier protocols of the pipelined tensor-core
+kernels (csrc/attn_tc.cu, csrc/map_tc.cu and csrc/estimate_tc.cu).
 
 Each role of a kernel (TMA producer, MMA issuer, softmax or epilogue warps) is
 a Python generator that takes the kernel's waits, arrivals and buffer accesses
@@ -285,11 +285,99 @@ def test_map_protocol(ntile, nc, seed):
     run(roles, pipe, random.Random(seed * 1000 + ntile))
 
 
+# -------------------------------------------------------- estimate passes --
+# estimate_tc.cu: the last block's queries of two heads loaded once, key tiles
+# through a ring of 3, S double-buffered per head in TMEM (both heads' S of a
+# tile in one buffer index), four consumer warps per head; in the second pass
+# each head's warps exchange diagonal bins through shared memory between two
+# warpgroup barriers per tile.
+
+def estimate_roles(ntile, RING=3, heads=2, warps_per_head=4, line_pass=True, drop=None):
+    pipe = Pipe()
+    q_full = Bar("q_full", 1)
+    ring_full = [Bar(f"ring_full{r}", 1) for r in range(RING)]
+    ring_empty = [Bar(f"ring_empty{r}", 1) for r in range(RING)]
+    s_full = [Bar(f"s_full{b}", 1) for b in range(2)]
+    s_free = [Bar(f"s_free{b}", heads * warps_per_head) for b in range(2)]
+    wg = [Bar(f"wg{h}", warps_per_head) for h in range(heads)]  # bar.sync per head
+    Q = Buf("Q")
+    ring = [Buf(f"ring{r}") for r in range(RING)]
+    S = [[Buf(f"S{h}_{b}") for b in range(2)] for h in range(heads)]
+    bins = [Buf(f"bins{h}") for h in range(heads)]
+    bin_stores = {}
+
+    def producer():
+        Q.write(0)
+        q_full.arrive()
+        for t in range(ntile):
+            slot = t % RING
+            yield from wait(ring_empty[slot], ((t // RING) & 1) ^ 1, drop == "ring_empty")
+            ring[slot].write(t // RING)
+            ring_full[slot].arrive()
+            yield
+
+    def mma():
+        yield from wait(q_full, 0)
+        for t in range(ntile):
+            slot, buf = t % RING, t & 1
+            yield from wait(ring_full[slot], (t // RING) & 1)
+            yield from wait(s_free[buf], ((t >> 1) & 1) ^ 1, drop == "s_free")
+            for h in range(heads):
+                pipe.mma([(Q, 0), (ring[slot], t // RING)], [(S[h][buf], t >> 1, True)])
+            pipe.commit(ring_empty[slot])
+            pipe.commit(s_full[buf])
+            yield
+
+    def bar_sync(b, gen):
+        # bar.sync over the head's warps: arrive, then wait for this generation
+        b.arrive()
+        while b.done <= gen:
+            yield
+
+    def consumer(h):
+        syncs = 0
+        for t in range(ntile):
+            buf = t & 1
+            yield from wait(s_full[buf], (t >> 1) & 1, drop == "s_full")
+            S[h][buf].read_begin(t >> 1)
+            yield
+            S[h][buf].read_end()
+            s_free[buf].arrive()
+            if line_pass:
+                key = (h, t)
+                n = bin_stores.get(key, 0)
+                bins[h].write(t, fresh=n == 0)  # this warp's diagonal bins
+                bin_stores[key] = n + 1
+                yield from bar_sync(wg[h], syncs)  # every warp's bins are written
+                syncs += 1
+                bins[h].read_begin(t)
+                yield
+                bins[h].read_end()
+                if drop != "wg_after":
+                    yield from bar_sync(wg[h], syncs)  # bins are rewritten by the next tile
+                    syncs += 1
+            yield
+
+    roles = [producer(), mma()]
+    roles += [consumer(h) for h in range(heads) for _ in range(warps_per_head)]
+    return roles, pipe
+
+
+@pytest.mark.parametrize("ntile", [1, 2, 3, 5, 16])
+@pytest.mark.parametrize("line_pass", [False, True])
+@pytest.mark.parametrize("seed", range(25))
+def test_estimate_pass_protocol(ntile, line_pass, seed):
+    roles, pipe = estimate_roles(ntile, line_pass=line_pass)
+    run(roles, pipe, random.Random(seed * 1000 + ntile + 7 * line_pass))
+
+
 @pytest.mark.parametrize("model,drop", [
     ("attention", "k_empty"), ("attention", "v_empty"), ("attention", "s_free"),
     ("attention", "s_full"), ("attention", "p_empty"), ("attention", "p_full"),
     ("map", "empty"), ("map", "q_ready"), ("map", "acc_empty"), ("map", "acc_full"),
     ("map", "st_free"), ("map", "st_full"),
+    ("estimate", "ring_empty"), ("estimate", "s_free"), ("estimate", "s_full"),
+    ("estimate", "wg_after"),
 ])
 def test_each_wait_is_needed(model, drop):
     """With any one of the kernel's waits taken out, some interleaving
@@ -298,8 +386,10 @@ def test_each_wait_is_needed(model, drop):
     for seed in range(60):
         if model == "attention":
             roles, pipe = attention_roles(8, drop=drop)
-        else:
+        elif model == "map":
             roles, pipe = map_roles(6, drop=drop)
+        else:
+            roles, pipe = estimate_roles(6, drop=drop)
         try:
             run(roles, pipe, random.Random(seed))
         except AssertionError:
