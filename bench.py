@@ -39,10 +39,10 @@ import torch  # noqa: E402
 from dynamic_block_sparse_fp_b200 import synth  # noqa: E402
 
 METRIC = "prefill-attn tokens/s and effective TFLOPS (% bf16 peak) at 128k; speedup vs dense"
-# the library's kernels per step of fp_prefill_attn: estimate 12 (7 for the
+# the library's kernels per step of fp_prefill_attn: estimate 11 (6 for the
 # pattern's inputs, 3 for the query-aware heads' map, 2 for the vertical-slash
 # heads' lines), pattern 1, select 6, attention 1
-LAUNCHES_PER_STEP = 20
+LAUNCHES_PER_STEP = 19
 
 
 def kernel_traffic(source: str, workload: str):

@@ -429,11 +429,16 @@ cudaError_t run_map(const Dims &Dm, const T *q, float *qbar, const float *kbar_h
   return cudaGetLastError();
 }
 
-// The true last-block distribution (every head).
+// The true last-block distribution (every head), and K pooled into kbar with
+// its tf32 halves: by the tensor-core pass from the key tiles it streams, or
+// by its own pooling launch before the CUDA-core passes.
 template <class T>
-cudaError_t run_true_last(const Dims &Dm, const T *q, const T *k, float *true_last, void *ws,
-                          cudaStream_t st) {
-  if (last_block_tc_supported(Dm)) return launch_last_block_rows_tc(Dm, q, k, true_last, ws, st);
+cudaError_t run_true_last(const Dims &Dm, const T *q, const T *k, float *true_last, float *kbar,
+                          float *kbar_hi, float *kbar_lo, void *ws, cudaStream_t st) {
+  if (last_block_tc_supported(Dm))
+    return launch_last_block_rows_tc(Dm, q, k, true_last, kbar, kbar_hi, kbar_lo, ws, st);
+  pool_kernel<T><<<dim3(Dm.nb, Dm.hkv, Dm.bt), 256, 0, st>>>(k, kbar, Dm.n, Dm.d, Dm.bs, Dm.nb,
+                                                              0, nullptr, kbar_hi, kbar_lo);
   if (Dm.bs == 128 && Dm.d == 128) return run_last_rows<128, 128, T>(Dm, q, k, true_last, ws, st);
   if (Dm.bs == 128 && Dm.d == 64) return run_last_rows<128, 64, T>(Dm, q, k, true_last, ws, st);
   if (Dm.bs == 64 && Dm.d == 128) return run_last_rows<64, 128, T>(Dm, q, k, true_last, ws, st);
@@ -464,13 +469,17 @@ cudaError_t run_lines(const Dims &Dm, const T *q, const T *k, float *vert, float
   return run_last_lines<64, 64, T>(Dm, q, k, vert, slash, vs_only, ws, st);
 }
 
-// The pooled keys' tf32 halves, carved from the start of a workspace (the
-// staged estimate: they are dead before the last-block passes reuse it).
+// The pooled keys' tf32 halves in the staged estimate's workspace, after the
+// last-block passes' region (both are live at once: the first pass writes
+// them and the map reads them).
+size_t passes_ws_bytes(const Dims &D) {
+  return last_block_tc_supported(D) ? last_block_tc_ws_bytes(D) : carve_core(D, nullptr).bytes;
+}
 struct Split {
   float *hi, *lo;
 };
 Split carve_split(const Dims &Dm, void *ws) {
-  Carver c{static_cast<char *>(ws), 0};
+  Carver c{static_cast<char *>(ws), (passes_ws_bytes(Dm) + 255) & ~size_t(255)};
   const size_t n = size_t(Dm.bt) * Dm.hkv * Dm.nb * Dm.d;
   Split sp;
   sp.hi = c.take<float>(n);
@@ -483,11 +492,9 @@ cudaError_t run_estimate(const Dims &Dm, const T *q, const T *k, float *qbar, fl
                          float *map, float *est_last, float *true_last, float *vert,
                          float *slash, void *ws, cudaStream_t st) {
   const Split sp = carve_split(Dm, ws);
-  pool_kernel<T><<<dim3(Dm.nb, Dm.hkv, Dm.bt), 256, 0, st>>>(k, kbar, Dm.n, Dm.d, Dm.bs, Dm.nb,
-                                                              0, nullptr, sp.hi, sp.lo);
-  cudaError_t e = run_map<T>(Dm, q, qbar, sp.hi, sp.lo, map, est_last, nullptr, st);
+  cudaError_t e = run_true_last<T>(Dm, q, k, true_last, kbar, sp.hi, sp.lo, ws, st);
   if (e != cudaSuccess) return e;
-  e = run_true_last<T>(Dm, q, k, true_last, ws, st);
+  e = run_map<T>(Dm, q, qbar, sp.hi, sp.lo, map, est_last, nullptr, st);
   if (e != cudaSuccess) return e;
   return run_lines<T>(Dm, q, k, vert, slash, nullptr, ws, st);
 }
@@ -499,24 +506,20 @@ template <class T>
 cudaError_t run_decision(const Dims &Dm, const T *q, const T *k, float *qbar, float *kbar,
                          float *kbar_hi, float *kbar_lo, float *map, float *est_last,
                          float *true_last, void *ws, cudaStream_t st) {
-  pool_kernel<T><<<dim3(Dm.nb, Dm.hkv, Dm.bt), 256, 0, st>>>(k, kbar, Dm.n, Dm.d, Dm.bs, Dm.nb,
-                                                              0, nullptr, kbar_hi, kbar_lo);
+  cudaError_t e = run_true_last<T>(Dm, q, k, true_last, kbar, kbar_hi, kbar_lo, ws, st);
+  if (e != cudaSuccess) return e;
   pool_kernel<T><<<dim3(1, Dm.hq, Dm.bt), 256, 0, st>>>(q, qbar, Dm.n, Dm.d, Dm.bs, Dm.nb,
                                                          Dm.nb - 1, nullptr);
-  cudaError_t e = launch_map_logits_tc(Dm, qbar, kbar_hi, kbar_lo, map, nullptr, true, st);
+  e = launch_map_logits_tc(Dm, qbar, kbar_hi, kbar_lo, map, nullptr, true, st);
   if (e != cudaSuccess) return e;
   map_last_softmax_kernel<<<unsigned(Dm.bt * Dm.hq), 32, 0, st>>>(map, est_last, Dm.nb);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  return run_true_last<T>(Dm, q, k, true_last, ws, st);
+  return cudaGetLastError();
 }
 
 }  // namespace
 
 size_t estimate_ws_bytes(const Dims &D) {
-  const size_t passes =
-      last_block_tc_supported(D) ? last_block_tc_ws_bytes(D) : carve_core(D, nullptr).bytes;
-  return std::max(passes, map_split_bytes(D));
+  return ((passes_ws_bytes(D) + 255) & ~size_t(255)) + map_split_bytes(D);
 }
 
 cudaError_t launch_estimate_decision(const Dims &D, const void *q, const void *k, float *qbar,

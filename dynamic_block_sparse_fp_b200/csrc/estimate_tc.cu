@@ -27,8 +27,11 @@
 // CTA: one kv head, a pair of its query heads (A, B), a chunk of key tiles.
 // 12 warps: 0-3 consumer of head A, 4-7 consumer of head B, 8 TMA producer
 // (Q_last of both heads, K tiles through a 3-entry ring), 9 MMA issuer,
-// 10-11 idle (registers are granted per warpgroup).  TMEM 512 columns: S
-// double-buffered per head, head A [0,256), head B [256,512).
+// 10-11 pass 1 of a kv head's first pair: the block means of K (kbar and its
+// tf32 halves) from the key tiles already in the ring, so K is not streamed
+// a second time for its pooling; otherwise idle (registers are granted per
+// warpgroup).  TMEM 512 columns: S double-buffered per head, head A [0,256),
+// head B [256,512).
 #include <math.h>
 
 #include "fp_internal.cuh"
@@ -83,6 +86,7 @@ __global__ void __launch_bounds__(kThreads, 1) last_block_tc_kernel(
     int hq, int g, int n_tok, int nb, int q0, int qrows, int n_chunks, float *__restrict__ pm,
     float *__restrict__ pl, float *__restrict__ ptile, const float *__restrict__ lse2g,
     float *__restrict__ vert, float *__restrict__ sp, const int32_t *__restrict__ vs_only,
+    float *__restrict__ kbar, float *__restrict__ kbar_hi, float *__restrict__ kbar_lo,
     int *status) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   EstSmem &sm = *reinterpret_cast<EstSmem *>(
@@ -105,12 +109,15 @@ __global__ void __launch_bounds__(kThreads, 1) last_block_tc_kernel(
   const int j0 = chunk * kChunk;
   const int j1 = min(nb, j0 + kChunk);
   const int ntiles = j1 - j0;
+  // pass 1 of the first pair of a kv head also pools the kv head's keys
+  const bool pool = PASS == 1 && kbar != nullptr && pair == 0;
 
   if (threadIdx.x == 0) {
     mbar_init(&sm.q_full, 1);
     for (int r = 0; r < RING; ++r) {
       mbar_init(&sm.ring_full[r], 1);
-      mbar_init(&sm.ring_empty[r], 1);
+      // freed by the MMAs' commit, and by both pooling warps when they pool
+      mbar_init(&sm.ring_empty[r], pool ? 3 : 1);
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&sm.s_full[s], 1);
@@ -198,6 +205,58 @@ __global__ void __launch_bounds__(kThreads, 1) last_block_tc_kernel(
       if (!ok) {
         report(status, FP_ERR_TIMEOUT);
         *abort_flag = 1;
+      }
+    }
+  } else if (warp >= 10) {
+    // ------------------------------------------- K block means (pass 1) --
+    // thread p (0..63) takes d = 2p, 2p+1: one 32-bit word per key row of
+    // the 128-B swizzled tile half p / 32; the rows of a block are summed in
+    // order in fp32, and the mean written with its tf32 halves.
+    if (pool) {
+      const int p = threadIdx.x - 320;
+      // word p % 32 of the 128-B rows of tile half p / 32; its 16-B chunk sits
+      // at chunk ^ (row % 8) under the 128-B swizzle
+      const uint32_t half_off = uint32_t(p / 32) * HALF_BYTES;
+      const int wchunk = (p % 32) / 4, wbyte = (p % 4) * 4;
+      constexpr int kBpt = QLO ? 2 : 1;        // blocks per 128-key tile
+      constexpr int kBrows = BS / kBpt;        // rows of a block
+      const int nbk = (n_tok + kBrows - 1) / kBrows;  // blocks of the sequence
+      const size_t kv0 = (size_t(b) * hkv + kv) * nbk;
+      for (int t = 0; t < ntiles; ++t) {
+        const int slot = t % RING;
+        if (!__all_sync(0xffffffffu, mbar_wait(&sm.ring_full[slot], (t / RING) & 1, abort_flag))) {
+          if (lane == 0) {
+            report(status, FP_ERR_TIMEOUT);
+            *abort_flag = 1;
+          }
+          break;
+        }
+        const uint32_t base = smem_u32(sm.ring[slot]) + half_off + uint32_t(wbyte);
+        const int j = j0 + t;
+        const int krows = min(BS, n_tok - j * BS);  // keys of the tile (a partial last tile)
+#pragma unroll
+        for (int blk = 0; blk < kBpt; ++blk) {
+          const int r0 = blk * kBrows, r1 = min(krows, r0 + kBrows);
+          if (r1 <= r0) continue;
+          float s0 = 0.f, s1 = 0.f;  // d = 2p, 2p + 1
+          for (int r = r0; r < r1; ++r) {
+            uint32_t w;
+            asm volatile("ld.shared.b32 %0, [%1];"
+                         : "=r"(w)
+                         : "r"(base + uint32_t(r * 128 + ((wchunk ^ (r % 8)) * 16))));
+            s0 += __uint_as_float(w << 16);
+            s1 += __uint_as_float(w & 0xFFFF0000u);
+          }
+          const size_t o = (kv0 + size_t(j) * kBpt + blk) * HD + 2 * p;
+          const float m0 = s0 / float(r1 - r0), m1 = s1 / float(r1 - r0);
+          const float h0 = tf32_hi(m0), h1 = tf32_hi(m1);
+          *reinterpret_cast<float2 *>(kbar + o) = make_float2(m0, m1);
+          *reinterpret_cast<float2 *>(kbar_hi + o) = make_float2(h0, h1);
+          *reinterpret_cast<float2 *>(kbar_lo + o) = make_float2(m0 - h0, m1 - h1);
+        }
+        // every lane's reads of the slot are done before it may be refilled
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.ring_empty[slot]);
       }
     }
   } else if (warp < 8) {
@@ -483,9 +542,12 @@ bool encode_qk(const Dims &D, const void *q, const void *k, CUtensorMap *mq, CUt
 
 size_t last_block_tc_ws_bytes(const Dims &D) { return carve_tc(D, nullptr).bytes; }
 
-// Pass 1, the log-sum-exps and the pooled true distribution, for every head.
+// Pass 1, the log-sum-exps and the pooled true distribution, for every head;
+// with kbar (and its halves) non-null, pass 1 also writes the block means of
+// K from the key tiles it streams.
 cudaError_t launch_last_block_rows_tc(const Dims &D, const void *q, const void *k,
-                                      float *true_last, void *ws, cudaStream_t st) {
+                                      float *true_last, float *kbar, float *kbar_hi,
+                                      float *kbar_lo, void *ws, cudaStream_t st) {
   CUtensorMap mq, mk;
   if (!encode_qk(D, q, k, &mq, &mk)) return cudaErrorInvalidValue;
   const TcWs w = carve_tc(D, ws);
@@ -500,7 +562,7 @@ cudaError_t launch_last_block_rows_tc(const Dims &D, const void *q, const void *
     cudaFuncSetAttribute(pass1, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmemBytes));
     pass1<<<grid, kThreads, kSmemBytes, st>>>(mq, mk, D.hq, D.g, D.n, nt, q0, qrows, n_chunks,
                                               w.pm, w.pl, w.ptile, nullptr, nullptr, nullptr,
-                                              nullptr, status);
+                                              nullptr, kbar, kbar_hi, kbar_lo, status);
     lse2_combine_kernel<<<(rows + 127) / 128, 128, 0, st>>>(w.pm, w.pl, w.lse2, rows, n_chunks);
     mass<<<dim3((nt + 7) / 8, unsigned(heads)), 256, 0, st>>>(w.ptile, w.lse2, true_last, nt,
                                                               qrows);
@@ -535,7 +597,7 @@ cudaError_t launch_last_block_lines_tc(const Dims &D, const void *q, const void 
     cudaFuncSetAttribute(pass2, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmemBytes));
     pass2<<<grid, kThreads, kSmemBytes, st>>>(mq, mk, D.hq, D.g, D.n, nt, q0, qrows, n_chunks,
                                               nullptr, nullptr, nullptr, w.lse2, vert, w.sp,
-                                              vs_only, status);
+                                              vs_only, nullptr, nullptr, nullptr, status);
   };
   if (D.bs == BS && qrows == BS)
     run(last_block_tc_kernel<2, 0, false>);

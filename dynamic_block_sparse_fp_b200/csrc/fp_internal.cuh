@@ -76,8 +76,11 @@ cudaError_t launch_estimate_lines_vs(const Dims &D, const void *q, const void *k
 bool last_block_tc_supported(const Dims &D);
 int last_block_tc_tiles(const Dims &D);
 size_t last_block_tc_ws_bytes(const Dims &D);
+// (with kbar non-null, pass 1 also writes the block means of K with their
+// tf32 halves, in place of a separate pooling of K)
 cudaError_t launch_last_block_rows_tc(const Dims &D, const void *q, const void *k,
-                                      float *true_last, void *ws, cudaStream_t st);
+                                      float *true_last, float *kbar, float *kbar_hi,
+                                      float *kbar_lo, void *ws, cudaStream_t st);
 cudaError_t launch_last_block_lines_tc(const Dims &D, const void *q, const void *k, float *vert,
                                        const int32_t *vs_only, float **sp_out, void *ws,
                                        cudaStream_t st);

@@ -290,13 +290,16 @@ def test_map_protocol(ntile, nc, seed):
 # through a ring of 3, S double-buffered per head in TMEM (both heads' S of a
 # tile in one buffer index), four consumer warps per head; in the second pass
 # each head's warps exchange diagonal bins through shared memory between two
-# warpgroup barriers per tile.
+# warpgroup barriers per tile; in the first pass of a kv head's first pair two
+# more warps read every key tile of the ring for the block means of K, and a
+# ring slot is free once the MMAs and both of them are done with it.
 
-def estimate_roles(ntile, RING=3, heads=2, warps_per_head=4, line_pass=True, drop=None):
+def estimate_roles(ntile, RING=3, heads=2, warps_per_head=4, line_pass=True, pool=False,
+                   drop=None):
     pipe = Pipe()
     q_full = Bar("q_full", 1)
     ring_full = [Bar(f"ring_full{r}", 1) for r in range(RING)]
-    ring_empty = [Bar(f"ring_empty{r}", 1) for r in range(RING)]
+    ring_empty = [Bar(f"ring_empty{r}", 3 if pool else 1) for r in range(RING)]
     s_full = [Bar(f"s_full{b}", 1) for b in range(2)]
     s_free = [Bar(f"s_free{b}", heads * warps_per_head) for b in range(2)]
     wg = [Bar(f"wg{h}", warps_per_head) for h in range(heads)]  # bar.sync per head
@@ -358,17 +361,28 @@ def estimate_roles(ntile, RING=3, heads=2, warps_per_head=4, line_pass=True, dro
                     syncs += 1
             yield
 
+    def pooler():
+        for t in range(ntile):
+            slot = t % RING
+            yield from wait(ring_full[slot], (t // RING) & 1, drop == "pool_full")
+            ring[slot].read_begin(t // RING)
+            yield
+            ring[slot].read_end()
+            ring_empty[slot].arrive()
+
     roles = [producer(), mma()]
     roles += [consumer(h) for h in range(heads) for _ in range(warps_per_head)]
+    if pool:
+        roles += [pooler(), pooler()]
     return roles, pipe
 
 
 @pytest.mark.parametrize("ntile", [1, 2, 3, 5, 16])
-@pytest.mark.parametrize("line_pass", [False, True])
+@pytest.mark.parametrize("line_pass,pool", [(False, False), (False, True), (True, False)])
 @pytest.mark.parametrize("seed", range(25))
-def test_estimate_pass_protocol(ntile, line_pass, seed):
-    roles, pipe = estimate_roles(ntile, line_pass=line_pass)
-    run(roles, pipe, random.Random(seed * 1000 + ntile + 7 * line_pass))
+def test_estimate_pass_protocol(ntile, line_pass, pool, seed):
+    roles, pipe = estimate_roles(ntile, line_pass=line_pass, pool=pool)
+    run(roles, pipe, random.Random(seed * 1000 + ntile + 7 * line_pass + 13 * pool))
 
 
 @pytest.mark.parametrize("model,drop", [
@@ -377,7 +391,7 @@ def test_estimate_pass_protocol(ntile, line_pass, seed):
     ("map", "empty"), ("map", "q_ready"), ("map", "acc_empty"), ("map", "acc_full"),
     ("map", "st_free"), ("map", "st_full"),
     ("estimate", "ring_empty"), ("estimate", "s_free"), ("estimate", "s_full"),
-    ("estimate", "wg_after"),
+    ("estimate", "wg_after"), ("estimate_pool", "pool_full"), ("estimate_pool", "ring_empty"),
 ])
 def test_each_wait_is_needed(model, drop):
     """With any one of the kernel's waits taken out, some interleaving
@@ -388,8 +402,10 @@ def test_each_wait_is_needed(model, drop):
             roles, pipe = attention_roles(8, drop=drop)
         elif model == "map":
             roles, pipe = map_roles(6, drop=drop)
-        else:
+        elif model == "estimate":
             roles, pipe = estimate_roles(6, drop=drop)
+        else:
+            roles, pipe = estimate_roles(6, line_pass=False, pool=True, drop=drop)
         try:
             run(roles, pipe, random.Random(seed))
         except AssertionError:
