@@ -164,6 +164,10 @@ size_t fp_workspace_size(const fp_shape *shape, int which_call);
  *   slash     [Bt,Hq,N]     fp32  slash[o] = sum over r of P[r, N-R+r-o]
  * where P is the causal softmax of q.k/sqrt(d) for the last block's R
  * queries (R = B, or the partial last block's length).
+ * Arithmetic: fp32 accumulation throughout.  The map's logits are tensor-core
+ * products of the fp32 pooled vectors split into tf32 halves (3 products per
+ * pair), off by at most about 2^-19 of sum_k |qbar_k kbar_k| / sqrt(d); the
+ * last block's scores are bf16 tensor-core products of q and k.
  * Workspace: fp_workspace_size(shape, FP_CALL_ESTIMATE).
  */
 fp_status fp_estimate(const fp_shape *shape, const void *q, const void *k,
