@@ -166,8 +166,9 @@ size_t fp_workspace_size(const fp_shape *shape, int which_call);
  * queries (R = B, or the partial last block's length).
  * Arithmetic: fp32 accumulation throughout.  The map's logits are tensor-core
  * products of the fp32 pooled vectors split into tf32 halves (3 products per
- * pair), off by at most about 2^-19 of sum_k |qbar_k kbar_k| / sqrt(d); the
- * last block's scores are bf16 tensor-core products of q and k.
+ * pair), off by at most about 2^-19 of sum_k |qbar_k kbar_k| / sqrt(d); for
+ * bf16 inputs the last block's scores are tensor-core products of q and k
+ * (fp32 inputs: fp32 products on the CUDA cores).
  * Workspace: fp_workspace_size(shape, FP_CALL_ESTIMATE).
  */
 fp_status fp_estimate(const fp_shape *shape, const void *q, const void *k,
