@@ -551,16 +551,8 @@ __global__ void __launch_bounds__(192, 2) attn_tc_kernel(
 
 // 2-D bf16 tensor map over [rows x 128] with a box of [box_rows x 64].
 bool encode_map(CUtensorMap *map, const void *ptr, uint64_t rows, uint32_t box_rows) {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (!fn) {
-    cudaDriverEntryPointQueryResult qr;
-    void *p = nullptr;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &qr) !=
-            cudaSuccess ||
-        qr != cudaDriverEntryPointSuccess || !p)
-      return false;
-    fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  }
+  const PFN_cuTensorMapEncodeTiled_v12000 fn = tensor_map_encoder();
+  if (!fn) return false;
   const cuuint64_t dims[2] = {cuuint64_t(HD), cuuint64_t(rows)};
   const cuuint64_t strides[1] = {cuuint64_t(HD) * 2};
   const cuuint32_t box[2] = {64, box_rows};

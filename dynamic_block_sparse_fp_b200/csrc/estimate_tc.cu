@@ -481,16 +481,8 @@ __global__ void __launch_bounds__(256) tile_mass_kernel(const float *__restrict_
 }
 
 bool encode_rows(CUtensorMap *map, const void *ptr, uint64_t rows) {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (!fn) {
-    cudaDriverEntryPointQueryResult qr;
-    void *p = nullptr;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &qr) !=
-            cudaSuccess ||
-        qr != cudaDriverEntryPointSuccess || !p)
-      return false;
-    fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  }
+  const PFN_cuTensorMapEncodeTiled_v12000 fn = tensor_map_encoder();
+  if (!fn) return false;
   const cuuint64_t dims[2] = {cuuint64_t(HD), cuuint64_t(rows)};
   const cuuint64_t strides[1] = {cuuint64_t(HD) * 2};
   const cuuint32_t box[2] = {64, 128};

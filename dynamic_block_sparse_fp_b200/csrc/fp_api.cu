@@ -4,6 +4,7 @@
 #include <math.h>
 
 #include <algorithm>
+#include <atomic>
 #include <mutex>
 #include <vector>
 
@@ -26,6 +27,20 @@ int *device_status_ptr() {
     if (cudaGetSymbolAddress(&p, g_fp_status) == cudaSuccess) ptrs[dev] = static_cast<int *>(p);
   }
   return ptrs[dev];
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  // a function-local static is initialised once, under the C++ runtime's lock
+  static const PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
+    cudaDriverEntryPointQueryResult qr;
+    void *p = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &qr) !=
+            cudaSuccess ||
+        qr != cudaDriverEntryPointSuccess)
+      p = nullptr;
+    return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }();
+  return fn;
 }
 
 // The streams of fp_prefill_attn_host besides the caller's: host-to-device
@@ -124,16 +139,16 @@ fp_status check_ws(void *ws, size_t have, size_t need) {
 }
 
 fp_status check_device() {
-  static int cc[64] = {0};
+  static std::atomic<int> cc[64];  // compute capability major, 0 = not yet read
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return FP_ERR_CUDA;
-  if (cc[dev] == 0) {
-    int major = 0;
+  int major = cc[dev].load(std::memory_order_relaxed);
+  if (major == 0) {
     if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
       return FP_ERR_CUDA;
-    cc[dev] = major;
+    cc[dev].store(major, std::memory_order_relaxed);
   }
-  return cc[dev] == 10 ? FP_OK : FP_ERR_UNSUPPORTED;
+  return major == 10 ? FP_OK : FP_ERR_UNSUPPORTED;
 }
 
 fp_status cuda_status(cudaError_t e) { return e == cudaSuccess ? FP_OK : FP_ERR_CUDA; }

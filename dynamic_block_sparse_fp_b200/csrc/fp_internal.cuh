@@ -38,6 +38,8 @@ struct Carver {
 };
 
 int *device_status_ptr();  // per-device status word (fp_api.cu)
+// The driver's cuTensorMapEncodeTiled (looked up once, thread-safe), or null.
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder();
 
 // Stage launchers (each returns cudaGetLastError() of its launches).
 size_t estimate_ws_bytes(const Dims &D);

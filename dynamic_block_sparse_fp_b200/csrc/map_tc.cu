@@ -305,16 +305,8 @@ __global__ void __launch_bounds__(320, 1) map_logits_tc_kernel(
 
 // 2-D fp32 tensor map over [rows x d] with a box of [128 rows x 32].
 bool encode_f32(CUtensorMap *m, const void *ptr, uint64_t rows, int d) {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (!fn) {
-    cudaDriverEntryPointQueryResult qr;
-    void *p = nullptr;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &qr) !=
-            cudaSuccess ||
-        qr != cudaDriverEntryPointSuccess || !p)
-      return false;
-    fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  }
+  const PFN_cuTensorMapEncodeTiled_v12000 fn = tensor_map_encoder();
+  if (!fn) return false;
   const cuuint64_t dims[2] = {cuuint64_t(d), cuuint64_t(rows)};
   const cuuint64_t strides[1] = {cuuint64_t(d) * 4};
   const cuuint32_t box[2] = {KC, MT};

@@ -35,6 +35,7 @@
 // which the radix select then takes as lines of a sequence of nb tokens
 // with block size 1 (a column is a key block, an offset one block distance).
 #include <algorithm>
+#include <atomic>
 #include <mutex>
 
 #include "fp_internal.cuh"
@@ -1060,16 +1061,16 @@ __global__ void stats_kernel(const int32_t *__restrict__ counts,
 
 // Streaming multiprocessors of the current device (cached per device).
 int sm_count() {
-  static int cache[64] = {0};
+  static std::atomic<int> cache[64];  // 0 = not yet read
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
-  if (cache[dev] == 0) {
-    int n = 0;
+  int n = cache[dev].load(std::memory_order_relaxed);
+  if (n == 0) {
     if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1)
       n = 148;
-    cache[dev] = n;
+    cache[dev].store(n, std::memory_order_relaxed);
   }
-  return cache[dev];
+  return n;
 }
 
 size_t select_ws_bytes(const Dims &D) {
