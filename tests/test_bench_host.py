@@ -59,3 +59,25 @@ def test_committed_record_names_a_real_kernel_and_the_bench_workload():
     assert rec["workload"] == "llama8b_n131072"
     assert len(rec["source_sha256"]) == 64
     assert rec["bytes_per_launch"] >= 2 * 1_073_741_824 + 2 * 268_435_456
+
+
+def test_reference_arm_prints_the_contract_line():
+    """`bench.py --impl reference` (the oracle timed on the host cores) prints
+    one JSON line with the headline metric, the reference tag, a cpu_baseline
+    describing the run and an e2e entry with no host-device copies."""
+    import subprocess
+    import sys
+    r = subprocess.run([sys.executable, os.path.join(bench.ROOT, "bench.py"), "--impl",
+                        "reference", "--workload", "tiny_n1024", "--steps", "1", "--warmup", "0"],
+                       capture_output=True, text=True, timeout=600, cwd=bench.ROOT)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [json.loads(x) for x in r.stdout.splitlines() if x.startswith("{")]
+    assert len(lines) == 1
+    d = lines[0]
+    assert d["impl"] == "reference" and d["metric"] == bench.METRIC
+    assert d["unit"] == "tokens/s" and d["higher_is_better"] is True and d["value"] > 0
+    assert d["config"]["workload"] == "tiny_n1024"
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
+    assert d["cpu_baseline"]["value"] == d["value"]
+    assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}
